@@ -1,0 +1,890 @@
+// Chunkwise-parallel forward pass of the Muir gated delta rule.
+//
+// Notation for one chunk of C tokens (local index t = 0..C-1) with start state
+// S0, per (batch, head):
+//   Gam_{t<-s} = prod_{u=s+1..t} alpha_u (per key channel), Gam_t = prod_{u<=t},
+//   Gsuf_t = prod_{u>t} (to the chunk end), Gam_C = prod over the chunk.
+//   K, A = e*k, Qt = r*g*q (key rows), U = w*v (value columns).
+//   M^kk_ts = k_t.Gam_{t<-s}.k_s, M^ka_ts = k_t.Gam_{t<-s}.a_s          (s < t)
+//   N^qk_ts = qt_t.Gam_{t<-s}.k_s, N^qa_ts = qt_t.Gam_{t<-s}.a_s        (s <= t)
+//   T = (I + M^ka)^-1,  W = T (K*Gam),  Ut = T M^kk U
+//   Phi  = Diag(Gam_C) - (A*Gsuf)^T W            (dk x dk)
+//   Psi  = (K*Gsuf)^T U - (A*Gsuf)^T Ut          (dk x dv)
+//   Q'   = Qt*Gam - N^qa W                        (C x dk)
+//   Oloc = N^qk U - N^qa Ut                       (C x dv)
+// and the chunk acts on the state as an affine map:
+//   S_C = Phi S0 + Psi,   O = Q' S0 + Oloc,   y = z * O.
+// (Derivation: unroll the recurrence inside the chunk; the prediction vector P
+// of all tokens solves (I + M^ka) P = (K*Gam) S0 + M^kk U.)
+//
+// Decay products are boundary-pivoted (openai-hub article, section on the TPU
+// chunkwise algorithm; liuch.name post, third bullet): the chunk is cut into
+// blocks of SB = 16 tokens. For s in block I and t in a later block J,
+//   Gam_{t<-s} = suf_s * mid(I,J) * pre_t
+// with suf_s = prod_{u=s+1..end(I)}, pre_t = prod_{u=start(J)..t} and mid the
+// product of whole blocks in between: every factor is a product of alphas, so
+// it lies in [0, 1] and nothing is divided. Off-diagonal Gram blocks then are
+// tensor-core GEMMs of pivot-scaled operands; the 16x16 diagonal blocks are
+// computed exactly on the CUDA cores with running products.
+//
+// Kernels (one CTA of 128 threads per (batch, head, chunk) unless noted):
+//   decay_kernel      pre, suf, Gam_t, Gsuf_t            -> workspace
+//   gram_off_kernel   off-diagonal blocks of the 4 Grams (tcgen05)
+//   gram_diag_kernel  diagonal 16x16 blocks (CUDA cores), one CTA per block
+//   solve_kernel      T: exact 16x16 leaves, then recursive 2x2 block merges
+//                     T21 = -T22 M21 T11 on tcgen05 (block-Neumann recursion)
+//   maps_kernel       W, Ut, Phi, Psi, Q', Oloc (tcgen05)  -> workspace
+//   compose_kernel    (chunk 256) composes two 128-token half-chunk maps
+//   scan_kernel       sequential over chunks per (batch, head, 32-column slab):
+//                     [S_C; O] = [Phi; Q'] S0 + [Psi; Oloc], y = z*O (tcgen05)
+#pragma once
+
+#include "tc.cuh"
+
+namespace muir {
+
+constexpr int SB = 16;  // pivot block length (tokens)
+
+struct ChunkParams {
+  int B;
+  int64_t T;
+  int H, dk, dv;
+  int Cs;    // tokens per local unit (min(chunk, 128))
+  int nsub;  // T / Cs
+  int C;     // chunk length of the state scan (Cs or 2*Cs)
+  const void *q, *k, *v, *e, *w, *g, *z;
+  const float* la;
+  const float* r;
+  const float* S0;
+  // workspace
+  float* dec;  // [nsubtot][4][Cs][dk]: pre, suf, Gam, Gsuf
+  float* gr;   // [nsubtot][4][Cs][Cs]: M^kk, M^ka, N^qk, N^qa
+  float* tt;   // [nsubtot][Cs][Cs]
+  float* ma;   // [nunits][dk + C][dk]: Phi ; Q'
+  float* mb;   // [nunits][dk + C][dv]: Psi ; Oloc
+  float* ma2;  // composition scratch for chunk 256 (same layout as ma at C = 2*Cs)
+  float* mb2;
+  // outputs
+  void* y;
+  float* S_T;
+  float* S_chunks;  // optional [B,H,T/C,dk,dv]: state at the start of every chunk
+};
+
+struct SubIdx {
+  int b, h, n;
+  int64_t tok0;
+};
+
+__device__ __forceinline__ SubIdx sub_of(const ChunkParams& p, int sid, int units_per_seq, int unit_len) {
+  SubIdx s;
+  s.n = sid % units_per_seq;
+  const int bh = sid / units_per_seq;
+  s.h = bh % p.H;
+  s.b = bh / p.H;
+  s.tok0 = (int64_t)s.n * unit_len;
+  return s;
+}
+
+// Offset of element 0 of token `tok` of (b, h) in a [B,T,H,d] tensor.
+__device__ __forceinline__ int64_t toff(const ChunkParams& p, int b, int64_t tok, int h, int d) {
+  return (((int64_t)b * p.T + tok) * p.H + h) * d;
+}
+
+__device__ __forceinline__ void ld8f(const float* p, float (&o)[8]) { Elt<float>::ld8(p, o); }
+
+__device__ __forceinline__ Tile sub_tile(const Tile& t, int k0, int mn0) {
+  const uint32_t off = (uint32_t)(k0 >> 3) * 128u + (uint32_t)(mn0 >> 3) * t.sbo;
+  return Tile{t.hi + off, t.lo + off, t.sbo};
+}
+
+__device__ __forceinline__ void zero_smem(uint32_t base, uint32_t bytes) {
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  for (uint32_t o = threadIdx.x * 16u; o < bytes; o += blockDim.x * 16u) sts128(base + o, z);
+}
+
+__device__ __forceinline__ uint32_t tmem_cols_for(int n) {
+  return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : n <= 256 ? 256u : 512u;
+}
+
+// CTA prologue shared by the tensor-core kernels: TMEM allocation + mbarrier.
+struct TcCta {
+  uint32_t tmem;
+  uint32_t ncols;
+  __device__ __forceinline__ void init(uint32_t* slot, uint64_t* bar, uint32_t cols) {
+    ncols = cols;
+    if ((threadIdx.x >> 5) == 0) tmem_alloc(slot, cols);
+    if (threadIdx.x == 0) mbar_init(bar, 1);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    tmem = *slot;
+  }
+  __device__ __forceinline__ void finish() {
+    tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, ncols);
+  }
+};
+
+// Input row helpers: 8 consecutive channels of token `tok`.
+template <typename T>
+struct Rows {
+  const ChunkParams& p;
+  int b, h;
+  __device__ __forceinline__ void k(int64_t tok, int c8, float (&o)[8]) const {
+    Elt<T>::ld8(static_cast<const T*>(p.k) + toff(p, b, tok, h, p.dk) + c8, o);
+  }
+  __device__ __forceinline__ void a(int64_t tok, int c8, float (&o)[8]) const {
+    float kk[8], ee[8];
+    Elt<T>::ld8(static_cast<const T*>(p.k) + toff(p, b, tok, h, p.dk) + c8, kk);
+    Elt<T>::ld8(static_cast<const T*>(p.e) + toff(p, b, tok, h, p.dk) + c8, ee);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = ee[i] * kk[i];
+  }
+  __device__ __forceinline__ void qt(int64_t tok, int c8, float (&o)[8]) const {
+    float qq[8], gg[8], rr[8];
+    Elt<T>::ld8(static_cast<const T*>(p.q) + toff(p, b, tok, h, p.dk) + c8, qq);
+    Elt<T>::ld8(static_cast<const T*>(p.g) + toff(p, b, tok, h, p.dk) + c8, gg);
+    ld8f(p.r + (int64_t)h * p.dk + c8, rr);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = rr[i] * gg[i] * qq[i];
+  }
+  __device__ __forceinline__ void u(int64_t tok, int c8, float (&o)[8]) const {
+    float vv[8], ww[8];
+    Elt<T>::ld8(static_cast<const T*>(p.v) + toff(p, b, tok, h, p.dv) + c8, vv);
+    Elt<T>::ld8(static_cast<const T*>(p.w) + toff(p, b, tok, h, p.dv) + c8, ww);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = ww[i] * vv[i];
+  }
+};
+
+// ---------------------------------------------------------------------------
+// decay_kernel: one CTA per unit, thread = key channel.
+//   pre[t]  = prod_{u=start(block)..t} alpha_u     suf[t]  = prod_{u=t+1..end(block)} alpha_u
+//   gam[t]  = prod_{u=0..t} alpha_u               gsuf[t] = prod_{u=t+1..Cs-1} alpha_u
+// built as running products of alphas inside blocks and products of whole-block
+// totals across blocks (no division, every factor in [0, 1]).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) decay_kernel(ChunkParams p) {
+  const int dk = p.dk, Cs = p.Cs;
+  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  const int i = threadIdx.x;
+  if (i >= dk) return;
+  float* pre = p.dec + (int64_t)blockIdx.x * 4 * Cs * dk;
+  float* suf = pre + Cs * dk;
+  float* gam = suf + Cs * dk;
+  float* gsuf = gam + Cs * dk;
+  const float* la = p.la + toff(p, s.b, s.tok0, s.h, dk) + i;
+  const int64_t stride = (int64_t)p.H * dk;
+  float run = 1.f, before = 1.f;
+  for (int t = 0; t < Cs; ++t) {
+    const float a = expf(__ldg(la + t * stride));
+    if ((t & (SB - 1)) == 0) {
+      before *= run;
+      run = a;
+    } else {
+      run *= a;
+    }
+    pre[t * dk + i] = run;
+    gam[t * dk + i] = before * run;
+  }
+  float after = 1.f, srun = 1.f;
+  for (int t = Cs - 1; t >= 0; --t) {
+    if ((t & (SB - 1)) == SB - 1) {
+      srun = 1.f;
+      if (t + SB < Cs) after *= pre[(t + SB) * dk + i];
+    }
+    suf[t * dk + i] = srun;
+    gsuf[t * dk + i] = srun * after;
+    srun *= expf(__ldg(la + t * stride));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// gram_off_kernel: off-diagonal 16-blocks of M^kk, M^ka, N^qk, N^qa.
+// For column block I (pivot = its last token), rows t in later blocks J:
+//   G[t, s] = sum_i (X_t,i pre_t,i mid(I,J)_i) (Y_s,i suf_s,i)
+// M = 128 rows (t), N = 16 (s in block I), K = dk. Column blocks are visited
+// from the last to the first so mid(I,J) = mid(I+1,J) * tot_{I+1} stays a
+// product of block totals. Writes every entry except the diagonal blocks
+// (upper blocks get 0).
+// ---------------------------------------------------------------------------
+template <int DK, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) gram_off_kernel(ChunkParams p) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int Cs = p.Cs, nb = Cs / SB;
+  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  constexpr uint32_t LB = 128u * DK * 2u, RB = SB * DK * 2u;
+  const uint32_t base = smem_u32(sm);
+  const Tile L{base, base + LB, DK * 16u};
+  const Tile RK{base + 2 * LB, base + 2 * LB + RB, DK * 16u};
+  const Tile RA{base + 2 * LB + 2 * RB, base + 2 * LB + 3 * RB, DK * 16u};
+  float* midtab = reinterpret_cast<float*>(sm + 2 * LB + 4 * RB);  // [nb][DK]
+  zero_smem(base, 2 * LB);
+  TcCta cta;
+  cta.init(&tslot, &bar, tmem_cols_for(4 * Cs));
+  const float* pre = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
+  const float* suf = pre + Cs * DK;
+  const Rows<T> rows{p, s.b, s.h};
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t id = idesc_bf16(128, SB, 0, 0);
+  for (int I = nb - 2; I >= 0 && drv.ok; --I) {
+    for (int x = tid; x < nb * DK; x += 128) {
+      const int J = x / DK, i = x % DK;
+      if (J == I + 1) midtab[x] = 1.f;
+      else if (J > I + 1) midtab[x] *= pre[(SB * (I + 1) + SB - 1) * DK + i];
+    }
+    for (int x = tid; x < SB * (DK / 8); x += 128) {
+      const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      const int t = SB * I + rr;
+      float kk[8], aa[8], sf[8], vk[8], va[8];
+      rows.k(s.tok0 + t, c8, kk);
+      rows.a(s.tok0 + t, c8, aa);
+      ld8f(suf + t * DK + c8, sf);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { vk[j] = kk[j] * sf[j]; va[j] = aa[j] * sf[j]; }
+      put_k(RK, rr, c8, vk);
+      put_k(RA, rr, c8, va);
+    }
+    __syncthreads();
+    const int t0 = SB * (I + 1);
+    for (int pass = 0; pass < 2 && drv.ok; ++pass) {
+      for (int x = tid; x < (Cs - t0) * (DK / 8); x += 128) {
+        const int t = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+        float xv[8], pr[8], md[8];
+        if (pass == 0) rows.k(s.tok0 + t, c8, xv);
+        else rows.qt(s.tok0 + t, c8, xv);
+        ld8f(pre + t * DK + c8, pr);
+        const float* mp = midtab + (t / SB) * DK + c8;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) md[j] = mp[j];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xv[j] *= pr[j] * md[j];
+        put_k(L, t, c8, xv);
+      }
+      const uint32_t c0 = (pass == 0 ? 0u : 2u * Cs) + SB * I;
+      drv.run([&] {
+        mma_tiles(cta.tmem + c0, L, RK, DK / 16, id, NS, false);
+        mma_tiles(cta.tmem + c0 + Cs, L, RA, DK / 16, id, NS, false);
+      });
+    }
+  }
+  // Epilogue: thread = row t.
+  const int t = tid;
+  const int J = t / SB;
+  float* out = p.gr + (int64_t)blockIdx.x * 4 * Cs * Cs;
+  for (int gidx = 0; gidx < 4; ++gidx) {
+    for (int c0 = 0; c0 < Cs; c0 += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + tmem_lane_base(warp) + gidx * Cs + c0, v);
+      const int I = c0 / SB;
+      if (t < Cs && I != J && drv.ok) {
+        float* o = out + ((int64_t)gidx * Cs + t) * Cs + c0;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+          float4 w4 = (I < J) ? make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(o + j) = w4;
+        }
+      }
+    }
+  }
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// gram_diag_kernel: the 16x16 diagonal blocks, exactly, on CUDA cores.
+// One CTA per (unit, block); thread = (row t, channel group cg of DK/8 channels).
+// For s = t, t-1, ..., the running product Gam_{t<-s} = Gam_{t<-s+1} * alpha_{s+1}
+// multiplies both key rows; partial sums over the channel group are reduced
+// across the 8 lanes of the row.
+// ---------------------------------------------------------------------------
+template <int DK, typename T>
+__global__ void __launch_bounds__(128) gram_diag_kernel(ChunkParams p) {
+  constexpr int CH = DK / 8;
+  __shared__ __align__(16) float sk[SB][DK], sq[SB][DK], sa[SB][DK], sal[SB][DK];
+  const int Cs = p.Cs, nb = Cs / SB;
+  const int sid = blockIdx.x / nb, J = blockIdx.x % nb;
+  const SubIdx s = sub_of(p, sid, p.nsub, Cs);
+  const Rows<T> rows{p, s.b, s.h};
+  for (int x = threadIdx.x; x < SB * (DK / 8); x += 128) {
+    const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+    const int64_t tok = s.tok0 + SB * J + rr;
+    float kk[8], aa[8], qq[8], la[8];
+    rows.k(tok, c8, kk);
+    rows.a(tok, c8, aa);
+    rows.qt(tok, c8, qq);
+    ld8f(p.la + toff(p, s.b, tok, s.h, DK) + c8, la);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      sk[rr][c8 + j] = kk[j];
+      sa[rr][c8 + j] = aa[j];
+      sq[rr][c8 + j] = qq[j];
+      sal[rr][c8 + j] = expf(la[j]);
+    }
+  }
+  __syncthreads();
+  const int t = threadIdx.x >> 3, cg = threadIdx.x & 7;
+  const int c0 = cg * CH;
+  float xk[CH], xq[CH], gm[CH];
+#pragma unroll
+  for (int j = 0; j < CH; ++j) { xk[j] = sk[t][c0 + j]; xq[j] = sq[t][c0 + j]; gm[j] = 1.f; }
+  float acc[4][SB];
+#pragma unroll
+  for (int ss = SB - 1; ss >= 0; --ss) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    if (ss <= t) {
+#pragma unroll
+      for (int j = 0; j < CH; ++j) {
+        const float yk = sk[ss][c0 + j] * gm[j], ya = sa[ss][c0 + j] * gm[j];
+        a0 += xk[j] * yk; a1 += xk[j] * ya; a2 += xq[j] * yk; a3 += xq[j] * ya;
+      }
+#pragma unroll
+      for (int j = 0; j < CH; ++j) gm[j] *= sal[ss][c0 + j];
+    }
+    acc[0][ss] = a0; acc[1][ss] = a1; acc[2][ss] = a2; acc[3][ss] = a3;
+  }
+#pragma unroll
+  for (int gidx = 0; gidx < 4; ++gidx)
+#pragma unroll
+    for (int ss = 0; ss < SB; ++ss) {
+      float v = acc[gidx][ss];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      acc[gidx][ss] = v;
+    }
+#pragma unroll
+  for (int gidx = 0; gidx < 4; ++gidx) {
+    if (cg != gidx) continue;  // lane cg of the row writes Gram cg
+    float* o = p.gr + (((int64_t)sid * 4 + gidx) * Cs + SB * J + t) * Cs + SB * J;
+    const bool strict = gidx < 2;  // M^kk, M^ka exclude the diagonal
+#pragma unroll
+    for (int ss = 0; ss < SB; ss += 4) {
+      float4 w4;
+      w4.x = (ss + 0 < t || (!strict && ss + 0 == t)) ? acc[gidx][ss + 0] : 0.f;
+      w4.y = (ss + 1 < t || (!strict && ss + 1 == t)) ? acc[gidx][ss + 1] : 0.f;
+      w4.z = (ss + 2 < t || (!strict && ss + 2 == t)) ? acc[gidx][ss + 2] : 0.f;
+      w4.w = (ss + 3 < t || (!strict && ss + 3 == t)) ? acc[gidx][ss + 3] : 0.f;
+      *reinterpret_cast<float4*>(o + ss) = w4;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// solve_kernel: T = (I + M^ka)^-1 (unit lower triangular) by the recursive
+// block method: exact 16x16 leaves by forward substitution, then for block size
+// h = 16, 32, 64 every pair [[A,0],[B,D]] of adjacent h-blocks gets the lower
+// left block -D^-1 B A^-1 = -T_D (M_B T_A): two batches of tcgen05 MMAs per
+// level (X = M_B T_A, then Y = T_D X).
+// ---------------------------------------------------------------------------
+template <int NS>
+__global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int Cs = p.Cs, nb = Cs / SB;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  float* Tf = reinterpret_cast<float*>(sm);  // [Cs][Cs]
+  const uint32_t base = smem_u32(sm) + 128u * 128u * 4u;
+  constexpr uint32_t TB = 128u * 128u * 2u;
+  const Tile TA{base, base + TB, (uint32_t)Cs * 16u};           // K-major A tiles (K = Cs)
+  const Tile TBt{base + 2 * TB, base + 3 * TB, (uint32_t)Cs * 16u};  // MN-major B tiles (K = Cs)
+  const float* M = p.gr + ((int64_t)blockIdx.x * 4 + 1) * Cs * Cs;
+  for (int x = tid; x < Cs * Cs; x += 128) Tf[x] = 0.f;
+  zero_smem(base, 4 * TB);
+  TcCta cta;
+  cta.init(&tslot, &bar, 256);
+  {
+    const int J = tid >> 4, j = tid & 15;
+    if (J < nb) {
+      float x[SB];
+#pragma unroll
+      for (int i = 0; i < SB; ++i) x[i] = (i == j) ? 1.f : 0.f;
+      const float* Mb = M + (int64_t)(SB * J) * Cs + SB * J;
+#pragma unroll
+      for (int i = 1; i < SB; ++i) {
+        float acc = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < i; ++kk) acc += __ldg(Mb + i * Cs + kk) * x[kk];
+        if (i > j) x[i] = -acc;
+      }
+#pragma unroll
+      for (int i = 0; i < SB; ++i) Tf[(SB * J + i) * Cs + SB * J + j] = x[i];
+    }
+  }
+  __syncthreads();
+  MmaSync drv{&bar, 0u, true};
+  const int t = tid;
+  for (int h = SB; h < Cs && drv.ok; h *= 2) {
+    // A = off-diagonal blocks (2m+1, 2m) of M (zeros elsewhere), K-major; B = Tcur, MN-major.
+    for (int x = tid; x < 128 * (Cs / 8); x += 128) {
+      const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
+      float v[8];
+      const bool on = r < Cs && ((r / h) & 1) && (c8 / h) == (r / h) - 1;
+      if (on) ld8f(M + (int64_t)r * Cs + c8, v);
+      else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      }
+      put_k(TA, r, c8, v);
+    }
+    for (int x = tid; x < Cs * (Cs / 8); x += 128) {
+      const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = Tf[r * Cs + c8 + j];
+      put_mn(TBt, r, c8, v);
+    }
+    const int nm = Cs / (2 * h);
+    const uint32_t idh = idesc_bf16(128, h, 0, 1);
+    drv.run([&] {
+      for (int m = 0; m < nm; ++m)
+        mma_tiles(cta.tmem + 2 * m * h, sub_tile(TA, 2 * m * h, 0), sub_tile(TBt, 2 * m * h, 2 * m * h), h / 16, idh,
+                  NS, false);
+    });
+    if (!drv.ok) break;
+    // X (rows of odd blocks, columns of the preceding even block) -> B tile, MN-major.
+    {
+      const int m = t / (2 * h);
+      const bool odd = t < Cs && ((t / h) & 1);
+      for (int c = 0; c < h; c += 16) {
+        float v[16];
+        tmem_ld16(cta.tmem + tmem_lane_base(warp) + 2 * m * h + c, v);
+        if (odd) {
+          float a[8], b8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) { a[j] = v[j]; b8[j] = v[8 + j]; }
+          put_mn(TBt, t, 2 * m * h + c, a);
+          put_mn(TBt, t, 2 * m * h + c + 8, b8);
+        }
+      }
+    }
+    // A = Tcur, K-major.
+    for (int x = tid; x < Cs * (Cs / 8); x += 128) {
+      const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = Tf[r * Cs + c8 + j];
+      put_k(TA, r, c8, v);
+    }
+    drv.run([&] {
+      for (int m = 0; m < nm; ++m)
+        mma_tiles(cta.tmem + 128 + 2 * m * h, sub_tile(TA, (2 * m + 1) * h, 0),
+                  sub_tile(TBt, (2 * m + 1) * h, 2 * m * h), h / 16, idh, NS, false);
+    });
+    if (!drv.ok) break;
+    {
+      const int m = t / (2 * h);
+      const bool odd = t < Cs && ((t / h) & 1);
+      for (int c = 0; c < h; c += 16) {
+        float v[16];
+        tmem_ld16(cta.tmem + tmem_lane_base(warp) + 128 + 2 * m * h + c, v);
+        if (odd) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) Tf[t * Cs + 2 * m * h + c + j] = -v[j];
+        }
+      }
+    }
+    __syncthreads();
+  }
+  float* out = p.tt + (int64_t)blockIdx.x * Cs * Cs;
+  if (drv.ok)
+    for (int x = tid; x < Cs * Cs / 4; x += 128)
+      reinterpret_cast<float4*>(out)[x] = reinterpret_cast<const float4*>(Tf)[x];
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// maps_kernel: the chunk's affine map. TMEM column bases (fp32, 128 lanes):
+//   phase 1: W -> 0, Z = M^kk U -> 128, Ut = T Z -> 256
+//   phase 2: Phi -> 0, Q' -> 384, Oloc -> 256 (after Ut left TMEM), Psi -> 128
+// Shared memory: one A tile and two MN-major B tiles (128 x 128 bf16 hi+lo
+// each). Negated operands are staged negated.
+// ---------------------------------------------------------------------------
+template <int DK, int DV, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int Cs = p.Cs;
+  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  constexpr uint32_t TBY = 128u * 128u * 2u;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t kstride = (uint32_t)Cs * 16u;  // every tile here contracts over the Cs tokens
+  const Tile A{base, base + TBY, kstride};
+  const Tile B1{base + 2 * TBY, base + 3 * TBY, kstride};
+  const Tile B2{base + 4 * TBY, base + 5 * TBY, kstride};
+  zero_smem(base, 6 * TBY);
+  TcCta cta;
+  cta.init(&tslot, &bar, 512);
+  const float* dec = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
+  const float* gam = dec + 2 * Cs * DK;
+  const float* gsuf = dec + 3 * Cs * DK;
+  const float* G = p.gr + (int64_t)blockIdx.x * 4 * Cs * Cs;
+  const float* Tm = p.tt + (int64_t)blockIdx.x * Cs * Cs;
+  const Rows<T> rows{p, s.b, s.h};
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t lane = tmem_lane_base(warp);
+  const int t = tid;
+  constexpr uint32_t cW = 0, cZ = 128, cUt = 256, cPhi = 0, cPsi = 128, cOl = 256, cQ = 384;
+
+  auto stage_k_matrix = [&](const Tile& dst, const float* src, float sign) {  // rows t, K = s (Cs x Cs)
+    for (int x = tid; x < Cs * (Cs / 8); x += 128) {
+      const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
+      float v[8];
+      ld8f(src + (int64_t)r * Cs + c8, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] *= sign;
+      put_k(dst, r, c8, v);
+    }
+  };
+  // TMEM columns [col, col+n) of this thread's row -> MN-major B tile row t.
+  auto tmem_to_b = [&](const Tile& dst, uint32_t col, int n) {
+    for (int c = 0; c < n; c += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + lane + col + c, v);
+      if (t < Cs) {
+        float a[8], b8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { a[j] = v[j]; b8[j] = v[8 + j]; }
+        put_mn(dst, t, c, a);
+        put_mn(dst, t, c + 8, b8);
+      }
+    }
+  };
+  // (X * Gsuf)^T as an MN-major A operand (M = channel, K = token), scaled by sign.
+  auto stage_suffixed = [&](bool erase, float sign) {
+    for (int x = tid; x < Cs * (DK / 8); x += 128) {
+      const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      float xx[8], gs[8];
+      if (erase) rows.a(s.tok0 + r, c8, xx);
+      else rows.k(s.tok0 + r, c8, xx);
+      ld8f(gsuf + r * DK + c8, gs);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xx[j] *= sign * gs[j];
+      put_mn(A, r, c8, xx);
+    }
+  };
+  const uint32_t idK = idesc_bf16(128, DK, 0, 1), idV = idesc_bf16(128, DV, 0, 1);
+  const uint32_t idKt = idesc_bf16(128, DK, 1, 1), idVt = idesc_bf16(128, DV, 1, 1);
+  // ---- phase 1: W = T (K*Gam), Z = M^kk U, Ut = T Z
+  stage_k_matrix(A, Tm, 1.f);
+  for (int x = tid; x < Cs * (DK / 8); x += 128) {  // B1 = K*Gam (K = token, N = channel)
+    const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+    float kk[8], gm[8];
+    rows.k(s.tok0 + r, c8, kk);
+    ld8f(gam + r * DK + c8, gm);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) kk[j] *= gm[j];
+    put_mn(B1, r, c8, kk);
+  }
+  for (int x = tid; x < Cs * (DV / 8); x += 128) {  // B2 = U
+    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+    float uu[8];
+    rows.u(s.tok0 + r, c8, uu);
+    put_mn(B2, r, c8, uu);
+  }
+  drv.run([&] { mma_tiles(cta.tmem + cW, A, B1, Cs / 16, idK, NS, false); });
+  stage_k_matrix(A, G + 0 * Cs * Cs, 1.f);  // M^kk
+  drv.run([&] { mma_tiles(cta.tmem + cZ, A, B2, Cs / 16, idV, NS, false); });
+  tmem_to_b(B1, cZ, DV);
+  stage_k_matrix(A, Tm, 1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cUt, A, B1, Cs / 16, idV, NS, false); });
+  // ---- phase 2 with W in B1: Phi = Diag(Gam_C) - (A*Gsuf)^T W, Q' = Qt*Gam - N^qa W
+  tmem_to_b(B1, cW, DK);
+  stage_suffixed(true, -1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cPhi, A, B1, Cs / 16, idKt, NS, false); });
+  stage_k_matrix(A, G + 3 * Cs * Cs, -1.f);  // -N^qa
+  drv.run([&] { mma_tiles(cta.tmem + cQ, A, B1, Cs / 16, idK, NS, false); });
+  // ---- phase 3 with Ut in B1, U in B2: Oloc = N^qk U - N^qa Ut, Psi = (K*Gsuf)^T U - (A*Gsuf)^T Ut
+  tmem_to_b(B1, cUt, DV);
+  drv.run([&] { mma_tiles(cta.tmem + cOl, A, B1, Cs / 16, idV, NS, false); });  // A still holds -N^qa
+  stage_k_matrix(A, G + 2 * Cs * Cs, 1.f);                                         // N^qk
+  drv.run([&] { mma_tiles(cta.tmem + cOl, A, B2, Cs / 16, idV, NS, true); });
+  stage_suffixed(false, 1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B2, Cs / 16, idVt, NS, false); });
+  stage_suffixed(true, -1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B1, Cs / 16, idVt, NS, true); });
+  // ---- epilogue: [Phi; Q'] -> ma, [Psi; Oloc] -> mb (fp32, row-major)
+  float* ma = p.ma + (int64_t)blockIdx.x * (DK + Cs) * DK;
+  float* mb = p.mb + (int64_t)blockIdx.x * (DK + Cs) * DV;
+  const float* gC = gam + (Cs - 1) * DK;
+  for (int c = 0; c < DK; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + cPhi + c, v);
+    if (t < DK && drv.ok) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (c + j == t) v[j] += gC[t];
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(ma + (int64_t)t * DK + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  }
+  for (int c = 0; c < DV; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + cPsi + c, v);
+    if (t < DK && drv.ok) {
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(mb + (int64_t)t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  }
+  for (int c = 0; c < DK; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + cQ + c, v);
+    if (t < Cs && drv.ok) {
+      float qq[8], gm[8];
+#pragma unroll
+      for (int h8 = 0; h8 < 16; h8 += 8) {
+        rows.qt(s.tok0 + t, c + h8, qq);
+        ld8f(gam + t * DK + c + h8, gm);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[h8 + j] += qq[j] * gm[j];
+      }
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(ma + (int64_t)(DK + t) * DK + c + j) =
+            make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  }
+  for (int c = 0; c < DV; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + cOl + c, v);
+    if (t < Cs && drv.ok) {
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(mb + (int64_t)(DK + t) * DV + c + j) =
+            make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  }
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// compose_kernel (chunk = 256): the map of a 256-token chunk from the maps of
+// its two 128-token halves (h0 then h1), which is the top-level merge of the
+// recursive block solve applied to the chunk map:
+//   Phi = Phi1 Phi0,  Psi = Phi1 Psi0 + Psi1
+//   rows of the first half:  Q'0, Oloc0 (unchanged)
+//   rows of the second half: Q'1 Phi0, Q'1 Psi0 + Oloc1
+// One CTA per chunk: A = [Phi1; Q'1] (two 128-row K-major tiles, K = dk),
+// B = Phi0 then Psi0 (MN-major, K = dk).
+// ---------------------------------------------------------------------------
+template <int DK, int DV, int NS>
+__global__ void __launch_bounds__(128, 1) compose_kernel(ChunkParams p) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int Cs = p.Cs;  // 128
+  const int tid = threadIdx.x, warp = tid >> 5;
+  constexpr uint32_t TBY = 128u * DK * 2u;
+  const uint32_t base = smem_u32(sm);
+  const Tile A0{base, base + TBY, DK * 16u};
+  const Tile A1{base + 2 * TBY, base + 3 * TBY, DK * 16u};
+  const Tile Bt{base + 4 * TBY, base + 4 * TBY + 128u * DK * 2u, DK * 16u};
+  zero_smem(base, 4 * TBY + 2u * 128u * DK * 2u);
+  TcCta cta;
+  cta.init(&tslot, &bar, 512);
+  const int64_t u0 = 2 * (int64_t)blockIdx.x, u1 = u0 + 1;
+  const int rows1 = DK + Cs;
+  const float* ma0 = p.ma + u0 * rows1 * DK;
+  const float* ma1 = p.ma + u1 * rows1 * DK;
+  const float* mb0 = p.mb + u0 * rows1 * DV;
+  const float* mb1 = p.mb + u1 * rows1 * DV;
+  for (int x = tid; x < rows1 * (DK / 8); x += 128) {
+    const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+    float v[8];
+    ld8f(ma1 + (int64_t)r * DK + c8, v);
+    put_k(r < 128 ? A0 : A1, r & 127, c8, v);
+  }
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t lane = tmem_lane_base(warp);
+  for (int x = tid; x < DK * (DK / 8); x += 128) {  // Phi0 (K = row, N = col)
+    const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+    float v[8];
+    ld8f(ma0 + (int64_t)r * DK + c8, v);
+    put_mn(Bt, r, c8, v);
+  }
+  const int ntile = (rows1 + 127) / 128;
+  drv.run([&] {
+    mma_tiles(cta.tmem + 0, A0, Bt, DK / 16, idesc_bf16(128, DK, 0, 1), NS, false);
+    if (ntile > 1) mma_tiles(cta.tmem + 128, A1, Bt, DK / 16, idesc_bf16(128, DK, 0, 1), NS, false);
+  });
+  for (int x = tid; x < DK * (DV / 8); x += 128) {  // Psi0
+    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+    float v[8];
+    ld8f(mb0 + (int64_t)r * DV + c8, v);
+    put_mn(Bt, r, c8, v);
+  }
+  drv.run([&] {
+    mma_tiles(cta.tmem + 256, A0, Bt, DK / 16, idesc_bf16(128, DV, 0, 1), NS, false);
+    if (ntile > 1) mma_tiles(cta.tmem + 384, A1, Bt, DK / 16, idesc_bf16(128, DV, 0, 1), NS, false);
+  });
+  const int rows2 = DK + 2 * Cs;
+  float* ma = p.ma2 + (int64_t)blockIdx.x * rows2 * DK;
+  float* mb = p.mb2 + (int64_t)blockIdx.x * rows2 * DV;
+  // rows of the composite: [0,DK) state, [DK, DK+Cs) first half, [DK+Cs, DK+2Cs) second half
+  for (int tile = 0; tile < ntile; ++tile) {
+    const int r1 = tile * 128 + tid;  // row of [Phi1; Q'1]
+    const int r2 = r1 < DK ? r1 : r1 + Cs;
+    for (int c = 0; c < DK; c += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + lane + tile * 128 + c, v);
+      if (r1 < rows1 && drv.ok)
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(ma + (int64_t)r2 * DK + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+    for (int c = 0; c < DV; c += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + lane + 256 + tile * 128 + c, v);
+      if (r1 < rows1 && drv.ok) {
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(mb1 + (int64_t)r1 * DV + c + j);
+          *reinterpret_cast<float4*>(mb + (int64_t)r2 * DV + c + j) =
+              make_float4(v[j] + a.x, v[j + 1] + a.y, v[j + 2] + a.z, v[j + 3] + a.w);
+        }
+      }
+    }
+  }
+  // first-half rows copied: [Q'0; Oloc0]
+  for (int x = tid; x < Cs * DK / 4; x += 128)
+    reinterpret_cast<float4*>(ma + (int64_t)DK * DK)[x] = reinterpret_cast<const float4*>(ma0 + (int64_t)DK * DK)[x];
+  for (int x = tid; x < Cs * DV / 4; x += 128)
+    reinterpret_cast<float4*>(mb + (int64_t)DK * DV)[x] = reinterpret_cast<const float4*>(mb0 + (int64_t)DK * DV)[x];
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// scan_kernel: one CTA per (batch, head, 32-column slab of the state); walks the
+// chunks in order. The state slab S (dk x 32 fp32) stays on chip: in registers
+// (thread = key row) and, split into bf16 hi/lo, as the MMA's B operand.
+//   D = [Phi; Q'] S   (M = dk + C rows in 128-row tiles, N = 32, K = dk)
+//   S <- D[0:dk] + Psi,   y = z * (D[dk:] + Oloc)
+// ---------------------------------------------------------------------------
+template <int DK, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const float* ma, const float* mb, int units,
+                                                      int ulen) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  constexpr int NW = 32;  // slab width
+  const int dv = p.dv, slabs = dv / NW;
+  const int slab = blockIdx.x % slabs;
+  const int bh = blockIdx.x / slabs;
+  const int h = bh % p.H, b = bh / p.H;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int rows_total = DK + ulen;
+  const int ntile = (rows_total + 127) / 128;
+  constexpr uint32_t ATB = 128u * DK * 2u;
+  const uint32_t base = smem_u32(sm);
+  const Tile Sb{base, base + NW * DK * 2u, DK * 16u};  // B: K = key row, N = slab column (MN-major)
+  const uint32_t abase = base + 2u * NW * DK * 2u;
+  zero_smem(base, 2u * NW * DK * 2u + 2u * ATB * ntile);
+  TcCta cta;
+  cta.init(&tslot, &bar, tmem_cols_for(NW * ntile));
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t lane = tmem_lane_base(warp);
+  // state slab in registers: thread = key row i < DK
+  float st[NW];
+  {
+    const float* s0 = p.S0 ? p.S0 + (((int64_t)b * p.H + h) * DK) * dv + slab * NW : nullptr;
+#pragma unroll
+    for (int j = 0; j < NW; ++j) st[j] = (s0 && tid < DK) ? s0[(int64_t)tid * dv + j] : 0.f;
+  }
+  const uint32_t id = idesc_bf16(128, NW, 0, 1);
+  for (int n = 0; n < units && drv.ok; ++n) {
+    const int64_t uid = ((int64_t)b * p.H + h) * units + n;
+    if (p.S_chunks && tid < DK) {
+      float* o = p.S_chunks + ((uid * DK) + tid) * dv + slab * NW;
+#pragma unroll
+      for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(st[j], st[j + 1], st[j + 2], st[j + 3]);
+    }
+    if (tid < DK) {
+#pragma unroll
+      for (int j = 0; j < NW; j += 8) {
+        float v[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) v[e2] = st[j + e2];
+        put_mn(Sb, tid, j, v);
+      }
+    }
+    const float* A = ma + uid * rows_total * DK;
+    for (int x = tid; x < ntile * 128 * (DK / 8); x += 128) {
+      const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      float v[8];
+      if (r < rows_total) ld8f(A + (int64_t)r * DK + c8, v);
+      else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      }
+      const int tile = r >> 7;
+      const Tile At{abase + tile * 2u * ATB, abase + tile * 2u * ATB + ATB, DK * 16u};
+      put_k(At, r & 127, c8, v);
+    }
+    drv.run([&] {
+      for (int tile = 0; tile < ntile; ++tile) {
+        const Tile At{abase + tile * 2u * ATB, abase + tile * 2u * ATB + ATB, DK * 16u};
+        mma_tiles(cta.tmem + tile * NW, At, Sb, DK / 16, id, NS, false);
+      }
+    });
+    if (!drv.ok) break;
+    const float* Bm = mb + uid * rows_total * dv + slab * NW;
+    for (int tile = 0; tile < ntile; ++tile) {
+      float v[NW];
+      tmem_ld16(cta.tmem + lane + tile * NW, *reinterpret_cast<float(*)[16]>(&v[0]));
+      tmem_ld16(cta.tmem + lane + tile * NW + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+      const int r = tile * 128 + tid;
+      if (r < DK) {
+#pragma unroll
+        for (int j = 0; j < NW; j += 4) {
+          const float4 add = *reinterpret_cast<const float4*>(Bm + (int64_t)r * dv + j);
+          st[j] = v[j] + add.x; st[j + 1] = v[j + 1] + add.y; st[j + 2] = v[j + 2] + add.z; st[j + 3] = v[j + 3] + add.w;
+        }
+      } else if (r < rows_total) {
+        const int tt = r - DK;
+        const int64_t tok = (int64_t)n * ulen + tt;
+        float o[NW];
+#pragma unroll
+        for (int j = 0; j < NW; j += 4) {
+          const float4 add = *reinterpret_cast<const float4*>(Bm + (int64_t)r * dv + j);
+          o[j] = v[j] + add.x; o[j + 1] = v[j + 1] + add.y; o[j + 2] = v[j + 2] + add.z; o[j + 3] = v[j + 3] + add.w;
+        }
+        const int64_t yo = toff(p, b, tok, h, dv) + slab * NW;
+        if (p.z) {
+#pragma unroll
+          for (int j = 0; j < NW; j += 8) {
+            float zz[8];
+            Elt<T>::ld8(static_cast<const T*>(p.z) + yo + j, zz);
+#pragma unroll
+            for (int e2 = 0; e2 < 8; ++e2) o[j + e2] *= zz[e2];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < NW; j += 8) {
+          float w8[8];
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) w8[e2] = o[j + e2];
+          Elt<T>::st8(static_cast<T*>(p.y) + yo + j, w8);
+        }
+      }
+    }
+    // registers of `st` now hold the next chunk's start state; the next loop
+    // iteration restages them (the MMA above has completed).
+    __syncthreads();
+  }
+  if (p.S_T && tid < DK && drv.ok) {
+    float* o = p.S_T + (((int64_t)b * p.H + h) * DK + tid) * dv + slab * NW;
+#pragma unroll
+    for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(st[j], st[j + 1], st[j + 2], st[j + 3]);
+  }
+  cta.finish();
+}
+
+}  // namespace muir

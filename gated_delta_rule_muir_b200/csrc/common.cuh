@@ -1,0 +1,87 @@
+// Shared device helpers: element loads/stores for the two input dtypes, and the
+// library's device status word (set when a bounded wait runs out).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace muir {
+
+// Device-side status word: bit 0 = a bounded wait expired. Read and cleared by
+// muir_device_status(). One word per device context of the library.
+__device__ unsigned int g_status;
+
+constexpr unsigned int kStatusTimeout = 1u;
+
+__device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, kStatusTimeout); }
+
+// ---- element access -----------------------------------------------------
+
+template <typename T> struct Elt;
+
+template <> struct Elt<float> {
+  static __device__ __forceinline__ float ld(const float* p) { return __ldg(p); }
+  static __device__ __forceinline__ void st(float* p, float x) { *p = x; }
+  // 8 consecutive elements (p 32-byte aligned).
+  static __device__ __forceinline__ void ld8(const float* p, float (&o)[8]) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+  static __device__ __forceinline__ void ld4(const float* p, float (&o)[4]) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  }
+  static __device__ __forceinline__ void st4(float* p, const float (&o)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
+  }
+  static __device__ __forceinline__ void st8(float* p, const float (&o)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(o[4], o[5], o[6], o[7]);
+  }
+};
+
+template <> struct Elt<__nv_bfloat16> {
+  using T = __nv_bfloat16;
+  static __device__ __forceinline__ float ld(const T* p) { return __bfloat162float(p[0]); }
+  static __device__ __forceinline__ void st(T* p, float x) { *p = __float2bfloat16_rn(x); }
+  static __device__ __forceinline__ void ld8(const T* p, float (&o)[8]) {
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      o[2 * i] = f.x; o[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void ld4(const T* p, float (&o)[4]) {
+    uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+    float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+    o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+  }
+  static __device__ __forceinline__ void st4(T* p, const float (&o)[4]) {
+    uint2 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+    h[0] = __floats2bfloat162_rn(o[0], o[1]);
+    h[1] = __floats2bfloat162_rn(o[2], o[3]);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+  static __device__ __forceinline__ void st8(T* p, const float (&o)[8]) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+}  // namespace muir

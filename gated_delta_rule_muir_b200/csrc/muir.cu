@@ -1,0 +1,127 @@
+// libmuir.so: the C ABI declared in include/muir.h. Validates arguments, sizes
+// workspaces and launches the kernels; all arithmetic of the operator happens
+// in the kernels included below.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/muir.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "selftest.cuh"
+#include "chunk.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MUIR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return MUIR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+}  // namespace
+
+extern "C" {
+
+int muir_version(void) { return 100; }
+
+const char* muir_last_error(void) { return g_err.c_str(); }
+
+int muir_device_status(void* stream) {
+  g_err.clear();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_check("cudaStreamSynchronize");
+  unsigned int host = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&host, muir::g_status, sizeof host) != cudaSuccess) return cuda_check("read status");
+  if (cudaMemcpyToSymbol(muir::g_status, &zero, sizeof zero) != cudaSuccess) return cuda_check("clear status");
+  if (host & muir::kStatusTimeout) return fail(MUIR_ERR_TIMEOUT, "a bounded device wait expired");
+  return MUIR_OK;
+}
+
+int muir_state_init(float* S, const float* S_src, int64_t n_seq, int32_t H, int32_t dk, int32_t dv, void* stream) {
+  g_err.clear();
+  if (!S) return fail(MUIR_ERR_INVALID_ARG, "state_init: S is NULL");
+  if (n_seq < 0 || H <= 0 || !dim_ok(dk) || !dim_ok(dv))
+    return fail(MUIR_ERR_UNSUPPORTED, "state_init: unsupported sizes n_seq=%lld H=%d dk=%d dv=%d", (long long)n_seq, H,
+                dk, dv);
+  if (!aligned16(S) || (S_src && !aligned16(S_src))) return fail(MUIR_ERR_INVALID_ARG, "state_init: misaligned pointer");
+  const int64_t n4 = n_seq * H * (int64_t)dk * dv / 4;
+  if (n4 == 0) return MUIR_OK;
+  int64_t blocks = (n4 + 255) / 256;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  muir::state_init_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<float4*>(S), reinterpret_cast<const float4*>(S_src), n4);
+  return cuda_check("state_init launch");
+}
+
+int muir_decode_step(const muir_decode_args* a, void* stream) {
+  g_err.clear();
+  if (!a) return fail(MUIR_ERR_INVALID_ARG, "decode: args is NULL");
+  if (a->n_seq == 0) return MUIR_OK;  // nothing to do (empty tensors may carry NULL pointers)
+  if (!a->S || !a->q || !a->k || !a->v || !a->e || !a->w || !a->g || !a->log_alpha || !a->r || !a->y)
+    return fail(MUIR_ERR_INVALID_ARG, "decode: a required pointer is NULL");
+  if (a->n_seq < 0 || a->H <= 0 || !dim_ok(a->dk) || !dim_ok(a->dv))
+    return fail(MUIR_ERR_UNSUPPORTED, "decode: unsupported sizes H=%d dk=%d dv=%d", a->H, a->dk, a->dv);
+  if (a->dtype != MUIR_F32 && a->dtype != MUIR_BF16) return fail(MUIR_ERR_UNSUPPORTED, "decode: dtype %d", a->dtype);
+  if (a->r_seq_stride < 0) return fail(MUIR_ERR_INVALID_ARG, "decode: negative r_seq_stride");
+  const void* ptrs[] = {a->S, a->q, a->k, a->v, a->e, a->w, a->g, a->z, a->log_alpha, a->r, a->y};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(MUIR_ERR_INVALID_ARG, "decode: pointer not 16-byte aligned");
+  if (a->n_seq == 0) return MUIR_OK;
+  muir::DecodeParams p{a->n_seq, a->H, a->dk, a->dv, a->S, a->q, a->k, a->v, a->e, a->w, a->g, a->z,
+                       a->log_alpha, a->r, a->r_seq_stride, a->y};
+  const int64_t blocks = a->n_seq * a->H * (a->dv / 32);
+  if (blocks > 0x7fffffff) return fail(MUIR_ERR_UNSUPPORTED, "decode: too many rows");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf = a->dtype == MUIR_BF16;
+#define MUIR_DECODE(DK)                                                                  \
+  if (bf)                                                                                \
+    muir::decode_step_kernel<DK, __nv_bfloat16><<<(unsigned)blocks, 128, 0, s>>>(p);     \
+  else                                                                                   \
+    muir::decode_step_kernel<DK, float><<<(unsigned)blocks, 128, 0, s>>>(p);
+  switch (a->dk) {
+    case 32: MUIR_DECODE(32) break;
+    case 64: MUIR_DECODE(64) break;
+    default: MUIR_DECODE(128) break;
+  }
+#undef MUIR_DECODE
+  return cuda_check("decode launch");
+}
+
+// Diagnostic entry point: D[128,N] = A[128,K] * B[K,N] through the tensor-core
+// operand layouts the chunk kernels use. a_mn/b_mn select MN-major staging,
+// nsplit is 1 or 3. Not part of the operator.
+int muir_selftest_gemm(const float* A, const float* B, float* D, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn,
+                       int32_t nsplit, void* stream) {
+  g_err.clear();
+  if (!A || !B || !D) return fail(MUIR_ERR_INVALID_ARG, "selftest: NULL pointer");
+  if (N < 16 || N > 256 || N % 16 || K < 16 || K > 128 || K % 16 || (nsplit != 1 && nsplit != 3))
+    return fail(MUIR_ERR_UNSUPPORTED, "selftest: N=%d K=%d nsplit=%d", N, K, nsplit);
+  const size_t smem = 2u * (128u * K * 2u) + 2u * ((size_t)N * K * 2u);
+  if (cudaFuncSetAttribute(muir::selftest_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return cuda_check("selftest attribute");
+  muir::selftest_gemm_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(A, B, D, N, K, a_mn, b_mn, nsplit);
+  return cuda_check("selftest launch");
+}
+
+}  // extern "C"
+
+#include "api_chunk.inc"

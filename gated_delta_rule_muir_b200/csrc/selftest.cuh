@@ -1,0 +1,74 @@
+// Diagnostic GEMM exercising the tcgen05 operand layouts of tc.cuh:
+// D[M=128, N] = A[128, K] * B[K, N] with fp32 row-major A and B in global
+// memory, staged K-major or MN-major, 1-pass or 3-pass bf16. One CTA.
+#pragma once
+
+#include "tc.cuh"
+
+namespace muir {
+
+__global__ void __launch_bounds__(128) selftest_gemm_kernel(const float* __restrict__ A, const float* __restrict__ B,
+                                                            float* __restrict__ D, int N, int K, int a_mn, int b_mn,
+                                                            int nsplit) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_base;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t base = smem_u32(smem);
+  const uint32_t a_bytes = 128u * K * 2u, b_bytes = (uint32_t)N * K * 2u;
+  Tile ta{base, base + a_bytes, (uint32_t)K * 16u};
+  Tile tb{base + 2 * a_bytes, base + 2 * a_bytes + b_bytes, (uint32_t)K * 16u};
+  if (warp == 0) tmem_alloc(&tmem_base, N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256)));
+  if (tid == 0) mbar_init(&bar, 1);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  // A: element (m, k) = A[m*K + k]
+  for (int idx = tid; idx < 128 * (K / 8); idx += 128) {
+    float x[8];
+    if (!a_mn) {
+      const int m = idx / (K / 8), k8 = (idx % (K / 8)) * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = A[m * K + k8 + e];
+      put_k(ta, m, k8, x);
+    } else {
+      const int k = idx / 16, m8 = (idx % 16) * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = A[(m8 + e) * K + k];
+      put_mn(ta, k, m8, x);
+    }
+  }
+  // B: element (k, n) = B[k*N + n]
+  for (int idx = tid; idx < N * (K / 8); idx += 128) {
+    float x[8];
+    if (!b_mn) {
+      const int n = idx / (K / 8), k8 = (idx % (K / 8)) * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = B[(k8 + e) * N + n];
+      put_k(tb, n, k8, x);
+    } else {
+      const int k = idx / (N / 8), n8 = (idx % (N / 8)) * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = B[k * N + n8 + e];
+      put_mn(tb, k, n8, x);
+    }
+  }
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t id = idesc_bf16(128, N, a_mn, b_mn);
+  drv.run([&] { mma_tiles(tmem, ta, tb, K / 16, id, nsplit, false); });
+  if (drv.ok) {
+    for (int c = 0; c < N; c += 16) {
+      float v[16];
+      tmem_ld16(tmem + tmem_lane_base(warp) + c, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) D[tid * N + c + i] = v[i];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256)));
+}
+
+}  // namespace muir

@@ -1,0 +1,247 @@
+// Blackwell (sm_100a) tensor-core primitives: tcgen05.mma with shared-memory
+// operand descriptors, fp32 accumulators in tensor memory (TMEM), completion
+// tracked through an mbarrier, and TMEM -> register loads.
+//
+// Operand tiles live in shared memory in the "no-swizzle" canonical layout made
+// of 8 x 16-byte core matrices (8 rows of 8 bf16). A tile covering MN rows
+// (multiple of 8) and KT contraction indices (multiple of 16) is stored as
+// MN/8 groups, each group holding KT/8 core matrices back to back:
+//
+//   K-major tile  (row = MN index m, 8 consecutive k per 16-byte row):
+//       byte(m, k) = (m/8)*SBO + (k/8)*128 + (m%8)*16 + (k%8)*2
+//   MN-major tile (row = contraction index k, 8 consecutive m per 16-byte row):
+//       byte(k, m) = (m/8)*SBO + (k/8)*128 + (k%8)*16 + (m%8)*2
+//
+// with SBO = KT*16 (distance between MN groups) and LBO = 128 (distance between
+// core matrices adjacent along K). One MMA consumes K = 16 = two core matrices
+// along K, so the k-th MMA step starts 256 bytes further. The same physical
+// tile of a row-major matrix X[rows][cols] can be fed as a K-major operand
+// (contract over cols) or as an MN-major operand (contract over rows).
+//
+// fp32 operands are split into bf16 hi + lo parts (x = hi + lo + O(2^-17 |x|));
+// a product is accumulated as hi*hi + hi*lo + lo*hi, which keeps ~2^-16
+// relative accuracy at bf16 tensor-core rate ("3-pass bf16").
+#pragma once
+
+#include "common.cuh"
+
+namespace muir {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier --------------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete. Bounded: gives up after
+// about one second, records the timeout in the device status word and returns
+// false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((it & 63) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > 1000000000ull) { flag_timeout(); return false; }
+    }
+  }
+}
+
+// ---- fences ----------------------------------------------------------------
+
+// Generic-proxy shared-memory writes -> visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// ---- TMEM allocation (whole warp) ------------------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// ---- descriptors -----------------------------------------------------------
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, dense.
+// a_mn / b_mn: 0 = K-major, 1 = MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                        // D format: f32
+         | (1u << 7)                      // A format: bf16
+         | (1u << 10)                     // B format: bf16
+         | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) |
+         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor, no swizzle (layout type 0), sm_100 version bit.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
+         (1ull << 46);
+}
+
+// ---- MMA issue (single thread) ---------------------------------------------
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+// Arrive once on `bar` when all previously issued MMAs of this thread complete.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// A staged operand tile: bf16 hi and lo parts in shared memory.
+struct Tile {
+  uint32_t hi, lo;  // shared addresses (16-byte aligned)
+  uint32_t sbo;     // KT * 16
+};
+
+// D[tmem] (+)= A * B for one tile pair covering `ksteps` MMA steps of K = 16.
+// M = 128 rows of A (lanes of D), N columns of B. nsplit = 1 (hi*hi) or 3.
+__device__ __forceinline__ void mma_tiles(uint32_t d_tmem, const Tile& A, const Tile& B, int ksteps, uint32_t idesc,
+                                          int nsplit, bool accumulate) {
+  for (int j = 0; j < ksteps; ++j) {
+    const uint32_t off = j * 256u;
+    const uint64_t ah = sdesc(A.hi + off, 128, A.sbo), bh = sdesc(B.hi + off, 128, B.sbo);
+    mma_bf16(d_tmem, ah, bh, idesc, (accumulate || j > 0) ? 1u : 0u);
+    if (nsplit == 3) {
+      const uint64_t al = sdesc(A.lo + off, 128, A.sbo), bl = sdesc(B.lo + off, 128, B.sbo);
+      mma_bf16(d_tmem, ah, bl, idesc, 1u);
+      mma_bf16(d_tmem, al, bh, idesc, 1u);
+    }
+  }
+}
+
+// ---- operand staging (any thread) ------------------------------------------
+
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
+  __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    const float2 hf = __bfloat1622float2(hh);
+    h[i] = hh;
+    l[i] = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+  }
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// K-major: 8 consecutive contraction indices k8..k8+7 of MN row m.
+__device__ __forceinline__ void put_k(const Tile& t, int m, int k8, const float (&x)[8]) {
+  uint4 hi, lo;
+  split8(x, hi, lo);
+  const uint32_t off = (uint32_t)(m >> 3) * t.sbo + (uint32_t)(k8 >> 3) * 128u + (uint32_t)(m & 7) * 16u;
+  sts128(t.hi + off, hi);
+  sts128(t.lo + off, lo);
+}
+
+// MN-major: 8 consecutive MN indices m8..m8+7 of contraction row k.
+__device__ __forceinline__ void put_mn(const Tile& t, int k, int m8, const float (&x)[8]) {
+  uint4 hi, lo;
+  split8(x, hi, lo);
+  const uint32_t off = (uint32_t)(m8 >> 3) * t.sbo + (uint32_t)(k >> 3) * 128u + (uint32_t)(k & 7) * 16u;
+  sts128(t.hi + off, hi);
+  sts128(t.lo + off, lo);
+}
+
+// ---- TMEM -> registers -----------------------------------------------------
+
+// Lane base of warp w's TMEM sub-partition.
+__device__ __forceinline__ uint32_t tmem_lane_base(int warp) { return (uint32_t)((warp & 3) * 32) << 16; }
+
+// 16 consecutive fp32 columns of this thread's lane (row), completes before return.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 8 consecutive fp32 columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---- a tiny synchronous MMA driver ----------------------------------------
+//
+// Holds the mbarrier phase. Usage (all threads of a 128-thread CTA):
+//   stage operands; drv.run([&]{ mma_tiles(...); ... });   // waits for completion
+struct MmaSync {
+  uint64_t* bar;
+  uint32_t phase;
+  bool ok;
+
+  // All threads: publish staged smem to the tensor core, let thread 0 issue the
+  // MMAs given by `issue`, commit, and wait for completion. Returns false (and
+  // leaves `ok` false) if the bounded wait expired.
+  template <typename F>
+  __device__ __forceinline__ bool run(F issue) {
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue();
+      mma_commit(bar);
+    }
+    const bool done = __syncthreads_and(mbar_wait(bar, phase) ? 1 : 0) != 0;
+    phase ^= 1u;
+    tc_fence_after();
+    ok = ok && done;
+    return done;
+  }
+};
+
+}  // namespace muir

@@ -1,0 +1,168 @@
+/*
+ * muir.h — C ABI of the Muir gated delta-rule operator library (libmuir.so),
+ * hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * The operator (arXiv 2611.08376, "Muir: Linear Attention with
+ * Sensitivity-Allocated Gating and Matched-Filter Readout", abstract "Full
+ * text"; openai-hub article, sections on the matched-filter readout and on
+ * the TPU chunkwise algorithm). Per batch b, head h, token t:
+ *
+ *   x_t = Diag(alpha_t) S_{t-1}                     channel-wise decay of the rows of S
+ *   p_t = x_t^T k_t                                 prediction for the incoming key
+ *   S_t = x_t - (e_t*k_t) p_t^T + k_t (w_t*v_t)^T   gated erase of the prediction, gated write
+ *   o_t = S_t^T (r * g_t * q_t)                     matched-filter readout: static row scale r,
+ *                                                   dynamic per-token query gate g_t
+ *   y_t = z_t * o_t                                 output gate (z may be omitted: y = o)
+ *
+ * S is a dk x dv fp32 matrix per (sequence, head). alpha is passed as
+ * log_alpha <= 0 (fp32). q and k are expected to be already activated and
+ * unit-normalised by the caller; the operator does not normalise.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are CUDA device pointers owned by the caller; the library never
+ *     allocates, frees or retains them. Scratch memory ("workspace") is passed
+ *     in by the caller after a size query.
+ *   - Tensors are dense, row-major, in the layouts stated per argument, and
+ *     every pointer must be 16-byte aligned.
+ *   - "dtype" selects the element type of q, k, v, e, w, g, z, y and of the
+ *     gradients of those: MUIR_F32 (float) or MUIR_BF16 (bfloat16). log_alpha,
+ *     r, states and their gradients are always float.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t, NULL = the
+ *     legacy default stream). Return values report argument validation and
+ *     launch errors only; a kernel's bounded waits that ran out are reported by
+ *     muir_device_status().
+ *   - Return: MUIR_OK (0) or one of the MUIR_ERR_* codes below; a message for
+ *     the calling thread is available from muir_last_error(). Nothing is thrown
+ *     across this interface.
+ *   - Supported sizes: dk, dv in {32, 64, 128}; chunk in {64, 128, 256};
+ *     T % chunk == 0 (callers pad with identity tokens: log_alpha = 0, k = 0,
+ *     e = 0, w = 0, which leave the state unchanged).
+ */
+#ifndef MUIR_H
+#define MUIR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MUIR_OK 0
+#define MUIR_ERR_INVALID_ARG 1 /* null pointer, bad stride/alignment, inconsistent sizes */
+#define MUIR_ERR_UNSUPPORTED 2 /* valid but unsupported size, chunk or dtype */
+#define MUIR_ERR_WORKSPACE 3   /* workspace pointer NULL/misaligned or smaller than the query */
+#define MUIR_ERR_CUDA 4        /* a CUDA runtime call failed (launch, attribute) */
+#define MUIR_ERR_TIMEOUT 5     /* a bounded device wait expired (from muir_device_status) */
+
+#define MUIR_F32 0
+#define MUIR_BF16 1
+
+/* Inputs of the chunkwise forward and backward passes. */
+typedef struct muir_chunk_args {
+  int64_t B;      /* batch size (independent sequences) */
+  int64_t T;      /* tokens per sequence; T % chunk == 0 */
+  int32_t H;      /* heads */
+  int32_t dk;     /* key dimension = rows of the state */
+  int32_t dv;     /* value dimension = columns of the state */
+  int32_t chunk;  /* chunk length C of the chunkwise algorithm: 64, 128 or 256 */
+  int32_t dtype;  /* MUIR_F32 or MUIR_BF16 */
+  int32_t reserved;
+  const void* q;  /* [B,T,H,dk] query (activated, unit-norm) */
+  const void* k;  /* [B,T,H,dk] key (activated, unit-norm) */
+  const void* v;  /* [B,T,H,dv] value */
+  const void* e;  /* [B,T,H,dk] erase gate, acts on key rows */
+  const void* w;  /* [B,T,H,dv] write gate, acts on value columns */
+  const void* g;  /* [B,T,H,dk] dynamic query (read) gate */
+  const void* z;  /* [B,T,H,dv] output gate, or NULL for none */
+  const float* log_alpha; /* [B,T,H,dk] log of the channel decay, <= 0 */
+  const float* r; /* [H,dk] static matched-filter row scale */
+  const float* S0;/* [B,H,dk,dv] initial state, or NULL for zeros */
+} muir_chunk_args;
+
+/*
+ * Chunkwise-parallel forward pass (openai-hub article, section on the TPU
+ * chunkwise algorithm; liuch.name post, bullet "Numerically-stable,
+ * large-chunk parallel kernel"): intra-chunk decay products are
+ * boundary-pivoted and multiplicative (each factor in [0,1], no division), the
+ * unit-lower-triangular chunk system is inverted by a recursive block method on
+ * the tensor cores, and the state is passed from chunk to chunk on chip.
+ *   y   [B,T,H,dv] output (dtype).
+ *   S_T [B,H,dk,dv] final state, or NULL if not wanted.
+ *   ws  workspace of at least muir_chunk_fwd_workspace(a) bytes, 256-byte
+ *       aligned; contents on entry are ignored.
+ */
+size_t muir_chunk_fwd_workspace(const muir_chunk_args* a);
+int muir_chunk_fwd(const muir_chunk_args* a, void* y, float* S_T, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* Gradients for muir_chunk_bwd. Outputs are written (not accumulated). */
+typedef struct muir_chunk_grads {
+  const void* dy;      /* [B,T,H,dv] cotangent of y (dtype) */
+  const float* dS_T;   /* [B,H,dk,dv] cotangent of the final state, or NULL for zeros */
+  void* dq;            /* [B,T,H,dk] (dtype) */
+  void* dk;            /* [B,T,H,dk] (dtype) */
+  void* dv;            /* [B,T,H,dv] (dtype) */
+  void* de;            /* [B,T,H,dk] (dtype) */
+  void* dw;            /* [B,T,H,dv] (dtype) */
+  void* dg;            /* [B,T,H,dk] (dtype) */
+  void* dz;            /* [B,T,H,dv] (dtype), or NULL; ignored when z is NULL */
+  float* dlog_alpha;   /* [B,T,H,dk]; d/d(alpha) = dlog_alpha / alpha */
+  float* dS0;          /* [B,H,dk,dv], or NULL */
+  float* dr;           /* [H,dk], or NULL */
+} muir_chunk_grads;
+
+/*
+ * Backward pass of muir_chunk_fwd with the same arguments. The per-chunk
+ * states are recomputed (a forward sweep into the workspace), then one reverse
+ * sweep carries the state cotangent, and chunk-parallel kernels form every
+ * input gradient (arXiv abstract: a parallel update for training).
+ *   ws  workspace of at least muir_chunk_bwd_workspace(a) bytes.
+ */
+size_t muir_chunk_bwd_workspace(const muir_chunk_args* a);
+int muir_chunk_bwd(const muir_chunk_args* a, const muir_chunk_grads* gr, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* One recurrent step for n_seq independent sequences (streaming decode,
+ * openai-hub article, section on 10M-token streaming). */
+typedef struct muir_decode_args {
+  int64_t n_seq;       /* number of (sequence, layer) rows */
+  int32_t H, dk, dv;
+  int32_t dtype;       /* of q,k,v,e,w,g,z,y */
+  float* S;            /* [n_seq,H,dk,dv] state, updated in place */
+  const void* q;       /* [n_seq,H,dk] */
+  const void* k;       /* [n_seq,H,dk] */
+  const void* v;       /* [n_seq,H,dv] */
+  const void* e;       /* [n_seq,H,dk] */
+  const void* w;       /* [n_seq,H,dv] */
+  const void* g;       /* [n_seq,H,dk] */
+  const void* z;       /* [n_seq,H,dv] or NULL */
+  const float* log_alpha; /* [n_seq,H,dk] */
+  const float* r;      /* [H,dk] when r_seq_stride == 0, else row n at r + n*r_seq_stride */
+  int64_t r_seq_stride;/* elements between consecutive rows' r (0 = shared, H*dk = per row) */
+  void* y;             /* [n_seq,H,dv] output */
+} muir_decode_args;
+
+/* Reads and writes each state element exactly once (memory-bound). */
+int muir_decode_step(const muir_decode_args* a, void* stream);
+
+/* S [n_seq,H,dk,dv] := S_src, or zeros when S_src is NULL. In-place safe. */
+int muir_state_init(float* S, const float* S_src, int64_t n_seq, int32_t H, int32_t dk, int32_t dv,
+                    void* stream);
+
+/* Synchronises `stream`, then returns and clears the device-side status word:
+ * MUIR_OK, or MUIR_ERR_TIMEOUT if a kernel's bounded wait expired since the
+ * last call (that kernel's outputs are then invalid), or MUIR_ERR_CUDA. */
+int muir_device_status(void* stream);
+
+/* Message describing the last error on the calling thread ("" if none). */
+const char* muir_last_error(void);
+
+/* Library ABI version (major*100 + minor). */
+int muir_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUIR_H */

@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_muir_b200 import _native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "muir.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(muir_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_muir_b200 import build
+    build.build()
+    return N.load()
+
+
+def test_header_declares_the_operator_api():
+    names = _header_functions()
+    for n in ("muir_chunk_fwd", "muir_chunk_bwd", "muir_decode_step", "muir_state_init",
+              "muir_chunk_fwd_workspace", "muir_chunk_bwd_workspace", "muir_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in _header_functions():
+        assert hasattr(lib, n), n
+        assert n in N.SIGNATURES, f"binding lacks a signature for {n}"
+
+
+def test_version(lib):
+    assert lib.muir_version() == 100
+
+
+def test_decode_rejects_null_and_bad_sizes(lib):
+    assert lib.muir_decode_step(None, None) == N.MUIR_ERR_INVALID_ARG
+    a = N.DecodeArgs(n_seq=1, H=1, dk=128, dv=128, dtype=N.MUIR_F32)
+    assert lib.muir_decode_step(C.byref(a), None) == N.MUIR_ERR_INVALID_ARG
+    assert b"NULL" in lib.muir_last_error()
+    fake = C.c_void_p(1 << 20)
+    for f in ("S", "q", "k", "v", "e", "w", "g", "log_alpha", "r", "y"):
+        setattr(a, f, fake)
+    a.dk = 96
+    assert lib.muir_decode_step(C.byref(a), None) == N.MUIR_ERR_UNSUPPORTED
+    a.dk = 128
+    a.dtype = 7
+    assert lib.muir_decode_step(C.byref(a), None) == N.MUIR_ERR_UNSUPPORTED
+    a.dtype = N.MUIR_BF16
+    a.q = C.c_void_p((1 << 20) + 2)
+    assert lib.muir_decode_step(C.byref(a), None) == N.MUIR_ERR_INVALID_ARG
+    assert b"aligned" in lib.muir_last_error()
+
+
+def test_state_init_rejects_bad_args(lib):
+    assert lib.muir_state_init(None, None, 1, 1, 32, 32, None) == N.MUIR_ERR_INVALID_ARG
+    assert lib.muir_state_init(C.c_void_p(1 << 20), None, 1, 1, 48, 32, None) == N.MUIR_ERR_UNSUPPORTED
+    assert lib.muir_state_init(C.c_void_p((1 << 20) + 4), None, 1, 1, 32, 32, None) == N.MUIR_ERR_INVALID_ARG
+
+
+def _chunk_args(**kw):
+    fake = C.c_void_p(1 << 20)
+    a = N.ChunkArgs(B=1, T=256, H=2, dk=32, dv=32, chunk=64, dtype=N.MUIR_F32, reserved=0,
+                    q=fake, k=fake, v=fake, e=fake, w=fake, g=fake, z=None, log_alpha=fake, r=fake, S0=None)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("chunk", 96, N.MUIR_ERR_UNSUPPORTED),
+    ("T", 250, N.MUIR_ERR_UNSUPPORTED),
+    ("dk", 48, N.MUIR_ERR_UNSUPPORTED),
+    ("dtype", 3, N.MUIR_ERR_UNSUPPORTED),
+    ("q", None, N.MUIR_ERR_INVALID_ARG),
+    ("log_alpha", C.c_void_p((1 << 20) + 8), N.MUIR_ERR_INVALID_ARG),
+])
+def test_chunk_fwd_rejects_bad_args(lib, field, value, code):
+    a = _chunk_args(**{field: value})
+    y = C.c_void_p(1 << 20)
+    assert lib.muir_chunk_fwd(C.byref(a), y, None, C.c_void_p(1 << 20), 1 << 30, None) == code
+
+
+def test_chunk_workspace_is_checked(lib):
+    a = _chunk_args()
+    need = lib.muir_chunk_fwd_workspace(C.byref(a))
+    assert need > 0
+    y = C.c_void_p(1 << 20)
+    assert lib.muir_chunk_fwd(C.byref(a), y, None, C.c_void_p(1 << 20), need - 1, None) == N.MUIR_ERR_WORKSPACE
+    assert lib.muir_chunk_fwd(C.byref(a), y, None, None, need, None) == N.MUIR_ERR_WORKSPACE
+    assert lib.muir_chunk_bwd_workspace(C.byref(a)) >= need
+    g = N.ChunkGrads()
+    assert lib.muir_chunk_bwd(C.byref(a), C.byref(g), C.c_void_p(1 << 20), 1 << 40, None) == N.MUIR_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op(lib):
+    a = _chunk_args(B=0)
+    assert lib.muir_chunk_fwd(C.byref(a), C.c_void_p(1 << 20), None, None, 0, None) == N.MUIR_OK
