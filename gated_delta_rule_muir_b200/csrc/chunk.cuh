@@ -67,7 +67,12 @@ struct ChunkParams {
   // outputs
   void* y;
   float* S_T;
-  float* S_chunks;  // optional [B,H,T/C,dk,dv]: state at the start of every chunk
+  float* S_chunks;  // optional [units][dk][dv]: state at the start of every unit
+  // backward
+  float* wsave;     // optional [nsubtot][Cs][dk]: W
+  float* usave;     // optional [nsubtot][Cs][dv]: Ut
+  const void* dy;   // [B,T,H,dv]
+  void* dz;         // [B,T,H,dv] or null
 };
 
 struct SubIdx {
@@ -93,8 +98,8 @@ __device__ __forceinline__ int64_t toff(const ChunkParams& p, int b, int64_t tok
 __device__ __forceinline__ void ld8f(const float* p, float (&o)[8]) { Elt<float>::ld8(p, o); }
 
 __device__ __forceinline__ Tile sub_tile(const Tile& t, int k0, int mn0) {
-  const uint32_t off = (uint32_t)(k0 >> 3) * 128u + (uint32_t)(mn0 >> 3) * t.sbo;
-  return Tile{t.hi + off, t.lo + off, t.sbo};
+  const uint32_t off = (uint32_t)(k0 >> 3) * t.lbo + (uint32_t)(mn0 >> 3) * t.sbo;
+  return Tile{t.hi + off, t.lo + off, t.lbo, t.sbo};
 }
 
 __device__ __forceinline__ void zero_smem(uint32_t base, uint32_t bytes) {
@@ -219,9 +224,9 @@ __global__ void __launch_bounds__(128, 1) gram_off_kernel(ChunkParams p) {
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr uint32_t LB = 128u * DK * 2u, RB = SB * DK * 2u;
   const uint32_t base = smem_u32(sm);
-  const Tile L{base, base + LB, DK * 16u};
-  const Tile RK{base + 2 * LB, base + 2 * LB + RB, DK * 16u};
-  const Tile RA{base + 2 * LB + 2 * RB, base + 2 * LB + 3 * RB, DK * 16u};
+  const Tile L{base, base + LB, 128u, DK * 16u};
+  const Tile RK{base + 2 * LB, base + 2 * LB + RB, 128u, DK * 16u};
+  const Tile RA{base + 2 * LB + 2 * RB, base + 2 * LB + 3 * RB, 128u, DK * 16u};
   float* midtab = reinterpret_cast<float*>(sm + 2 * LB + 4 * RB);  // [nb][DK]
   zero_smem(base, 2 * LB);
   TcCta cta;
@@ -390,8 +395,8 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
   float* Tf = reinterpret_cast<float*>(sm);  // [Cs][Cs]
   const uint32_t base = smem_u32(sm) + 128u * 128u * 4u;
   constexpr uint32_t TB = 128u * 128u * 2u;
-  const Tile TA{base, base + TB, (uint32_t)Cs * 16u};           // K-major A tiles (K = Cs)
-  const Tile TBt{base + 2 * TB, base + 3 * TB, (uint32_t)Cs * 16u};  // MN-major B tiles (K = Cs)
+  const Tile TA{base, base + TB, 128u, (uint32_t)Cs * 16u};           // K-major A tiles (K = Cs)
+  const Tile TBt{base + 2 * TB, base + 3 * TB, 128u, (uint32_t)Cs * 16u};  // MN-major B tiles (K = Cs)
   const float* M = p.gr + ((int64_t)blockIdx.x * 4 + 1) * Cs * Cs;
   for (int x = tid; x < Cs * Cs; x += 128) Tf[x] = 0.f;
   zero_smem(base, 4 * TB);
@@ -515,9 +520,9 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   constexpr uint32_t TBY = 128u * 128u * 2u;
   const uint32_t base = smem_u32(sm);
   const uint32_t kstride = (uint32_t)Cs * 16u;  // every tile here contracts over the Cs tokens
-  const Tile A{base, base + TBY, kstride};
-  const Tile B1{base + 2 * TBY, base + 3 * TBY, kstride};
-  const Tile B2{base + 4 * TBY, base + 5 * TBY, kstride};
+  const Tile A{base, base + TBY, 128u, kstride};
+  const Tile B1{base + 2 * TBY, base + 3 * TBY, 128u, kstride};
+  const Tile B2{base + 4 * TBY, base + 5 * TBY, 128u, kstride};
   zero_smem(base, 6 * TBY);
   TcCta cta;
   cta.init(&tslot, &bar, 512);
@@ -594,6 +599,26 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   tmem_to_b(B1, cZ, DV);
   stage_k_matrix(A, Tm, 1.f);
   drv.run([&] { mma_tiles(cta.tmem + cUt, A, B1, Cs / 16, idV, NS, false); });
+  if (p.wsave) {  // the backward pass reuses W and Ut
+    float* wo = p.wsave + (int64_t)blockIdx.x * Cs * DK;
+    float* uo = p.usave + (int64_t)blockIdx.x * Cs * DV;
+    for (int c = 0; c < DK; c += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + lane + cW + c, v);
+      if (t < Cs)
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(wo + t * DK + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+    for (int c = 0; c < DV; c += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + lane + cUt + c, v);
+      if (t < Cs)
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(uo + t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  }
   // ---- phase 2 with W in B1: Phi = Diag(Gam_C) - (A*Gsuf)^T W, Q' = Qt*Gam - N^qa W
   tmem_to_b(B1, cW, DK);
   stage_suffixed(true, -1.f);
@@ -684,9 +709,9 @@ __global__ void __launch_bounds__(128, 1) compose_kernel(ChunkParams p) {
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr uint32_t TBY = 128u * DK * 2u;
   const uint32_t base = smem_u32(sm);
-  const Tile A0{base, base + TBY, DK * 16u};
-  const Tile A1{base + 2 * TBY, base + 3 * TBY, DK * 16u};
-  const Tile Bt{base + 4 * TBY, base + 4 * TBY + 128u * DK * 2u, DK * 16u};
+  const Tile A0{base, base + TBY, 128u, DK * 16u};
+  const Tile A1{base + 2 * TBY, base + 3 * TBY, 128u, DK * 16u};
+  const Tile Bt{base + 4 * TBY, base + 4 * TBY + 128u * DK * 2u, 128u, DK * 16u};
   zero_smem(base, 4 * TBY + 2u * 128u * DK * 2u);
   TcCta cta;
   cta.init(&tslot, &bar, 512);
@@ -784,7 +809,7 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const float
   const int ntile = (rows_total + 127) / 128;
   constexpr uint32_t ATB = 128u * DK * 2u;
   const uint32_t base = smem_u32(sm);
-  const Tile Sb{base, base + NW * DK * 2u, DK * 16u};  // B: K = key row, N = slab column (MN-major)
+  const Tile Sb{base, base + NW * DK * 2u, 128u, DK * 16u};  // B: K = key row, N = slab column (MN-major)
   const uint32_t abase = base + 2u * NW * DK * 2u;
   zero_smem(base, 2u * NW * DK * 2u + 2u * ATB * ntile);
   TcCta cta;
@@ -825,12 +850,12 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const float
         for (int j = 0; j < 8; ++j) v[j] = 0.f;
       }
       const int tile = r >> 7;
-      const Tile At{abase + tile * 2u * ATB, abase + tile * 2u * ATB + ATB, DK * 16u};
+      const Tile At{abase + tile * 2u * ATB, abase + tile * 2u * ATB + ATB, 128u, DK * 16u};
       put_k(At, r & 127, c8, v);
     }
     drv.run([&] {
       for (int tile = 0; tile < ntile; ++tile) {
-        const Tile At{abase + tile * 2u * ATB, abase + tile * 2u * ATB + ATB, DK * 16u};
+        const Tile At{abase + tile * 2u * ATB, abase + tile * 2u * ATB + ATB, 128u, DK * 16u};
         mma_tiles(cta.tmem + tile * NW, At, Sb, DK / 16, id, NS, false);
       }
     });
@@ -857,6 +882,19 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const float
           o[j] = v[j] + add.x; o[j + 1] = v[j + 1] + add.y; o[j + 2] = v[j + 2] + add.z; o[j + 3] = v[j + 3] + add.w;
         }
         const int64_t yo = toff(p, b, tok, h, dv) + slab * NW;
+        if (!p.y) {  // backward recompute: only dz = O * dy is wanted
+          if (p.dz && p.z) {
+#pragma unroll
+            for (int j = 0; j < NW; j += 8) {
+              float dd[8], w8[8];
+              Elt<T>::ld8(static_cast<const T*>(p.dy) + yo + j, dd);
+#pragma unroll
+              for (int e2 = 0; e2 < 8; ++e2) w8[e2] = o[j + e2] * dd[e2];
+              Elt<T>::st8(static_cast<T*>(p.dz) + yo + j, w8);
+            }
+          }
+          continue;
+        }
         if (p.z) {
 #pragma unroll
           for (int j = 0; j < NW; j += 8) {

@@ -1,0 +1,697 @@
+// Chunkwise backward pass (reverse mode of the chunk map in chunk.cuh).
+//
+// Per unit (chunk of Cs <= 128 tokens) with start state S0, forward quantities
+//   Z = (K*Gam) S0 + M^kk U,  P = T Z,  O = (Qt*Gam) S0 + N^qk U - N^qa P,
+//   S_C = Diag(Gam_C) S0 + (K*Gsuf)^T U - (A*Gsuf)^T P,  y = z*O,
+// and cotangents dO = z*dy, dS_C (state cotangent at the unit end):
+//   dP   = -N^qa^T dO - (A*Gsuf) dS_C          dZ = T^T dP
+//   dU   = N^qk^T dO + (K*Gsuf) dS_C + M^kk^T dZ
+//   dQp  = dO S0^T      dKp = dZ S0^T      dKs = U dS_C^T      dAs = -P dS_C^T
+//   dN^qk = dO U^T, dN^qa = -dO P^T (s <= t);  dM^kk = dZ U^T, dM^ka = -dZ P^T (s < t)
+//   dGam_C = rowsum(dS_C * S0)
+// (dM^ka uses d(T) = -T d(M^ka) T, so -T^T dP Z^T T^T = -dZ P^T.) The state
+// cotangent entering the unit is the adjoint of the unit's affine map:
+//   dS0 = Phi^T dS_C + Q'^T dO.
+// A decayed Gram G_ts = sum_i X_ti Y_si Gam_{t<-s,i} sends
+//   dX_t = sum_s dG_ts Y_s*Gam_{t<-s},  dY_s = sum_t dG_ts X_t*Gam_{t<-s},
+// and, since Gam_{t<-s} = exp(L_t - L_s) with L the in-chunk cumulative sum of
+// log alpha, dL_t += X_t*dX_t and dL_s -= Y_s*dY_s. dlog_alpha is the reverse
+// cumulative sum of dL inside the unit.
+//
+// Kernels:
+//   rscan_kernel       reverse sweep over units per (b, h, 32-column slab)
+//   bwd_p_kernel       P = W S0 + Ut, dGam_C
+//   bwd_dz_kernel      dP, dZ, dU
+//   bwd_grads_kernel   dQp, dKp, dKs, dAs and the four Gram cotangents
+//   bwd_gram_off_kernel  off-diagonal blocks of the Gram backward (tcgen05):
+//                      dX with the pivot at the start of the row block,
+//                      dY with the pivot at the end of the column block
+//   bwd_gram_diag_kernel diagonal 16x16 blocks (CUDA cores, thread = channel)
+//   bwd_final_kernel   decay cotangents, reverse cumsum, chain rule to inputs
+#pragma once
+
+#include "chunk.cuh"
+
+namespace muir {
+
+struct BwdBufs {
+  float* S_chunks;  // [nst][dk][dv]
+  float* dSC;       // [nst][dk][dv]   state cotangent at each unit's end
+  float* P;         // [nst][Cs][dv]
+  float* dZ;        // [nst][Cs][dv]
+  float* dU;        // [nst][Cs][dv]
+  float* dgc;       // [nst][dk]
+  float* g4;        // [nst][4][Cs][dk]: dQp, dKp, dKs, dAs
+  float* dG;        // [nst][4][Cs][Cs]: dM^kk, dM^ka, dN^qk, dN^qa
+  float* gl;        // [nst][4][Cs][dk]: dK_left, dQ_left, dK_right, dA_right
+  const float* dS_T;
+  float* dS0;
+  void *dq, *dk, *dv, *de, *dw, *dg;
+  float* dla;
+  float* dr;
+};
+
+// ---------------------------------------------------------------------------
+// rscan_kernel: for n = last..0: dSC[n] = dS;  dS <- [Phi; Q']^T [dS; dO_n].
+// A = [Phi; Q']^T (M = key channel, K = rows of the map), MN-major;
+// B = [dS; dO] (K = rows, N = 32 slab columns), MN-major.
+// ---------------------------------------------------------------------------
+template <int DK, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  constexpr int NW = 32;
+  const int dv = p.dv, slabs = dv / NW, Cs = p.Cs;
+  const int slab = blockIdx.x % slabs;
+  const int bh = blockIdx.x / slabs;
+  const int h = bh % p.H, b = bh / p.H;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int R = DK + Cs;  // rows of the map = contraction length
+  const uint32_t base = smem_u32(sm);
+  const uint32_t AB = 128u * (uint32_t)R * 2u, BB = (uint32_t)NW * R * 2u;
+  const Tile At{base, base + AB, 128u, (uint32_t)R * 16u};
+  const Tile Bt{base + 2 * AB, base + 2 * AB + BB, 128u, (uint32_t)R * 16u};
+  zero_smem(base, 2 * AB + 2 * BB);
+  TcCta cta;
+  cta.init(&tslot, &bar, 32);
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t lane = tmem_lane_base(warp);
+  float ds[NW];
+  {
+    const float* src = q.dS_T ? q.dS_T + (((int64_t)b * p.H + h) * DK) * dv + slab * NW : nullptr;
+#pragma unroll
+    for (int j = 0; j < NW; ++j) ds[j] = (src && tid < DK) ? src[(int64_t)tid * dv + j] : 0.f;
+  }
+  const uint32_t id = idesc_bf16(128, NW, 1, 1);
+  for (int n = p.nsub - 1; n >= 0 && drv.ok; --n) {
+    const int64_t uid = ((int64_t)b * p.H + h) * p.nsub + n;
+    if (tid < DK) {
+      float* o = q.dSC + (uid * DK + tid) * dv + slab * NW;
+#pragma unroll
+      for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(ds[j], ds[j + 1], ds[j + 2], ds[j + 3]);
+#pragma unroll
+      for (int j = 0; j < NW; j += 8) {
+        float v[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) v[e2] = ds[j + e2];
+        put_mn(Bt, tid, j, v);
+      }
+    }
+    // dO rows of this unit: tokens n*Cs + t
+    for (int x = tid; x < Cs * (NW / 8); x += 128) {
+      const int t = x / (NW / 8), c8 = (x % (NW / 8)) * 8;
+      const int64_t o = toff(p, b, (int64_t)n * Cs + t, h, dv) + slab * NW + c8;
+      float dd[8], zz[8];
+      Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
+      if (p.z) {
+        Elt<T>::ld8(static_cast<const T*>(p.z) + o, zz);
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) dd[e2] *= zz[e2];
+      }
+      put_mn(Bt, DK + t, c8, dd);
+    }
+    const float* A = p.ma + uid * R * DK;
+    for (int x = tid; x < R * (DK / 8); x += 128) {
+      const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      float v[8];
+      ld8f(A + (int64_t)r * DK + c8, v);
+      put_mn(At, r, c8, v);
+    }
+    drv.run([&] { mma_tiles(cta.tmem, At, Bt, R / 16, id, NS, false); });
+    if (!drv.ok) break;
+    float v[NW];
+    tmem_ld16(cta.tmem + lane, *reinterpret_cast<float(*)[16]>(&v[0]));
+    tmem_ld16(cta.tmem + lane + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+#pragma unroll
+    for (int j = 0; j < NW; ++j) ds[j] = v[j];
+    __syncthreads();
+  }
+  if (q.dS0 && tid < DK && drv.ok) {
+    float* o = q.dS0 + (((int64_t)b * p.H + h) * DK + tid) * dv + slab * NW;
+#pragma unroll
+    for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(ds[j], ds[j + 1], ds[j + 2], ds[j + 3]);
+  }
+  cta.finish();
+}
+
+// Stage a row-major fp32 matrix src[rows][cols] (row stride ld) as a K-major
+// operand contracting over cols (put_k), values scaled by sign. rows <= 128.
+__device__ __forceinline__ void stage_rows_k(const Tile& t, const float* src, int rows, int cols, int64_t ld,
+                                             float sign) {
+  for (int x = threadIdx.x; x < rows * (cols / 8); x += blockDim.x) {
+    const int r = x / (cols / 8), c8 = (x % (cols / 8)) * 8;
+    float v[8];
+    ld8f(src + r * ld + c8, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] *= sign;
+    put_k(t, r, c8, v);
+  }
+}
+// Same matrix as an MN-major operand contracting over rows (put_mn).
+__device__ __forceinline__ void stage_rows_mn(const Tile& t, const float* src, int rows, int cols, int64_t ld,
+                                              float sign) {
+  for (int x = threadIdx.x; x < rows * (cols / 8); x += blockDim.x) {
+    const int r = x / (cols / 8), c8 = (x % (cols / 8)) * 8;
+    float v[8];
+    ld8f(src + r * ld + c8, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] *= sign;
+    put_mn(t, r, c8, v);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_p_kernel: P = W S0 + Ut (A = W K-major over channels, B = S0 MN-major),
+// and dGam_C[i] = sum_j dS_C[i][j] S0[i][j].
+// ---------------------------------------------------------------------------
+template <int DK, int DV, int NS>
+__global__ void __launch_bounds__(128, 1) bwd_p_kernel(ChunkParams p, BwdBufs q) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int Cs = p.Cs;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t u = blockIdx.x;
+  const uint32_t base = smem_u32(sm);
+  constexpr uint32_t TB = 128u * 128u * 2u;
+  const Tile A{base, base + TB, 128u, DK * 16u};
+  const Tile B{base + 2 * TB, base + 3 * TB, 128u, DK * 16u};
+  zero_smem(base, 4 * TB);
+  TcCta cta;
+  cta.init(&tslot, &bar, 128);
+  MmaSync drv{&bar, 0u, true};
+  const float* S0 = q.S_chunks + u * DK * DV;
+  stage_rows_k(A, p.wsave + u * Cs * DK, Cs, DK, DK, 1.f);
+  stage_rows_mn(B, S0, DK, DV, DV, 1.f);
+  drv.run([&] { mma_tiles(cta.tmem, A, B, DK / 16, idesc_bf16(128, DV, 0, 1), NS, false); });
+  const int t = tid;
+  const float* Ut = p.usave + u * Cs * DV;
+  float* P = q.P + u * Cs * DV;
+  for (int c = 0; c < DV; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + tmem_lane_base(warp) + c, v);
+    if (t < Cs && drv.ok)
+#pragma unroll
+      for (int j = 0; j < 16; j += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(Ut + t * DV + c + j);
+        *reinterpret_cast<float4*>(P + t * DV + c + j) = make_float4(v[j] + a.x, v[j + 1] + a.y, v[j + 2] + a.z, v[j + 3] + a.w);
+      }
+  }
+  if (tid < DK) {
+    const float* d = q.dSC + u * DK * DV + tid * DV;
+    const float* s0 = S0 + tid * DV;
+    float acc = 0.f;
+    for (int j = 0; j < DV; ++j) acc += d[j] * s0[j];
+    q.dgc[u * DK + tid] = acc;
+  }
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// bwd_dz_kernel: dP = -N^qa^T dO - (A*Gsuf) dS_C;  dZ = T^T dP;
+//                dU = N^qk^T dO + (K*Gsuf) dS_C + M^kk^T dZ.
+// TMEM: dP -> 0, dU -> 128, dZ -> 256. Tiles: A, B1 (dO), B2 (dS_C; later dZ).
+// ---------------------------------------------------------------------------
+template <int DK, int DV, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int Cs = p.Cs;
+  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t u = blockIdx.x;
+  const uint32_t base = smem_u32(sm);
+  constexpr uint32_t TB = 128u * 128u * 2u;
+  const uint32_t ks = (uint32_t)Cs * 16u;
+  const Tile A{base, base + TB, 128u, ks};             // A over tokens (K = Cs)
+  const Tile Ak{base, base + TB, 128u, DK * 16u};      // A over channels (K = DK)
+  const Tile B1{base + 2 * TB, base + 3 * TB, 128u, ks};
+  const Tile B2{base + 4 * TB, base + 5 * TB, 128u, DK * 16u};
+  const Tile B3{base + 4 * TB, base + 5 * TB, 128u, ks};
+  zero_smem(base, 6 * TB);
+  TcCta cta;
+  cta.init(&tslot, &bar, 512);
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t lane = tmem_lane_base(warp);
+  const Rows<T> rows{p, s.b, s.h};
+  const float* G = p.gr + u * 4 * Cs * Cs;
+  const float* gsuf = p.dec + (u * 4 + 3) * Cs * DK;
+  const int t = tid;
+  constexpr uint32_t cP = 0, cU = 128, cZ = 256;
+  // B1 = dO (K = token, N = value column)
+  for (int x = tid; x < Cs * (DV / 8); x += 128) {
+    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+    const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
+    float dd[8], zz[8];
+    Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
+    if (p.z) {
+      Elt<T>::ld8(static_cast<const T*>(p.z) + o, zz);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dd[j] *= zz[j];
+    }
+    put_mn(B1, r, c8, dd);
+  }
+  stage_rows_mn(B2, q.dSC + u * DK * DV, DK, DV, DV, 1.f);  // dS_C (K = channel)
+  stage_rows_mn(A, G + 3 * Cs * Cs, Cs, Cs, Cs, -1.f);      // (-N^qa)^T: K = t, M = s
+  const uint32_t idT = idesc_bf16(128, DV, 1, 1), idK = idesc_bf16(128, DV, 0, 1);
+  drv.run([&] { mma_tiles(cta.tmem + cP, A, B1, Cs / 16, idT, NS, false); });
+  stage_rows_mn(A, G + 2 * Cs * Cs, Cs, Cs, Cs, 1.f);       // N^qk^T
+  drv.run([&] { mma_tiles(cta.tmem + cU, A, B1, Cs / 16, idT, NS, false); });
+  // -(A*Gsuf) and (K*Gsuf): rows s, K = channel (K-major)
+  auto stage_suf = [&](bool erase, float sign) {
+    for (int x = tid; x < Cs * (DK / 8); x += 128) {
+      const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      float xx[8], gs[8];
+      if (erase) rows.a(s.tok0 + r, c8, xx);
+      else rows.k(s.tok0 + r, c8, xx);
+      ld8f(gsuf + r * DK + c8, gs);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xx[j] *= sign * gs[j];
+      put_k(Ak, r, c8, xx);
+    }
+  };
+  stage_suf(true, -1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cP, Ak, B2, DK / 16, idK, NS, true); });
+  stage_suf(false, 1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cU, Ak, B2, DK / 16, idK, NS, true); });
+  // dP (TMEM) -> B3 (K = token), then dZ = T^T dP
+  for (int c = 0; c < DV; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + cP + c, v);
+    if (t < Cs) {
+      float a8[8], b8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
+      put_mn(B3, t, c, a8);
+      put_mn(B3, t, c + 8, b8);
+    }
+  }
+  stage_rows_mn(A, p.tt + u * Cs * Cs, Cs, Cs, Cs, 1.f);  // T^T: K = t, M = s
+  drv.run([&] { mma_tiles(cta.tmem + cZ, A, B3, Cs / 16, idT, NS, false); });
+  float* dZo = q.dZ + u * Cs * DV;
+  for (int c = 0; c < DV; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + cZ + c, v);
+    if (t < Cs) {
+      float a8[8], b8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
+      put_mn(B3, t, c, a8);
+      put_mn(B3, t, c + 8, b8);
+      if (drv.ok)
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(dZo + t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+  }
+  stage_rows_mn(A, G + 0 * Cs * Cs, Cs, Cs, Cs, 1.f);  // M^kk^T
+  drv.run([&] { mma_tiles(cta.tmem + cU, A, B3, Cs / 16, idT, NS, true); });
+  float* dUo = q.dU + u * Cs * DV;
+  for (int c = 0; c < DV; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + cU + c, v);
+    if (t < Cs && drv.ok)
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<float4*>(dUo + t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  }
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// bwd_grads_kernel: products that contract over the value dimension (K = DV),
+// every operand a K-major tile of a [rows][DV] matrix:
+//   pass 1: dKs = U dS_C^T, dAs = -P dS_C^T
+//   pass 2: dN^qk = dO U^T, dN^qa = -dO P^T, dM^kk = dZ U^T, dM^ka = -dZ P^T (masked)
+//   pass 3: dQp = dO S0^T, dKp = dZ S0^T
+// ---------------------------------------------------------------------------
+template <int DK, int DV, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBufs q) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int Cs = p.Cs;
+  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t u = blockIdx.x;
+  const uint32_t base = smem_u32(sm);
+  constexpr uint32_t TB = 128u * 128u * 2u;
+  const Tile R0{base, base + TB, 128u, DV * 16u};
+  const Tile R1{base + 2 * TB, base + 3 * TB, 128u, DV * 16u};
+  const Tile R2{base + 4 * TB, base + 5 * TB, 128u, DV * 16u};
+  zero_smem(base, 6 * TB);
+  TcCta cta;
+  cta.init(&tslot, &bar, 512);
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t lane = tmem_lane_base(warp);
+  const int t = tid;
+  auto stage_dO = [&](const Tile& dst) {
+    for (int x = tid; x < Cs * (DV / 8); x += 128) {
+      const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+      const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
+      float dd[8], zz[8];
+      Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
+      if (p.z) {
+        Elt<T>::ld8(static_cast<const T*>(p.z) + o, zz);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dd[j] *= zz[j];
+      }
+      put_k(dst, r, c8, dd);
+    }
+  };
+  auto stage_U = [&](const Tile& dst) {
+    const Rows<T> rows{p, s.b, s.h};
+    for (int x = tid; x < Cs * (DV / 8); x += 128) {
+      const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+      float uu[8];
+      rows.u(s.tok0 + r, c8, uu);
+      put_k(dst, r, c8, uu);
+    }
+  };
+  // Row t of a [Cs][N] TMEM result -> dst (fp32, row-major, row stride ld), optional mask.
+  auto drain = [&](uint32_t col, int n, float* dst, int64_t ld, int mask) {
+    for (int c = 0; c < n; c += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + lane + col + c, v);
+      if (t < Cs && drv.ok) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int sidx = c + j;
+          if (mask == 1 && sidx >= t) v[j] = 0.f;  // strictly lower
+          if (mask == 2 && sidx > t) v[j] = 0.f;   // lower incl. diagonal
+        }
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(dst + t * ld + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      }
+    }
+  };
+  const uint32_t idK = idesc_bf16(128, DK, 0, 0), idC = idesc_bf16(128, Cs, 0, 0);
+  float* g4 = q.g4 + u * 4 * Cs * DK;
+  float* dG = q.dG + u * 4 * Cs * Cs;
+  // pass 1
+  stage_rows_k(R0, q.dSC + u * DK * DV, DK, DV, DV, 1.f);
+  stage_U(R1);
+  stage_rows_k(R2, q.P + u * Cs * DV, Cs, DV, DV, -1.f);
+  drv.run([&] {
+    mma_tiles(cta.tmem + 0, R1, R0, DV / 16, idK, NS, false);
+    mma_tiles(cta.tmem + 128, R2, R0, DV / 16, idK, NS, false);
+  });
+  drain(0, DK, g4 + 2 * Cs * DK, DK, 0);    // dKs
+  drain(128, DK, g4 + 3 * Cs * DK, DK, 0);  // dAs
+  // pass 2: R1 = U, R2 = -P stay
+  stage_dO(R0);
+  drv.run([&] {
+    mma_tiles(cta.tmem + 0, R0, R1, DV / 16, idC, NS, false);    // dN^qk
+    mma_tiles(cta.tmem + 128, R0, R2, DV / 16, idC, NS, false);  // dN^qa
+  });
+  stage_rows_k(R0, q.dZ + u * Cs * DV, Cs, DV, DV, 1.f);
+  drv.run([&] {
+    mma_tiles(cta.tmem + 256, R0, R1, DV / 16, idC, NS, false);  // dM^kk
+    mma_tiles(cta.tmem + 384, R0, R2, DV / 16, idC, NS, false);  // dM^ka
+  });
+  drain(0, Cs, dG + 2 * Cs * Cs, Cs, 2);
+  drain(128, Cs, dG + 3 * Cs * Cs, Cs, 2);
+  drain(256, Cs, dG + 0 * Cs * Cs, Cs, 1);
+  drain(384, Cs, dG + 1 * Cs * Cs, Cs, 1);
+  // pass 3: R1 = S0, R0 = dO, R2 = dZ
+  stage_rows_k(R1, q.S_chunks + u * DK * DV, DK, DV, DV, 1.f);
+  stage_dO(R0);
+  stage_rows_k(R2, q.dZ + u * Cs * DV, Cs, DV, DV, 1.f);
+  drv.run([&] {
+    mma_tiles(cta.tmem + 0, R0, R1, DV / 16, idK, NS, false);    // dQp
+    mma_tiles(cta.tmem + 128, R2, R1, DV / 16, idK, NS, false);  // dKp
+  });
+  drain(0, DK, g4 + 0 * Cs * DK, DK, 0);
+  drain(128, DK, g4 + 1 * Cs * DK, DK, 0);
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// bwd_gram_off_kernel: off-diagonal blocks of the Gram backward. Results are
+// accumulated transposed in TMEM (lane = key channel, column = token):
+//   left  (rows t of block J, pivot = last token of block J-1):
+//     dX_t = pre_t * sum_{s < start(J)} dG_ts (Y_s * suf_s * mid(I(s), J))
+//     A = (Y*suf*mid)^T (MN-major over s), B = dG[J rows, s]^T (K-major, N = 16)
+//   right (columns s of block I, pivot = last token of block I):
+//     dY_s = suf_s * sum_{t > end(I)} dG_ts (X_t * pre_t * mid(I, J(t)))
+//     A = (X*pre*mid)^T (MN-major over t), B = dG[t, I cols] (MN-major, N = 16)
+// Region columns: dK_left 0, dQ_left Cs, dK_right 2Cs, dA_right 3Cs.
+// ---------------------------------------------------------------------------
+template <int DK, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, BwdBufs q) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  const int Cs = p.Cs, nb = Cs / SB;
+  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t u = blockIdx.x;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t AB = 128u * (uint32_t)Cs * 2u;  // M = 128 channels (padded) x K = Cs tokens
+  const uint32_t BB = (uint32_t)SB * Cs * 2u;    // N = 16 x K = Cs
+  const Tile A1{base, base + AB, 128u, (uint32_t)Cs * 16u};
+  const Tile A2{base + 2 * AB, base + 3 * AB, 128u, (uint32_t)Cs * 16u};
+  Tile Bk[4], Bm[4];
+  for (int g = 0; g < 4; ++g) {
+    const uint32_t b0 = base + 4 * AB + g * 2 * BB;
+    Bk[g] = Tile{b0, b0 + BB, 128u, (uint32_t)Cs * 16u};  // K-major: row = t (N), K = s
+    Bm[g] = Tile{b0, b0 + BB, 128u, (uint32_t)Cs * 16u};  // MN-major: row = t (K), N = s (16)
+  }
+  float* midtab = reinterpret_cast<float*>(sm + 4 * AB + 8 * BB);  // [nb][DK]
+  zero_smem(base, 4 * AB + 8 * BB);
+  TcCta cta;
+  cta.init(&tslot, &bar, tmem_cols_for(4 * Cs));
+  MmaSync drv{&bar, 0u, true};
+  const float* pre = p.dec + u * 4 * Cs * DK;
+  const float* suf = pre + Cs * DK;
+  const float* dG = q.dG + u * 4 * Cs * Cs;
+  const Rows<T> rows{p, s.b, s.h};
+  const uint32_t id16 = idesc_bf16(128, SB, 1, 0), id16m = idesc_bf16(128, SB, 1, 1);
+  // ---- left gradients: J ascending, mid(I, J) for I < J
+  for (int J = 1; J < nb && drv.ok; ++J) {
+    for (int x = tid; x < nb * DK; x += 128) {
+      const int I = x / DK, i = x % DK;
+      if (I == J - 1) midtab[x] = 1.f;
+      else if (I < J - 1) midtab[x] *= pre[(SB * (J - 1) + SB - 1) * DK + i];  // tot_{J-1}
+    }
+    __syncthreads();
+    for (int x = tid; x < SB * J * (DK / 8); x += 128) {
+      const int ss = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      float kk[8], aa[8], sf[8];
+      rows.k(s.tok0 + ss, c8, kk);
+      rows.a(s.tok0 + ss, c8, aa);
+      ld8f(suf + ss * DK + c8, sf);
+      const float* mp = midtab + (ss / SB) * DK + c8;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { const float f = sf[j] * mp[j]; kk[j] *= f; aa[j] *= f; }
+      put_mn(A1, ss, c8, kk);
+      put_mn(A2, ss, c8, aa);
+    }
+    for (int x = tid; x < 4 * SB * (SB * J / 8); x += 128) {
+      const int g = x / (SB * (SB * J / 8)), rem = x % (SB * (SB * J / 8));
+      const int rr = rem / (SB * J / 8), c8 = (rem % (SB * J / 8)) * 8;
+      float v[8];
+      ld8f(dG + ((int64_t)g * Cs + SB * J + rr) * Cs + c8, v);
+      put_k(Bk[g], rr, c8, v);
+    }
+    drv.run([&] {
+      const uint32_t c = SB * J;
+      mma_tiles(cta.tmem + 0 * Cs + c, A1, Bk[0], J, id16, NS, false);  // dM^kk . K
+      mma_tiles(cta.tmem + 0 * Cs + c, A2, Bk[1], J, id16, NS, true);   // dM^ka . A
+      mma_tiles(cta.tmem + 1 * Cs + c, A1, Bk[2], J, id16, NS, false);  // dN^qk . K
+      mma_tiles(cta.tmem + 1 * Cs + c, A2, Bk[3], J, id16, NS, true);   // dN^qa . A
+    });
+  }
+  // ---- right gradients: I descending, mid(I, J) for J > I
+  for (int I = nb - 2; I >= 0 && drv.ok; --I) {
+    for (int x = tid; x < nb * DK; x += 128) {
+      const int J = x / DK, i = x % DK;
+      if (J == I + 1) midtab[x] = 1.f;
+      else if (J > I + 1) midtab[x] *= pre[(SB * (I + 1) + SB - 1) * DK + i];
+    }
+    __syncthreads();
+    const int t0 = SB * (I + 1);
+    for (int x = tid; x < (Cs - t0) * (DK / 8); x += 128) {
+      const int tt = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      float kk[8], qq[8], pr[8];
+      rows.k(s.tok0 + tt, c8, kk);
+      rows.qt(s.tok0 + tt, c8, qq);
+      ld8f(pre + tt * DK + c8, pr);
+      const float* mp = midtab + (tt / SB) * DK + c8;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { const float f = pr[j] * mp[j]; kk[j] *= f; qq[j] *= f; }
+      put_mn(A1, tt, c8, kk);
+      put_mn(A2, tt, c8, qq);
+    }
+    for (int x = tid; x < 4 * (Cs - t0) * 2; x += 128) {
+      const int g = x / ((Cs - t0) * 2), rem = x % ((Cs - t0) * 2);
+      const int tt = t0 + rem / 2, c8 = (rem % 2) * 8;
+      float v[8];
+      ld8f(dG + ((int64_t)g * Cs + tt) * Cs + SB * I + c8, v);
+      put_mn(Bm[g], tt, c8, v);
+    }
+    drv.run([&] {
+      const uint32_t c = SB * I;
+      const int k0 = t0, ks = (Cs - t0) / 16;
+      mma_tiles(cta.tmem + 2 * Cs + c, sub_tile(A1, k0, 0), sub_tile(Bm[0], k0, 0), ks, id16m, NS, false);
+      mma_tiles(cta.tmem + 2 * Cs + c, sub_tile(A2, k0, 0), sub_tile(Bm[2], k0, 0), ks, id16m, NS, true);
+      mma_tiles(cta.tmem + 3 * Cs + c, sub_tile(A1, k0, 0), sub_tile(Bm[1], k0, 0), ks, id16m, NS, false);
+      mma_tiles(cta.tmem + 3 * Cs + c, sub_tile(A2, k0, 0), sub_tile(Bm[3], k0, 0), ks, id16m, NS, true);
+    });
+  }
+  // ---- epilogue: lane = channel i; scale by pre (left) or suf (right); blocks
+  // without contributions (J = 0 left, I = nb-1 right) are written as zeros.
+  const int i = tid;
+  float* gl = q.gl + u * 4 * Cs * DK;
+  for (int reg = 0; reg < 4; ++reg) {
+    const bool left = reg < 2;
+    const float* sc = left ? pre : suf;
+    for (int c = 0; c < Cs; c += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + tmem_lane_base(warp) + reg * Cs + c, v);
+      const int blk = c / SB;
+      const bool zero = left ? (blk == 0) : (blk == nb - 1);
+      if (i < DK && drv.ok) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int tt = c + j;
+          gl[((int64_t)reg * Cs + tt) * DK + i] = zero ? 0.f : v[j] * sc[tt * DK + i];
+        }
+      }
+    }
+  }
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// bwd_gram_diag_kernel: diagonal 16x16 blocks of the Gram backward, exactly.
+// One CTA per (unit, block), thread = key channel (running products).
+// ---------------------------------------------------------------------------
+template <int DK, typename T>
+__global__ void __launch_bounds__(128) bwd_gram_diag_kernel(ChunkParams p, BwdBufs q) {
+  __shared__ float sdg[4][SB][SB];
+  const int Cs = p.Cs, nb = Cs / SB;
+  const int64_t u = blockIdx.x / nb;
+  const int J = blockIdx.x % nb;
+  const SubIdx s = sub_of(p, (int)u, p.nsub, Cs);
+  const int i = threadIdx.x;
+  for (int x = threadIdx.x; x < 4 * SB * SB; x += blockDim.x) {
+    const int g = x / (SB * SB), tt = (x / SB) % SB, ss = x % SB;
+    sdg[g][tt][ss] = q.dG[((u * 4 + g) * Cs + SB * J + tt) * Cs + SB * J + ss];
+  }
+  __syncthreads();
+  if (i >= DK) return;
+  float K[SB], A[SB], Q[SB], al[SB];
+  const int64_t stride = (int64_t)p.H * DK;
+  const int64_t o0 = toff(p, s.b, s.tok0 + SB * J, s.h, DK) + i;
+  const float rr = p.r[(int64_t)s.h * DK + i];
+#pragma unroll
+  for (int tt = 0; tt < SB; ++tt) {
+    const int64_t o = o0 + tt * stride;
+    const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
+    K[tt] = kk;
+    A[tt] = Elt<T>::ld(static_cast<const T*>(p.e) + o) * kk;
+    Q[tt] = rr * Elt<T>::ld(static_cast<const T*>(p.g) + o) * Elt<T>::ld(static_cast<const T*>(p.q) + o);
+    al[tt] = expf(p.la[o]);
+  }
+  float dKl[SB], dQl[SB], dKr[SB], dAr[SB];
+#pragma unroll
+  for (int tt = 0; tt < SB; ++tt) { dKl[tt] = 0.f; dQl[tt] = 0.f; dKr[tt] = 0.f; dAr[tt] = 0.f; }
+#pragma unroll
+  for (int ss = 0; ss < SB; ++ss) {
+    float gm = 1.f;
+#pragma unroll
+    for (int tt = ss; tt < SB; ++tt) {
+      if (tt > ss) gm *= al[tt];
+      const float mkk = sdg[0][tt][ss], mka = sdg[1][tt][ss], nqk = sdg[2][tt][ss], nqa = sdg[3][tt][ss];
+      dKl[tt] += (mkk * K[ss] + mka * A[ss]) * gm;
+      dQl[tt] += (nqk * K[ss] + nqa * A[ss]) * gm;
+      dKr[ss] += (mkk * K[tt] + nqk * Q[tt]) * gm;
+      dAr[ss] += (mka * K[tt] + nqa * Q[tt]) * gm;
+    }
+  }
+  float* gl = q.gl + u * 4 * Cs * DK + (int64_t)(SB * J) * DK + i;
+#pragma unroll
+  for (int tt = 0; tt < SB; ++tt) {
+    gl[(0 * Cs + tt) * DK] += dKl[tt];
+    gl[(1 * Cs + tt) * DK] += dQl[tt];
+    gl[(2 * Cs + tt) * DK] += dKr[tt];
+    gl[(3 * Cs + tt) * DK] += dAr[tt];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_final_kernel: per unit, thread = key channel i (then value channel j):
+//   dL_t = k dKl + qt dQl - k dKr - a dAr + Kp dKp + Qp dQp - Ks dKs - As dAs
+//   dL_{C-1} += sum_s (Ks dKs + As dAs) + Gam_C dGam_C
+//   dlog_alpha_t = sum_{u >= t} dL_u
+//   dqt = dQl + Gam dQp, da = dAr + Gsuf dAs, dk = dKl + dKr + Gam dKp + Gsuf dKs + e da
+//   dq = r g dqt, dg = r q dqt, dr += g q dqt, de = k da, dv = w dU, dw = v dU
+// ---------------------------------------------------------------------------
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q) {
+  const int Cs = p.Cs;
+  const int64_t u = blockIdx.x;
+  const SubIdx s = sub_of(p, (int)u, p.nsub, Cs);
+  const int i = threadIdx.x;
+  const int64_t stride_k = (int64_t)p.H * DK, stride_v = (int64_t)p.H * DV;
+  if (i < DK) {
+    const float* gam = p.dec + (u * 4 + 2) * Cs * DK;
+    const float* gsuf = p.dec + (u * 4 + 3) * Cs * DK;
+    const float* g4 = q.g4 + u * 4 * Cs * DK;
+    const float* gl = q.gl + u * 4 * Cs * DK;
+    const float rr = p.r[(int64_t)s.h * DK + i];
+    const int64_t o0 = toff(p, s.b, s.tok0, s.h, DK) + i;
+    // The terms that land on the last token's cumulative log-decay enter every
+    // dlog_alpha of the unit: gather them first.
+    float E = gam[(Cs - 1) * DK + i] * q.dgc[u * DK + i];
+    for (int tt = 0; tt < Cs; ++tt) {
+      const int64_t o = o0 + tt * stride_k;
+      const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
+      const float ee = Elt<T>::ld(static_cast<const T*>(p.e) + o);
+      const int ti = tt * DK + i;
+      E += kk * gsuf[ti] * (g4[2 * Cs * DK + ti] + ee * g4[3 * Cs * DK + ti]);
+    }
+    float run = E, dr_acc = 0.f;
+    for (int tt = Cs - 1; tt >= 0; --tt) {
+      const int64_t o = o0 + tt * stride_k;
+      const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
+      const float ee = Elt<T>::ld(static_cast<const T*>(p.e) + o);
+      const float gg = Elt<T>::ld(static_cast<const T*>(p.g) + o);
+      const float qq = Elt<T>::ld(static_cast<const T*>(p.q) + o);
+      const float a = ee * kk, qt = rr * gg * qq;
+      const int ti = tt * DK + i;
+      const float G = gam[ti], Gs = gsuf[ti];
+      const float dQp = g4[0 * Cs * DK + ti], dKp = g4[1 * Cs * DK + ti];
+      const float dKs = g4[2 * Cs * DK + ti], dAs = g4[3 * Cs * DK + ti];
+      const float dKl = gl[0 * Cs * DK + ti], dQl = gl[1 * Cs * DK + ti];
+      const float dKr = gl[2 * Cs * DK + ti], dAr = gl[3 * Cs * DK + ti];
+      run += kk * dKl + qt * dQl - kk * dKr - a * dAr + kk * G * dKp + qt * G * dQp - kk * Gs * dKs - a * Gs * dAs;
+      q.dla[o] = run;
+      const float dqt = dQl + G * dQp;
+      const float da = dAr + Gs * dAs;
+      const float dkt = dKl + dKr + G * dKp + Gs * dKs + ee * da;
+      Elt<T>::st(static_cast<T*>(q.dq) + o, rr * gg * dqt);
+      Elt<T>::st(static_cast<T*>(q.dg) + o, rr * qq * dqt);
+      Elt<T>::st(static_cast<T*>(q.dk) + o, dkt);
+      Elt<T>::st(static_cast<T*>(q.de) + o, kk * da);
+      dr_acc += gg * qq * dqt;
+    }
+    if (q.dr) atomicAdd(q.dr + (int64_t)s.h * DK + i, dr_acc);
+  }
+  if (i < DV) {
+    const float* dU = q.dU + u * Cs * DV;
+    const int64_t o0 = toff(p, s.b, s.tok0, s.h, DV) + i;
+    for (int tt = 0; tt < Cs; ++tt) {
+      const int64_t o = o0 + tt * stride_v;
+      const float du = dU[tt * DV + i];
+      Elt<T>::st(static_cast<T*>(q.dv) + o, Elt<T>::ld(static_cast<const T*>(p.w) + o) * du);
+      Elt<T>::st(static_cast<T*>(q.dw) + o, Elt<T>::ld(static_cast<const T*>(p.v) + o) * du);
+    }
+  }
+}
+
+}  // namespace muir

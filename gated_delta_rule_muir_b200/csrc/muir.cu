@@ -11,6 +11,7 @@
 #include "decode.cuh"
 #include "selftest.cuh"
 #include "chunk.cuh"
+#include "chunk_bwd.cuh"
 
 namespace {
 

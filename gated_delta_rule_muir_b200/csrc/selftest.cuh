@@ -16,8 +16,8 @@ __global__ void __launch_bounds__(128) selftest_gemm_kernel(const float* __restr
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t base = smem_u32(smem);
   const uint32_t a_bytes = 128u * K * 2u, b_bytes = (uint32_t)N * K * 2u;
-  Tile ta{base, base + a_bytes, (uint32_t)K * 16u};
-  Tile tb{base + 2 * a_bytes, base + 2 * a_bytes + b_bytes, (uint32_t)K * 16u};
+  Tile ta{base, base + a_bytes, 128u, (uint32_t)K * 16u};
+  Tile tb{base + 2 * a_bytes, base + 2 * a_bytes + b_bytes, 128u, (uint32_t)K * 16u};
   if (warp == 0) tmem_alloc(&tmem_base, N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256)));
   if (tid == 0) mbar_init(&bar, 1);
   tc_fence_before();
@@ -25,38 +25,50 @@ __global__ void __launch_bounds__(128) selftest_gemm_kernel(const float* __restr
   tc_fence_after();
   const uint32_t tmem = tmem_base;
 
+  // Operand modes: bit 0 = major (0 K-major, 1 MN-major); bit 1 = the tile is
+  // written in the other arrangement and read through transposed().
+  const int a_major = a_mn & 1, b_major = b_mn & 1;
+  Tile ta_w = ta, tb_w = tb;
+  if (a_mn & 2) ta_w.sbo = 128u * 16u;     // arrangement stride over the 128 rows/cols of A
+  if (b_mn & 2) tb_w.sbo = (uint32_t)N * 16u;
   // A: element (m, k) = A[m*K + k]
   for (int idx = tid; idx < 128 * (K / 8); idx += 128) {
     float x[8];
-    if (!a_mn) {
+    if (a_mn == 0 || a_mn == 2) {  // rows m, 8 consecutive k
       const int m = idx / (K / 8), k8 = (idx % (K / 8)) * 8;
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = A[m * K + k8 + e];
-      put_k(ta, m, k8, x);
-    } else {
+      if (a_mn == 0) put_k(ta_w, m, k8, x);
+      else put_mn(ta_w, m, k8, x);
+    } else {                        // rows k, 8 consecutive m
       const int k = idx / 16, m8 = (idx % 16) * 8;
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = A[(m8 + e) * K + k];
-      put_mn(ta, k, m8, x);
+      if (a_mn == 1) put_mn(ta_w, k, m8, x);
+      else put_k(ta_w, k, m8, x);
     }
   }
   // B: element (k, n) = B[k*N + n]
   for (int idx = tid; idx < N * (K / 8); idx += 128) {
     float x[8];
-    if (!b_mn) {
+    if (b_mn == 0 || b_mn == 2) {  // rows n, 8 consecutive k
       const int n = idx / (K / 8), k8 = (idx % (K / 8)) * 8;
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = B[(k8 + e) * N + n];
-      put_k(tb, n, k8, x);
-    } else {
+      if (b_mn == 0) put_k(tb_w, n, k8, x);
+      else put_mn(tb_w, n, k8, x);
+    } else {                        // rows k, 8 consecutive n
       const int k = idx / (N / 8), n8 = (idx % (N / 8)) * 8;
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = B[k * N + n8 + e];
-      put_mn(tb, k, n8, x);
+      if (b_mn == 1) put_mn(tb_w, k, n8, x);
+      else put_k(tb_w, k, n8, x);
     }
   }
+  if (a_mn & 2) ta = transposed(ta_w);
+  if (b_mn & 2) tb = transposed(tb_w);
   MmaSync drv{&bar, 0u, true};
-  const uint32_t id = idesc_bf16(128, N, a_mn, b_mn);
+  const uint32_t id = idesc_bf16(128, N, a_major, b_major);
   drv.run([&] { mma_tiles(tmem, ta, tb, K / 16, id, nsplit, false); });
   if (drv.ok) {
     for (int c = 0; c < N; c += 16) {

@@ -123,22 +123,30 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// A staged operand tile: bf16 hi and lo parts in shared memory.
+// A staged operand tile: bf16 hi and lo parts in shared memory, with the byte
+// distance between core matrices adjacent along K (lbo) and along M/N (sbo).
+// put_k / put_mn below write tiles whose natural view has lbo = 128. The same
+// memory read with lbo and sbo swapped (transposed()) is the other major: a
+// tile written by put_k as a K-major operand is, transposed, an MN-major
+// operand of the transposed matrix, and vice versa.
 struct Tile {
   uint32_t hi, lo;  // shared addresses (16-byte aligned)
-  uint32_t sbo;     // KT * 16
+  uint32_t lbo;     // K-direction core-matrix stride
+  uint32_t sbo;     // MN-direction core-matrix stride
 };
+
+__device__ __forceinline__ Tile transposed(const Tile& t) { return Tile{t.hi, t.lo, t.sbo, t.lbo}; }
 
 // D[tmem] (+)= A * B for one tile pair covering `ksteps` MMA steps of K = 16.
 // M = 128 rows of A (lanes of D), N columns of B. nsplit = 1 (hi*hi) or 3.
 __device__ __forceinline__ void mma_tiles(uint32_t d_tmem, const Tile& A, const Tile& B, int ksteps, uint32_t idesc,
                                           int nsplit, bool accumulate) {
   for (int j = 0; j < ksteps; ++j) {
-    const uint32_t off = j * 256u;
-    const uint64_t ah = sdesc(A.hi + off, 128, A.sbo), bh = sdesc(B.hi + off, 128, B.sbo);
+    const uint32_t oa = j * 2u * A.lbo, ob = j * 2u * B.lbo;
+    const uint64_t ah = sdesc(A.hi + oa, A.lbo, A.sbo), bh = sdesc(B.hi + ob, B.lbo, B.sbo);
     mma_bf16(d_tmem, ah, bh, idesc, (accumulate || j > 0) ? 1u : 0u);
     if (nsplit == 3) {
-      const uint64_t al = sdesc(A.lo + off, 128, A.sbo), bl = sdesc(B.lo + off, 128, B.sbo);
+      const uint64_t al = sdesc(A.lo + oa, A.lbo, A.sbo), bl = sdesc(B.lo + ob, B.lbo, B.sbo);
       mma_bf16(d_tmem, ah, bl, idesc, 1u);
       mma_bf16(d_tmem, al, bh, idesc, 1u);
     }
@@ -164,7 +172,7 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
-// K-major: 8 consecutive contraction indices k8..k8+7 of MN row m.
+// K-major (natural view, lbo = 128): 8 consecutive contraction indices k8..k8+7 of MN row m.
 __device__ __forceinline__ void put_k(const Tile& t, int m, int k8, const float (&x)[8]) {
   uint4 hi, lo;
   split8(x, hi, lo);
@@ -173,7 +181,7 @@ __device__ __forceinline__ void put_k(const Tile& t, int m, int k8, const float 
   sts128(t.lo + off, lo);
 }
 
-// MN-major: 8 consecutive MN indices m8..m8+7 of contraction row k.
+// MN-major (natural view, lbo = 128): 8 consecutive MN indices m8..m8+7 of contraction row k.
 __device__ __forceinline__ void put_mn(const Tile& t, int k, int m8, const float (&x)[8]) {
   uint4 hi, lo;
   split8(x, hi, lo);

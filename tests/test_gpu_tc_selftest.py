@@ -11,8 +11,8 @@ from gated_delta_rule_muir_b200 import _native as N
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("a_mn", [0, 1])
-@pytest.mark.parametrize("b_mn", [0, 1])
+@pytest.mark.parametrize("a_mn", [0, 1, 2, 3])
+@pytest.mark.parametrize("b_mn", [0, 1, 2, 3])
 @pytest.mark.parametrize("N_,K", [(16, 16), (64, 128), (128, 64), (256, 128), (48, 32)])
 @pytest.mark.parametrize("nsplit", [1, 3])
 def test_selftest_gemm(cuda_ok, a_mn, b_mn, N_, K, nsplit):
