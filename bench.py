@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the Muir gated delta-rule hot path on B200.
+
+One step = the chunkwise forward and backward pass (libmuir.so) over the
+training-shape workload B=1, T=32768, H=16, dk=dv=128, chunk=128, bf16 inputs,
+fp32 state, random upstream gradient. The same run measures the streaming decode
+step (24 layers x 16 heads x 128x128 fp32 state, batch 1/8/64) as GB/s of state
+traffic. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl muir|reference]
+
+N > 1 runs under torch.distributed (one process per GPU, NCCL): every rank runs
+its own replica of the workload (the operator has no cross-GPU exchange at this
+shape), the timed region is bracketed by barriers and the slowest rank's time
+is reported. --impl reference times the fp64 CPU oracle on a bounded sample of
+the same workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "chunk fwd+bwd tokens/s (H=16,d=128) & % TC peak; decode GB/s % HBM"
+WL = dict(name="train_fwdbwd_bf16_B1_T32768_H16_d128_C128", B=1, T=32768, H=16, dk=128, dv=128, chunk=128,
+          dtype="bf16", rate_lo=1e-4, rate_hi=0.7, seed=2)
+DECODE = dict(layers=24, H=16, dk=128, dv=128, batches=(1, 8, 64))
+CPU_SAMPLE_T = 1024  # oracle sample: all 16 heads, first 1024 tokens, fwd + bwd
+REF_SAMPLE_T = 256   # per-step sample of the reference arm
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"], src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work per unit (one chunk of C tokens of one (batch, head)) for each
+# kernel: (flops, bytes). Flops count each multiply-add as 2, triangles once,
+# and the math once (the 3-pass bf16 split is an implementation cost, not work).
+# Bytes are the kernel's compulsory global traffic for its interface.
+# ---------------------------------------------------------------------------
+def kernel_model(C, dk, dv, es):
+    f4 = 4
+    tri = C * C / 2
+    m = {}
+    m["decay"] = (0.0, C * dk * f4 + 4 * C * dk * f4)
+    m["gram_off"] = (4 * 2 * (tri - C * 8) * dk, 4 * C * dk * es + 2 * C * dk * f4 + 4 * C * C * f4)
+    m["gram_diag"] = (4 * 2 * C * 8.5 * dk, 4 * C * dk * es + C * dk * f4 + 4 * C * 16 * f4)
+    m["solve"] = (C ** 3 / 3.0, 2 * C * C * f4)
+    maps_fl = 2 * (tri * dk + tri * dv + tri * dv + C * dk * dk + tri * dk + 2 * tri * dv + 2 * C * dk * dv)
+    m["maps"] = (maps_fl, 4 * C * C * f4 + 6 * C * dk * es + 2 * C * dk * f4 + (dk + C) * (dk + dv) * f4)
+    m["scan"] = (2 * (dk + C) * dk * dv, (dk + C) * (dk + dv) * f4 + 2 * C * dv * es)
+    m["scan_recompute"] = (2 * (dk + C) * dk * dv, (dk + C) * (dk + dv) * f4 + dk * dv * f4 + 2 * C * dv * es)
+    m["rscan"] = (2 * (dk + C) * dk * dv, (dk + C) * dk * f4 + 2 * dk * dv * f4 + 2 * C * dv * es)
+    m["bwd_p"] = (2 * C * dk * dv, C * dk * f4 + 2 * dk * dv * f4 + 2 * C * dv * f4)
+    m["bwd_dz"] = (2 * (tri * dv + C * dk * dv + tri * dv + tri * dv + C * dk * dv + tri * dv),
+                   3 * C * C * f4 + 2 * C * dv * es + dk * dv * f4 + 2 * C * dk * es + 2 * C * dv * f4)
+    m["bwd_grads"] = (2 * (4 * C * dk * dv + 4 * tri * dv),
+                      4 * C * dv * f4 + 2 * dk * dv * f4 + 2 * C * dv * es + 4 * C * dk * f4 + 4 * C * C * f4)
+    m["bwd_gram_off"] = (4 * 2 * 2 * (tri - C * 8) * dk, 4 * C * C * f4 + 4 * C * dk * es + 2 * C * dk * f4 + 4 * C * dk * f4)
+    m["bwd_gram_diag"] = (4 * 2 * 2 * C * 8.5 * dk, 4 * C * 16 * f4 + 4 * C * dk * es + 8 * C * dk * f4)
+    m["bwd_final"] = (0.0, 14 * C * dk * f4 + 6 * C * dk * es + C * dv * f4 + 4 * C * dv * es)
+    return m
+
+
+def algorithmic_step():
+    """Work of one fwd+bwd step of the whole path (per head-token figures of the
+    survey's measurement section, at C = 128, d = 128): flops and bytes."""
+    C, d = WL["chunk"], WL["dk"]
+    ht = WL["B"] * WL["T"] * WL["H"]
+    fwd_fl = 8 * C * d + C * C / 3 + 8 * d * d
+    bwd_fl = 22 * C * d + C * C / 3 + 22 * d * d
+    return ht * (fwd_fl + bwd_fl), ht * (2560 + 5888)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def make_workload(dev):
+    import torch
+    from gated_delta_rule_muir_b200.inputs import device_inputs
+    d = device_inputs(WL["B"], WL["T"], WL["H"], WL["dk"], WL["dv"], dtype=WL["dtype"], rate_lo=WL["rate_lo"],
+                      rate_hi=WL["rate_hi"], bimodal=False, seed=WL["seed"], device=dev, with_grads=True)
+    torch.cuda.synchronize()
+    return d
+
+
+NAMES = ("q", "k", "v", "e", "w", "g", "z", "log_alpha", "r")
+
+
+class Step:
+    """Preallocated fwd+bwd step through the public binding."""
+
+    def __init__(self, d):
+        import torch
+        import gated_delta_rule_muir_b200 as muir
+        self.muir = muir
+        self.d = d
+        self.args = [d[n] for n in NAMES]
+        C = WL["chunk"]
+        self.y = torch.empty_like(d["v"])
+        self.S = torch.empty(WL["B"], WL["H"], WL["dk"], WL["dv"], device=d["q"].device)
+        nf = muir.chunk_fwd_workspace_bytes(*self.args, C)
+        nb = muir.chunk_bwd_workspace_bytes(*self.args, C)
+        self.ws = torch.empty(max(nf, nb), dtype=torch.uint8, device=d["q"].device)
+        self.grads = muir.chunk_bwd(*self.args, d["dy"], chunk=C, workspace=self.ws)
+
+    def __call__(self):
+        C = WL["chunk"]
+        self.muir.chunk_fwd(*self.args, chunk=C, y=self.y, S_T=self.S, workspace=self.ws)
+        self.muir.chunk_bwd(*self.args, self.d["dy"], chunk=C, workspace=self.ws, outputs=self.grads)
+
+
+def time_steps(fn, steps, dist_on):
+    import torch
+    import torch.distributed as dist
+    if dist_on:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if dist_on:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    return ms
+
+
+def bench_decode(dev, steps, warmup, pk):
+    """Decode GB/s: one launch over all 24 layers x batch rows (per-row readout scale)."""
+    import torch
+    import gated_delta_rule_muir_b200 as muir
+    out = {}
+    L, H, dk, dv = DECODE["layers"], DECODE["H"], DECODE["dk"], DECODE["dv"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    for nb in DECODE["batches"]:
+        n = L * nb
+        S = 0.1 * torch.randn(n, H, dk, dv, device=dev, generator=g)
+        mk = lambda d: torch.randn(n, H, d, device=dev, generator=g)
+        q = torch.nn.functional.normalize(torch.nn.functional.silu(mk(dk)), dim=-1).bfloat16()
+        k = torch.nn.functional.normalize(torch.nn.functional.silu(mk(dk)), dim=-1).bfloat16()
+        v = mk(dv).bfloat16()
+        e, gg = torch.sigmoid(mk(dk)).bfloat16(), torch.sigmoid(mk(dk)).bfloat16()
+        w, z = torch.sigmoid(mk(dv)).bfloat16(), torch.sigmoid(mk(dv)).bfloat16()
+        la = -0.01 * torch.rand(n, H, dk, device=dev, generator=g)
+        r = torch.rand(n, H, dk, device=dev, generator=g)
+        y = torch.empty(n, H, dv, device=dev, dtype=torch.bfloat16)
+        fn = lambda: muir.decode_step(S, q, k, v, e, w, gg, z, la, r, y=y)
+        for _ in range(max(warmup, 3)):
+            fn()
+        reps = max(steps, 20)
+        ms = time_steps(fn, reps, False) / reps
+        state_bytes = 2.0 * n * H * dk * dv * 4
+        io_bytes = n * H * (5 * dk * 2 + dk * 4 + dk * 4 + 3 * dv * 2 + dv * 2)
+        gbs = (state_bytes + io_bytes) / (ms * 1e-3) / 1e9
+        out[f"batch{nb}"] = {"ms_per_token": round(ms, 4), "GB_s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 3),
+                             "state_MB": round(n * H * dk * dv * 4 / 1e6, 1),
+                             "note": "state fits in L2: effective bandwidth" if n * H * dk * dv * 4 < 100e6 else "HBM"}
+        del S, q, k, v, e, gg, w, z, la, r, y
+    return out
+
+
+def e2e_pass(d, steps, warmup):
+    """Same fwd+bwd through the public API with host (pinned) inputs copied in and
+    all outputs copied back inside the timed region."""
+    import torch
+    import gated_delta_rule_muir_b200 as muir
+    dev = d["q"].device
+    host = {n: d[n].cpu().pin_memory() for n in NAMES + ("dy",)}
+    dbuf = {n: torch.empty_like(d[n]) for n in NAMES + ("dy",)}
+    st = Step({**dbuf})
+    outs_h = {"y": torch.empty_like(st.y, device="cpu").pin_memory(),
+              "S_T": torch.empty_like(st.S, device="cpu").pin_memory()}
+    for n, t in st.grads.items():
+        if t is not None:
+            outs_h[n] = torch.empty_like(t, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_h.values())
+
+    def one():
+        for n in host:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        st()
+        outs_h["y"].copy_(st.y, non_blocking=True)
+        outs_h["S_T"].copy_(st.S, non_blocking=True)
+        for n, t in st.grads.items():
+            if t is not None:
+                outs_h[n].copy_(t, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    ms = time_steps(one, steps, False) / steps
+    tok = WL["B"] * WL["T"]
+    return {"value": round(tok / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def oracle_sample(T_sample):
+    """fwd + bwd of the fp64 oracle on all heads of the first T_sample tokens."""
+    from gated_delta_rule_muir_b200.inputs import make_inputs
+    from oracle import muir_oracle as orc
+    d = make_inputs(WL["B"], T_sample, WL["H"], WL["dk"], WL["dv"], dtype=WL["dtype"], rate_lo=WL["rate_lo"],
+                    rate_hi=WL["rate_hi"], seed=WL["seed"], with_grads=True)
+    a = [d[n] for n in NAMES]
+    t0 = time.perf_counter()
+    orc.forward(*a)
+    orc.backward(*a, d["dy"])
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline():
+    sec = oracle_sample(CPU_SAMPLE_T)
+    tok = WL["B"] * CPU_SAMPLE_T
+    return {"value": round(tok / sec, 2), "unit": "tokens/s", "cores": blas_threads(), "host_cpus": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"fp64 numpy oracle fwd+bwd, all {WL['H']} heads, first {CPU_SAMPLE_T} of {WL['T']} tokens "
+                      f"({sec:.1f} s)"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(REF_SAMPLE_T)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(REF_SAMPLE_T)
+    sec = time.perf_counter() - t0
+    tok = WL["B"] * REF_SAMPLE_T * args.steps
+    v = round(tok / sec, 2)
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sec / args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WL["name"], "B": WL["B"], "T": WL["T"], "H": WL["H"], "dk": WL["dk"],
+                       "dv": WL["dv"], "chunk": WL["chunk"], "sample_tokens_per_step": REF_SAMPLE_T},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"fp64 numpy oracle fwd+bwd, all {WL['H']} heads, {REF_SAMPLE_T} tokens per step"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="muir", choices=["muir", "reference"])
+    ap.add_argument("--skip-extras", action="store_true", help="only the timed step (for profiling)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import gated_delta_rule_muir_b200 as muir
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    pk = peaks()
+    d = make_workload(dev)
+    step = Step(d)
+    with ClockSampler(local) as clk:  # started before the warm-up so its start-up stays outside the timing
+        for _ in range(args.warmup):
+            step()
+        n0 = muir.launch_count()
+        ms = time_steps(step, args.steps, dist_on) / args.steps
+        launches = (muir.launch_count() - n0)
+    tok = WL["B"] * WL["T"]
+    value = world * tok / (ms * 1e-3)
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WL["name"], "B": WL["B"], "T": WL["T"], "H": WL["H"], "dk": WL["dk"],
+                       "dv": WL["dv"], "chunk": WL["chunk"], "global_batch": world * WL["B"], "seq_len": WL["T"],
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (about 1.3 GB read per step)",
+                       "state": "fp32", "tensor_core": "tcgen05 kind::f16, 3-pass bf16 split, fp32 accumulate"},
+            "gpu_launches": int(launches), "clocks": clk.summary()}
+    # per-kernel device times (library events on the launch stream), same workload
+    with muir.KernelTimer() as kt:
+        for _ in range(args.steps):
+            step()
+    kern = {k: {"launches": c, "ms_per_step": round(t / args.steps, 4)} for k, (c, t) in kt.result.items()}
+    line["kernels"] = kern
+    C, dk, dv = WL["chunk"], WL["dk"], WL["dv"]
+    model = kernel_model(C, dk, dv, 2)
+    units = WL["B"] * WL["H"] * (WL["T"] // C)
+    top = max(kt.result.items(), key=lambda kv: kv[1][1])
+    name, (cnt, tot) = top
+    base = name.split(":")[-1]
+    fl, by = model[base]
+    per_launch_ms = tot / cnt
+    launches_per_step = cnt / args.steps
+    fl_l, by_l = fl * units / launches_per_step, by * units / launches_per_step
+    t_s = per_launch_ms * 1e-3
+    tc_bound, hbm_bound = fl_l / (pk["bf16_sus"] * 1e12), by_l / (pk["hbm"] * 1e9)
+    if tc_bound >= hbm_bound:
+        ach = fl_l / t_s / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": pk["bf16_sus"], "unit": "TFLOP/s"}
+    else:
+        ach = by_l / t_s / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s"}
+    roof["frac"] = round(ach / roof["peak"], 4)
+    roof["traffic"] = None
+    roof["kernel"] = name
+    roof["peak_source"] = pk["src"]
+    line["roofline"] = roof
+    sfl, sby = algorithmic_step()
+    t_step = ms * 1e-3
+    line["step_roofline"] = {"algorithmic_TFLOP_s": round(sfl / t_step / 1e12, 2),
+                             "frac_tc_peak": round(sfl / t_step / 1e12 / pk["bf16_sus"], 4),
+                             "algorithmic_GB_s": round(sby / t_step / 1e9, 1),
+                             "frac_hbm_peak": round(sby / t_step / 1e9 / pk["hbm"], 4),
+                             "roofline_ms": round(1e3 * max(sfl / (pk["bf16_sus"] * 1e12), sby / (pk["hbm"] * 1e9)), 3)}
+    if not args.skip_extras and rank == 0:
+        line["decode"] = bench_decode(dev, args.steps, args.warmup, pk)
+        line["e2e"] = e2e_pass(d, max(2, min(args.steps, 5)), 1)
+        if world == 1:
+            line["cpu_baseline"] = cpu_baseline()
+    if dist_on:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

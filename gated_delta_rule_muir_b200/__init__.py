@@ -14,7 +14,7 @@ import torch
 from . import _native as N
 
 __all__ = ["chunk_fwd", "chunk_bwd", "decode_step", "state_init", "device_status", "chunk_fwd_workspace_bytes",
-           "chunk_bwd_workspace_bytes", "MuirError"]
+           "chunk_bwd_workspace_bytes", "MuirError", "KernelTimer", "launch_count"]
 
 MuirError = N.MuirError
 
@@ -99,15 +99,24 @@ def chunk_fwd(q, k, v, e, w, g, z, log_alpha, r, *, chunk=128, S0=None, want_sta
 
 
 def chunk_bwd(q, k, v, e, w, g, z, log_alpha, r, dy, *, chunk=128, S0=None, dS_T=None, want_dS0=True,
-              want_dr=False, workspace=None, stream=None):
+              want_dr=False, workspace=None, outputs=None, stream=None):
     """Backward pass of chunk_fwd. Returns a dict of gradients (dq, dk, dv, de, dw, dg, dz, dlog_alpha,
-    dS0, dr), each shaped like its input."""
+    dS0, dr), each shaped like its input. `outputs` (a dict from an earlier call) is reused if given."""
     lib = N.load()
     a, (B, T, H, dk, dv, dt) = _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0)
     _need(dy, "dy", (B, T, H, dv), dt)
     if dS_T is not None:
         _need(dS_T, "dS_T", (B, H, dk, dv), torch.float32)
     dev = q.device
+    if outputs is not None:
+        out = outputs
+        gr = N.ChunkGrads(dy=_ptr(dy), dS_T=_ptr(dS_T), dq=_ptr(out["dq"]), dk=_ptr(out["dk"]), dv=_ptr(out["dv"]),
+                          de=_ptr(out["de"]), dw=_ptr(out["dw"]), dg=_ptr(out["dg"]), dz=_ptr(out["dz"]),
+                          dlog_alpha=_ptr(out["dlog_alpha"]), dS0=_ptr(out["dS0"]), dr=_ptr(out["dr"]))
+        nbytes = int(lib.muir_chunk_bwd_workspace(C.byref(a)))
+        ws = _workspace(nbytes, dev, workspace)
+        N.check(lib.muir_chunk_bwd(C.byref(a), C.byref(gr), _ptr(ws), nbytes, _stream(stream)), "muir_chunk_bwd")
+        return out
     out = {n: torch.empty(B, T, H, dk, dtype=dt, device=dev) for n in ("dq", "dk", "de", "dg")}
     out.update({n: torch.empty(B, T, H, dv, dtype=dt, device=dev) for n in ("dv", "dw")})
     out["dz"] = torch.empty(B, T, H, dv, dtype=dt, device=dev) if z is not None else None
@@ -159,6 +168,34 @@ def state_init(S, S_src=None, *, stream=None):
         _need(S_src, "S_src", (n, H, dk, dv), torch.float32)
     N.check(lib.muir_state_init(_ptr(S), _ptr(S_src), n, H, dk, dv, _stream(stream)), "muir_state_init")
     return S
+
+
+def launch_count() -> int:
+    """Number of kernels libmuir has launched in this process."""
+    return int(N.load().muir_launch_count())
+
+
+class KernelTimer:
+    """Per-kernel device time from CUDA events the library records around each of
+    its launches (on the launch stream). Use as a context manager; .result maps
+    'phase:kernel' -> (launches, total_ms)."""
+
+    def __enter__(self):
+        N.load().muir_profile_begin()
+        return self
+
+    def __exit__(self, *exc):
+        lib = N.load()
+        cap, maxn = 1 << 14, 64
+        buf = C.create_string_buffer(cap)
+        ms = (C.c_float * maxn)()
+        cnt = (C.c_int64 * maxn)()
+        n = lib.muir_profile_end(buf, cap, ms, cnt, maxn)
+        if n < 0:
+            raise MuirError(N.MUIR_ERR_CUDA, "muir_profile_end", "event timing failed")
+        names = buf.value.decode().split("\n")[:n]
+        self.result = {nm: (int(cnt[i]), float(ms[i])) for i, nm in enumerate(names)}
+        return False
 
 
 def device_status(stream=None) -> int:

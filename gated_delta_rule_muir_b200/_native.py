@@ -47,9 +47,12 @@ SIGNATURES = {
     "muir_version": (C.c_int, []),
 }
 
-# Diagnostic exports that are not part of the header's operator API.
+# Diagnostic exports declared in include/muir_profile.h.
 EXTRA_SIGNATURES = {
     "muir_selftest_gemm": (C.c_int, [vp, vp, vp, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32, vp]),
+    "muir_profile_begin": (None, []),
+    "muir_profile_end": (C.c_int, [C.c_char_p, C.c_size_t, C.POINTER(C.c_float), C.POINTER(C.c_int64), C.c_int]),
+    "muir_launch_count": (C.c_int64, []),
 }
 
 _lib = None

@@ -5,8 +5,10 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <vector>
 
 #include "../../include/muir.h"
+#include "../../include/muir_profile.h"
 #include "common.cuh"
 #include "decode.cuh"
 #include "selftest.cuh"
@@ -35,6 +37,51 @@ int cuda_check(const char* what) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- launch accounting and optional per-launch event timing ---------------
+struct ProfRec {
+  const char* phase;
+  const char* name;
+  cudaEvent_t a, b;
+};
+thread_local const char* g_phase = "";  // "fwd" / "bwd" while inside a chunk entry point
+struct Prof {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  int64_t launches = 0;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Prof g_prof;
+
+// Brackets one kernel launch on stream s (construct right before the launch).
+struct Launch {
+  cudaStream_t s;
+  const char* name;
+  cudaEvent_t b = nullptr;
+  ProfRec* rec = nullptr;
+  Launch(const char* n, cudaStream_t st) : s(st), name(n) {
+    ++g_prof.launches;
+    if (g_prof.on) {
+      ProfRec r{g_phase, n, g_prof.get(), g_prof.get()};
+      cudaEventRecord(r.a, s);
+      g_prof.recs.push_back(r);
+      b = r.b;
+    }
+  }
+  ~Launch() {
+    if (b) cudaEventRecord(b, s);
+  }
+};
 bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 
 }  // namespace
@@ -67,6 +114,7 @@ int muir_state_init(float* S, const float* S_src, int64_t n_seq, int32_t H, int3
   if (n4 == 0) return MUIR_OK;
   int64_t blocks = (n4 + 255) / 256;
   if (blocks > 148 * 32) blocks = 148 * 32;
+  Launch L_("state_init", static_cast<cudaStream_t>(stream));
   muir::state_init_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<float4*>(S), reinterpret_cast<const float4*>(S_src), n4);
   return cuda_check("state_init launch");
@@ -92,6 +140,7 @@ int muir_decode_step(const muir_decode_args* a, void* stream) {
   if (blocks > 0x7fffffff) return fail(MUIR_ERR_UNSUPPORTED, "decode: too many rows");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf = a->dtype == MUIR_BF16;
+  Launch L_("decode_step", s);
 #define MUIR_DECODE(DK)                                                                  \
   if (bf)                                                                                \
     muir::decode_step_kernel<DK, __nv_bfloat16><<<(unsigned)blocks, 128, 0, s>>>(p);     \
@@ -119,9 +168,57 @@ int muir_selftest_gemm(const float* A, const float* B, float* D, int32_t N, int3
   if (cudaFuncSetAttribute(muir::selftest_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return cuda_check("selftest attribute");
+  Launch L_("selftest_gemm", static_cast<cudaStream_t>(stream));
   muir::selftest_gemm_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(A, B, D, N, K, a_mn, b_mn, nsplit);
   return cuda_check("selftest launch");
 }
+
+void muir_profile_begin(void) {
+  for (auto& r : g_prof.recs) {
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.recs.clear();
+  g_prof.on = true;
+}
+
+int muir_profile_end(char* names_buf, size_t names_cap, float* ms, int64_t* launches, int max_entries) {
+  g_prof.on = false;
+  std::vector<std::string> names;
+  std::vector<double> tot;
+  std::vector<int64_t> cnt;
+  for (auto& r : g_prof.recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return -1;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return -1;
+    const std::string key = (r.phase[0] ? std::string(r.phase) + ":" : std::string()) + r.name;
+    size_t k = 0;
+    while (k < names.size() && names[k] != key) ++k;
+    if (k == names.size()) {
+      names.emplace_back(key);
+      tot.push_back(0.0);
+      cnt.push_back(0);
+    }
+    tot[k] += t;
+    cnt[k] += 1;
+  }
+  std::string joined;
+  const int n = (int)names.size() < max_entries ? (int)names.size() : max_entries;
+  for (int i = 0; i < n; ++i) {
+    joined += names[i];
+    joined += '\n';
+    ms[i] = (float)tot[i];
+    launches[i] = cnt[i];
+  }
+  if (names_buf && names_cap) {
+    const size_t m = joined.size() < names_cap - 1 ? joined.size() : names_cap - 1;
+    memcpy(names_buf, joined.data(), m);
+    names_buf[m] = 0;
+  }
+  return n;
+}
+
+int64_t muir_launch_count(void) { return g_prof.launches; }
 
 }  // extern "C"
 

@@ -1,0 +1,41 @@
+/*
+ * muir_profile.h — diagnostics of libmuir.so (not part of the operator API).
+ *
+ * Kernel timing: between muir_profile_begin() and muir_profile_end(), every
+ * kernel the library launches is bracketed by a pair of CUDA events recorded on
+ * the stream it is launched on. muir_profile_end() synchronises those events and
+ * returns, per kernel name, the number of launches and the summed device time.
+ * Profiling is process-wide and not thread-safe; it costs two event records per
+ * launch, so time throughput with it off.
+ *
+ * muir_launch_count(): number of kernels the library has launched since load.
+ *
+ * muir_selftest_gemm(): D[128,N] = A[128,K] * B[K,N] (fp32 row-major device
+ * buffers) through the tensor-core operand layouts the chunk kernels use;
+ * a_mode/b_mode bit 0 = MN-major operand, bit 1 = read through the transposed
+ * view of a tile written in the other arrangement; nsplit 1 or 3 bf16 passes.
+ */
+#ifndef MUIR_PROFILE_H
+#define MUIR_PROFILE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+void muir_profile_begin(void);
+/* names: '\n'-separated kernel names written into names_buf (NUL-terminated);
+ * ms[i], launches[i]: totals for the i-th name. Returns the number of names
+ * (at most max_entries), or -1 on a CUDA error. */
+int muir_profile_end(char* names_buf, size_t names_cap, float* ms, int64_t* launches, int max_entries);
+int64_t muir_launch_count(void);
+int muir_selftest_gemm(const float* A, const float* B, float* D, int32_t N, int32_t K, int32_t a_mode,
+                       int32_t b_mode, int32_t nsplit, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUIR_PROFILE_H */
