@@ -38,6 +38,7 @@ class DecodeArgs(C.Structure):
 SIGNATURES = {
     "muir_chunk_fwd_workspace": (C.c_size_t, [C.POINTER(ChunkArgs)]),
     "muir_chunk_fwd": (C.c_int, [C.POINTER(ChunkArgs), vp, vp, vp, C.c_size_t, vp]),
+    "muir_chunk_fwd_noalloc": (C.c_int, [C.POINTER(ChunkArgs), vp, vp, vp]),
     "muir_chunk_bwd_workspace": (C.c_size_t, [C.POINTER(ChunkArgs)]),
     "muir_chunk_bwd": (C.c_int, [C.POINTER(ChunkArgs), C.POINTER(ChunkGrads), vp, C.c_size_t, vp]),
     "muir_decode_step": (C.c_int, [C.POINTER(DecodeArgs), vp]),

@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -223,3 +224,60 @@ int64_t muir_launch_count(void) { return g_prof.launches; }
 }  // extern "C"
 
 #include "api_chunk.inc"
+
+// ---------------------------------------------------------------------------
+// Allocation-free chunkwise forward.
+//
+// Some callers cannot allocate device memory: a host that embeds this library
+// as a plug-in and hands it only its input and output buffers, or a
+// latency-critical loop that must not call cudaMalloc/cudaFree because those
+// calls can synchronise the whole device. For them the forward pass can run on
+// a scratch area compiled into the library: a file-scope device array of
+// kNoAllocScratchBytes, which every GPU that loads the library holds until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+}
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. In host code the
+// array's name is only a host-side stand-in, so the address must come from
+// cudaGetSymbolAddress, once per device, with that device current.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_check("chunk_fwd_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MUIR_ERR_UNSUPPORTED, "chunk_fwd_noalloc: device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess)
+      return fail(MUIR_ERR_CUDA, "chunk_fwd_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MUIR_OK;
+}
+}  // namespace
+
+extern "C" int muir_chunk_fwd_noalloc(const muir_chunk_args* a, void* y, float* S_T, void* stream) {
+  g_err.clear();
+  int rc = validate_chunk_args(a, "chunk_fwd_noalloc");
+  if (rc) return rc;
+  const size_t need = muir_chunk_fwd_workspace(a);
+  if (need > kNoAllocScratchBytes)
+    return fail(MUIR_ERR_UNSUPPORTED,
+                "chunk_fwd_noalloc: this problem needs %zu bytes of scratch but the built-in scratch holds %zu; "
+                "use muir_chunk_fwd with a caller-provided workspace",
+                need, kNoAllocScratchBytes);
+  void* ws = nullptr;
+  if ((rc = noalloc_scratch(&ws))) return rc;
+  return muir_chunk_fwd(a, y, S_T, ws, kNoAllocScratchBytes, stream);
+}

@@ -123,6 +123,27 @@ size_t muir_chunk_bwd_workspace(const muir_chunk_args* a);
 int muir_chunk_bwd(const muir_chunk_args* a, const muir_chunk_grads* gr, void* ws, size_t ws_bytes,
                    void* stream);
 
+/*
+ * Allocation-free variant of muir_chunk_fwd (the pages have no counterpart;
+ * this is a packaging choice of the library). For callers that cannot allocate
+ * device memory — a host that embeds the library as a plug-in and owns all
+ * allocations, or a latency-critical loop that must not call cudaMalloc or
+ * cudaFree because they can synchronise the device — the forward pass runs on
+ * a 32 MiB scratch area compiled into the library (every GPU that loads the
+ * library holds it until the process exits). The caller still passes inputs
+ * and outputs exactly as for muir_chunk_fwd; this call allocates nothing.
+ *   - Problems whose muir_chunk_fwd_workspace() exceeds 32 MiB are rejected
+ *     with MUIR_ERR_UNSUPPORTED before any GPU work.
+ *   - The first call on a device looks up the scratch address with
+ *     cudaGetSymbolAddress (once per device, with that device current); make
+ *     that first call before any stream capture on the device.
+ *   - All calls on a device share the one scratch area and it keeps the last
+ *     call's contents; the kernels write every scratch byte they read within
+ *     the same call, so nothing needs clearing. Calls that overlap on the GPU
+ *     (e.g. on two streams at once) race on the scratch: serialise them.
+ */
+int muir_chunk_fwd_noalloc(const muir_chunk_args* a, void* y, float* S_T, void* stream);
+
 /* One recurrent step for n_seq independent sequences (streaming decode,
  * openai-hub article, section on 10M-token streaming). */
 typedef struct muir_decode_args {
