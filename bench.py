@@ -153,6 +153,8 @@ NAMES = ("q", "k", "v", "e", "w", "g", "z", "log_alpha", "r")
 class Step:
     """Preallocated fwd+bwd step through the public binding."""
 
+    fwd_only = False
+
     def __init__(self, d):
         import torch
         import gated_delta_rule_muir_b200 as muir
@@ -165,12 +167,14 @@ class Step:
         nf = muir.chunk_fwd_workspace_bytes(*self.args, C)
         nb = muir.chunk_bwd_workspace_bytes(*self.args, C)
         self.ws = torch.empty(max(nf, nb), dtype=torch.uint8, device=d["q"].device)
-        self.grads = muir.chunk_bwd(*self.args, d["dy"], chunk=C, workspace=self.ws)
+        if not self.fwd_only:
+            self.grads = muir.chunk_bwd(*self.args, d["dy"], chunk=C, workspace=self.ws)
 
     def __call__(self):
         C = WL["chunk"]
         self.muir.chunk_fwd(*self.args, chunk=C, y=self.y, S_T=self.S, workspace=self.ws)
-        self.muir.chunk_bwd(*self.args, self.d["dy"], chunk=C, workspace=self.ws, outputs=self.grads)
+        if not self.fwd_only:
+            self.muir.chunk_bwd(*self.args, self.d["dy"], chunk=C, workspace=self.ws, outputs=self.grads)
 
 
 def time_steps(fn, steps, dist_on):
@@ -323,7 +327,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="muir", choices=["muir", "reference"])
     ap.add_argument("--skip-extras", action="store_true", help="only the timed step (for profiling)")
+    ap.add_argument("--T", type=int, default=None, help="override the sequence length (profiling runs)")
+    ap.add_argument("--fwd-only", action="store_true", help="time the forward pass only (profiling runs)")
     args = ap.parse_args()
+    if args.T:
+        WL["T"] = args.T
+        WL["name"] = f"train_fwdbwd_bf16_B1_T{args.T}_H16_d128_C128"
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -343,6 +352,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pk = peaks()
+    Step.fwd_only = args.fwd_only
     d = make_workload(dev)
     step = Step(d)
     with ClockSampler(local) as clk:  # started before the warm-up so its start-up stays outside the timing

@@ -60,10 +60,12 @@ struct ChunkParams {
   float* dec;  // [nsubtot][4][Cs][dk]: pre, suf, Gam, Gsuf
   float* gr;   // [nsubtot][4][Cs][Cs]: M^kk, M^ka, N^qk, N^qa
   float* tt;   // [nsubtot][Cs][Cs]
-  float* ma;   // [nunits][dk + C][dk]: Phi ; Q'
-  float* mb;   // [nunits][dk + C][dv]: Psi ; Oloc
-  float* ma2;  // composition scratch for chunk 256 (same layout as ma at C = 2*Cs)
-  float* mb2;
+  uint8_t* ma;  // [nunits] images of Phi and Q' (see MapGeom)
+  float* psi;   // [nunits][dv/32][dk][32]: Psi in 32-column slabs
+  float* ol;    // [nunits][Cs][dv]: Oloc
+  uint8_t* ma2; // the same three for chunk-256 maps composed from two 128-token units
+  float* psi2;
+  float* ol2;   // [nunits/2][256][dv]
   // outputs
   void* y;
   float* S_T;
@@ -109,6 +111,42 @@ __device__ __forceinline__ void zero_smem(uint32_t base, uint32_t bytes) {
 
 __device__ __forceinline__ uint32_t tmem_cols_for(int n) {
   return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : n <= 256 ? 256u : 512u;
+}
+
+// Workspace image of a chunk map with L tokens: tile 0 holds Phi (dk x dk),
+// tiles 1.. hold Q' (128 token rows each). Every tile is a bf16 hi block then a
+// lo block of 128 rows x dk in the K-major canonical layout (sbo = dk*16),
+// exactly as the MMA reads it, so consumers fetch tiles with bulk copies.
+struct MapGeom {
+  int ntile;      // 1 + ceil(L / 128)
+  uint32_t half;  // bytes of one hi (or lo) block
+  uint32_t tile;  // hi + lo
+  uint32_t unit;  // all tiles of one map
+};
+__host__ __device__ inline MapGeom map_geom(int dk, int L) {
+  MapGeom g;
+  g.ntile = 1 + (L + 127) / 128;
+  g.half = 128u * (uint32_t)dk * 2u;
+  g.tile = 2u * g.half;
+  g.unit = (uint32_t)g.ntile * g.tile;
+  return g;
+}
+
+// Row i of Phi, 8 consecutive columns c8.., as bf16 hi/lo.
+__device__ __forceinline__ void map_put_phi(uint8_t* img, const MapGeom& g, int dk, int i, int c8, const float (&x)[8]) {
+  gput_k(img, g.half, (uint32_t)dk * 16u, i, c8, x);
+}
+// Row t (token) of Q'.
+__device__ __forceinline__ void map_put_q(uint8_t* img, const MapGeom& g, int dk, int t, int c8, const float (&x)[8]) {
+  gput_k(img + (uint32_t)(1 + (t >> 7)) * g.tile, g.half, (uint32_t)dk * 16u, t & 127, c8, x);
+}
+
+// Bulk copy of `bytes` (multiple of 16) in pieces of at most 32 KB.
+__device__ __forceinline__ void bulk_g2s_big(uint32_t dst, const uint8_t* src, uint32_t bytes, uint64_t* bar) {
+  for (uint32_t o = 0; o < bytes; o += 32768u) {
+    const uint32_t n = bytes - o < 32768u ? bytes - o : 32768u;
+    bulk_g2s(dst + o, src + o, n, bar);
+  }
 }
 
 // CTA prologue shared by the tensor-core kernels: TMEM allocation + mbarrier.
@@ -237,11 +275,13 @@ __global__ void __launch_bounds__(128, 1) gram_off_kernel(ChunkParams p) {
   MmaSync drv{&bar, 0u, true};
   const uint32_t id = idesc_bf16(128, SB, 0, 0);
   for (int I = nb - 2; I >= 0 && drv.ok; --I) {
+    #pragma unroll 4
     for (int x = tid; x < nb * DK; x += 128) {
       const int J = x / DK, i = x % DK;
       if (J == I + 1) midtab[x] = 1.f;
       else if (J > I + 1) midtab[x] *= pre[(SB * (I + 1) + SB - 1) * DK + i];
     }
+    #pragma unroll 4
     for (int x = tid; x < SB * (DK / 8); x += 128) {
       const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       const int t = SB * I + rr;
@@ -257,6 +297,7 @@ __global__ void __launch_bounds__(128, 1) gram_off_kernel(ChunkParams p) {
     __syncthreads();
     const int t0 = SB * (I + 1);
     for (int pass = 0; pass < 2 && drv.ok; ++pass) {
+      #pragma unroll 4
       for (int x = tid; x < (Cs - t0) * (DK / 8); x += 128) {
         const int t = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
         float xv[8], pr[8], md[8];
@@ -314,6 +355,7 @@ __global__ void __launch_bounds__(128) gram_diag_kernel(ChunkParams p) {
   const int sid = blockIdx.x / nb, J = blockIdx.x % nb;
   const SubIdx s = sub_of(p, sid, p.nsub, Cs);
   const Rows<T> rows{p, s.b, s.h};
+  #pragma unroll 4
   for (int x = threadIdx.x; x < SB * (DK / 8); x += 128) {
     const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
     const int64_t tok = s.tok0 + SB * J + rr;
@@ -425,6 +467,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
   const int t = tid;
   for (int h = SB; h < Cs && drv.ok; h *= 2) {
     // A = off-diagonal blocks (2m+1, 2m) of M (zeros elsewhere), K-major; B = Tcur, MN-major.
+    #pragma unroll 4
     for (int x = tid; x < 128 * (Cs / 8); x += 128) {
       const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
       float v[8];
@@ -436,6 +479,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
       }
       put_k(TA, r, c8, v);
     }
+    #pragma unroll 4
     for (int x = tid; x < Cs * (Cs / 8); x += 128) {
       const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
       float v[8];
@@ -468,6 +512,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
       }
     }
     // A = Tcur, K-major.
+    #pragma unroll 4
     for (int x = tid; x < Cs * (Cs / 8); x += 128) {
       const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
       float v[8];
@@ -538,6 +583,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   constexpr uint32_t cW = 0, cZ = 128, cUt = 256, cPhi = 0, cPsi = 128, cOl = 256, cQ = 384;
 
   auto stage_k_matrix = [&](const Tile& dst, const float* src, float sign) {  // rows t, K = s (Cs x Cs)
+    #pragma unroll 4
     for (int x = tid; x < Cs * (Cs / 8); x += 128) {
       const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
       float v[8];
@@ -563,6 +609,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   };
   // (X * Gsuf)^T as an MN-major A operand (M = channel, K = token), scaled by sign.
   auto stage_suffixed = [&](bool erase, float sign) {
+    #pragma unroll 4
     for (int x = tid; x < Cs * (DK / 8); x += 128) {
       const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float xx[8], gs[8];
@@ -578,6 +625,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   const uint32_t idKt = idesc_bf16(128, DK, 1, 1), idVt = idesc_bf16(128, DV, 1, 1);
   // ---- phase 1: W = T (K*Gam), Z = M^kk U, Ut = T Z
   stage_k_matrix(A, Tm, 1.f);
+  #pragma unroll 4
   for (int x = tid; x < Cs * (DK / 8); x += 128) {  // B1 = K*Gam (K = token, N = channel)
     const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
     float kk[8], gm[8];
@@ -587,6 +635,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
     for (int j = 0; j < 8; ++j) kk[j] *= gm[j];
     put_mn(B1, r, c8, kk);
   }
+  #pragma unroll 4
   for (int x = tid; x < Cs * (DV / 8); x += 128) {  // B2 = U
     const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
     float uu[8];
@@ -634,9 +683,11 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B2, Cs / 16, idVt, NS, false); });
   stage_suffixed(true, -1.f);
   drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B1, Cs / 16, idVt, NS, true); });
-  // ---- epilogue: [Phi; Q'] -> ma, [Psi; Oloc] -> mb (fp32, row-major)
-  float* ma = p.ma + (int64_t)blockIdx.x * (DK + Cs) * DK;
-  float* mb = p.mb + (int64_t)blockIdx.x * (DK + Cs) * DV;
+  // ---- epilogue: Phi, Q' -> map image (bf16 hi/lo tiles); Psi -> 32-column slabs; Oloc -> row-major
+  const MapGeom mg = map_geom(DK, Cs);
+  uint8_t* ma = p.ma + (int64_t)blockIdx.x * mg.unit;
+  float* psi = p.psi + (int64_t)blockIdx.x * DK * DV;
+  float* ol = p.ol + (int64_t)blockIdx.x * Cs * DV;
   const float* gC = gam + (Cs - 1) * DK;
   for (int c = 0; c < DK; c += 16) {
     float v[16];
@@ -645,18 +696,20 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
 #pragma unroll
       for (int j = 0; j < 16; ++j)
         if (c + j == t) v[j] += gC[t];
+      float a8[8], b8[8];
 #pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(ma + (int64_t)t * DK + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
+      map_put_phi(ma, mg, DK, t, c, a8);
+      map_put_phi(ma, mg, DK, t, c + 8, b8);
     }
   }
   for (int c = 0; c < DV; c += 16) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cPsi + c, v);
     if (t < DK && drv.ok) {
+      float* o = psi + ((int64_t)(c >> 5) * DK + t) * 32 + (c & 31);
 #pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(mb + (int64_t)t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
   }
   for (int c = 0; c < DK; c += 16) {
@@ -671,10 +724,11 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[h8 + j] += qq[j] * gm[j];
       }
+      float a8[8], b8[8];
 #pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(ma + (int64_t)(DK + t) * DK + c + j) =
-            make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
+      map_put_q(ma, mg, DK, t, c, a8);
+      map_put_q(ma, mg, DK, t, c + 8, b8);
     }
   }
   for (int c = 0; c < DV; c += 16) {
@@ -683,8 +737,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
     if (t < Cs && drv.ok) {
 #pragma unroll
       for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(mb + (int64_t)(DK + t) * DV + c + j) =
-            make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        *reinterpret_cast<float4*>(ol + (int64_t)t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
   }
   cta.finish();
@@ -695,143 +748,165 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
 // its two 128-token halves (h0 then h1), which is the top-level merge of the
 // recursive block solve applied to the chunk map:
 //   Phi = Phi1 Phi0,  Psi = Phi1 Psi0 + Psi1
-//   rows of the first half:  Q'0, Oloc0 (unchanged)
-//   rows of the second half: Q'1 Phi0, Q'1 Psi0 + Oloc1
-// One CTA per chunk: A = [Phi1; Q'1] (two 128-row K-major tiles, K = dk),
-// B = Phi0 then Psi0 (MN-major, K = dk).
+//   first-half outputs: Q'0, Oloc0 (unchanged)
+//   second-half outputs: Q'1 Phi0, Q'1 Psi0 + Oloc1
+// One CTA per chunk. A = [Phi1; Q'1] (tiles 0, 1 of the second half's image,
+// bulk copy, K-major over key channels); B = Phi0 (tile 0 of the first half's
+// image read through the transposed view), then Psi0 staged by the threads.
 // ---------------------------------------------------------------------------
 template <int DK, int DV, int NS>
 __global__ void __launch_bounds__(128, 1) compose_kernel(ChunkParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;  // 128
   const int tid = threadIdx.x, warp = tid >> 5;
-  constexpr uint32_t TBY = 128u * DK * 2u;
+  const MapGeom g1 = map_geom(DK, Cs), g2 = map_geom(DK, 2 * Cs);
   const uint32_t base = smem_u32(sm);
-  const Tile A0{base, base + TBY, 128u, DK * 16u};
-  const Tile A1{base + 2 * TBY, base + 3 * TBY, 128u, DK * 16u};
-  const Tile Bt{base + 4 * TBY, base + 4 * TBY + 128u * DK * 2u, 128u, DK * 16u};
-  zero_smem(base, 4 * TBY + 2u * 128u * DK * 2u);
+  const uint32_t bbase = base + 2 * g1.tile;
+  if (tid == 0) mbar_init(&bar_cp, 1);
   TcCta cta;
   cta.init(&tslot, &bar, 512);
   const int64_t u0 = 2 * (int64_t)blockIdx.x, u1 = u0 + 1;
-  const int rows1 = DK + Cs;
-  const float* ma0 = p.ma + u0 * rows1 * DK;
-  const float* ma1 = p.ma + u1 * rows1 * DK;
-  const float* mb0 = p.mb + u0 * rows1 * DV;
-  const float* mb1 = p.mb + u1 * rows1 * DV;
-  for (int x = tid; x < rows1 * (DK / 8); x += 128) {
-    const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-    float v[8];
-    ld8f(ma1 + (int64_t)r * DK + c8, v);
-    put_k(r < 128 ? A0 : A1, r & 127, c8, v);
+  const uint8_t* img0 = p.ma + u0 * g1.unit;
+  const uint8_t* img1 = p.ma + u1 * g1.unit;
+  if (tid == 0) {
+    mbar_expect_tx(&bar_cp, 3 * g1.tile);
+    bulk_g2s_big(base, img1, 2 * g1.tile, &bar_cp);
+    bulk_g2s_big(bbase, img0, g1.tile, &bar_cp);
   }
   MmaSync drv{&bar, 0u, true};
+  drv.ok = __syncthreads_and(mbar_wait(&bar_cp, 0) ? 1 : 0) != 0;
   const uint32_t lane = tmem_lane_base(warp);
-  for (int x = tid; x < DK * (DK / 8); x += 128) {  // Phi0 (K = row, N = col)
-    const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-    float v[8];
-    ld8f(ma0 + (int64_t)r * DK + c8, v);
-    put_mn(Bt, r, c8, v);
-  }
-  const int ntile = (rows1 + 127) / 128;
-  drv.run([&] {
-    mma_tiles(cta.tmem + 0, A0, Bt, DK / 16, idesc_bf16(128, DK, 0, 1), NS, false);
-    if (ntile > 1) mma_tiles(cta.tmem + 128, A1, Bt, DK / 16, idesc_bf16(128, DK, 0, 1), NS, false);
-  });
-  for (int x = tid; x < DK * (DV / 8); x += 128) {  // Psi0
+  auto At = [&](int j) { return Tile{base + j * g1.tile, base + j * g1.tile + g1.half, 128u, DK * 16u}; };
+  const Tile Bphi{bbase, bbase + g1.half, DK * 16u, 128u};  // Phi0: K = row, N = column
+  if (drv.ok)
+    drv.run([&] {
+      for (int j = 0; j < 2; ++j)
+        mma_tiles(cta.tmem + j * 128, At(j), Bphi, DK / 16, idesc_bf16(128, DK, 0, 1), NS, false);
+    });
+  const Tile Bpsi{bbase, bbase + DK * DV * 2u, 128u, DK * 16u};  // Psi0: K = row, N = column
+  const float* psi0 = p.psi + u0 * DK * DV;
+#pragma unroll 4
+  for (int x = tid; x < DK * (DV / 8); x += 128) {
     const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
     float v[8];
-    ld8f(mb0 + (int64_t)r * DV + c8, v);
-    put_mn(Bt, r, c8, v);
+    ld8f(psi0 + ((int64_t)(c8 >> 5) * DK + r) * 32 + (c8 & 31), v);
+    put_mn(Bpsi, r, c8, v);
   }
-  drv.run([&] {
-    mma_tiles(cta.tmem + 256, A0, Bt, DK / 16, idesc_bf16(128, DV, 0, 1), NS, false);
-    if (ntile > 1) mma_tiles(cta.tmem + 384, A1, Bt, DK / 16, idesc_bf16(128, DV, 0, 1), NS, false);
-  });
-  const int rows2 = DK + 2 * Cs;
-  float* ma = p.ma2 + (int64_t)blockIdx.x * rows2 * DK;
-  float* mb = p.mb2 + (int64_t)blockIdx.x * rows2 * DV;
-  // rows of the composite: [0,DK) state, [DK, DK+Cs) first half, [DK+Cs, DK+2Cs) second half
-  for (int tile = 0; tile < ntile; ++tile) {
-    const int r1 = tile * 128 + tid;  // row of [Phi1; Q'1]
-    const int r2 = r1 < DK ? r1 : r1 + Cs;
+  if (drv.ok)
+    drv.run([&] {
+      for (int j = 0; j < 2; ++j)
+        mma_tiles(cta.tmem + 256 + j * 128, At(j), Bpsi, DK / 16, idesc_bf16(128, DV, 0, 1), NS, false);
+    });
+  uint8_t* ma = p.ma2 + (int64_t)blockIdx.x * g2.unit;
+  float* psi = p.psi2 + (int64_t)blockIdx.x * DK * DV;
+  float* ol = p.ol2 + (int64_t)blockIdx.x * 2 * Cs * DV;
+  const float* psi1 = p.psi + u1 * DK * DV;
+  const float* ol1 = p.ol + u1 * Cs * DV;
+  // tile 0 rows: Phi1 Phi0 (-> Phi), Phi1 Psi0 + Psi1 (-> Psi); tile 1 rows: Q'1 Phi0, Q'1 Psi0 + Oloc1
+  for (int j = 0; j < 2; ++j) {
+    const bool on = (j == 0 ? tid < DK : true) && drv.ok;
     for (int c = 0; c < DK; c += 16) {
       float v[16];
-      tmem_ld16(cta.tmem + lane + tile * 128 + c, v);
-      if (r1 < rows1 && drv.ok)
+      tmem_ld16(cta.tmem + lane + j * 128 + c, v);
+      if (on) {
+        float a8[8], b8[8];
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(ma + (int64_t)r2 * DK + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int e = 0; e < 8; ++e) { a8[e] = v[e]; b8[e] = v[8 + e]; }
+        if (j == 0) { map_put_phi(ma, g2, DK, tid, c, a8); map_put_phi(ma, g2, DK, tid, c + 8, b8); }
+        else { map_put_q(ma, g2, DK, Cs + tid, c, a8); map_put_q(ma, g2, DK, Cs + tid, c + 8, b8); }
+      }
     }
     for (int c = 0; c < DV; c += 16) {
       float v[16];
-      tmem_ld16(cta.tmem + lane + 256 + tile * 128 + c, v);
-      if (r1 < rows1 && drv.ok) {
+      tmem_ld16(cta.tmem + lane + 256 + j * 128 + c, v);
+      if (on) {
+        const float* a = j == 0 ? psi1 + ((int64_t)(c >> 5) * DK + tid) * 32 + (c & 31) : ol1 + (int64_t)tid * DV + c;
+        float* o = j == 0 ? psi + ((int64_t)(c >> 5) * DK + tid) * 32 + (c & 31) : ol + (int64_t)(Cs + tid) * DV + c;
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-          const float4 a = *reinterpret_cast<const float4*>(mb1 + (int64_t)r1 * DV + c + j);
-          *reinterpret_cast<float4*>(mb + (int64_t)r2 * DV + c + j) =
-              make_float4(v[j] + a.x, v[j + 1] + a.y, v[j + 2] + a.z, v[j + 3] + a.w);
-        }
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4*>(o + e) = make_float4(v[e] + a[e], v[e + 1] + a[e + 1], v[e + 2] + a[e + 2],
+                                                          v[e + 3] + a[e + 3]);
       }
     }
   }
-  // first-half rows copied: [Q'0; Oloc0]
-  for (int x = tid; x < Cs * DK / 4; x += 128)
-    reinterpret_cast<float4*>(ma + (int64_t)DK * DK)[x] = reinterpret_cast<const float4*>(ma0 + (int64_t)DK * DK)[x];
-  for (int x = tid; x < Cs * DV / 4; x += 128)
-    reinterpret_cast<float4*>(mb + (int64_t)DK * DV)[x] = reinterpret_cast<const float4*>(mb0 + (int64_t)DK * DV)[x];
+  // first half: Q'0 (tile 1 of h0 -> tile 1 of the chunk) and Oloc0 unchanged
+  if (drv.ok) {
+    const uint4* src = reinterpret_cast<const uint4*>(img0 + g1.tile);
+    uint4* dst = reinterpret_cast<uint4*>(ma + g2.tile);
+#pragma unroll 4
+    for (int x = tid; x < (int)(g1.tile / 16); x += 128) dst[x] = src[x];
+    const float4* s4 = reinterpret_cast<const float4*>(p.ol + u0 * Cs * DV);
+    float4* d4 = reinterpret_cast<float4*>(ol);
+#pragma unroll 4
+    for (int x = tid; x < Cs * DV / 4; x += 128) d4[x] = s4[x];
+  }
   cta.finish();
 }
 
 // ---------------------------------------------------------------------------
-// scan_kernel: one CTA per (batch, head, 32-column slab of the state); walks the
-// chunks in order. The state slab S (dk x 32 fp32) stays on chip: in registers
-// (thread = key row) and, split into bf16 hi/lo, as the MMA's B operand.
-//   D = [Phi; Q'] S   (M = dk + C rows in 128-row tiles, N = 32, K = dk)
-//   S <- D[0:dk] + Psi,   y = z * (D[dk:] + Oloc)
+// scan_kernel: the only sequential step. One CTA per (batch, head, 32-column
+// slab of the state) walks the chunks in order:
+//   S_chunks[n] = S;   S <- Phi_n S + Psi_n
+// The state slab stays on chip (registers, and bf16 hi/lo as the MMA's B
+// operand). Phi_n (one tile) and the Psi_n slab arrive by bulk copies into two
+// alternating buffers, issued two chunks ahead. The outputs, which need only
+// the chunk-start states, are formed afterwards by out_kernel in parallel.
 // ---------------------------------------------------------------------------
-template <int DK, typename T, int NS>
-__global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const float* ma, const float* mb, int units,
+template <int DK, int NS>
+__global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8_t* ma, const float* psi, int units,
                                                       int ulen) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_c[2];
   __shared__ uint32_t tslot;
-  constexpr int NW = 32;  // slab width
+  constexpr int NW = 32;
   const int dv = p.dv, slabs = dv / NW;
   const int slab = blockIdx.x % slabs;
   const int bh = blockIdx.x / slabs;
   const int h = bh % p.H, b = bh / p.H;
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int rows_total = DK + ulen;
-  const int ntile = (rows_total + 127) / 128;
-  constexpr uint32_t ATB = 128u * DK * 2u;
+  const MapGeom g = map_geom(DK, ulen);
+  const uint32_t PS = DK * NW * 4u;  // Psi slab bytes
   const uint32_t base = smem_u32(sm);
-  const Tile Sb{base, base + NW * DK * 2u, 128u, DK * 16u};  // B: K = key row, N = slab column (MN-major)
-  const uint32_t abase = base + 2u * NW * DK * 2u;
-  zero_smem(base, 2u * NW * DK * 2u + 2u * ATB * ntile);
+  const uint32_t psi_off = 2 * g.tile;
+  const uint32_t s_off = psi_off + 2 * PS;
+  const Tile Sb{base + s_off, base + s_off + NW * DK * 2u, 128u, DK * 16u};  // B: K = key row, N = column
+  if (tid == 0) {
+    mbar_init(&bar_c[0], 1);
+    mbar_init(&bar_c[1], 1);
+  }
   TcCta cta;
-  cta.init(&tslot, &bar, tmem_cols_for(NW * ntile));
+  cta.init(&tslot, &bar, 32);
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
-  // state slab in registers: thread = key row i < DK
+  const float* psi_s = reinterpret_cast<const float*>(static_cast<const uint8_t*>(sm) + psi_off);
+  auto uid_of = [&](int n) { return ((int64_t)b * p.H + h) * units + n; };
+  auto issue = [&](int n, int buf) {
+    if (tid == 0) {
+      mbar_expect_tx(&bar_c[buf], g.tile + PS);
+      bulk_g2s_big(base + buf * g.tile, ma + uid_of(n) * g.unit, g.tile, &bar_c[buf]);
+      bulk_g2s_big(base + psi_off + buf * PS,
+                   reinterpret_cast<const uint8_t*>(psi + (uid_of(n) * slabs + slab) * DK * NW), PS, &bar_c[buf]);
+    }
+  };
   float st[NW];
   {
     const float* s0 = p.S0 ? p.S0 + (((int64_t)b * p.H + h) * DK) * dv + slab * NW : nullptr;
 #pragma unroll
     for (int j = 0; j < NW; ++j) st[j] = (s0 && tid < DK) ? s0[(int64_t)tid * dv + j] : 0.f;
   }
+  issue(0, 0);
+  if (units > 1) issue(1, 1);
   const uint32_t id = idesc_bf16(128, NW, 0, 1);
   for (int n = 0; n < units && drv.ok; ++n) {
-    const int64_t uid = ((int64_t)b * p.H + h) * units + n;
-    if (p.S_chunks && tid < DK) {
-      float* o = p.S_chunks + ((uid * DK) + tid) * dv + slab * NW;
-#pragma unroll
-      for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(st[j], st[j + 1], st[j + 2], st[j + 3]);
-    }
+    const int buf = n & 1;
     if (tid < DK) {
+      if (p.S_chunks) {
+        float* o = p.S_chunks + ((uid_of(n) * DK) + tid) * dv + slab * NW;
+#pragma unroll
+        for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(st[j], st[j + 1], st[j + 2], st[j + 3]);
+      }
 #pragma unroll
       for (int j = 0; j < NW; j += 8) {
         float v[8];
@@ -840,87 +915,105 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const float
         put_mn(Sb, tid, j, v);
       }
     }
-    const float* A = ma + uid * rows_total * DK;
-    for (int x = tid; x < ntile * 128 * (DK / 8); x += 128) {
-      const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-      float v[8];
-      if (r < rows_total) ld8f(A + (int64_t)r * DK + c8, v);
-      else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = 0.f;
-      }
-      const int tile = r >> 7;
-      const Tile At{abase + tile * 2u * ATB, abase + tile * 2u * ATB + ATB, 128u, DK * 16u};
-      put_k(At, r & 127, c8, v);
-    }
-    drv.run([&] {
-      for (int tile = 0; tile < ntile; ++tile) {
-        const Tile At{abase + tile * 2u * ATB, abase + tile * 2u * ATB + ATB, 128u, DK * 16u};
-        mma_tiles(cta.tmem + tile * NW, At, Sb, DK / 16, id, NS, false);
-      }
-    });
+    const bool c_ok = mbar_wait(&bar_c[buf], (uint32_t)(n >> 1) & 1u);
+    if (!__syncthreads_and(c_ok ? 1 : 0)) { drv.ok = false; break; }
+    const Tile Phi{base + buf * g.tile, base + buf * g.tile + g.half, 128u, DK * 16u};
+    drv.run([&] { mma_tiles(cta.tmem, Phi, Sb, DK / 16, id, NS, false); });
     if (!drv.ok) break;
-    const float* Bm = mb + uid * rows_total * dv + slab * NW;
-    for (int tile = 0; tile < ntile; ++tile) {
-      float v[NW];
-      tmem_ld16(cta.tmem + lane + tile * NW, *reinterpret_cast<float(*)[16]>(&v[0]));
-      tmem_ld16(cta.tmem + lane + tile * NW + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
-      const int r = tile * 128 + tid;
-      if (r < DK) {
+    float v[NW];
+    tmem_ld16(cta.tmem + lane, *reinterpret_cast<float(*)[16]>(&v[0]));
+    tmem_ld16(cta.tmem + lane + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+    if (tid < DK) {
+      const float* add = psi_s + buf * (PS / 4) + tid * NW;
 #pragma unroll
-        for (int j = 0; j < NW; j += 4) {
-          const float4 add = *reinterpret_cast<const float4*>(Bm + (int64_t)r * dv + j);
-          st[j] = v[j] + add.x; st[j + 1] = v[j + 1] + add.y; st[j + 2] = v[j + 2] + add.z; st[j + 3] = v[j + 3] + add.w;
-        }
-      } else if (r < rows_total) {
-        const int tt = r - DK;
-        const int64_t tok = (int64_t)n * ulen + tt;
-        float o[NW];
-#pragma unroll
-        for (int j = 0; j < NW; j += 4) {
-          const float4 add = *reinterpret_cast<const float4*>(Bm + (int64_t)r * dv + j);
-          o[j] = v[j] + add.x; o[j + 1] = v[j + 1] + add.y; o[j + 2] = v[j + 2] + add.z; o[j + 3] = v[j + 3] + add.w;
-        }
-        const int64_t yo = toff(p, b, tok, h, dv) + slab * NW;
-        if (!p.y) {  // backward recompute: only dz = O * dy is wanted
-          if (p.dz && p.z) {
-#pragma unroll
-            for (int j = 0; j < NW; j += 8) {
-              float dd[8], w8[8];
-              Elt<T>::ld8(static_cast<const T*>(p.dy) + yo + j, dd);
-#pragma unroll
-              for (int e2 = 0; e2 < 8; ++e2) w8[e2] = o[j + e2] * dd[e2];
-              Elt<T>::st8(static_cast<T*>(p.dz) + yo + j, w8);
-            }
-          }
-          continue;
-        }
-        if (p.z) {
-#pragma unroll
-          for (int j = 0; j < NW; j += 8) {
-            float zz[8];
-            Elt<T>::ld8(static_cast<const T*>(p.z) + yo + j, zz);
-#pragma unroll
-            for (int e2 = 0; e2 < 8; ++e2) o[j + e2] *= zz[e2];
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < NW; j += 8) {
-          float w8[8];
-#pragma unroll
-          for (int e2 = 0; e2 < 8; ++e2) w8[e2] = o[j + e2];
-          Elt<T>::st8(static_cast<T*>(p.y) + yo + j, w8);
-        }
+      for (int j = 0; j < NW; j += 4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(add + j);
+        st[j] = v[j] + a4.x; st[j + 1] = v[j + 1] + a4.y; st[j + 2] = v[j + 2] + a4.z; st[j + 3] = v[j + 3] + a4.w;
       }
     }
-    // registers of `st` now hold the next chunk's start state; the next loop
-    // iteration restages them (the MMA above has completed).
-    __syncthreads();
+    __syncthreads();  // buffer `buf` (Phi, Psi) is free again
+    if (n + 2 < units) issue(n + 2, buf);
   }
   if (p.S_T && tid < DK && drv.ok) {
     float* o = p.S_T + (((int64_t)b * p.H + h) * DK + tid) * dv + slab * NW;
 #pragma unroll
     for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(st[j], st[j + 1], st[j + 2], st[j + 3]);
+  }
+  cta.finish();
+}
+
+// ---------------------------------------------------------------------------
+// out_kernel: outputs of one chunk from its start state, all chunks in
+// parallel:  y = z * (Q' S0 + Oloc).
+// A = Q' tiles of the map image (bulk copy, K-major over key channels),
+// B = S0 (MN-major: K = key channel, N = value column), staged by the threads.
+// ---------------------------------------------------------------------------
+template <int DK, int DV, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) out_kernel(ChunkParams p, const uint8_t* ma, const float* ol, int units,
+                                                     int ulen) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar, bar_cp;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t uid = blockIdx.x;
+  const int n = (int)(uid % units);
+  const int bh = (int)(uid / units);
+  const int h = bh % p.H, b = bh / p.H;
+  const MapGeom g = map_geom(DK, ulen);
+  const int nq = g.ntile - 1;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t s_off = (uint32_t)nq * g.tile;
+  const Tile Sb{base + s_off, base + s_off + DK * DV * 2u, 128u, DK * 16u};
+  if (tid == 0) mbar_init(&bar_cp, 1);
+  TcCta cta;
+  cta.init(&tslot, &bar, tmem_cols_for(nq * DV));
+  if (tid == 0) {
+    mbar_expect_tx(&bar_cp, nq * g.tile);
+    bulk_g2s_big(base, ma + uid * g.unit + g.tile, nq * g.tile, &bar_cp);
+  }
+  const float* S0 = p.S_chunks + uid * DK * DV;
+#pragma unroll 4
+  for (int x = tid; x < DK * (DV / 8); x += 128) {
+    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+    float v[8];
+    ld8f(S0 + (int64_t)r * DV + c8, v);
+    put_mn(Sb, r, c8, v);
+  }
+  MmaSync drv{&bar, 0u, true};
+  drv.ok = __syncthreads_and(mbar_wait(&bar_cp, 0) ? 1 : 0) != 0;
+  const uint32_t id = idesc_bf16(128, DV, 0, 1);
+  if (drv.ok)
+    drv.run([&] {
+      for (int j = 0; j < nq; ++j) {
+        const Tile Q{base + j * g.tile, base + j * g.tile + g.half, 128u, DK * 16u};
+        mma_tiles(cta.tmem + j * DV, Q, Sb, DK / 16, id, NS, false);
+      }
+    });
+  const uint32_t lane = tmem_lane_base(warp);
+  const float* olu = ol + uid * ulen * DV;
+  for (int j = 0; j < nq; ++j) {
+    const int tt = j * 128 + tid;
+    const bool on = tt < ulen && drv.ok;
+    const int64_t yo = toff(p, b, (int64_t)n * ulen + tt, h, DV);
+    for (int c = 0; c < DV; c += 16) {
+      float v[16];
+      tmem_ld16(cta.tmem + lane + j * DV + c, v);
+      if (!on) continue;
+#pragma unroll
+      for (int h8 = 0; h8 < 16; h8 += 8) {
+        float o8[8], a8[8];
+        ld8f(olu + (int64_t)tt * DV + c + h8, a8);
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) o8[e2] = v[h8 + e2] + a8[e2];
+        if (p.z) {
+          float zz[8];
+          Elt<T>::ld8(static_cast<const T*>(p.z) + yo + c + h8, zz);
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) o8[e2] *= zz[e2];
+        }
+        Elt<T>::st8(static_cast<T*>(p.y) + yo + c + h8, o8);
+      }
+    }
   }
   cta.finish();
 }

@@ -19,10 +19,11 @@
 // cumulative sum of dL inside the unit.
 //
 // Kernels:
-//   rscan_kernel       reverse sweep over units per (b, h, 32-column slab)
-//   bwd_p_kernel       P = W S0 + Ut, dGam_C
+//   bwd_pe_kernel      P = W S0 + Ut, dz = dy * (Q' S0 + Oloc), E = Q'^T dO
+//   rscan_kernel       reverse sweep over units per (b, h, 32-column slab):
+//                      dS <- Phi^T dS + E (the adjoint of the state map)
 //   bwd_dz_kernel      dP, dZ, dU
-//   bwd_grads_kernel   dQp, dKp, dKs, dAs and the four Gram cotangents
+//   bwd_grads_kernel   dQp, dKp, dKs, dAs, dGam_C and the four Gram cotangents
 //   bwd_gram_off_kernel  off-diagonal blocks of the Gram backward (tcgen05):
 //                      dX with the pivot at the start of the row block,
 //                      dY with the pivot at the end of the column block
@@ -41,6 +42,7 @@ struct BwdBufs {
   float* dZ;        // [nst][Cs][dv]
   float* dU;        // [nst][Cs][dv]
   float* dgc;       // [nst][dk]
+  float* E;         // [nst][dv/32][dk][32]: Q'^T dO per unit, 32-column slabs
   float* g4;        // [nst][4][Cs][dk]: dQp, dKp, dKs, dAs
   float* dG;        // [nst][4][Cs][Cs]: dM^kk, dM^ka, dN^qk, dN^qa
   float* gl;        // [nst][4][Cs][dk]: dK_left, dQ_left, dK_right, dA_right
@@ -52,31 +54,47 @@ struct BwdBufs {
 };
 
 // ---------------------------------------------------------------------------
-// rscan_kernel: for n = last..0: dSC[n] = dS;  dS <- [Phi; Q']^T [dS; dO_n].
-// A = [Phi; Q']^T (M = key channel, K = rows of the map), MN-major;
-// B = [dS; dO] (K = rows, N = 32 slab columns), MN-major.
+// rscan_kernel: the sequential part of the backward pass. For n = last..0:
+//   dSC[n] = dS;   dS <- Phi_n^T dS + E_n,   E_n = Q'_n^T dO_n (from bwd_pe)
+// A = Phi^T: tile 0 of the map image read through the transposed view; B = dS
+// (K = key row, N = 32 slab columns, MN-major) from registers. Phi_n and the
+// E_n slab arrive by bulk copies into two alternating buffers, two units ahead.
 // ---------------------------------------------------------------------------
-template <int DK, typename T, int NS>
+template <int DK, int NS>
 __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_c[2];
   __shared__ uint32_t tslot;
   constexpr int NW = 32;
-  const int dv = p.dv, slabs = dv / NW, Cs = p.Cs;
+  const int dv = p.dv, slabs = dv / NW;
   const int slab = blockIdx.x % slabs;
   const int bh = blockIdx.x / slabs;
   const int h = bh % p.H, b = bh / p.H;
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int R = DK + Cs;  // rows of the map = contraction length
+  const MapGeom g = map_geom(DK, p.Cs);
+  const uint32_t ES = DK * NW * 4u;
   const uint32_t base = smem_u32(sm);
-  const uint32_t AB = 128u * (uint32_t)R * 2u, BB = (uint32_t)NW * R * 2u;
-  const Tile At{base, base + AB, 128u, (uint32_t)R * 16u};
-  const Tile Bt{base + 2 * AB, base + 2 * AB + BB, 128u, (uint32_t)R * 16u};
-  zero_smem(base, 2 * AB + 2 * BB);
+  const uint32_t e_off = 2 * g.tile;  // the transposed view may read up to 2 KB past a Phi tile: E follows
+  const uint32_t b_off = e_off + 2 * ES;
+  const Tile Bt{base + b_off, base + b_off + NW * DK * 2u, 128u, DK * 16u};
+  if (tid == 0) {
+    mbar_init(&bar_c[0], 1);
+    mbar_init(&bar_c[1], 1);
+  }
   TcCta cta;
   cta.init(&tslot, &bar, 32);
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
+  const float* e_s = reinterpret_cast<const float*>(static_cast<const uint8_t*>(sm) + e_off);
+  auto uid_of = [&](int n) { return ((int64_t)b * p.H + h) * p.nsub + n; };
+  auto issue = [&](int n, int buf) {
+    if (tid == 0) {
+      mbar_expect_tx(&bar_c[buf], g.tile + ES);
+      bulk_g2s_big(base + buf * g.tile, p.ma + uid_of(n) * g.unit, g.tile, &bar_c[buf]);
+      bulk_g2s_big(base + e_off + buf * ES, reinterpret_cast<const uint8_t*>(q.E + (uid_of(n) * slabs + slab) * DK * NW),
+                   ES, &bar_c[buf]);
+    }
+  };
   float ds[NW];
   {
     const float* src = q.dS_T ? q.dS_T + (((int64_t)b * p.H + h) * DK) * dv + slab * NW : nullptr;
@@ -84,10 +102,13 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
     for (int j = 0; j < NW; ++j) ds[j] = (src && tid < DK) ? src[(int64_t)tid * dv + j] : 0.f;
   }
   const uint32_t id = idesc_bf16(128, NW, 1, 1);
-  for (int n = p.nsub - 1; n >= 0 && drv.ok; --n) {
-    const int64_t uid = ((int64_t)b * p.H + h) * p.nsub + n;
+  issue(p.nsub - 1, 0);
+  if (p.nsub > 1) issue(p.nsub - 2, 1);
+  for (int k = 0; k < p.nsub && drv.ok; ++k) {
+    const int n = p.nsub - 1 - k;
+    const int buf = k & 1;
     if (tid < DK) {
-      float* o = q.dSC + (uid * DK + tid) * dv + slab * NW;
+      float* o = q.dSC + (uid_of(n) * DK + tid) * dv + slab * NW;
 #pragma unroll
       for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(ds[j], ds[j + 1], ds[j + 2], ds[j + 3]);
 #pragma unroll
@@ -98,34 +119,24 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
         put_mn(Bt, tid, j, v);
       }
     }
-    // dO rows of this unit: tokens n*Cs + t
-    for (int x = tid; x < Cs * (NW / 8); x += 128) {
-      const int t = x / (NW / 8), c8 = (x % (NW / 8)) * 8;
-      const int64_t o = toff(p, b, (int64_t)n * Cs + t, h, dv) + slab * NW + c8;
-      float dd[8], zz[8];
-      Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
-      if (p.z) {
-        Elt<T>::ld8(static_cast<const T*>(p.z) + o, zz);
-#pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) dd[e2] *= zz[e2];
-      }
-      put_mn(Bt, DK + t, c8, dd);
-    }
-    const float* A = p.ma + uid * R * DK;
-    for (int x = tid; x < R * (DK / 8); x += 128) {
-      const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-      float v[8];
-      ld8f(A + (int64_t)r * DK + c8, v);
-      put_mn(At, r, c8, v);
-    }
-    drv.run([&] { mma_tiles(cta.tmem, At, Bt, R / 16, id, NS, false); });
+    const bool c_ok = mbar_wait(&bar_c[buf], (uint32_t)(k >> 1) & 1u);
+    if (!__syncthreads_and(c_ok ? 1 : 0)) { drv.ok = false; break; }
+    const Tile PhiT{base + buf * g.tile, base + buf * g.tile + g.half, DK * 16u, 128u};
+    drv.run([&] { mma_tiles(cta.tmem, PhiT, Bt, DK / 16, id, NS, false); });
     if (!drv.ok) break;
     float v[NW];
     tmem_ld16(cta.tmem + lane, *reinterpret_cast<float(*)[16]>(&v[0]));
     tmem_ld16(cta.tmem + lane + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+    if (tid < DK) {
+      const float* add = e_s + buf * (ES / 4) + tid * NW;
 #pragma unroll
-    for (int j = 0; j < NW; ++j) ds[j] = v[j];
+      for (int j = 0; j < NW; j += 4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(add + j);
+        ds[j] = v[j] + a4.x; ds[j + 1] = v[j + 1] + a4.y; ds[j + 2] = v[j + 2] + a4.z; ds[j + 3] = v[j + 3] + a4.w;
+      }
+    }
     __syncthreads();
+    if (k + 2 < p.nsub) issue(n - 2, buf);
   }
   if (q.dS0 && tid < DK && drv.ok) {
     float* o = q.dS0 + (((int64_t)b * p.H + h) * DK + tid) * dv + slab * NW;
@@ -139,6 +150,7 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
 // operand contracting over cols (put_k), values scaled by sign. rows <= 128.
 __device__ __forceinline__ void stage_rows_k(const Tile& t, const float* src, int rows, int cols, int64_t ld,
                                              float sign) {
+  #pragma unroll 4
   for (int x = threadIdx.x; x < rows * (cols / 8); x += blockDim.x) {
     const int r = x / (cols / 8), c8 = (x % (cols / 8)) * 8;
     float v[8];
@@ -151,6 +163,7 @@ __device__ __forceinline__ void stage_rows_k(const Tile& t, const float* src, in
 // Same matrix as an MN-major operand contracting over rows (put_mn).
 __device__ __forceinline__ void stage_rows_mn(const Tile& t, const float* src, int rows, int cols, int64_t ld,
                                               float sign) {
+  #pragma unroll 4
   for (int x = threadIdx.x; x < rows * (cols / 8); x += blockDim.x) {
     const int r = x / (cols / 8), c8 = (x % (cols / 8)) * 8;
     float v[8];
@@ -162,49 +175,103 @@ __device__ __forceinline__ void stage_rows_mn(const Tile& t, const float* src, i
 }
 
 // ---------------------------------------------------------------------------
-// bwd_p_kernel: P = W S0 + Ut (A = W K-major over channels, B = S0 MN-major),
-// and dGam_C[i] = sum_j dS_C[i][j] S0[i][j].
+// bwd_pe_kernel (per unit, after the recompute sweep):
+//   P  = W S0 + Ut                  A = W (K-major over key channels), B = S0
+//   dz = dy * (Q' S0 + Oloc)        A = Q' (tile 1 of the map image, bulk copy)
+//   E  = Q'^T dO,  dO = z * dy      A = Q' through the transposed view, B = dO
+// TMEM: P -> 0, O -> 128, E -> 256.
 // ---------------------------------------------------------------------------
-template <int DK, int DV, int NS>
-__global__ void __launch_bounds__(128, 1) bwd_p_kernel(ChunkParams p, BwdBufs q) {
+template <int DK, int DV, typename T, int NS>
+__global__ void __launch_bounds__(128, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
+  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
+  const MapGeom g = map_geom(DK, Cs);
   const uint32_t base = smem_u32(sm);
   constexpr uint32_t TB = 128u * 128u * 2u;
-  const Tile A{base, base + TB, 128u, DK * 16u};
-  const Tile B{base + 2 * TB, base + 3 * TB, 128u, DK * 16u};
-  zero_smem(base, 4 * TB);
+  const Tile Qt{base, base + g.half, 128u, DK * 16u};        // Q': rows = tokens, K = key channel
+  const Tile QtT{base, base + g.half, DK * 16u, 128u};       // Q'^T: M = key channel, K = token
+  const Tile A{base + 2 * TB, base + 3 * TB, 128u, DK * 16u};  // W: rows = tokens, K = key channel
+  const Tile B{base + 4 * TB, base + 5 * TB, 128u, DK * 16u};  // S0: K = key channel, N = value column
+  const Tile Bo{base + 4 * TB, base + 5 * TB, 128u, (uint32_t)Cs * 16u};  // dO: K = token, N = value column
+  if (tid == 0) mbar_init(&bar_cp, 1);
   TcCta cta;
-  cta.init(&tslot, &bar, 128);
+  cta.init(&tslot, &bar, 512);
+  if (tid == 0) {
+    mbar_expect_tx(&bar_cp, g.tile);
+    bulk_g2s_big(base, p.ma + u * g.unit + g.tile, g.tile, &bar_cp);
+  }
   MmaSync drv{&bar, 0u, true};
+  const uint32_t lane = tmem_lane_base(warp);
   const float* S0 = q.S_chunks + u * DK * DV;
   stage_rows_k(A, p.wsave + u * Cs * DK, Cs, DK, DK, 1.f);
   stage_rows_mn(B, S0, DK, DV, DV, 1.f);
-  drv.run([&] { mma_tiles(cta.tmem, A, B, DK / 16, idesc_bf16(128, DV, 0, 1), NS, false); });
+  drv.ok = __syncthreads_and(mbar_wait(&bar_cp, 0) ? 1 : 0) != 0;
+  const uint32_t id = idesc_bf16(128, DV, 0, 1);
+  if (drv.ok)
+    drv.run([&] {
+      mma_tiles(cta.tmem + 0, A, B, DK / 16, id, NS, false);
+      mma_tiles(cta.tmem + 128, Qt, B, DK / 16, id, NS, false);
+    });
   const int t = tid;
+  const Rows<T> rows{p, s.b, s.h};
+  // dO = z * dy (B region is free: both MMAs above have completed)
+#pragma unroll 4
+  for (int x = tid; x < Cs * (DV / 8); x += 128) {
+    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+    const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
+    float dd[8], zz[8];
+    Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
+    if (p.z) {
+      Elt<T>::ld8(static_cast<const T*>(p.z) + o, zz);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dd[j] *= zz[j];
+    }
+    put_mn(Bo, r, c8, dd);
+  }
+  if (drv.ok) drv.run([&] { mma_tiles(cta.tmem + 256, QtT, Bo, Cs / 16, idesc_bf16(128, DV, 1, 1), NS, false); });
   const float* Ut = p.usave + u * Cs * DV;
+  const float* olu = p.ol + u * Cs * DV;
   float* P = q.P + u * Cs * DV;
   for (int c = 0; c < DV; c += 16) {
-    float v[16];
-    tmem_ld16(cta.tmem + tmem_lane_base(warp) + c, v);
-    if (t < Cs && drv.ok)
+    float v[16], w[16];
+    tmem_ld16(cta.tmem + lane + c, v);
+    tmem_ld16(cta.tmem + lane + 128 + c, w);
+    if (t < Cs && drv.ok) {
 #pragma unroll
       for (int j = 0; j < 16; j += 4) {
         const float4 a = *reinterpret_cast<const float4*>(Ut + t * DV + c + j);
         *reinterpret_cast<float4*>(P + t * DV + c + j) = make_float4(v[j] + a.x, v[j + 1] + a.y, v[j + 2] + a.z, v[j + 3] + a.w);
       }
+      if (p.dz && p.z) {
+        const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DV) + c;
+#pragma unroll
+        for (int h8 = 0; h8 < 16; h8 += 8) {
+          float dd[8], ol8[8], out[8];
+          Elt<T>::ld8(static_cast<const T*>(p.dy) + o + h8, dd);
+          ld8f(olu + (int64_t)t * DV + c + h8, ol8);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) out[j] = dd[j] * (w[h8 + j] + ol8[j]);
+          Elt<T>::st8(static_cast<T*>(p.dz) + o + h8, out);
+        }
+      }
+    }
   }
-  if (tid < DK) {
-    const float* d = q.dSC + u * DK * DV + tid * DV;
-    const float* s0 = S0 + tid * DV;
-    float acc = 0.f;
-    for (int j = 0; j < DV; ++j) acc += d[j] * s0[j];
-    q.dgc[u * DK + tid] = acc;
+  float* E = q.E + u * DK * DV;
+  for (int c = 0; c < DV; c += 16) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + 256 + c, v);
+    if (t < DK && drv.ok) {
+      float* o = E + ((int64_t)(c >> 5) * DK + t) * 32 + (c & 31);
+#pragma unroll
+      for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
   }
+  (void)rows;
   cta.finish();
 }
 
@@ -241,6 +308,7 @@ __global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   const int t = tid;
   constexpr uint32_t cP = 0, cU = 128, cZ = 256;
   // B1 = dO (K = token, N = value column)
+  #pragma unroll 4
   for (int x = tid; x < Cs * (DV / 8); x += 128) {
     const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
     const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
@@ -261,6 +329,7 @@ __global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   drv.run([&] { mma_tiles(cta.tmem + cU, A, B1, Cs / 16, idT, NS, false); });
   // -(A*Gsuf) and (K*Gsuf): rows s, K = channel (K-major)
   auto stage_suf = [&](bool erase, float sign) {
+    #pragma unroll 4
     for (int x = tid; x < Cs * (DK / 8); x += 128) {
       const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float xx[8], gs[8];
@@ -348,6 +417,7 @@ __global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   const uint32_t lane = tmem_lane_base(warp);
   const int t = tid;
   auto stage_dO = [&](const Tile& dst) {
+    #pragma unroll 4
     for (int x = tid; x < Cs * (DV / 8); x += 128) {
       const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
       const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
@@ -363,6 +433,7 @@ __global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   };
   auto stage_U = [&](const Tile& dst) {
     const Rows<T> rows{p, s.b, s.h};
+    #pragma unroll 4
     for (int x = tid; x < Cs * (DV / 8); x += 128) {
       const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
       float uu[8];
@@ -390,6 +461,17 @@ __global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   };
   const uint32_t idK = idesc_bf16(128, DK, 0, 0), idC = idesc_bf16(128, Cs, 0, 0);
   float* g4 = q.g4 + u * 4 * Cs * DK;
+  if (tid < DK) {  // dGam_C[i] = sum_j dS_C[i][j] S0[i][j]
+    const float* d = q.dSC + u * DK * DV + tid * DV;
+    const float* s0 = q.S_chunks + u * DK * DV + tid * DV;
+    float acc = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < DV; j += 4) {
+      const float4 a = *reinterpret_cast<const float4*>(d + j), c = *reinterpret_cast<const float4*>(s0 + j);
+      acc += a.x * c.x + a.y * c.y + a.z * c.z + a.w * c.w;
+    }
+    q.dgc[u * DK + tid] = acc;
+  }
   float* dG = q.dG + u * 4 * Cs * Cs;
   // pass 1
   stage_rows_k(R0, q.dSC + u * DK * DV, DK, DV, DV, 1.f);
@@ -472,12 +554,14 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
   const uint32_t id16 = idesc_bf16(128, SB, 1, 0), id16m = idesc_bf16(128, SB, 1, 1);
   // ---- left gradients: J ascending, mid(I, J) for I < J
   for (int J = 1; J < nb && drv.ok; ++J) {
+    #pragma unroll 4
     for (int x = tid; x < nb * DK; x += 128) {
       const int I = x / DK, i = x % DK;
       if (I == J - 1) midtab[x] = 1.f;
       else if (I < J - 1) midtab[x] *= pre[(SB * (J - 1) + SB - 1) * DK + i];  // tot_{J-1}
     }
     __syncthreads();
+    #pragma unroll 4
     for (int x = tid; x < SB * J * (DK / 8); x += 128) {
       const int ss = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float kk[8], aa[8], sf[8];
@@ -490,6 +574,7 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
       put_mn(A1, ss, c8, kk);
       put_mn(A2, ss, c8, aa);
     }
+    #pragma unroll 4
     for (int x = tid; x < 4 * SB * (SB * J / 8); x += 128) {
       const int g = x / (SB * (SB * J / 8)), rem = x % (SB * (SB * J / 8));
       const int rr = rem / (SB * J / 8), c8 = (rem % (SB * J / 8)) * 8;
@@ -507,6 +592,7 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
   }
   // ---- right gradients: I descending, mid(I, J) for J > I
   for (int I = nb - 2; I >= 0 && drv.ok; --I) {
+    #pragma unroll 4
     for (int x = tid; x < nb * DK; x += 128) {
       const int J = x / DK, i = x % DK;
       if (J == I + 1) midtab[x] = 1.f;
@@ -514,6 +600,7 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
     }
     __syncthreads();
     const int t0 = SB * (I + 1);
+    #pragma unroll 4
     for (int x = tid; x < (Cs - t0) * (DK / 8); x += 128) {
       const int tt = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float kk[8], qq[8], pr[8];
@@ -526,6 +613,7 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
       put_mn(A1, tt, c8, kk);
       put_mn(A2, tt, c8, qq);
     }
+    #pragma unroll 4
     for (int x = tid; x < 4 * (Cs - t0) * 2; x += 128) {
       const int g = x / ((Cs - t0) * 2), rem = x % ((Cs - t0) * 2);
       const int tt = t0 + rem / 2, c8 = (rem % 2) * 8;
@@ -578,6 +666,7 @@ __global__ void __launch_bounds__(128) bwd_gram_diag_kernel(ChunkParams p, BwdBu
   const int J = blockIdx.x % nb;
   const SubIdx s = sub_of(p, (int)u, p.nsub, Cs);
   const int i = threadIdx.x;
+  #pragma unroll 4
   for (int x = threadIdx.x; x < 4 * SB * SB; x += blockDim.x) {
     const int g = x / (SB * SB), tt = (x / SB) % SB, ss = x % SB;
     sdg[g][tt][ss] = q.dG[((u * 4 + g) * Cs + SB * J + tt) * Cs + SB * J + ss];

@@ -22,6 +22,12 @@ template <typename T> struct Elt;
 
 template <> struct Elt<float> {
   static __device__ __forceinline__ float ld(const float* p) { return __ldg(p); }
+  // 8 consecutive elements through a generic pointer (e.g. shared memory).
+  static __device__ __forceinline__ void ld8g(const float* p, float (&o)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
   static __device__ __forceinline__ void st(float* p, float x) { *p = x; }
   // 8 consecutive elements (p 32-byte aligned).
   static __device__ __forceinline__ void ld8(const float* p, float (&o)[8]) {
@@ -46,6 +52,15 @@ template <> struct Elt<float> {
 template <> struct Elt<__nv_bfloat16> {
   using T = __nv_bfloat16;
   static __device__ __forceinline__ float ld(const T* p) { return __bfloat162float(p[0]); }
+  static __device__ __forceinline__ void ld8g(const T* p, float (&o)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      o[2 * i] = f.x; o[2 * i + 1] = f.y;
+    }
+  }
   static __device__ __forceinline__ void st(T* p, float x) { *p = __float2bfloat16_rn(x); }
   static __device__ __forceinline__ void ld8(const T* p, float (&o)[8]) {
     uint4 u = __ldg(reinterpret_cast<const uint4*>(p));

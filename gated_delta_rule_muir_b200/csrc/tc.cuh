@@ -68,6 +68,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// ---- bulk asynchronous copies (global -> shared, completion on an mbarrier) --
+
+// Arrive on `bar` (count 1) and announce `bytes` of incoming bulk-copy traffic.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+// Copy `bytes` (multiple of 16, both addresses 16-byte aligned) from global to
+// shared memory; completes as transaction bytes on `bar`. No multicast.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // ---- fences ----------------------------------------------------------------
 
 // Generic-proxy shared-memory writes -> visible to the tensor core (async proxy).
@@ -167,9 +182,13 @@ __device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo
   }
 }
 
+// 16-byte store to a shared-memory address. A plain C++ store through the
+// generic alias of the address: the compiler sees a shared-memory store and can
+// keep issuing the next staging iteration's global loads ahead of it (an asm
+// store with a memory clobber would serialise every staging loop). Ordering
+// with the tensor core is established by fence_async_smem() + a CTA barrier.
 __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
+  *reinterpret_cast<uint4*>(__cvta_shared_to_generic(addr)) = v;
 }
 
 // K-major (natural view, lbo = 128): 8 consecutive contraction indices k8..k8+7 of MN row m.
@@ -188,6 +207,17 @@ __device__ __forceinline__ void put_mn(const Tile& t, int k, int m8, const float
   const uint32_t off = (uint32_t)(m8 >> 3) * t.sbo + (uint32_t)(k >> 3) * 128u + (uint32_t)(k & 7) * 16u;
   sts128(t.hi + off, hi);
   sts128(t.lo + off, lo);
+}
+
+// Global-memory image of staged tiles: the same byte layout as put_k, written to
+// global memory so that a consumer can bring it into shared memory with one bulk
+// copy. `hi` points at the hi block, the lo block follows `lo_off` bytes later.
+__device__ __forceinline__ void gput_k(uint8_t* hi, uint32_t lo_off, uint32_t sbo, int m, int k8, const float (&x)[8]) {
+  uint4 h, l;
+  split8(x, h, l);
+  const uint32_t off = (uint32_t)(m >> 3) * sbo + (uint32_t)(k8 >> 3) * 128u + (uint32_t)(m & 7) * 16u;
+  *reinterpret_cast<uint4*>(hi + off) = h;
+  *reinterpret_cast<uint4*>(hi + lo_off + off) = l;
 }
 
 // ---- TMEM -> registers -----------------------------------------------------
