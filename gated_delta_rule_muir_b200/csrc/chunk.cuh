@@ -253,20 +253,22 @@ __global__ void __launch_bounds__(128) decay_kernel(ChunkParams p) {
 // (upper blocks get 0).
 // ---------------------------------------------------------------------------
 template <int DK, typename T, int NS>
-__global__ void __launch_bounds__(128, 1) gram_off_kernel(ChunkParams p) {
+__global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
+  constexpr int NT = 256;
   const int Cs = p.Cs, nb = Cs / SB;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr uint32_t LB = 128u * DK * 2u, RB = SB * DK * 2u;
   const uint32_t base = smem_u32(sm);
-  const Tile L{base, base + LB, 128u, DK * 16u};
-  const Tile RK{base + 2 * LB, base + 2 * LB + RB, 128u, DK * 16u};
-  const Tile RA{base + 2 * LB + 2 * RB, base + 2 * LB + 3 * RB, 128u, DK * 16u};
-  float* midtab = reinterpret_cast<float*>(sm + 2 * LB + 4 * RB);  // [nb][DK]
-  zero_smem(base, 2 * LB);
+  const Tile LK{base, base + LB, 128u, DK * 16u};                   // K-side left operand
+  const Tile LQ{base + 2 * LB, base + 3 * LB, 128u, DK * 16u};      // Q-side left operand
+  const Tile RK{base + 4 * LB, base + 4 * LB + RB, 128u, DK * 16u};
+  const Tile RA{base + 4 * LB + 2 * RB, base + 4 * LB + 3 * RB, 128u, DK * 16u};
+  float* midtab = reinterpret_cast<float*>(sm + 4 * LB + 4 * RB);  // [nb][DK]
+  zero_smem(base, 4 * LB);
   TcCta cta;
   cta.init(&tslot, &bar, tmem_cols_for(4 * Cs));
   const float* pre = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
@@ -275,14 +277,14 @@ __global__ void __launch_bounds__(128, 1) gram_off_kernel(ChunkParams p) {
   MmaSync drv{&bar, 0u, true};
   const uint32_t id = idesc_bf16(128, SB, 0, 0);
   for (int I = nb - 2; I >= 0 && drv.ok; --I) {
-    #pragma unroll 4
-    for (int x = tid; x < nb * DK; x += 128) {
+#pragma unroll 4
+    for (int x = tid; x < nb * DK; x += NT) {
       const int J = x / DK, i = x % DK;
       if (J == I + 1) midtab[x] = 1.f;
       else if (J > I + 1) midtab[x] *= pre[(SB * (I + 1) + SB - 1) * DK + i];
     }
-    #pragma unroll 4
-    for (int x = tid; x < SB * (DK / 8); x += 128) {
+#pragma unroll 2
+    for (int x = tid; x < SB * (DK / 8); x += NT) {
       const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       const int t = SB * I + rr;
       float kk[8], aa[8], sf[8], vk[8], va[8];
@@ -296,34 +298,39 @@ __global__ void __launch_bounds__(128, 1) gram_off_kernel(ChunkParams p) {
     }
     __syncthreads();
     const int t0 = SB * (I + 1);
-    for (int pass = 0; pass < 2 && drv.ok; ++pass) {
-      #pragma unroll 4
-      for (int x = tid; x < (Cs - t0) * (DK / 8); x += 128) {
-        const int t = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-        float xv[8], pr[8], md[8];
-        if (pass == 0) rows.k(s.tok0 + t, c8, xv);
-        else rows.qt(s.tok0 + t, c8, xv);
-        ld8f(pre + t * DK + c8, pr);
-        const float* mp = midtab + (t / SB) * DK + c8;
+#pragma unroll 2
+    for (int x = tid; x < (Cs - t0) * (DK / 8); x += NT) {
+      const int t = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      float kv[8], qv[8], pr[8];
+      rows.k(s.tok0 + t, c8, kv);
+      rows.qt(s.tok0 + t, c8, qv);
+      ld8f(pre + t * DK + c8, pr);
+      const float4* mp = reinterpret_cast<const float4*>(midtab + (t / SB) * DK + c8);
+      const float4 m0 = mp[0], m1 = mp[1];
+      const float md[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) md[j] = mp[j];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xv[j] *= pr[j] * md[j];
-        put_k(L, t, c8, xv);
+      for (int j = 0; j < 8; ++j) {
+        const float f = pr[j] * md[j];
+        kv[j] *= f;
+        qv[j] *= f;
       }
-      const uint32_t c0 = (pass == 0 ? 0u : 2u * Cs) + SB * I;
-      drv.run([&] {
-        mma_tiles(cta.tmem + c0, L, RK, DK / 16, id, NS, false);
-        mma_tiles(cta.tmem + c0 + Cs, L, RA, DK / 16, id, NS, false);
-      });
+      put_k(LK, t, c8, kv);
+      put_k(LQ, t, c8, qv);
     }
+    const uint32_t c0 = SB * I;
+    drv.run([&] {
+      mma_tiles(cta.tmem + c0, LK, RK, DK / 16, id, NS, false);
+      mma_tiles(cta.tmem + c0 + Cs, LK, RA, DK / 16, id, NS, false);
+      mma_tiles(cta.tmem + c0 + 2 * Cs, LQ, RK, DK / 16, id, NS, false);
+      mma_tiles(cta.tmem + c0 + 3 * Cs, LQ, RA, DK / 16, id, NS, false);
+    });
   }
-  // Epilogue: thread = row t.
-  const int t = tid;
+  // Epilogue: row t = TMEM lane; the two warpgroups take alternate 16-column chunks.
+  const int t = tid & 127, wg = tid >> 7;
   const int J = t / SB;
   float* out = p.gr + (int64_t)blockIdx.x * 4 * Cs * Cs;
   for (int gidx = 0; gidx < 4; ++gidx) {
-    for (int c0 = 0; c0 < Cs; c0 += 16) {
+    for (int c0 = wg * 16; c0 < Cs; c0 += 32) {
       float v[16];
       tmem_ld16(cta.tmem + tmem_lane_base(warp) + gidx * Cs + c0, v);
       const int I = c0 / SB;
@@ -428,11 +435,12 @@ __global__ void __launch_bounds__(128) gram_diag_kernel(ChunkParams p) {
 // level (X = M_B T_A, then Y = T_D X).
 // ---------------------------------------------------------------------------
 template <int NS>
-__global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
+__global__ void __launch_bounds__(256, 1) solve_kernel(ChunkParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs, nb = Cs / SB;
+  constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
   float* Tf = reinterpret_cast<float*>(sm);  // [Cs][Cs]
   const uint32_t base = smem_u32(sm) + 128u * 128u * 4u;
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
   const Tile TA{base, base + TB, 128u, (uint32_t)Cs * 16u};           // K-major A tiles (K = Cs)
   const Tile TBt{base + 2 * TB, base + 3 * TB, 128u, (uint32_t)Cs * 16u};  // MN-major B tiles (K = Cs)
   const float* M = p.gr + ((int64_t)blockIdx.x * 4 + 1) * Cs * Cs;
-  for (int x = tid; x < Cs * Cs; x += 128) Tf[x] = 0.f;
+  for (int x = tid; x < Cs * Cs; x += NT) Tf[x] = 0.f;
   zero_smem(base, 4 * TB);
   TcCta cta;
   cta.init(&tslot, &bar, 256);
@@ -464,11 +472,11 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
   }
   __syncthreads();
   MmaSync drv{&bar, 0u, true};
-  const int t = tid;
+  const int t = tid & 127, wg = tid >> 7;
   for (int h = SB; h < Cs && drv.ok; h *= 2) {
     // A = off-diagonal blocks (2m+1, 2m) of M (zeros elsewhere), K-major; B = Tcur, MN-major.
     #pragma unroll 4
-    for (int x = tid; x < 128 * (Cs / 8); x += 128) {
+    for (int x = tid; x < 128 * (Cs / 8); x += NT) {
       const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
       float v[8];
       const bool on = r < Cs && ((r / h) & 1) && (c8 / h) == (r / h) - 1;
@@ -480,7 +488,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
       put_k(TA, r, c8, v);
     }
     #pragma unroll 4
-    for (int x = tid; x < Cs * (Cs / 8); x += 128) {
+    for (int x = tid; x < Cs * (Cs / 8); x += NT) {
       const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
       float v[8];
 #pragma unroll
@@ -499,7 +507,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
     {
       const int m = t / (2 * h);
       const bool odd = t < Cs && ((t / h) & 1);
-      for (int c = 0; c < h; c += 16) {
+      for (int c = wg * 16; c < h; c += 32) {
         float v[16];
         tmem_ld16(cta.tmem + tmem_lane_base(warp) + 2 * m * h + c, v);
         if (odd) {
@@ -513,7 +521,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
     }
     // A = Tcur, K-major.
     #pragma unroll 4
-    for (int x = tid; x < Cs * (Cs / 8); x += 128) {
+    for (int x = tid; x < Cs * (Cs / 8); x += NT) {
       const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
       float v[8];
 #pragma unroll
@@ -529,7 +537,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
     {
       const int m = t / (2 * h);
       const bool odd = t < Cs && ((t / h) & 1);
-      for (int c = 0; c < h; c += 16) {
+      for (int c = wg * 16; c < h; c += 32) {
         float v[16];
         tmem_ld16(cta.tmem + tmem_lane_base(warp) + 128 + 2 * m * h + c, v);
         if (odd) {
@@ -542,7 +550,7 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
   }
   float* out = p.tt + (int64_t)blockIdx.x * Cs * Cs;
   if (drv.ok)
-    for (int x = tid; x < Cs * Cs / 4; x += 128)
+    for (int x = tid; x < Cs * Cs / 4; x += NT)
       reinterpret_cast<float4*>(out)[x] = reinterpret_cast<const float4*>(Tf)[x];
   cta.finish();
 }
@@ -555,12 +563,13 @@ __global__ void __launch_bounds__(128, 1) solve_kernel(ChunkParams p) {
 // each). Negated operands are staged negated.
 // ---------------------------------------------------------------------------
 template <int DK, int DV, typename T, int NS>
-__global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
+__global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr uint32_t TBY = 128u * 128u * 2u;
   const uint32_t base = smem_u32(sm);
@@ -579,12 +588,12 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   const Rows<T> rows{p, s.b, s.h};
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
-  const int t = tid;
+  const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroup takes alternate 16-column chunks
   constexpr uint32_t cW = 0, cZ = 128, cUt = 256, cPhi = 0, cPsi = 128, cOl = 256, cQ = 384;
 
   auto stage_k_matrix = [&](const Tile& dst, const float* src, float sign) {  // rows t, K = s (Cs x Cs)
     #pragma unroll 4
-    for (int x = tid; x < Cs * (Cs / 8); x += 128) {
+    for (int x = tid; x < Cs * (Cs / 8); x += NT) {
       const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
       float v[8];
       ld8f(src + (int64_t)r * Cs + c8, v);
@@ -595,7 +604,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   };
   // TMEM columns [col, col+n) of this thread's row -> MN-major B tile row t.
   auto tmem_to_b = [&](const Tile& dst, uint32_t col, int n) {
-    for (int c = 0; c < n; c += 16) {
+    for (int c = wg * 16; c < n; c += 32) {
       float v[16];
       tmem_ld16(cta.tmem + lane + col + c, v);
       if (t < Cs) {
@@ -610,7 +619,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   // (X * Gsuf)^T as an MN-major A operand (M = channel, K = token), scaled by sign.
   auto stage_suffixed = [&](bool erase, float sign) {
     #pragma unroll 4
-    for (int x = tid; x < Cs * (DK / 8); x += 128) {
+    for (int x = tid; x < Cs * (DK / 8); x += NT) {
       const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float xx[8], gs[8];
       if (erase) rows.a(s.tok0 + r, c8, xx);
@@ -626,7 +635,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   // ---- phase 1: W = T (K*Gam), Z = M^kk U, Ut = T Z
   stage_k_matrix(A, Tm, 1.f);
   #pragma unroll 4
-  for (int x = tid; x < Cs * (DK / 8); x += 128) {  // B1 = K*Gam (K = token, N = channel)
+  for (int x = tid; x < Cs * (DK / 8); x += NT) {  // B1 = K*Gam (K = token, N = channel)
     const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
     float kk[8], gm[8];
     rows.k(s.tok0 + r, c8, kk);
@@ -636,7 +645,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
     put_mn(B1, r, c8, kk);
   }
   #pragma unroll 4
-  for (int x = tid; x < Cs * (DV / 8); x += 128) {  // B2 = U
+  for (int x = tid; x < Cs * (DV / 8); x += NT) {  // B2 = U
     const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
     float uu[8];
     rows.u(s.tok0 + r, c8, uu);
@@ -651,7 +660,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   if (p.wsave) {  // the backward pass reuses W and Ut
     float* wo = p.wsave + (int64_t)blockIdx.x * Cs * DK;
     float* uo = p.usave + (int64_t)blockIdx.x * Cs * DV;
-    for (int c = 0; c < DK; c += 16) {
+    for (int c = wg * 16; c < DK; c += 32) {
       float v[16];
       tmem_ld16(cta.tmem + lane + cW + c, v);
       if (t < Cs)
@@ -659,7 +668,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
         for (int j = 0; j < 16; j += 4)
           *reinterpret_cast<float4*>(wo + t * DK + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
-    for (int c = 0; c < DV; c += 16) {
+    for (int c = wg * 16; c < DV; c += 32) {
       float v[16];
       tmem_ld16(cta.tmem + lane + cUt + c, v);
       if (t < Cs)
@@ -689,7 +698,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
   float* psi = p.psi + (int64_t)blockIdx.x * DK * DV;
   float* ol = p.ol + (int64_t)blockIdx.x * Cs * DV;
   const float* gC = gam + (Cs - 1) * DK;
-  for (int c = 0; c < DK; c += 16) {
+  for (int c = wg * 16; c < DK; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cPhi + c, v);
     if (t < DK && drv.ok) {
@@ -703,7 +712,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
       map_put_phi(ma, mg, DK, t, c + 8, b8);
     }
   }
-  for (int c = 0; c < DV; c += 16) {
+  for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cPsi + c, v);
     if (t < DK && drv.ok) {
@@ -712,7 +721,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
       for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
   }
-  for (int c = 0; c < DK; c += 16) {
+  for (int c = wg * 16; c < DK; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cQ + c, v);
     if (t < Cs && drv.ok) {
@@ -731,7 +740,7 @@ __global__ void __launch_bounds__(128, 1) maps_kernel(ChunkParams p) {
       map_put_q(ma, mg, DK, t, c + 8, b8);
     }
   }
-  for (int c = 0; c < DV; c += 16) {
+  for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cOl + c, v);
     if (t < Cs && drv.ok) {

@@ -182,12 +182,13 @@ __device__ __forceinline__ void stage_rows_mn(const Tile& t, const float* src, i
 // TMEM: P -> 0, O -> 128, E -> 256.
 // ---------------------------------------------------------------------------
 template <int DK, int DV, typename T, int NS>
-__global__ void __launch_bounds__(128, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q) {
+__global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
   const MapGeom g = map_geom(DK, Cs);
@@ -217,11 +218,11 @@ __global__ void __launch_bounds__(128, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
       mma_tiles(cta.tmem + 0, A, B, DK / 16, id, NS, false);
       mma_tiles(cta.tmem + 128, Qt, B, DK / 16, id, NS, false);
     });
-  const int t = tid;
+  const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
   const Rows<T> rows{p, s.b, s.h};
   // dO = z * dy (B region is free: both MMAs above have completed)
 #pragma unroll 4
-  for (int x = tid; x < Cs * (DV / 8); x += 128) {
+  for (int x = tid; x < Cs * (DV / 8); x += NT) {
     const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
     const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
     float dd[8], zz[8];
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(128, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
   const float* Ut = p.usave + u * Cs * DV;
   const float* olu = p.ol + u * Cs * DV;
   float* P = q.P + u * Cs * DV;
-  for (int c = 0; c < DV; c += 16) {
+  for (int c = wg * 16; c < DV; c += 32) {
     float v[16], w[16];
     tmem_ld16(cta.tmem + lane + c, v);
     tmem_ld16(cta.tmem + lane + 128 + c, w);
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(128, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
     }
   }
   float* E = q.E + u * DK * DV;
-  for (int c = 0; c < DV; c += 16) {
+  for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + 256 + c, v);
     if (t < DK && drv.ok) {
@@ -281,12 +282,13 @@ __global__ void __launch_bounds__(128, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
 // TMEM: dP -> 0, dU -> 128, dZ -> 256. Tiles: A, B1 (dO), B2 (dS_C; later dZ).
 // ---------------------------------------------------------------------------
 template <int DK, int DV, typename T, int NS>
-__global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q) {
+__global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
   const uint32_t base = smem_u32(sm);
@@ -305,11 +307,11 @@ __global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   const Rows<T> rows{p, s.b, s.h};
   const float* G = p.gr + u * 4 * Cs * Cs;
   const float* gsuf = p.dec + (u * 4 + 3) * Cs * DK;
-  const int t = tid;
+  const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
   constexpr uint32_t cP = 0, cU = 128, cZ = 256;
   // B1 = dO (K = token, N = value column)
   #pragma unroll 4
-  for (int x = tid; x < Cs * (DV / 8); x += 128) {
+  for (int x = tid; x < Cs * (DV / 8); x += NT) {
     const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
     const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
     float dd[8], zz[8];
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   // -(A*Gsuf) and (K*Gsuf): rows s, K = channel (K-major)
   auto stage_suf = [&](bool erase, float sign) {
     #pragma unroll 4
-    for (int x = tid; x < Cs * (DK / 8); x += 128) {
+    for (int x = tid; x < Cs * (DK / 8); x += NT) {
       const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float xx[8], gs[8];
       if (erase) rows.a(s.tok0 + r, c8, xx);
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   stage_suf(false, 1.f);
   drv.run([&] { mma_tiles(cta.tmem + cU, Ak, B2, DK / 16, idK, NS, true); });
   // dP (TMEM) -> B3 (K = token), then dZ = T^T dP
-  for (int c = 0; c < DV; c += 16) {
+  for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cP + c, v);
     if (t < Cs) {
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   stage_rows_mn(A, p.tt + u * Cs * Cs, Cs, Cs, Cs, 1.f);  // T^T: K = t, M = s
   drv.run([&] { mma_tiles(cta.tmem + cZ, A, B3, Cs / 16, idT, NS, false); });
   float* dZo = q.dZ + u * Cs * DV;
-  for (int c = 0; c < DV; c += 16) {
+  for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cZ + c, v);
     if (t < Cs) {
@@ -378,7 +380,7 @@ __global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   stage_rows_mn(A, G + 0 * Cs * Cs, Cs, Cs, Cs, 1.f);  // M^kk^T
   drv.run([&] { mma_tiles(cta.tmem + cU, A, B3, Cs / 16, idT, NS, true); });
   float* dUo = q.dU + u * Cs * DV;
-  for (int c = 0; c < DV; c += 16) {
+  for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cU + c, v);
     if (t < Cs && drv.ok)
@@ -397,12 +399,13 @@ __global__ void __launch_bounds__(128, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
 //   pass 3: dQp = dO S0^T, dKp = dZ S0^T
 // ---------------------------------------------------------------------------
 template <int DK, int DV, typename T, int NS>
-__global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBufs q) {
+__global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
   const uint32_t base = smem_u32(sm);
@@ -415,10 +418,10 @@ __global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   cta.init(&tslot, &bar, 512);
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
-  const int t = tid;
+  const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
   auto stage_dO = [&](const Tile& dst) {
     #pragma unroll 4
-    for (int x = tid; x < Cs * (DV / 8); x += 128) {
+    for (int x = tid; x < Cs * (DV / 8); x += NT) {
       const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
       const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
       float dd[8], zz[8];
@@ -434,7 +437,7 @@ __global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   auto stage_U = [&](const Tile& dst) {
     const Rows<T> rows{p, s.b, s.h};
     #pragma unroll 4
-    for (int x = tid; x < Cs * (DV / 8); x += 128) {
+    for (int x = tid; x < Cs * (DV / 8); x += NT) {
       const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
       float uu[8];
       rows.u(s.tok0 + r, c8, uu);
@@ -443,7 +446,7 @@ __global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   };
   // Row t of a [Cs][N] TMEM result -> dst (fp32, row-major, row stride ld), optional mask.
   auto drain = [&](uint32_t col, int n, float* dst, int64_t ld, int mask) {
-    for (int c = 0; c < n; c += 16) {
+    for (int c = wg * 16; c < n; c += 32) {
       float v[16];
       tmem_ld16(cta.tmem + lane + col + c, v);
       if (t < Cs && drv.ok) {
@@ -523,12 +526,13 @@ __global__ void __launch_bounds__(128, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
 // Region columns: dK_left 0, dQ_left Cs, dK_right 2Cs, dA_right 3Cs.
 // ---------------------------------------------------------------------------
 template <int DK, typename T, int NS>
-__global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, BwdBufs q) {
+__global__ void __launch_bounds__(256, 1) bwd_gram_off_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs, nb = Cs / SB;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
+  constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
   const uint32_t base = smem_u32(sm);
@@ -555,14 +559,14 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
   // ---- left gradients: J ascending, mid(I, J) for I < J
   for (int J = 1; J < nb && drv.ok; ++J) {
     #pragma unroll 4
-    for (int x = tid; x < nb * DK; x += 128) {
+    for (int x = tid; x < nb * DK; x += NT) {
       const int I = x / DK, i = x % DK;
       if (I == J - 1) midtab[x] = 1.f;
       else if (I < J - 1) midtab[x] *= pre[(SB * (J - 1) + SB - 1) * DK + i];  // tot_{J-1}
     }
     __syncthreads();
     #pragma unroll 4
-    for (int x = tid; x < SB * J * (DK / 8); x += 128) {
+    for (int x = tid; x < SB * J * (DK / 8); x += NT) {
       const int ss = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float kk[8], aa[8], sf[8];
       rows.k(s.tok0 + ss, c8, kk);
@@ -575,7 +579,7 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
       put_mn(A2, ss, c8, aa);
     }
     #pragma unroll 4
-    for (int x = tid; x < 4 * SB * (SB * J / 8); x += 128) {
+    for (int x = tid; x < 4 * SB * (SB * J / 8); x += NT) {
       const int g = x / (SB * (SB * J / 8)), rem = x % (SB * (SB * J / 8));
       const int rr = rem / (SB * J / 8), c8 = (rem % (SB * J / 8)) * 8;
       float v[8];
@@ -593,7 +597,7 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
   // ---- right gradients: I descending, mid(I, J) for J > I
   for (int I = nb - 2; I >= 0 && drv.ok; --I) {
     #pragma unroll 4
-    for (int x = tid; x < nb * DK; x += 128) {
+    for (int x = tid; x < nb * DK; x += NT) {
       const int J = x / DK, i = x % DK;
       if (J == I + 1) midtab[x] = 1.f;
       else if (J > I + 1) midtab[x] *= pre[(SB * (I + 1) + SB - 1) * DK + i];
@@ -601,7 +605,7 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
     __syncthreads();
     const int t0 = SB * (I + 1);
     #pragma unroll 4
-    for (int x = tid; x < (Cs - t0) * (DK / 8); x += 128) {
+    for (int x = tid; x < (Cs - t0) * (DK / 8); x += NT) {
       const int tt = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float kk[8], qq[8], pr[8];
       rows.k(s.tok0 + tt, c8, kk);
@@ -614,7 +618,7 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
       put_mn(A2, tt, c8, qq);
     }
     #pragma unroll 4
-    for (int x = tid; x < 4 * (Cs - t0) * 2; x += 128) {
+    for (int x = tid; x < 4 * (Cs - t0) * 2; x += NT) {
       const int g = x / ((Cs - t0) * 2), rem = x % ((Cs - t0) * 2);
       const int tt = t0 + rem / 2, c8 = (rem % 2) * 8;
       float v[8];
@@ -632,12 +636,12 @@ __global__ void __launch_bounds__(128, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
   }
   // ---- epilogue: lane = channel i; scale by pre (left) or suf (right); blocks
   // without contributions (J = 0 left, I = nb-1 right) are written as zeros.
-  const int i = tid;
+  const int i = tid & 127, wg = tid >> 7;  // TMEM lane = key channel; warpgroups split the columns
   float* gl = q.gl + u * 4 * Cs * DK;
   for (int reg = 0; reg < 4; ++reg) {
     const bool left = reg < 2;
     const float* sc = left ? pre : suf;
-    for (int c = 0; c < Cs; c += 16) {
+    for (int c = wg * 16; c < Cs; c += 32) {
       float v[16];
       tmem_ld16(cta.tmem + tmem_lane_base(warp) + reg * Cs + c, v);
       const int blk = c / SB;
