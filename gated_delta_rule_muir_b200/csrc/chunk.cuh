@@ -58,8 +58,8 @@ struct ChunkParams {
   const float* S0;
   // workspace
   float* dec;  // [nsubtot][4][Cs][dk]: pre, suf, Gam, Gsuf
-  float* gr;   // [nsubtot][4][Cs][Cs]: M^kk, M^ka, N^qk, N^qa
-  float* tt;   // [nsubtot][Cs][Cs]
+  uint8_t* gr; // [nsubtot][4] images of M^kk, M^ka, N^qk, N^qa (see sq_put)
+  uint8_t* tt; // [nsubtot] image of T
   uint8_t* ma;  // [nunits] images of Phi and Q' (see MapGeom)
   float* psi;   // [nunits][dv/32][dk][32]: Psi in 32-column slabs
   float* ol;    // [nunits][Cs][dv]: Oloc
@@ -139,6 +139,23 @@ __device__ __forceinline__ void map_put_phi(uint8_t* img, const MapGeom& g, int 
 // Row t (token) of Q'.
 __device__ __forceinline__ void map_put_q(uint8_t* img, const MapGeom& g, int dk, int t, int c8, const float (&x)[8]) {
   gput_k(img + (uint32_t)(1 + (t >> 7)) * g.tile, g.half, (uint32_t)dk * 16u, t & 127, c8, x);
+}
+
+// Workspace image of a Cs x Cs matrix (a Gram or T): bf16 hi block then lo
+// block of 128 rows x Cs columns in the K-major canonical layout (sbo = Cs*16),
+// row = first index. Consumers bulk-copy it; a K-major read contracts over the
+// columns, the transposed view (lbo = Cs*16, sbo = 128) over the rows.
+__host__ __device__ inline uint32_t sq_half(int Cs) { return 128u * (uint32_t)Cs * 2u; }
+__host__ __device__ inline uint32_t sq_bytes(int Cs) { return 2u * sq_half(Cs); }
+__device__ __forceinline__ void sq_put(uint8_t* img, int Cs, int r, int c8, const float (&x)[8]) {
+  gput_k(img, sq_half(Cs), (uint32_t)Cs * 16u, r, c8, x);
+}
+__device__ __forceinline__ float sq_get(const uint8_t* img, int Cs, int r, int c) {
+  const uint32_t off = (uint32_t)(r >> 3) * (uint32_t)Cs * 16u + (uint32_t)(c >> 3) * 128u + (uint32_t)(r & 7) * 16u +
+                       (uint32_t)(c & 7) * 2u;
+  const __nv_bfloat16 h = *reinterpret_cast<const __nv_bfloat16*>(img + off);
+  const __nv_bfloat16 l = *reinterpret_cast<const __nv_bfloat16*>(img + sq_half(Cs) + off);
+  return __bfloat162float(h) + __bfloat162float(l);
 }
 
 // Bulk copy of `bytes` (multiple of 16) in pieces of at most 32 KB.
@@ -328,19 +345,21 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
   // Epilogue: row t = TMEM lane; the two warpgroups take alternate 16-column chunks.
   const int t = tid & 127, wg = tid >> 7;
   const int J = t / SB;
-  float* out = p.gr + (int64_t)blockIdx.x * 4 * Cs * Cs;
+  uint8_t* out = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
   for (int gidx = 0; gidx < 4; ++gidx) {
     for (int c0 = wg * 16; c0 < Cs; c0 += 32) {
       float v[16];
       tmem_ld16(cta.tmem + tmem_lane_base(warp) + gidx * Cs + c0, v);
       const int I = c0 / SB;
       if (t < Cs && I != J && drv.ok) {
-        float* o = out + ((int64_t)gidx * Cs + t) * Cs + c0;
+        float a8[8], b8[8];
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-          float4 w4 = (I < J) ? make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
-          *reinterpret_cast<float4*>(o + j) = w4;
+        for (int j = 0; j < 8; ++j) {
+          a8[j] = I < J ? v[j] : 0.f;
+          b8[j] = I < J ? v[8 + j] : 0.f;
         }
+        sq_put(out + gidx * sq_bytes(Cs), Cs, t, c0, a8);
+        sq_put(out + gidx * sq_bytes(Cs), Cs, t, c0 + 8, b8);
       }
     }
   }
@@ -413,17 +432,16 @@ __global__ void __launch_bounds__(128) gram_diag_kernel(ChunkParams p) {
 #pragma unroll
   for (int gidx = 0; gidx < 4; ++gidx) {
     if (cg != gidx) continue;  // lane cg of the row writes Gram cg
-    float* o = p.gr + (((int64_t)sid * 4 + gidx) * Cs + SB * J + t) * Cs + SB * J;
+    uint8_t* img = p.gr + ((int64_t)sid * 4 + gidx) * sq_bytes(Cs);
     const bool strict = gidx < 2;  // M^kk, M^ka exclude the diagonal
+    float a8[8], b8[8];
 #pragma unroll
-    for (int ss = 0; ss < SB; ss += 4) {
-      float4 w4;
-      w4.x = (ss + 0 < t || (!strict && ss + 0 == t)) ? acc[gidx][ss + 0] : 0.f;
-      w4.y = (ss + 1 < t || (!strict && ss + 1 == t)) ? acc[gidx][ss + 1] : 0.f;
-      w4.z = (ss + 2 < t || (!strict && ss + 2 == t)) ? acc[gidx][ss + 2] : 0.f;
-      w4.w = (ss + 3 < t || (!strict && ss + 3 == t)) ? acc[gidx][ss + 3] : 0.f;
-      *reinterpret_cast<float4*>(o + ss) = w4;
+    for (int ss = 0; ss < 8; ++ss) {
+      a8[ss] = (ss < t || (!strict && ss == t)) ? acc[gidx][ss] : 0.f;
+      b8[ss] = (ss + 8 < t || (!strict && ss + 8 == t)) ? acc[gidx][ss + 8] : 0.f;
     }
+    sq_put(img, Cs, SB * J + t, SB * J, a8);
+    sq_put(img, Cs, SB * J + t, SB * J + 8, b8);
   }
 }
 
@@ -437,121 +455,107 @@ __global__ void __launch_bounds__(128) gram_diag_kernel(ChunkParams p) {
 template <int NS>
 __global__ void __launch_bounds__(256, 1) solve_kernel(ChunkParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs, nb = Cs / SB;
   constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
-  float* Tf = reinterpret_cast<float*>(sm);  // [Cs][Cs]
-  const uint32_t base = smem_u32(sm) + 128u * 128u * 4u;
-  constexpr uint32_t TB = 128u * 128u * 2u;
-  const Tile TA{base, base + TB, 128u, (uint32_t)Cs * 16u};           // K-major A tiles (K = Cs)
-  const Tile TBt{base + 2 * TB, base + 3 * TB, 128u, (uint32_t)Cs * 16u};  // MN-major B tiles (K = Cs)
-  const float* M = p.gr + ((int64_t)blockIdx.x * 4 + 1) * Cs * Cs;
-  for (int x = tid; x < Cs * Cs; x += NT) Tf[x] = 0.f;
-  zero_smem(base, 4 * TB);
+  const uint32_t H = sq_half(Cs);
+  const uint32_t base = smem_u32(sm);
+  const Tile TM{base, base + H, 128u, (uint32_t)Cs * 16u};                 // M^ka image, K-major
+  const Tile TA{base + 2 * H, base + 3 * H, 128u, (uint32_t)Cs * 16u};     // T so far, K-major
+  const Tile TBt{base + 4 * H, base + 5 * H, 128u, (uint32_t)Cs * 16u};    // T so far / X, MN-major
+  float* leaf = reinterpret_cast<float*>(sm + 6 * H);                      // [nb][16][16]
+  const uint8_t* smc = sm;
+  if (tid == 0) mbar_init(&bar_cp, 1);
+  zero_smem(base + 2 * H, 4 * H);
   TcCta cta;
   cta.init(&tslot, &bar, 256);
+  if (tid == 0) {
+    mbar_expect_tx(&bar_cp, 2 * H);
+    bulk_g2s_big(base, p.gr + ((int64_t)blockIdx.x * 4 + 1) * sq_bytes(Cs), 2 * H, &bar_cp);
+  }
+  MmaSync drv{&bar, 0u, true};
+  drv.ok = __syncthreads_and(mbar_wait(&bar_cp, 0) ? 1 : 0) != 0;
+  // exact 16x16 leaves: column j of (I + M_JJ)^-1 by forward substitution
   {
     const int J = tid >> 4, j = tid & 15;
     if (J < nb) {
       float x[SB];
 #pragma unroll
       for (int i = 0; i < SB; ++i) x[i] = (i == j) ? 1.f : 0.f;
-      const float* Mb = M + (int64_t)(SB * J) * Cs + SB * J;
 #pragma unroll
       for (int i = 1; i < SB; ++i) {
         float acc = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < i; ++kk) acc += __ldg(Mb + i * Cs + kk) * x[kk];
+        for (int kk = 0; kk < i; ++kk) acc += sq_get(smc, Cs, SB * J + i, SB * J + kk) * x[kk];
         if (i > j) x[i] = -acc;
       }
 #pragma unroll
-      for (int i = 0; i < SB; ++i) Tf[(SB * J + i) * Cs + SB * J + j] = x[i];
+      for (int i = 0; i < SB; ++i) leaf[(J * SB + i) * SB + j] = x[i];
     }
   }
   __syncthreads();
-  MmaSync drv{&bar, 0u, true};
+  for (int x = tid; x < nb * SB * 2; x += NT) {  // leaves -> both tiles
+    const int J = x / (SB * 2), i = (x / 2) % SB, c8 = (x & 1) * 8;
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = leaf[(J * SB + i) * SB + c8 + e];
+    put_k(TA, SB * J + i, SB * J + c8, v);
+    put_mn(TBt, SB * J + i, SB * J + c8, v);
+  }
   const int t = tid & 127, wg = tid >> 7;
   for (int h = SB; h < Cs && drv.ok; h *= 2) {
-    // A = off-diagonal blocks (2m+1, 2m) of M (zeros elsewhere), K-major; B = Tcur, MN-major.
-    #pragma unroll 4
-    for (int x = tid; x < 128 * (Cs / 8); x += NT) {
-      const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
-      float v[8];
-      const bool on = r < Cs && ((r / h) & 1) && (c8 / h) == (r / h) - 1;
-      if (on) ld8f(M + (int64_t)r * Cs + c8, v);
-      else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = 0.f;
-      }
-      put_k(TA, r, c8, v);
-    }
-    #pragma unroll 4
-    for (int x = tid; x < Cs * (Cs / 8); x += NT) {
-      const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
-      float v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = Tf[r * Cs + c8 + j];
-      put_mn(TBt, r, c8, v);
-    }
+    // X = M (K-range = the even block) * T_even: only rows of the odd block are used
     const int nm = Cs / (2 * h);
     const uint32_t idh = idesc_bf16(128, h, 0, 1);
     drv.run([&] {
       for (int m = 0; m < nm; ++m)
-        mma_tiles(cta.tmem + 2 * m * h, sub_tile(TA, 2 * m * h, 0), sub_tile(TBt, 2 * m * h, 2 * m * h), h / 16, idh,
+        mma_tiles(cta.tmem + 2 * m * h, sub_tile(TM, 2 * m * h, 0), sub_tile(TBt, 2 * m * h, 2 * m * h), h / 16, idh,
                   NS, false);
     });
     if (!drv.ok) break;
-    // X (rows of odd blocks, columns of the preceding even block) -> B tile, MN-major.
-    {
-      const int m = t / (2 * h);
-      const bool odd = t < Cs && ((t / h) & 1);
-      for (int c = wg * 16; c < h; c += 32) {
-        float v[16];
-        tmem_ld16(cta.tmem + tmem_lane_base(warp) + 2 * m * h + c, v);
-        if (odd) {
-          float a[8], b8[8];
+    const int m = t / (2 * h);
+    const bool odd = t < Cs && ((t / h) & 1);
+    for (int c = wg * 16; c < h; c += 32) {  // X (odd rows, even-block columns) -> B tile
+      float v[16];
+      tmem_ld16(cta.tmem + tmem_lane_base(warp) + 2 * m * h + c, v);
+      if (odd) {
+        float a[8], b8[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) { a[j] = v[j]; b8[j] = v[8 + j]; }
-          put_mn(TBt, t, 2 * m * h + c, a);
-          put_mn(TBt, t, 2 * m * h + c + 8, b8);
-        }
+        for (int j = 0; j < 8; ++j) { a[j] = v[j]; b8[j] = v[8 + j]; }
+        put_mn(TBt, t, 2 * m * h + c, a);
+        put_mn(TBt, t, 2 * m * h + c + 8, b8);
       }
-    }
-    // A = Tcur, K-major.
-    #pragma unroll 4
-    for (int x = tid; x < Cs * (Cs / 8); x += NT) {
-      const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
-      float v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = Tf[r * Cs + c8 + j];
-      put_k(TA, r, c8, v);
     }
     drv.run([&] {
-      for (int m = 0; m < nm; ++m)
-        mma_tiles(cta.tmem + 128 + 2 * m * h, sub_tile(TA, (2 * m + 1) * h, 0),
-                  sub_tile(TBt, (2 * m + 1) * h, 2 * m * h), h / 16, idh, NS, false);
+      for (int mm = 0; mm < nm; ++mm)
+        mma_tiles(cta.tmem + 128 + 2 * mm * h, sub_tile(TA, (2 * mm + 1) * h, 0),
+                  sub_tile(TBt, (2 * mm + 1) * h, 2 * mm * h), h / 16, idh, NS, false);
     });
     if (!drv.ok) break;
-    {
-      const int m = t / (2 * h);
-      const bool odd = t < Cs && ((t / h) & 1);
-      for (int c = wg * 16; c < h; c += 32) {
-        float v[16];
-        tmem_ld16(cta.tmem + tmem_lane_base(warp) + 128 + 2 * m * h + c, v);
-        if (odd) {
+    for (int c = wg * 16; c < h; c += 32) {  // new lower-left block -T_odd X into both tiles
+      float v[16];
+      tmem_ld16(cta.tmem + tmem_lane_base(warp) + 128 + 2 * m * h + c, v);
+      if (odd) {
+        float a[8], b8[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) Tf[t * Cs + 2 * m * h + c + j] = -v[j];
-        }
+        for (int j = 0; j < 8; ++j) { a[j] = -v[j]; b8[j] = -v[8 + j]; }
+        put_k(TA, t, 2 * m * h + c, a);
+        put_k(TA, t, 2 * m * h + c + 8, b8);
+        put_mn(TBt, t, 2 * m * h + c, a);
+        put_mn(TBt, t, 2 * m * h + c + 8, b8);
       }
     }
-    __syncthreads();
   }
-  float* out = p.tt + (int64_t)blockIdx.x * Cs * Cs;
-  if (drv.ok)
-    for (int x = tid; x < Cs * Cs / 4; x += NT)
-      reinterpret_cast<float4*>(out)[x] = reinterpret_cast<const float4*>(Tf)[x];
+  __syncthreads();
+  // the K-major tile of T is exactly its workspace image
+  if (drv.ok) {
+    uint4* out = reinterpret_cast<uint4*>(p.tt + (int64_t)blockIdx.x * sq_bytes(Cs));
+    const uint4* src = reinterpret_cast<const uint4*>(sm + 2 * H);
+#pragma unroll 4
+    for (int x = tid; x < (int)(2 * H / 16); x += NT) out[x] = src[x];
+  }
   cta.finish();
 }
 
@@ -565,7 +569,7 @@ __global__ void __launch_bounds__(256, 1) solve_kernel(ChunkParams p) {
 template <int DK, int DV, typename T, int NS>
 __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
@@ -574,43 +578,44 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   constexpr uint32_t TBY = 128u * 128u * 2u;
   const uint32_t base = smem_u32(sm);
   const uint32_t kstride = (uint32_t)Cs * 16u;  // every tile here contracts over the Cs tokens
-  const Tile A{base, base + TBY, 128u, kstride};
+  const uint32_t H = sq_half(Cs);
+  const Tile A{base, base + H, 128u, kstride};  // bulk-copied Gram / T image, or a staged operand
   const Tile B1{base + 2 * TBY, base + 3 * TBY, 128u, kstride};
   const Tile B2{base + 4 * TBY, base + 5 * TBY, 128u, kstride};
-  zero_smem(base, 6 * TBY);
+  if (tid == 0) mbar_init(&bar_cp, 1);
+  zero_smem(base + 2 * TBY, 4 * TBY);
   TcCta cta;
   cta.init(&tslot, &bar, 512);
   const float* dec = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
   const float* gam = dec + 2 * Cs * DK;
   const float* gsuf = dec + 3 * Cs * DK;
-  const float* G = p.gr + (int64_t)blockIdx.x * 4 * Cs * Cs;
-  const float* Tm = p.tt + (int64_t)blockIdx.x * Cs * Cs;
+  const uint8_t* G = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
+  const uint8_t* Tm = p.tt + (int64_t)blockIdx.x * sq_bytes(Cs);
   const Rows<T> rows{p, s.b, s.h};
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
-  const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroup takes alternate 16-column chunks
+  const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups take alternate 16-column chunks
   constexpr uint32_t cW = 0, cZ = 128, cUt = 256, cPhi = 0, cPsi = 128, cOl = 256, cQ = 384;
-
-  auto stage_k_matrix = [&](const Tile& dst, const float* src, float sign) {  // rows t, K = s (Cs x Cs)
-    #pragma unroll 4
-    for (int x = tid; x < Cs * (Cs / 8); x += NT) {
-      const int r = x / (Cs / 8), c8 = (x % (Cs / 8)) * 8;
-      float v[8];
-      ld8f(src + (int64_t)r * Cs + c8, v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] *= sign;
-      put_k(dst, r, c8, v);
+  uint32_t cp_phase = 0;
+  // A <- a Gram or T image (one bulk copy); the MMA that last read A has completed.
+  auto load_img = [&](const uint8_t* img) {
+    if (tid == 0) {
+      mbar_expect_tx(&bar_cp, 2 * H);
+      bulk_g2s_big(base, img, 2 * H, &bar_cp);
     }
+    const bool ok = mbar_wait(&bar_cp, cp_phase);
+    cp_phase ^= 1u;
+    if (!ok) drv.ok = false;
   };
-  // TMEM columns [col, col+n) of this thread's row -> MN-major B tile row t.
-  auto tmem_to_b = [&](const Tile& dst, uint32_t col, int n) {
+  // TMEM columns [col, col+n) of this thread's row (times sign) -> MN-major B tile row t.
+  auto tmem_to_b = [&](const Tile& dst, uint32_t col, int n, float sign) {
     for (int c = wg * 16; c < n; c += 32) {
       float v[16];
       tmem_ld16(cta.tmem + lane + col + c, v);
       if (t < Cs) {
         float a[8], b8[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) { a[j] = v[j]; b8[j] = v[8 + j]; }
+        for (int j = 0; j < 8; ++j) { a[j] = sign * v[j]; b8[j] = sign * v[8 + j]; }
         put_mn(dst, t, c, a);
         put_mn(dst, t, c + 8, b8);
       }
@@ -618,7 +623,7 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   };
   // (X * Gsuf)^T as an MN-major A operand (M = channel, K = token), scaled by sign.
   auto stage_suffixed = [&](bool erase, float sign) {
-    #pragma unroll 4
+#pragma unroll 4
     for (int x = tid; x < Cs * (DK / 8); x += NT) {
       const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float xx[8], gs[8];
@@ -633,8 +638,7 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   const uint32_t idK = idesc_bf16(128, DK, 0, 1), idV = idesc_bf16(128, DV, 0, 1);
   const uint32_t idKt = idesc_bf16(128, DK, 1, 1), idVt = idesc_bf16(128, DV, 1, 1);
   // ---- phase 1: W = T (K*Gam), Z = M^kk U, Ut = T Z
-  stage_k_matrix(A, Tm, 1.f);
-  #pragma unroll 4
+#pragma unroll 4
   for (int x = tid; x < Cs * (DK / 8); x += NT) {  // B1 = K*Gam (K = token, N = channel)
     const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
     float kk[8], gm[8];
@@ -644,18 +648,19 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
     for (int j = 0; j < 8; ++j) kk[j] *= gm[j];
     put_mn(B1, r, c8, kk);
   }
-  #pragma unroll 4
+#pragma unroll 4
   for (int x = tid; x < Cs * (DV / 8); x += NT) {  // B2 = U
     const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
     float uu[8];
     rows.u(s.tok0 + r, c8, uu);
     put_mn(B2, r, c8, uu);
   }
+  load_img(Tm);
   drv.run([&] { mma_tiles(cta.tmem + cW, A, B1, Cs / 16, idK, NS, false); });
-  stage_k_matrix(A, G + 0 * Cs * Cs, 1.f);  // M^kk
+  load_img(G + 0 * sq_bytes(Cs));  // M^kk
   drv.run([&] { mma_tiles(cta.tmem + cZ, A, B2, Cs / 16, idV, NS, false); });
-  tmem_to_b(B1, cZ, DV);
-  stage_k_matrix(A, Tm, 1.f);
+  tmem_to_b(B1, cZ, DV, 1.f);
+  load_img(Tm);
   drv.run([&] { mma_tiles(cta.tmem + cUt, A, B1, Cs / 16, idV, NS, false); });
   if (p.wsave) {  // the backward pass reuses W and Ut
     float* wo = p.wsave + (int64_t)blockIdx.x * Cs * DK;
@@ -677,20 +682,20 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
           *reinterpret_cast<float4*>(uo + t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
   }
-  // ---- phase 2 with W in B1: Phi = Diag(Gam_C) - (A*Gsuf)^T W, Q' = Qt*Gam - N^qa W
-  tmem_to_b(B1, cW, DK);
+  // ---- phase 2 with W in B1: Phi = Diag(Gam_C) - (A*Gsuf)^T W, N^qa W (Q' = Qt*Gam - N^qa W in the epilogue)
+  tmem_to_b(B1, cW, DK, 1.f);
   stage_suffixed(true, -1.f);
   drv.run([&] { mma_tiles(cta.tmem + cPhi, A, B1, Cs / 16, idKt, NS, false); });
-  stage_k_matrix(A, G + 3 * Cs * Cs, -1.f);  // -N^qa
+  load_img(G + 3 * sq_bytes(Cs));  // N^qa
   drv.run([&] { mma_tiles(cta.tmem + cQ, A, B1, Cs / 16, idK, NS, false); });
-  // ---- phase 3 with Ut in B1, U in B2: Oloc = N^qk U - N^qa Ut, Psi = (K*Gsuf)^T U - (A*Gsuf)^T Ut
-  tmem_to_b(B1, cUt, DV);
-  drv.run([&] { mma_tiles(cta.tmem + cOl, A, B1, Cs / 16, idV, NS, false); });  // A still holds -N^qa
-  stage_k_matrix(A, G + 2 * Cs * Cs, 1.f);                                         // N^qk
+  // ---- phase 3 with -Ut in B1, U in B2: Oloc = N^qa (-Ut) + N^qk U, Psi = (K*Gsuf)^T U + (A*Gsuf)^T (-Ut)
+  tmem_to_b(B1, cUt, DV, -1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cOl, A, B1, Cs / 16, idV, NS, false); });  // A still holds N^qa
+  load_img(G + 2 * sq_bytes(Cs));                                                 // N^qk
   drv.run([&] { mma_tiles(cta.tmem + cOl, A, B2, Cs / 16, idV, NS, true); });
   stage_suffixed(false, 1.f);
   drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B2, Cs / 16, idVt, NS, false); });
-  stage_suffixed(true, -1.f);
+  stage_suffixed(true, 1.f);
   drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B1, Cs / 16, idVt, NS, true); });
   // ---- epilogue: Phi, Q' -> map image (bf16 hi/lo tiles); Psi -> 32-column slabs; Oloc -> row-major
   const MapGeom mg = map_geom(DK, Cs);
@@ -731,7 +736,7 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
         rows.qt(s.tok0 + t, c + h8, qq);
         ld8f(gam + t * DK + c + h8, gm);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[h8 + j] += qq[j] * gm[j];
+        for (int j = 0; j < 8; ++j) v[h8 + j] = qq[j] * gm[j] - v[h8 + j];
       }
       float a8[8], b8[8];
 #pragma unroll

@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
 template <int DK, int DV, typename T, int NS>
 __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
@@ -294,23 +294,35 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   const uint32_t base = smem_u32(sm);
   constexpr uint32_t TB = 128u * 128u * 2u;
   const uint32_t ks = (uint32_t)Cs * 16u;
-  const Tile A{base, base + TB, 128u, ks};             // A over tokens (K = Cs)
-  const Tile Ak{base, base + TB, 128u, DK * 16u};      // A over channels (K = DK)
+  const uint32_t H = sq_half(Cs);
+  const Tile AT{base, base + H, ks, 128u};         // transposed view of a Gram / T image: M = column, K = row
+  const Tile Ak{base, base + TB, 128u, DK * 16u};  // staged operand over channels (K = DK)
   const Tile B1{base + 2 * TB, base + 3 * TB, 128u, ks};
   const Tile B2{base + 4 * TB, base + 5 * TB, 128u, DK * 16u};
   const Tile B3{base + 4 * TB, base + 5 * TB, 128u, ks};
-  zero_smem(base, 6 * TB);
+  if (tid == 0) mbar_init(&bar_cp, 1);
+  zero_smem(base + 2 * TB, 4 * TB);
   TcCta cta;
   cta.init(&tslot, &bar, 512);
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
   const Rows<T> rows{p, s.b, s.h};
-  const float* G = p.gr + u * 4 * Cs * Cs;
+  const uint8_t* G = p.gr + u * 4 * sq_bytes(Cs);
   const float* gsuf = p.dec + (u * 4 + 3) * Cs * DK;
   const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
   constexpr uint32_t cP = 0, cU = 128, cZ = 256;
+  uint32_t cp_phase = 0;
+  auto load_img = [&](const uint8_t* img) {
+    if (tid == 0) {
+      mbar_expect_tx(&bar_cp, 2 * H);
+      bulk_g2s_big(base, img, 2 * H, &bar_cp);
+    }
+    const bool ok = mbar_wait(&bar_cp, cp_phase);
+    cp_phase ^= 1u;
+    if (!ok) drv.ok = false;
+  };
   // B1 = dO (K = token, N = value column)
-  #pragma unroll 4
+#pragma unroll 4
   for (int x = tid; x < Cs * (DV / 8); x += NT) {
     const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
     const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
@@ -324,14 +336,14 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
     put_mn(B1, r, c8, dd);
   }
   stage_rows_mn(B2, q.dSC + u * DK * DV, DK, DV, DV, 1.f);  // dS_C (K = channel)
-  stage_rows_mn(A, G + 3 * Cs * Cs, Cs, Cs, Cs, -1.f);      // (-N^qa)^T: K = t, M = s
   const uint32_t idT = idesc_bf16(128, DV, 1, 1), idK = idesc_bf16(128, DV, 0, 1);
-  drv.run([&] { mma_tiles(cta.tmem + cP, A, B1, Cs / 16, idT, NS, false); });
-  stage_rows_mn(A, G + 2 * Cs * Cs, Cs, Cs, Cs, 1.f);       // N^qk^T
-  drv.run([&] { mma_tiles(cta.tmem + cU, A, B1, Cs / 16, idT, NS, false); });
-  // -(A*Gsuf) and (K*Gsuf): rows s, K = channel (K-major)
-  auto stage_suf = [&](bool erase, float sign) {
-    #pragma unroll 4
+  load_img(G + 3 * sq_bytes(Cs));  // N^qa -> -dP (partial): N^qa^T dO
+  drv.run([&] { mma_tiles(cta.tmem + cP, AT, B1, Cs / 16, idT, NS, false); });
+  load_img(G + 2 * sq_bytes(Cs));  // N^qk -> dU: N^qk^T dO
+  drv.run([&] { mma_tiles(cta.tmem + cU, AT, B1, Cs / 16, idT, NS, false); });
+  // (A*Gsuf) and (K*Gsuf): rows s, K = channel (K-major)
+  auto stage_suf = [&](bool erase) {
+#pragma unroll 4
     for (int x = tid; x < Cs * (DK / 8); x += NT) {
       const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
       float xx[8], gs[8];
@@ -339,28 +351,28 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
       else rows.k(s.tok0 + r, c8, xx);
       ld8f(gsuf + r * DK + c8, gs);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) xx[j] *= sign * gs[j];
+      for (int j = 0; j < 8; ++j) xx[j] *= gs[j];
       put_k(Ak, r, c8, xx);
     }
   };
-  stage_suf(true, -1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cP, Ak, B2, DK / 16, idK, NS, true); });
-  stage_suf(false, 1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cU, Ak, B2, DK / 16, idK, NS, true); });
-  // dP (TMEM) -> B3 (K = token), then dZ = T^T dP
+  stage_suf(true);
+  drv.run([&] { mma_tiles(cta.tmem + cP, Ak, B2, DK / 16, idK, NS, true); });  // -dP = N^qa^T dO + (A*Gsuf) dS_C
+  stage_suf(false);
+  drv.run([&] { mma_tiles(cta.tmem + cU, Ak, B2, DK / 16, idK, NS, true); });  // + (K*Gsuf) dS_C
+  // dP (TMEM, negated) -> B3 (K = token), then dZ = T^T dP
   for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cP + c, v);
     if (t < Cs) {
       float a8[8], b8[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
+      for (int j = 0; j < 8; ++j) { a8[j] = -v[j]; b8[j] = -v[8 + j]; }
       put_mn(B3, t, c, a8);
       put_mn(B3, t, c + 8, b8);
     }
   }
-  stage_rows_mn(A, p.tt + u * Cs * Cs, Cs, Cs, Cs, 1.f);  // T^T: K = t, M = s
-  drv.run([&] { mma_tiles(cta.tmem + cZ, A, B3, Cs / 16, idT, NS, false); });
+  load_img(p.tt + u * sq_bytes(Cs));  // T^T
+  drv.run([&] { mma_tiles(cta.tmem + cZ, AT, B3, Cs / 16, idT, NS, false); });
   float* dZo = q.dZ + u * Cs * DV;
   for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
@@ -377,8 +389,8 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
           *reinterpret_cast<float4*>(dZo + t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
   }
-  stage_rows_mn(A, G + 0 * Cs * Cs, Cs, Cs, Cs, 1.f);  // M^kk^T
-  drv.run([&] { mma_tiles(cta.tmem + cU, A, B3, Cs / 16, idT, NS, true); });
+  load_img(G + 0 * sq_bytes(Cs));  // M^kk^T
+  drv.run([&] { mma_tiles(cta.tmem + cU, AT, B3, Cs / 16, idT, NS, true); });
   float* dUo = q.dU + u * Cs * DV;
   for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
@@ -634,25 +646,73 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
       mma_tiles(cta.tmem + 3 * Cs + c, sub_tile(A2, k0, 0), sub_tile(Bm[3], k0, 0), ks, id16m, NS, true);
     });
   }
-  // ---- epilogue: lane = channel i; scale by pre (left) or suf (right); blocks
-  // without contributions (J = 0 left, I = nb-1 right) are written as zeros.
-  const int i = tid & 127, wg = tid >> 7;  // TMEM lane = key channel; warpgroups split the columns
+  // ---- epilogue, one 16-token block at a time; lane = key channel i.
+  // Off-diagonal parts come from TMEM, scaled by pre (left) or suf (right);
+  // blocks without them (J = 0 left, J = nb-1 right) contribute zero. The
+  // block's own 16x16 diagonal part is added exactly on the CUDA cores with
+  // running products: for s <= t in the block, Gam_{t<-s} = prod_{u=s+1..t} alpha_u,
+  //   dK_left_t  += (dM^kk_ts k_s + dM^ka_ts a_s) Gam      dQ_left_t += (dN^qk_ts k_s + dN^qa_ts a_s) Gam
+  //   dK_right_s += (dM^kk_ts k_t + dN^qk_ts qt_t) Gam     dA_right_s += (dM^ka_ts k_t + dN^qa_ts qt_t) Gam
+  const int i = tid & 127, wg = tid >> 7;  // TMEM lane = key channel; warpgroups take alternate blocks
+  float* dgd = reinterpret_cast<float*>(sm + 4 * AB + 8 * BB + nb * DK * 4);  // [nb][4][16][16]
+#pragma unroll 4
+  for (int x = tid; x < nb * 4 * SB * SB; x += NT) {
+    const int J = x / (4 * SB * SB), g = (x / (SB * SB)) % 4, tt = (x / SB) % SB, ss = x % SB;
+    dgd[x] = dG[((int64_t)g * Cs + SB * J + tt) * Cs + SB * J + ss];
+  }
+  __syncthreads();
   float* gl = q.gl + u * 4 * Cs * DK;
-  for (int reg = 0; reg < 4; ++reg) {
-    const bool left = reg < 2;
-    const float* sc = left ? pre : suf;
-    for (int c = wg * 16; c < Cs; c += 32) {
-      float v[16];
-      tmem_ld16(cta.tmem + tmem_lane_base(warp) + reg * Cs + c, v);
-      const int blk = c / SB;
-      const bool zero = left ? (blk == 0) : (blk == nb - 1);
-      if (i < DK && drv.ok) {
+  const int ic = i < DK ? i : DK - 1;
+  const float rr = p.r[(int64_t)s.h * DK + ic];
+  const int64_t kstride = (int64_t)p.H * DK;
+  for (int J = wg; J < nb; J += 2) {
+    float raw[4][SB];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int tt = c + j;
-          gl[((int64_t)reg * Cs + tt) * DK + i] = zero ? 0.f : v[j] * sc[tt * DK + i];
-        }
+    for (int reg = 0; reg < 4; ++reg) tmem_ld16(cta.tmem + tmem_lane_base(warp) + reg * Cs + SB * J, raw[reg]);
+    if (i >= DK || !drv.ok) continue;
+    float K[SB], Av[SB], Q[SB], al[SB];
+    const int64_t o0 = toff(p, s.b, s.tok0 + SB * J, s.h, DK) + i;
+#pragma unroll
+    for (int tt = 0; tt < SB; ++tt) {
+      const int64_t o = o0 + tt * kstride;
+      const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
+      K[tt] = kk;
+      Av[tt] = Elt<T>::ld(static_cast<const T*>(p.e) + o) * kk;
+      Q[tt] = rr * Elt<T>::ld(static_cast<const T*>(p.g) + o) * Elt<T>::ld(static_cast<const T*>(p.q) + o);
+      al[tt] = expf(__ldg(p.la + o));
+    }
+    float dKl[SB], dQl[SB], dKr[SB], dAr[SB];
+#pragma unroll
+    for (int tt = 0; tt < SB; ++tt) {
+      const int t = SB * J + tt;
+      const float pr = pre[t * DK + i], sf = suf[t * DK + i];
+      dKl[tt] = J == 0 ? 0.f : raw[0][tt] * pr;
+      dQl[tt] = J == 0 ? 0.f : raw[1][tt] * pr;
+      dKr[tt] = J == nb - 1 ? 0.f : raw[2][tt] * sf;
+      dAr[tt] = J == nb - 1 ? 0.f : raw[3][tt] * sf;
+    }
+    const float* dg = dgd + J * 4 * SB * SB;
+#pragma unroll
+    for (int ss = 0; ss < SB; ++ss) {
+      float gm = 1.f;
+#pragma unroll
+      for (int tt = ss; tt < SB; ++tt) {
+        if (tt > ss) gm *= al[tt];
+        const float mkk = dg[(0 * SB + tt) * SB + ss], mka = dg[(1 * SB + tt) * SB + ss];
+        const float nqk = dg[(2 * SB + tt) * SB + ss], nqa = dg[(3 * SB + tt) * SB + ss];
+        dKl[tt] += (mkk * K[ss] + mka * Av[ss]) * gm;
+        dQl[tt] += (nqk * K[ss] + nqa * Av[ss]) * gm;
+        dKr[ss] += (mkk * K[tt] + nqk * Q[tt]) * gm;
+        dAr[ss] += (mka * K[tt] + nqa * Q[tt]) * gm;
       }
+    }
+#pragma unroll
+    for (int tt = 0; tt < SB; ++tt) {
+      const int64_t o = (int64_t)(SB * J + tt) * DK + i;
+      gl[0 * Cs * DK + o] = dKl[tt];
+      gl[1 * Cs * DK + o] = dQl[tt];
+      gl[2 * Cs * DK + o] = dKr[tt];
+      gl[3 * Cs * DK + o] = dAr[tt];
     }
   }
   cta.finish();
