@@ -57,8 +57,9 @@ def kernel_model(C, dk, dv, es):
     tri = C * C / 2
     m = {}
     m["decay"] = (0.0, C * dk * f4 + 4 * C * dk * f4)
-    m["gram_off"] = (4 * 2 * (tri - C * 8) * dk, 4 * C * dk * es + 2 * C * dk * f4 + 4 * C * C * f4)
-    m["gram_diag"] = (4 * 2 * C * 8.5 * dk, 4 * C * dk * es + C * dk * f4 + 4 * C * 16 * f4)
+    # off-diagonal blocks (tensor cores) + the exact 16x16 diagonal blocks (CUDA cores)
+    m["gram_off"] = (4 * 2 * (tri - C * 8) * dk + 4 * 2 * C * 8.5 * dk,
+                     4 * C * dk * es + 3 * C * dk * f4 + 4 * C * C * f4)
     m["solve"] = (C ** 3 / 3.0, 2 * C * C * f4)
     maps_fl = 2 * (tri * dk + tri * dv + tri * dv + C * dk * dk + tri * dk + 2 * tri * dv + 2 * C * dk * dv)
     m["maps"] = (maps_fl, 4 * C * C * f4 + 6 * C * dk * es + 2 * C * dk * f4 + (dk + C) * (dk + dv) * f4)
@@ -70,8 +71,7 @@ def kernel_model(C, dk, dv, es):
                    3 * C * C * f4 + 2 * C * dv * es + dk * dv * f4 + 2 * C * dk * es + 2 * C * dv * f4)
     m["bwd_grads"] = (2 * (4 * C * dk * dv + 4 * tri * dv),
                       4 * C * dv * f4 + 2 * dk * dv * f4 + 2 * C * dv * es + 4 * C * dk * f4 + 4 * C * C * f4)
-    m["bwd_gram_off"] = (4 * 2 * 2 * (tri - C * 8) * dk, 4 * C * C * f4 + 4 * C * dk * es + 2 * C * dk * f4 + 4 * C * dk * f4)
-    m["bwd_gram_diag"] = (4 * 2 * 2 * C * 8.5 * dk, 4 * C * 16 * f4 + 4 * C * dk * es + 8 * C * dk * f4)
+    m["bwd_gram_off"] = (4 * 2 * 2 * (tri - C * 8) * dk + 4 * 2 * 2 * C * 8.5 * dk, 4 * C * C * f4 + 4 * C * dk * es + 2 * C * dk * f4 + 4 * C * dk * f4)
     m["bwd_final"] = (0.0, 14 * C * dk * f4 + 6 * C * dk * es + C * dv * f4 + 4 * C * dv * es)
     return m
 

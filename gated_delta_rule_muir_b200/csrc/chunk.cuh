@@ -27,16 +27,17 @@
 // tensor-core GEMMs of pivot-scaled operands; the 16x16 diagonal blocks are
 // computed exactly on the CUDA cores with running products.
 //
-// Kernels (one CTA of 128 threads per (batch, head, chunk) unless noted):
+// Kernels (one CTA per (batch, head, unit of Cs = min(chunk, 128) tokens) unless noted):
 //   decay_kernel      pre, suf, Gam_t, Gsuf_t            -> workspace
-//   gram_off_kernel   off-diagonal blocks of the 4 Grams (tcgen05)
-//   gram_diag_kernel  diagonal 16x16 blocks (CUDA cores), one CTA per block
+//   gram_off_kernel   the 4 Grams: off-diagonal blocks on tcgen05, while the
+//                     exact 16x16 diagonal blocks run on the CUDA cores
 //   solve_kernel      T: exact 16x16 leaves, then recursive 2x2 block merges
 //                     T21 = -T22 M21 T11 on tcgen05 (block-Neumann recursion)
 //   maps_kernel       W, Ut, Phi, Psi, Q', Oloc (tcgen05)  -> workspace
 //   compose_kernel    (chunk 256) composes two 128-token half-chunk maps
 //   scan_kernel       sequential over chunks per (batch, head, 32-column slab):
-//                     [S_C; O] = [Phi; Q'] S0 + [Psi; Oloc], y = z*O (tcgen05)
+//                     S_C = Phi S0 + Psi (tcgen05), states -> workspace
+//   out_kernel        chunk-parallel y = z * (Q' S0 + Oloc) (tcgen05)
 #pragma once
 
 #include "tc.cuh"
@@ -275,6 +276,7 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
   constexpr int NT = 256;
+  constexpr int CH = DK / 16;  // channels per thread in the diagonal blocks
   const int Cs = p.Cs, nb = Cs / SB;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -285,14 +287,85 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
   const Tile RK{base + 4 * LB, base + 4 * LB + RB, 128u, DK * 16u};
   const Tile RA{base + 4 * LB + 2 * RB, base + 4 * LB + 3 * RB, 128u, DK * 16u};
   float* midtab = reinterpret_cast<float*>(sm + 4 * LB + 4 * RB);  // [nb][DK]
+  float* drow = midtab + nb * DK;                                    // [4][16][DK]: k, qt, a, alpha of one block
   zero_smem(base, 4 * LB);
   TcCta cta;
   cta.init(&tslot, &bar, tmem_cols_for(4 * Cs));
   const float* pre = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
   const float* suf = pre + Cs * DK;
   const Rows<T> rows{p, s.b, s.h};
+  uint8_t* out = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
   MmaSync drv{&bar, 0u, true};
   const uint32_t id = idesc_bf16(128, SB, 0, 0);
+
+  // Diagonal 16x16 blocks, exactly, on the CUDA cores: rows of block J -> drow.
+  auto load_block = [&](int J) {
+    for (int x = tid; x < SB * (DK / 8); x += NT) {
+      const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      const int64_t tok = s.tok0 + SB * J + rr;
+      float kk[8], aa[8], qq[8], la[8];
+      rows.k(tok, c8, kk);
+      rows.a(tok, c8, aa);
+      rows.qt(tok, c8, qq);
+      ld8f(p.la + toff(p, s.b, tok, s.h, DK) + c8, la);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        drow[(0 * SB + rr) * DK + c8 + j] = kk[j];
+        drow[(1 * SB + rr) * DK + c8 + j] = qq[j];
+        drow[(2 * SB + rr) * DK + c8 + j] = aa[j];
+        drow[(3 * SB + rr) * DK + c8 + j] = expf(la[j]);
+      }
+    }
+  };
+  // thread = (row t, channel group cg of CH channels); for s = t, t-1, ... the
+  // running product Gam_{t<-s} = Gam_{t<-s+1} alpha_{s+1} scales both right
+  // operands; the 64 partial sums are reduced over the 16 lanes of the row by
+  // recursive halving, after which lane cg holds Gram cg/4, columns 4(cg%4)..+3.
+  auto diag_block = [&](int J) {
+    const int t = tid >> 4, cg = tid & 15, c0 = cg * CH;
+    float xk[CH], xq[CH], gm[CH];
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      xk[j] = drow[(0 * SB + t) * DK + c0 + j];
+      xq[j] = drow[(1 * SB + t) * DK + c0 + j];
+      gm[j] = 1.f;
+    }
+    float v[64];
+#pragma unroll
+    for (int ss = SB - 1; ss >= 0; --ss) {
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      if (ss <= t) {
+#pragma unroll
+        for (int j = 0; j < CH; ++j) {
+          const float yk = drow[(0 * SB + ss) * DK + c0 + j] * gm[j], ya = drow[(2 * SB + ss) * DK + c0 + j] * gm[j];
+          a0 += xk[j] * yk; a1 += xk[j] * ya; a2 += xq[j] * yk; a3 += xq[j] * ya;
+        }
+#pragma unroll
+        for (int j = 0; j < CH; ++j) gm[j] *= drow[(3 * SB + ss) * DK + c0 + j];
+      }
+      v[0 * 16 + ss] = a0; v[1 * 16 + ss] = a1; v[2 * 16 + ss] = a2; v[3 * 16 + ss] = a3;
+    }
+#pragma unroll
+    for (int m = 8, n = 32; m >= 1; m >>= 1, n >>= 1) {
+      const bool up = (cg & m) != 0;
+#pragma unroll
+      for (int j = 0; j < n; ++j) {
+        const float send = up ? v[j] : v[j + n];
+        const float keep = up ? v[j + n] : v[j];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+      }
+    }
+    const int g = cg >> 2, c4 = (cg & 3) * 4;
+    const bool strict = g < 2;  // M^kk, M^ka exclude the diagonal
+    float w4[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int ss = c4 + j;
+      w4[j] = (ss < t || (!strict && ss == t)) ? v[j] : 0.f;
+    }
+    gput_k4(out + g * sq_bytes(Cs), sq_half(Cs), (uint32_t)Cs * 16u, SB * J + t, SB * J + c4, w4);
+  };
+
   for (int I = nb - 2; I >= 0 && drv.ok; --I) {
 #pragma unroll 4
     for (int x = tid; x < nb * DK; x += NT) {
@@ -313,6 +386,7 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
       put_k(RK, rr, c8, vk);
       put_k(RA, rr, c8, va);
     }
+    load_block(I + 1);
     __syncthreads();
     const int t0 = SB * (I + 1);
 #pragma unroll 2
@@ -335,17 +409,23 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
       put_k(LQ, t, c8, qv);
     }
     const uint32_t c0 = SB * I;
-    drv.run([&] {
-      mma_tiles(cta.tmem + c0, LK, RK, DK / 16, id, NS, false);
-      mma_tiles(cta.tmem + c0 + Cs, LK, RA, DK / 16, id, NS, false);
-      mma_tiles(cta.tmem + c0 + 2 * Cs, LQ, RK, DK / 16, id, NS, false);
-      mma_tiles(cta.tmem + c0 + 3 * Cs, LQ, RA, DK / 16, id, NS, false);
-    });
+    drv.run_overlap(
+        [&] {
+          mma_tiles(cta.tmem + c0, LK, RK, DK / 16, id, NS, false);
+          mma_tiles(cta.tmem + c0 + Cs, LK, RA, DK / 16, id, NS, false);
+          mma_tiles(cta.tmem + c0 + 2 * Cs, LQ, RK, DK / 16, id, NS, false);
+          mma_tiles(cta.tmem + c0 + 3 * Cs, LQ, RA, DK / 16, id, NS, false);
+        },
+        [&] { diag_block(I + 1); });
+  }
+  if (drv.ok) {
+    load_block(0);
+    __syncthreads();
+    diag_block(0);
   }
   // Epilogue: row t = TMEM lane; the two warpgroups take alternate 16-column chunks.
   const int t = tid & 127, wg = tid >> 7;
   const int J = t / SB;
-  uint8_t* out = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
   for (int gidx = 0; gidx < 4; ++gidx) {
     for (int c0 = wg * 16; c0 < Cs; c0 += 32) {
       float v[16];
@@ -364,85 +444,6 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
     }
   }
   cta.finish();
-}
-
-// ---------------------------------------------------------------------------
-// gram_diag_kernel: the 16x16 diagonal blocks, exactly, on CUDA cores.
-// One CTA per (unit, block); thread = (row t, channel group cg of DK/8 channels).
-// For s = t, t-1, ..., the running product Gam_{t<-s} = Gam_{t<-s+1} * alpha_{s+1}
-// multiplies both key rows; partial sums over the channel group are reduced
-// across the 8 lanes of the row.
-// ---------------------------------------------------------------------------
-template <int DK, typename T>
-__global__ void __launch_bounds__(128) gram_diag_kernel(ChunkParams p) {
-  constexpr int CH = DK / 8;
-  __shared__ __align__(16) float sk[SB][DK], sq[SB][DK], sa[SB][DK], sal[SB][DK];
-  const int Cs = p.Cs, nb = Cs / SB;
-  const int sid = blockIdx.x / nb, J = blockIdx.x % nb;
-  const SubIdx s = sub_of(p, sid, p.nsub, Cs);
-  const Rows<T> rows{p, s.b, s.h};
-  #pragma unroll 4
-  for (int x = threadIdx.x; x < SB * (DK / 8); x += 128) {
-    const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-    const int64_t tok = s.tok0 + SB * J + rr;
-    float kk[8], aa[8], qq[8], la[8];
-    rows.k(tok, c8, kk);
-    rows.a(tok, c8, aa);
-    rows.qt(tok, c8, qq);
-    ld8f(p.la + toff(p, s.b, tok, s.h, DK) + c8, la);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      sk[rr][c8 + j] = kk[j];
-      sa[rr][c8 + j] = aa[j];
-      sq[rr][c8 + j] = qq[j];
-      sal[rr][c8 + j] = expf(la[j]);
-    }
-  }
-  __syncthreads();
-  const int t = threadIdx.x >> 3, cg = threadIdx.x & 7;
-  const int c0 = cg * CH;
-  float xk[CH], xq[CH], gm[CH];
-#pragma unroll
-  for (int j = 0; j < CH; ++j) { xk[j] = sk[t][c0 + j]; xq[j] = sq[t][c0 + j]; gm[j] = 1.f; }
-  float acc[4][SB];
-#pragma unroll
-  for (int ss = SB - 1; ss >= 0; --ss) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    if (ss <= t) {
-#pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        const float yk = sk[ss][c0 + j] * gm[j], ya = sa[ss][c0 + j] * gm[j];
-        a0 += xk[j] * yk; a1 += xk[j] * ya; a2 += xq[j] * yk; a3 += xq[j] * ya;
-      }
-#pragma unroll
-      for (int j = 0; j < CH; ++j) gm[j] *= sal[ss][c0 + j];
-    }
-    acc[0][ss] = a0; acc[1][ss] = a1; acc[2][ss] = a2; acc[3][ss] = a3;
-  }
-#pragma unroll
-  for (int gidx = 0; gidx < 4; ++gidx)
-#pragma unroll
-    for (int ss = 0; ss < SB; ++ss) {
-      float v = acc[gidx][ss];
-      v += __shfl_xor_sync(0xffffffffu, v, 1);
-      v += __shfl_xor_sync(0xffffffffu, v, 2);
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      acc[gidx][ss] = v;
-    }
-#pragma unroll
-  for (int gidx = 0; gidx < 4; ++gidx) {
-    if (cg != gidx) continue;  // lane cg of the row writes Gram cg
-    uint8_t* img = p.gr + ((int64_t)sid * 4 + gidx) * sq_bytes(Cs);
-    const bool strict = gidx < 2;  // M^kk, M^ka exclude the diagonal
-    float a8[8], b8[8];
-#pragma unroll
-    for (int ss = 0; ss < 8; ++ss) {
-      a8[ss] = (ss < t || (!strict && ss == t)) ? acc[gidx][ss] : 0.f;
-      b8[ss] = (ss + 8 < t || (!strict && ss + 8 == t)) ? acc[gidx][ss + 8] : 0.f;
-    }
-    sq_put(img, Cs, SB * J + t, SB * J, a8);
-    sq_put(img, Cs, SB * J + t, SB * J + 8, b8);
-  }
 }
 
 // ---------------------------------------------------------------------------

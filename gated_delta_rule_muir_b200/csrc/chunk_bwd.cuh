@@ -27,7 +27,6 @@
 //   bwd_gram_off_kernel  off-diagonal blocks of the Gram backward (tcgen05):
 //                      dX with the pivot at the start of the row block,
 //                      dY with the pivot at the end of the column block
-//   bwd_gram_diag_kernel diagonal 16x16 blocks (CUDA cores, thread = channel)
 //   bwd_final_kernel   decay cotangents, reverse cumsum, chain rule to inputs
 #pragma once
 
@@ -716,64 +715,6 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_off_kernel(ChunkParams p, Bwd
     }
   }
   cta.finish();
-}
-
-// ---------------------------------------------------------------------------
-// bwd_gram_diag_kernel: diagonal 16x16 blocks of the Gram backward, exactly.
-// One CTA per (unit, block), thread = key channel (running products).
-// ---------------------------------------------------------------------------
-template <int DK, typename T>
-__global__ void __launch_bounds__(128) bwd_gram_diag_kernel(ChunkParams p, BwdBufs q) {
-  __shared__ float sdg[4][SB][SB];
-  const int Cs = p.Cs, nb = Cs / SB;
-  const int64_t u = blockIdx.x / nb;
-  const int J = blockIdx.x % nb;
-  const SubIdx s = sub_of(p, (int)u, p.nsub, Cs);
-  const int i = threadIdx.x;
-  #pragma unroll 4
-  for (int x = threadIdx.x; x < 4 * SB * SB; x += blockDim.x) {
-    const int g = x / (SB * SB), tt = (x / SB) % SB, ss = x % SB;
-    sdg[g][tt][ss] = q.dG[((u * 4 + g) * Cs + SB * J + tt) * Cs + SB * J + ss];
-  }
-  __syncthreads();
-  if (i >= DK) return;
-  float K[SB], A[SB], Q[SB], al[SB];
-  const int64_t stride = (int64_t)p.H * DK;
-  const int64_t o0 = toff(p, s.b, s.tok0 + SB * J, s.h, DK) + i;
-  const float rr = p.r[(int64_t)s.h * DK + i];
-#pragma unroll
-  for (int tt = 0; tt < SB; ++tt) {
-    const int64_t o = o0 + tt * stride;
-    const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
-    K[tt] = kk;
-    A[tt] = Elt<T>::ld(static_cast<const T*>(p.e) + o) * kk;
-    Q[tt] = rr * Elt<T>::ld(static_cast<const T*>(p.g) + o) * Elt<T>::ld(static_cast<const T*>(p.q) + o);
-    al[tt] = expf(p.la[o]);
-  }
-  float dKl[SB], dQl[SB], dKr[SB], dAr[SB];
-#pragma unroll
-  for (int tt = 0; tt < SB; ++tt) { dKl[tt] = 0.f; dQl[tt] = 0.f; dKr[tt] = 0.f; dAr[tt] = 0.f; }
-#pragma unroll
-  for (int ss = 0; ss < SB; ++ss) {
-    float gm = 1.f;
-#pragma unroll
-    for (int tt = ss; tt < SB; ++tt) {
-      if (tt > ss) gm *= al[tt];
-      const float mkk = sdg[0][tt][ss], mka = sdg[1][tt][ss], nqk = sdg[2][tt][ss], nqa = sdg[3][tt][ss];
-      dKl[tt] += (mkk * K[ss] + mka * A[ss]) * gm;
-      dQl[tt] += (nqk * K[ss] + nqa * A[ss]) * gm;
-      dKr[ss] += (mkk * K[tt] + nqk * Q[tt]) * gm;
-      dAr[ss] += (mka * K[tt] + nqa * Q[tt]) * gm;
-    }
-  }
-  float* gl = q.gl + u * 4 * Cs * DK + (int64_t)(SB * J) * DK + i;
-#pragma unroll
-  for (int tt = 0; tt < SB; ++tt) {
-    gl[(0 * Cs + tt) * DK] += dKl[tt];
-    gl[(1 * Cs + tt) * DK] += dQl[tt];
-    gl[(2 * Cs + tt) * DK] += dKr[tt];
-    gl[(3 * Cs + tt) * DK] += dAr[tt];
-  }
 }
 
 // ---------------------------------------------------------------------------

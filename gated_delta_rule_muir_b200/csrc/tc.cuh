@@ -220,6 +220,23 @@ __device__ __forceinline__ void gput_k(uint8_t* hi, uint32_t lo_off, uint32_t sb
   *reinterpret_cast<uint4*>(hi + lo_off + off) = l;
 }
 
+// 4 consecutive columns (c4 % 4 == 0) of row m into a global tile image.
+__device__ __forceinline__ void gput_k4(uint8_t* hi, uint32_t lo_off, uint32_t sbo, int m, int c4, const float (&x)[4]) {
+  uint2 h, l;
+  __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&h);
+  __nv_bfloat162* ll = reinterpret_cast<__nv_bfloat162*>(&l);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    const float2 f = __bfloat1622float2(b);
+    hh[i] = b;
+    ll[i] = __floats2bfloat162_rn(x[2 * i] - f.x, x[2 * i + 1] - f.y);
+  }
+  const uint32_t off = (uint32_t)(m >> 3) * sbo + (uint32_t)(c4 >> 3) * 128u + (uint32_t)(m & 7) * 16u + (uint32_t)(c4 & 7) * 2u;
+  *reinterpret_cast<uint2*>(hi + off) = h;
+  *reinterpret_cast<uint2*>(hi + lo_off + off) = l;
+}
+
 // ---- TMEM -> registers -----------------------------------------------------
 
 // Lane base of warp w's TMEM sub-partition.
@@ -274,6 +291,26 @@ struct MmaSync {
       issue();
       mma_commit(bar);
     }
+    const bool done = __syncthreads_and(mbar_wait(bar, phase) ? 1 : 0) != 0;
+    phase ^= 1u;
+    tc_fence_after();
+    ok = ok && done;
+    return done;
+  }
+
+  // Same, but all threads run `work` (which must not touch the staged operands
+  // or the accumulators of these MMAs) while the tensor core executes.
+  template <typename F, typename W>
+  __device__ __forceinline__ bool run_overlap(F issue, W work) {
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue();
+      mma_commit(bar);
+    }
+    work();
     const bool done = __syncthreads_and(mbar_wait(bar, phase) ? 1 : 0) != 0;
     phase ^= 1u;
     tc_fence_after();
