@@ -168,13 +168,17 @@ class Step:
         nb = muir.chunk_bwd_workspace_bytes(*self.args, C)
         self.ws = torch.empty(max(nf, nb), dtype=torch.uint8, device=d["q"].device)
         if not self.fwd_only:
-            self.grads = muir.chunk_bwd(*self.args, d["dy"], chunk=C, workspace=self.ws)
+            # the forward keeps its chunk maps for the backward (no recomputation)
+            muir.chunk_fwd(*self.args, chunk=C, y=self.y, S_T=self.S, workspace=self.ws, save_for_bwd=True)
+            self.grads = muir.chunk_bwd(*self.args, d["dy"], chunk=C, workspace=self.ws, use_saved=True)
 
     def __call__(self):
         C = WL["chunk"]
-        self.muir.chunk_fwd(*self.args, chunk=C, y=self.y, S_T=self.S, workspace=self.ws)
-        if not self.fwd_only:
-            self.muir.chunk_bwd(*self.args, self.d["dy"], chunk=C, workspace=self.ws, outputs=self.grads)
+        save = not self.fwd_only
+        self.muir.chunk_fwd(*self.args, chunk=C, y=self.y, S_T=self.S, workspace=self.ws, save_for_bwd=save)
+        if save:
+            self.muir.chunk_bwd(*self.args, self.d["dy"], chunk=C, workspace=self.ws, outputs=self.grads,
+                                use_saved=True)
 
 
 def time_steps(fn, steps, dist_on):
@@ -370,7 +374,9 @@ def main():
                        "dv": WL["dv"], "chunk": WL["chunk"], "global_batch": world * WL["B"], "seq_len": WL["T"],
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs larger than L2 (about 1.3 GB read per step)",
-                       "state": "fp32", "tensor_core": "tcgen05 kind::f16, 3-pass bf16 split, fp32 accumulate"},
+                       "state": "fp32", "tensor_core": "tcgen05 kind::f16, 3-pass bf16 split, fp32 accumulate",
+                       "step": "forward only" if Step.fwd_only else
+                       "forward (saving its chunk maps) + backward (using them)"},
             "gpu_launches": int(launches), "clocks": clk.summary()}
     # per-kernel device times (library events on the launch stream), same workload
     with muir.KernelTimer() as kt:

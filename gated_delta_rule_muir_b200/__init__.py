@@ -45,7 +45,7 @@ def _need(t, name, shape, dtype=None):
         raise ValueError(f"{name}: must be a contiguous CUDA tensor")
 
 
-def _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0):
+def _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0, flags=0):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
@@ -57,14 +57,14 @@ def _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0):
     _need(r, "r", (H, dk), torch.float32)
     if S0 is not None:
         _need(S0, "S0", (B, H, dk, dv), torch.float32)
-    a = N.ChunkArgs(B=B, T=T, H=H, dk=dk, dv=dv, chunk=chunk, dtype=_dtype_code(dt), reserved=0,
+    a = N.ChunkArgs(B=B, T=T, H=H, dk=dk, dv=dv, chunk=chunk, dtype=_dtype_code(dt), flags=flags,
                     q=_ptr(q), k=_ptr(k), v=_ptr(v), e=_ptr(e), w=_ptr(w), g=_ptr(g), z=_ptr(z),
                     log_alpha=_ptr(log_alpha), r=_ptr(r), S0=_ptr(S0))
     return a, (B, T, H, dk, dv, dt)
 
 
-def chunk_fwd_workspace_bytes(q, k, v, e, w, g, z, log_alpha, r, chunk, S0=None) -> int:
-    a, _ = _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0)
+def chunk_fwd_workspace_bytes(q, k, v, e, w, g, z, log_alpha, r, chunk, S0=None, save_for_bwd=False) -> int:
+    a, _ = _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0, N.MUIR_SAVE_FOR_BWD if save_for_bwd else 0)
     return int(N.load().muir_chunk_fwd_workspace(C.byref(a)))
 
 
@@ -82,16 +82,21 @@ def _workspace(nbytes, device, ws):
 
 
 def chunk_fwd(q, k, v, e, w, g, z, log_alpha, r, *, chunk=128, S0=None, want_state=True, y=None, S_T=None,
-              workspace=None, stream=None):
+              workspace=None, save_for_bwd=False, stream=None):
     """Chunkwise forward pass. Inputs [B,T,H,d] (fp32 or bf16; log_alpha fp32), r [H,dk] fp32.
-    Returns (y [B,T,H,dv], S_T [B,H,dk,dv] fp32 or None)."""
+    Returns (y [B,T,H,dv], S_T [B,H,dk,dv] fp32 or None). With save_for_bwd=True the
+    workspace (pass one, of chunk_bwd_workspace_bytes) keeps what chunk_bwd(use_saved=True)
+    needs."""
     lib = N.load()
-    a, (B, T, H, dk, dv, dt) = _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0)
+    flags = N.MUIR_SAVE_FOR_BWD if save_for_bwd else 0
+    a, (B, T, H, dk, dv, dt) = _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0, flags)
     if y is None:
         y = torch.empty(B, T, H, dv, dtype=dt, device=q.device)
     if want_state and S_T is None:
         S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     nbytes = int(lib.muir_chunk_fwd_workspace(C.byref(a)))
+    if save_for_bwd and workspace is None:
+        raise ValueError("save_for_bwd needs a workspace to keep (chunk_bwd_workspace_bytes)")
     ws = _workspace(nbytes, q.device, workspace)
     N.check(lib.muir_chunk_fwd(C.byref(a), _ptr(y), _ptr(S_T if want_state else None), _ptr(ws), nbytes,
                                _stream(stream)), "muir_chunk_fwd")
@@ -99,11 +104,15 @@ def chunk_fwd(q, k, v, e, w, g, z, log_alpha, r, *, chunk=128, S0=None, want_sta
 
 
 def chunk_bwd(q, k, v, e, w, g, z, log_alpha, r, dy, *, chunk=128, S0=None, dS_T=None, want_dS0=True,
-              want_dr=False, workspace=None, outputs=None, stream=None):
+              want_dr=False, workspace=None, outputs=None, use_saved=False, stream=None):
     """Backward pass of chunk_fwd. Returns a dict of gradients (dq, dk, dv, de, dw, dg, dz, dlog_alpha,
-    dS0, dr), each shaped like its input. `outputs` (a dict from an earlier call) is reused if given."""
+    dS0, dr), each shaped like its input. `outputs` (a dict from an earlier call) is reused if given.
+    use_saved=True: `workspace` is the one a chunk_fwd(save_for_bwd=True) of the same inputs filled."""
     lib = N.load()
-    a, (B, T, H, dk, dv, dt) = _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0)
+    if use_saved and workspace is None:
+        raise ValueError("use_saved needs the workspace of chunk_fwd(save_for_bwd=True)")
+    flags = N.MUIR_USE_SAVED if use_saved else 0
+    a, (B, T, H, dk, dv, dt) = _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0, flags)
     _need(dy, "dy", (B, T, H, dv), dt)
     if dS_T is not None:
         _need(dS_T, "dS_T", (B, H, dk, dv), torch.float32)

@@ -9,6 +9,7 @@ LIB_PATH = os.path.join(_PKG, "libmuir.so")
 
 MUIR_OK, MUIR_ERR_INVALID_ARG, MUIR_ERR_UNSUPPORTED, MUIR_ERR_WORKSPACE, MUIR_ERR_CUDA, MUIR_ERR_TIMEOUT = range(6)
 MUIR_F32, MUIR_BF16 = 0, 1
+MUIR_SAVE_FOR_BWD, MUIR_USE_SAVED = 1, 2
 
 ERROR_NAMES = {MUIR_ERR_INVALID_ARG: "invalid argument", MUIR_ERR_UNSUPPORTED: "unsupported",
                MUIR_ERR_WORKSPACE: "workspace", MUIR_ERR_CUDA: "CUDA error", MUIR_ERR_TIMEOUT: "device timeout"}
@@ -18,7 +19,7 @@ vp = C.c_void_p
 
 class ChunkArgs(C.Structure):
     _fields_ = [("B", C.c_int64), ("T", C.c_int64), ("H", C.c_int32), ("dk", C.c_int32), ("dv", C.c_int32),
-                ("chunk", C.c_int32), ("dtype", C.c_int32), ("reserved", C.c_int32),
+                ("chunk", C.c_int32), ("dtype", C.c_int32), ("flags", C.c_int32),
                 ("q", vp), ("k", vp), ("v", vp), ("e", vp), ("w", vp), ("g", vp), ("z", vp),
                 ("log_alpha", vp), ("r", vp), ("S0", vp)]
 

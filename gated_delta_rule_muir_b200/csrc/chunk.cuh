@@ -100,6 +100,25 @@ __device__ __forceinline__ int64_t toff(const ChunkParams& p, int b, int64_t tok
 
 __device__ __forceinline__ void ld8f(const float* p, float (&o)[8]) { Elt<float>::ld8(p, o); }
 
+// N consecutive floats from shared memory (p aligned to 4 * min(N, 4) bytes), vectorised.
+template <int N>
+__device__ __forceinline__ void lds_vec(const float* p, float (&o)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 a = reinterpret_cast<const float4*>(p)[i];
+      o[4 * i] = a.x; o[4 * i + 1] = a.y; o[4 * i + 2] = a.z; o[4 * i + 3] = a.w;
+    }
+  } else {
+    static_assert(N % 2 == 0, "even length");
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const float2 a = reinterpret_cast<const float2*>(p)[i];
+      o[2 * i] = a.x; o[2 * i + 1] = a.y;
+    }
+  }
+}
+
 __device__ __forceinline__ Tile sub_tile(const Tile& t, int k0, int mn0) {
   const uint32_t off = (uint32_t)(k0 >> 3) * t.lbo + (uint32_t)(mn0 >> 3) * t.sbo;
   return Tile{t.hi + off, t.lo + off, t.lbo, t.sbo};
@@ -309,12 +328,11 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
       rows.qt(tok, c8, qq);
       ld8f(p.la + toff(p, s.b, tok, s.h, DK) + c8, la);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        drow[(0 * SB + rr) * DK + c8 + j] = kk[j];
-        drow[(1 * SB + rr) * DK + c8 + j] = qq[j];
-        drow[(2 * SB + rr) * DK + c8 + j] = aa[j];
-        drow[(3 * SB + rr) * DK + c8 + j] = expf(la[j]);
-      }
+      for (int j = 0; j < 8; ++j) la[j] = expf(la[j]);
+      Elt<float>::st8(drow + (0 * SB + rr) * DK + c8, kk);
+      Elt<float>::st8(drow + (1 * SB + rr) * DK + c8, qq);
+      Elt<float>::st8(drow + (2 * SB + rr) * DK + c8, aa);
+      Elt<float>::st8(drow + (3 * SB + rr) * DK + c8, la);
     }
   };
   // thread = (row t, channel group cg of CH channels); for s = t, t-1, ... the
@@ -324,24 +342,26 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
   auto diag_block = [&](int J) {
     const int t = tid >> 4, cg = tid & 15, c0 = cg * CH;
     float xk[CH], xq[CH], gm[CH];
+    lds_vec(drow + (0 * SB + t) * DK + c0, xk);
+    lds_vec(drow + (1 * SB + t) * DK + c0, xq);
 #pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      xk[j] = drow[(0 * SB + t) * DK + c0 + j];
-      xq[j] = drow[(1 * SB + t) * DK + c0 + j];
-      gm[j] = 1.f;
-    }
+    for (int j = 0; j < CH; ++j) gm[j] = 1.f;
     float v[64];
 #pragma unroll
     for (int ss = SB - 1; ss >= 0; --ss) {
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       if (ss <= t) {
+        float yk[CH], ya[CH], al[CH];
+        lds_vec(drow + (0 * SB + ss) * DK + c0, yk);
+        lds_vec(drow + (2 * SB + ss) * DK + c0, ya);
+        lds_vec(drow + (3 * SB + ss) * DK + c0, al);
 #pragma unroll
         for (int j = 0; j < CH; ++j) {
-          const float yk = drow[(0 * SB + ss) * DK + c0 + j] * gm[j], ya = drow[(2 * SB + ss) * DK + c0 + j] * gm[j];
-          a0 += xk[j] * yk; a1 += xk[j] * ya; a2 += xq[j] * yk; a3 += xq[j] * ya;
+          yk[j] *= gm[j];
+          ya[j] *= gm[j];
+          a0 += xk[j] * yk[j]; a1 += xk[j] * ya[j]; a2 += xq[j] * yk[j]; a3 += xq[j] * ya[j];
+          gm[j] *= al[j];
         }
-#pragma unroll
-        for (int j = 0; j < CH; ++j) gm[j] *= drow[(3 * SB + ss) * DK + c0 + j];
       }
       v[0 * 16 + ss] = a0; v[1 * 16 + ss] = a1; v[2 * 16 + ss] = a2; v[3 * 16 + ss] = a3;
     }

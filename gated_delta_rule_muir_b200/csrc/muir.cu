@@ -89,7 +89,7 @@ bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 
 extern "C" {
 
-int muir_version(void) { return 100; }
+int muir_version(void) { return 101; }
 
 const char* muir_last_error(void) { return g_err.c_str(); }
 
@@ -271,6 +271,7 @@ extern "C" int muir_chunk_fwd_noalloc(const muir_chunk_args* a, void* y, float* 
   g_err.clear();
   int rc = validate_chunk_args(a, "chunk_fwd_noalloc");
   if (rc) return rc;
+  if (a->flags != 0) return fail(MUIR_ERR_INVALID_ARG, "chunk_fwd_noalloc: flags must be 0");
   const size_t need = muir_chunk_fwd_workspace(a);
   if (need > kNoAllocScratchBytes)
     return fail(MUIR_ERR_UNSUPPORTED,

@@ -58,6 +58,10 @@ extern "C" {
 #define MUIR_F32 0
 #define MUIR_BF16 1
 
+/* Bits of muir_chunk_args.flags (every other bit must be 0). */
+#define MUIR_SAVE_FOR_BWD 1 /* muir_chunk_fwd: also leave in the workspace what muir_chunk_bwd needs */
+#define MUIR_USE_SAVED 2    /* muir_chunk_bwd: the workspace holds it; skip the recomputation */
+
 /* Inputs of the chunkwise forward and backward passes. */
 typedef struct muir_chunk_args {
   int64_t B;      /* batch size (independent sequences) */
@@ -67,7 +71,7 @@ typedef struct muir_chunk_args {
   int32_t dv;     /* value dimension = columns of the state */
   int32_t chunk;  /* chunk length C of the chunkwise algorithm: 64, 128 or 256 */
   int32_t dtype;  /* MUIR_F32 or MUIR_BF16 */
-  int32_t reserved;
+  int32_t flags;  /* 0, or MUIR_SAVE_FOR_BWD (forward) / MUIR_USE_SAVED (backward) */
   const void* q;  /* [B,T,H,dk] query (activated, unit-norm) */
   const void* k;  /* [B,T,H,dk] key (activated, unit-norm) */
   const void* v;  /* [B,T,H,dv] value */
@@ -95,6 +99,19 @@ typedef struct muir_chunk_args {
 size_t muir_chunk_fwd_workspace(const muir_chunk_args* a);
 int muir_chunk_fwd(const muir_chunk_args* a, void* y, float* S_T, void* ws, size_t ws_bytes,
                    void* stream);
+/*
+ * Saving for the backward pass (a packaging choice of the library; the pages
+ * describe the backward only as a parallel update). With MUIR_SAVE_FOR_BWD in
+ * a->flags, muir_chunk_fwd needs a workspace of muir_chunk_fwd_workspace(a)
+ * bytes, which then equals muir_chunk_bwd_workspace(a), and leaves in it the
+ * per-unit decay products, Gram and T images, chunk maps, W, Ut and the
+ * unit-start states. It works on units of min(chunk, 128) tokens (the
+ * backward's units; for chunk 256 the state is carried every 128 tokens, which
+ * is the same map). A following muir_chunk_bwd with MUIR_USE_SAVED in its
+ * flags (otherwise the same arguments, the same inputs and the same workspace,
+ * untouched in between) then skips the forward recomputation. Memory: about
+ * 1.1 MB per 128 tokens per (batch, head) at dk = dv = 128.
+ */
 
 /* Gradients for muir_chunk_bwd. Outputs are written (not accumulated). */
 typedef struct muir_chunk_grads {
@@ -117,7 +134,9 @@ typedef struct muir_chunk_grads {
  * states are recomputed (a forward sweep into the workspace), then one reverse
  * sweep carries the state cotangent, and chunk-parallel kernels form every
  * input gradient (arXiv abstract: a parallel update for training).
- *   ws  workspace of at least muir_chunk_bwd_workspace(a) bytes.
+ *   ws  workspace of at least muir_chunk_bwd_workspace(a) bytes; with
+ *       MUIR_USE_SAVED in a->flags, the workspace a forward pass with
+ *       MUIR_SAVE_FOR_BWD filled (see above).
  */
 size_t muir_chunk_bwd_workspace(const muir_chunk_args* a);
 int muir_chunk_bwd(const muir_chunk_args* a, const muir_chunk_grads* gr, void* ws, size_t ws_bytes,
@@ -132,6 +151,8 @@ int muir_chunk_bwd(const muir_chunk_args* a, const muir_chunk_grads* gr, void* w
  * a 32 MiB scratch area compiled into the library (every GPU that loads the
  * library holds it until the process exits). The caller still passes inputs
  * and outputs exactly as for muir_chunk_fwd; this call allocates nothing.
+ *   - a->flags must be 0 (MUIR_ERR_INVALID_ARG otherwise): nothing can be saved
+ *     for a backward pass in the library's scratch.
  *   - Problems whose muir_chunk_fwd_workspace() exceeds 32 MiB are rejected
  *     with MUIR_ERR_UNSUPPORTED before any GPU work.
  *   - The first call on a device looks up the scratch address with

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version(lib):
-    assert lib.muir_version() == 100
+    assert lib.muir_version() == 101
 
 
 def test_decode_rejects_null_and_bad_sizes(lib):
@@ -76,7 +76,7 @@ def test_state_init_rejects_bad_args(lib):
 
 def _chunk_args(**kw):
     fake = C.c_void_p(1 << 20)
-    a = N.ChunkArgs(B=1, T=256, H=2, dk=32, dv=32, chunk=64, dtype=N.MUIR_F32, reserved=0,
+    a = N.ChunkArgs(B=1, T=256, H=2, dk=32, dv=32, chunk=64, dtype=N.MUIR_F32, flags=0,
                     q=fake, k=fake, v=fake, e=fake, w=fake, g=fake, z=None, log_alpha=fake, r=fake, S0=None)
     for k, v in kw.items():
         setattr(a, k, v)
@@ -90,6 +90,7 @@ def _chunk_args(**kw):
     ("dtype", 3, N.MUIR_ERR_UNSUPPORTED),
     ("q", None, N.MUIR_ERR_INVALID_ARG),
     ("log_alpha", C.c_void_p((1 << 20) + 8), N.MUIR_ERR_INVALID_ARG),
+    ("flags", 4, N.MUIR_ERR_INVALID_ARG),
 ])
 def test_chunk_fwd_rejects_bad_args(lib, field, value, code):
     a = _chunk_args(**{field: value})
@@ -112,3 +113,21 @@ def test_chunk_workspace_is_checked(lib):
 def test_empty_batch_is_a_no_op(lib):
     a = _chunk_args(B=0)
     assert lib.muir_chunk_fwd(C.byref(a), C.c_void_p(1 << 20), None, None, 0, None) == N.MUIR_OK
+
+
+def test_save_for_bwd_workspace_is_the_backward_one(lib):
+    a = _chunk_args(T=512)
+    plain = lib.muir_chunk_fwd_workspace(C.byref(a))
+    bwd = lib.muir_chunk_bwd_workspace(C.byref(a))
+    a.flags = N.MUIR_SAVE_FOR_BWD
+    assert lib.muir_chunk_fwd_workspace(C.byref(a)) == bwd > plain
+    y = C.c_void_p(1 << 20)
+    assert lib.muir_chunk_fwd(C.byref(a), y, None, C.c_void_p(1 << 20), bwd - 1, None) == N.MUIR_ERR_WORKSPACE
+    a.flags = N.MUIR_USE_SAVED
+    assert lib.muir_chunk_bwd_workspace(C.byref(a)) == bwd
+
+
+def test_noalloc_rejects_flags(lib):
+    a = _chunk_args(flags=N.MUIR_SAVE_FOR_BWD)
+    assert lib.muir_chunk_fwd_noalloc(C.byref(a), C.c_void_p(1 << 20), None, None) == N.MUIR_ERR_INVALID_ARG
+    assert b"flags" in lib.muir_last_error()

@@ -45,14 +45,21 @@ def test_train_forward_full_size(cuda_ok, chunk):
         assert rel_err(S[b:b + 1, h:h + 1], S_ref) < 1e-3
 
 
-def test_train_forward_backward_full_size(cuda_ok):
+@pytest.mark.parametrize("saved", [False, True])
+def test_train_forward_backward_full_size(cuda_ok, saved):
     """B=1, T=32768, H=16, d=128, chunk 128, bf16, dy ~ N(0,1): head 5 checked for y,
-    the final state and every gradient."""
+    the final state and every gradient; with and without the forward saving for the
+    backward (the saving path is the one the benchmark times)."""
     dev = torch.device("cuda")
     d = _gen(TRAIN_FWD_BWD, dev, with_grads=True)
     a = [d[n] for n in INPUT_NAMES]
-    y, S = muir.chunk_fwd(*a, chunk=128)
-    gr = muir.chunk_bwd(*a, d["dy"], chunk=128, dS_T=d["dS_T"], want_dr=True)
+    if saved:
+        ws = torch.empty(muir.chunk_bwd_workspace_bytes(*a, 128), dtype=torch.uint8, device=dev)
+        y, S = muir.chunk_fwd(*a, chunk=128, workspace=ws, save_for_bwd=True)
+        gr = muir.chunk_bwd(*a, d["dy"], chunk=128, dS_T=d["dS_T"], want_dr=True, workspace=ws, use_saved=True)
+    else:
+        y, S = muir.chunk_fwd(*a, chunk=128)
+        gr = muir.chunk_bwd(*a, d["dy"], chunk=128, dS_T=d["dS_T"], want_dr=True)
     assert muir.device_status() == 0
     h = 5
     c = _chain(d, 0, h)

@@ -23,7 +23,7 @@ def _args(t, chunk, S0):
     dv = t["v"].shape[-1]
     p = lambda x: C.c_void_p(x.data_ptr()) if x is not None else None
     return N.ChunkArgs(B=B, T=T, H=H, dk=dk, dv=dv, chunk=chunk,
-                       dtype=N.MUIR_BF16 if t["q"].dtype == torch.bfloat16 else N.MUIR_F32, reserved=0,
+                       dtype=N.MUIR_BF16 if t["q"].dtype == torch.bfloat16 else N.MUIR_F32, flags=0,
                        q=p(t["q"]), k=p(t["k"]), v=p(t["v"]), e=p(t["e"]), w=p(t["w"]), g=p(t["g"]), z=p(t["z"]),
                        log_alpha=p(t["log_alpha"]), r=p(t["r"]), S0=p(S0))
 
@@ -61,7 +61,7 @@ def test_noalloc_rejects_problems_beyond_the_scratch():
     build.build()
     lib = N.load()
     fake = C.c_void_p(1 << 20)
-    a = N.ChunkArgs(B=4, T=8192, H=16, dk=128, dv=128, chunk=128, dtype=N.MUIR_BF16, reserved=0,
+    a = N.ChunkArgs(B=4, T=8192, H=16, dk=128, dv=128, chunk=128, dtype=N.MUIR_BF16, flags=0,
                     q=fake, k=fake, v=fake, e=fake, w=fake, g=fake, z=None, log_alpha=fake, r=fake, S0=None)
     assert lib.muir_chunk_fwd_workspace(C.byref(a)) > (32 << 20)
     assert lib.muir_chunk_fwd_noalloc(C.byref(a), fake, None, None) == N.MUIR_ERR_UNSUPPORTED
