@@ -58,7 +58,7 @@ def kernel_model(C, dk, dv, es):
     m = {}
     m["decay"] = (0.0, C * dk * f4 + 4 * C * dk * f4)
     # off-diagonal blocks (tensor cores) + the exact 16x16 diagonal blocks (CUDA cores)
-    m["gram_off"] = (4 * 2 * (tri - C * 8) * dk + 4 * 2 * C * 8.5 * dk,
+    m["gram"] = (4 * 2 * (tri - C * 8) * dk + 4 * 2 * C * 8.5 * dk,
                      4 * C * dk * es + 3 * C * dk * f4 + 4 * C * C * f4)
     m["solve"] = (C ** 3 / 3.0, 2 * C * C * f4)
     maps_fl = 2 * (tri * dk + tri * dv + tri * dv + C * dk * dk + tri * dk + 2 * tri * dv + 2 * C * dk * dv)

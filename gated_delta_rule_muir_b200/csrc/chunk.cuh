@@ -29,8 +29,9 @@
 //
 // Kernels (one CTA per (batch, head, unit of Cs = min(chunk, 128) tokens) unless noted):
 //   decay_kernel      pre, suf, Gam_t, Gsuf_t            -> workspace
-//   gram_off_kernel   the 4 Grams: off-diagonal blocks on tcgen05, while the
-//                     exact 16x16 diagonal blocks run on the CUDA cores
+//   gram_kernel       the 4 Grams: blocks across the binary tree of 16-token
+//                     blocks on tcgen05 (one product per level), the exact
+//                     16x16 diagonal blocks on the CUDA cores meanwhile
 //   solve_kernel      T: exact 16x16 leaves, then recursive 2x2 block merges
 //                     T21 = -T22 M21 T11 on tcgen05 (block-Neumann recursion)
 //   maps_kernel       W, Ut, Phi, Psi, Q', Oloc (tcgen05)  -> workspace
@@ -281,66 +282,133 @@ __global__ void __launch_bounds__(128) decay_kernel(ChunkParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// gram_off_kernel: off-diagonal 16-blocks of M^kk, M^ka, N^qk, N^qa.
-// For column block I (pivot = its last token), rows t in later blocks J:
-//   G[t, s] = sum_i (X_t,i pre_t,i mid(I,J)_i) (Y_s,i suf_s,i)
-// M = 128 rows (t), N = 16 (s in block I), K = dk. Column blocks are visited
-// from the last to the first so mid(I,J) = mid(I+1,J) * tot_{I+1} stays a
-// product of block totals. Writes every entry except the diagonal blocks
-// (upper blocks get 0).
+// gram_kernel: the four decayed Grams M^kk, M^ka (strictly lower), N^qk, N^qa
+// (lower, diagonal included) of one unit, written as bf16 hi/lo images.
+//
+// Pairs (t, s) in different 16-token blocks are taken level by level over the
+// binary tree of the unit's blocks: at level b (64, 32, 16 for Cs = 128) the
+// pivots are P = (2p+1) b, and every t in [P, P+b) meets every s in [P-b, P):
+//   Gam_{t<-s} = pre^b_t * suf^b_s,  pre^b_t = prod_{u=P..t} alpha_u,
+//                                    suf^b_s = prod_{u=s+1..P-1} alpha_u,
+// both products of alphas in [0, 1] (no division). With pre16 / suf16 the
+// in-block products and tot_J the block totals, pre^b_t = pre16_t F^b_J(t) and
+// suf^b_s = suf16_s F^b_J(s), where F^b_J is the product of the block totals
+// between block J and the pivot. One tcgen05 product per level:
+//   XL rows p*2b + X*b + r = [K; Qt]_t pre^b_t   (t = (2p+1)b + r, X = K, Qt)
+//   YL rows p*2b + Y*b + r = [K; A]_s  suf^b_s   (s = 2pb + r,     Y = K, A)
+//   D = XL YL^T (M = 128, N = Cs, K = dk): row block p, column block p holds
+//   the four Gram blocks of pivot p; the other blocks of D are not used.
+// The 16x16 diagonal blocks are computed exactly on the CUDA cores with
+// running products while the tensor core runs; entries above the diagonal
+// blocks are written as zeros.
 // ---------------------------------------------------------------------------
 template <int DK, typename T, int NS>
-__global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
+__global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
   constexpr int NT = 256;
   constexpr int CH = DK / 16;  // channels per thread in the diagonal blocks
+  constexpr int MAXLEV = 3;
   const int Cs = p.Cs, nb = Cs / SB;
+  const int nlev = Cs == 128 ? 3 : 2;  // b = Cs/2, ..., 16
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   const int tid = threadIdx.x, warp = tid >> 5;
-  constexpr uint32_t LB = 128u * DK * 2u, RB = SB * DK * 2u;
+  constexpr uint32_t LB = 128u * DK * 2u;
   const uint32_t base = smem_u32(sm);
-  const Tile LK{base, base + LB, 128u, DK * 16u};                   // K-side left operand
-  const Tile LQ{base + 2 * LB, base + 3 * LB, 128u, DK * 16u};      // Q-side left operand
-  const Tile RK{base + 4 * LB, base + 4 * LB + RB, 128u, DK * 16u};
-  const Tile RA{base + 4 * LB + 2 * RB, base + 4 * LB + 3 * RB, 128u, DK * 16u};
-  float* midtab = reinterpret_cast<float*>(sm + 4 * LB + 4 * RB);  // [nb][DK]
-  float* drow = midtab + nb * DK;                                    // [4][16][DK]: k, qt, a, alpha of one block
+  const Tile XL{base, base + LB, 128u, DK * 16u};
+  const Tile YL{base + 2 * LB, base + 3 * LB, 128u, DK * 16u};
+  float* ftab = reinterpret_cast<float*>(sm + 4 * LB);  // [MAXLEV][nb][DK]
+  float* drow = ftab + MAXLEV * nb * DK;                 // [4][16][DK]: k, qt, a, alpha of one block
   zero_smem(base, 4 * LB);
   TcCta cta;
-  cta.init(&tslot, &bar, tmem_cols_for(4 * Cs));
+  cta.init(&tslot, &bar, tmem_cols_for(128 * nlev));
   const float* pre = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
   const float* suf = pre + Cs * DK;
   const Rows<T> rows{p, s.b, s.h};
   uint8_t* out = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
   MmaSync drv{&bar, 0u, true};
-  const uint32_t id = idesc_bf16(128, SB, 0, 0);
+  const uint32_t id = idesc_bf16(128, Cs, 0, 0);
 
-  // Diagonal 16x16 blocks, exactly, on the CUDA cores: rows of block J -> drow.
-  auto load_block = [&](int J) {
-    for (int x = tid; x < SB * (DK / 8); x += NT) {
-      const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-      const int64_t tok = s.tok0 + SB * J + rr;
-      float kk[8], aa[8], qq[8], la[8];
-      rows.k(tok, c8, kk);
-      rows.a(tok, c8, aa);
-      rows.qt(tok, c8, qq);
-      ld8f(p.la + toff(p, s.b, tok, s.h, DK) + c8, la);
+  // F^b_J per level and channel: products of block totals toward the pivot.
+  if (tid < DK) {
+    float tot[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) la[j] = expf(la[j]);
-      Elt<float>::st8(drow + (0 * SB + rr) * DK + c8, kk);
-      Elt<float>::st8(drow + (1 * SB + rr) * DK + c8, qq);
-      Elt<float>::st8(drow + (2 * SB + rr) * DK + c8, aa);
-      Elt<float>::st8(drow + (3 * SB + rr) * DK + c8, la);
+    for (int J = 0; J < 8; ++J) tot[J] = J < nb ? pre[(SB * J + SB - 1) * DK + tid] : 1.f;
+    for (int lev = 0; lev < nlev; ++lev) {
+      const int hb = (Cs >> (lev + 1)) / SB;  // blocks per half at this level
+      for (int J0 = 0; J0 < nb; J0 += 2 * hb) {
+        float run = 1.f;
+        for (int J = J0 + hb; J < J0 + 2 * hb; ++J) {  // upper half: from the pivot forward
+          ftab[(lev * nb + J) * DK + tid] = run;
+          run *= tot[J];
+        }
+        run = 1.f;
+        for (int J = J0 + hb - 1; J >= J0; --J) {  // lower half: from the pivot backward
+          ftab[(lev * nb + J) * DK + tid] = run;
+          run *= tot[J];
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // Rows of block J for its exact diagonal block: fetched into registers one
+  // block ahead (the loads fly while the previous block is computed), then
+  // stored to drow as k, qt, a, alpha.
+  constexpr int FPT = (SB * (DK / 8) + NT - 1) / NT;  // 8-channel pieces per thread
+  Pack8<T> fk[FPT], fe[FPT], fq[FPT], fg[FPT];
+  Pack8<float> fl[FPT];
+  auto fetch_block = [&](int J) {
+#pragma unroll
+    for (int f = 0; f < FPT; ++f) {
+      const int x = tid + f * NT;
+      if (x < SB * (DK / 8)) {
+        const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+        const int64_t o = toff(p, s.b, s.tok0 + SB * J + rr, s.h, DK) + c8;
+        fk[f].ld(static_cast<const T*>(p.k) + o);
+        fe[f].ld(static_cast<const T*>(p.e) + o);
+        fq[f].ld(static_cast<const T*>(p.q) + o);
+        fg[f].ld(static_cast<const T*>(p.g) + o);
+        fl[f].ld(p.la + o);
+      }
+    }
+  };
+  auto store_block = [&] {
+#pragma unroll
+    for (int f = 0; f < FPT; ++f) {
+      const int x = tid + f * NT;
+      if (x < SB * (DK / 8)) {
+        const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+        float kk[8], ee[8], qq[8], gg[8], la[8], rr8[8];
+        fk[f].get(kk);
+        fe[f].get(ee);
+        fq[f].get(qq);
+        fg[f].get(gg);
+        fl[f].get(la);
+        ld8f(p.r + (int64_t)s.h * DK + c8, rr8);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          la[j] = expf(la[j]);
+          ee[j] *= kk[j];               // a = e k
+          qq[j] = rr8[j] * gg[j] * qq[j];  // qt = r g q
+        }
+        Elt<float>::st8(drow + (0 * SB + rr) * DK + c8, kk);
+        Elt<float>::st8(drow + (1 * SB + rr) * DK + c8, qq);
+        Elt<float>::st8(drow + (2 * SB + rr) * DK + c8, ee);
+        Elt<float>::st8(drow + (3 * SB + rr) * DK + c8, la);
+      }
     }
   };
   // thread = (row t, channel group cg of CH channels); for s = t, t-1, ... the
   // running product Gam_{t<-s} = Gam_{t<-s+1} alpha_{s+1} scales both right
   // operands; the 64 partial sums are reduced over the 16 lanes of the row by
   // recursive halving, after which lane cg holds Gram cg/4, columns 4(cg%4)..+3.
+  // Warps w and w + 4 share a scheduler: rows (2w, 2w+1) go with (14-2w, 15-2w)
+  // so that every scheduler runs 18 row steps.
   auto diag_block = [&](int J) {
-    const int t = tid >> 4, cg = tid & 15, c0 = cg * CH;
+    const int pair = warp < 4 ? warp : 11 - warp;
+    const int t = 2 * pair + ((tid >> 4) & 1), cg = tid & 15, c0 = cg * CH;
     float xk[CH], xq[CH], gm[CH];
     lds_vec(drow + (0 * SB + t) * DK + c0, xk);
     lds_vec(drow + (1 * SB + t) * DK + c0, xq);
@@ -385,81 +453,111 @@ __global__ void __launch_bounds__(256, 1) gram_off_kernel(ChunkParams p) {
     }
     gput_k4(out + g * sq_bytes(Cs), sq_half(Cs), (uint32_t)Cs * 16u, SB * J + t, SB * J + c4, w4);
   };
+  // Zeros above the diagonal blocks of the four images.
+  const int lcs = Cs == 128 ? 7 : 6;  // log2(Cs)
+  // In the image an 8-row group is Cs 16-byte chunks; chunk c holds columns
+  // 8 (c >> 3) .. + 7, so its part right of the diagonal block is contiguous.
+  auto zero_upper = [&] {
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int x = tid; x < 8 << (2 * lcs - 3); x += NT) {  // (image, hi/lo, row group, chunk)
+      const int c = x & (Cs - 1), rg = (x >> lcs) & ((Cs >> 3) - 1), gh = x >> (2 * lcs - 3);
+      if ((c >> 4) <= (rg >> 1)) continue;
+      uint8_t* img = out + (gh >> 1) * sq_bytes(Cs) + (gh & 1) * sq_half(Cs);
+      *reinterpret_cast<uint4*>(img + (uint32_t)rg * (uint32_t)Cs * 16u + (uint32_t)c * 16u) = z;
+    }
+  };
 
-  for (int I = nb - 2; I >= 0 && drv.ok; --I) {
-#pragma unroll 4
-    for (int x = tid; x < nb * DK; x += NT) {
-      const int J = x / DK, i = x % DK;
-      if (J == I + 1) midtab[x] = 1.f;
-      else if (J > I + 1) midtab[x] *= pre[(SB * (I + 1) + SB - 1) * DK + i];
-    }
-#pragma unroll 2
-    for (int x = tid; x < SB * (DK / 8); x += NT) {
-      const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-      const int t = SB * I + rr;
-      float kk[8], aa[8], sf[8], vk[8], va[8];
-      rows.k(s.tok0 + t, c8, kk);
-      rows.a(s.tok0 + t, c8, aa);
-      ld8f(suf + t * DK + c8, sf);
+  fetch_block(0);
+  float rv[8];  // r for this thread's 8 channels (fixed: NT is a multiple of DK / 8)
+  ld8f(p.r + (int64_t)s.h * DK + (tid % (DK / 8)) * 8, rv);
+  for (int lev = 0; lev < nlev && drv.ok; ++lev) {
+    const int lb = lcs - 1 - lev;  // b = 2^lb
+    const int b = 1 << lb;
+    const float* ft = ftab + lev * nb * DK;
+    // Stage XL / YL: four tokens per thread per batch, loads first. Upper tokens
+    // take (k, r g q, pre), lower ones (k, e k, suf); the sources are selected by
+    // pointer so that every load of the batch is issued before any is used.
+    constexpr int BT = sizeof(T) == 2 ? 4 : 2;  // tokens per thread per batch
+    auto tok_c8 = [&](int x, int& t, int& c8) {
+      t = x / (DK / 8);
+      c8 = (x % (DK / 8)) * 8;
+    };
+    for (int x0 = tid; x0 < Cs * (DK / 8); x0 += BT * NT) {
+      Pack8<T> pk[BT], p1[BT], p2[BT];
+      Pack8<float> ps[BT];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) { vk[j] = kk[j] * sf[j]; va[j] = aa[j] * sf[j]; }
-      put_k(RK, rr, c8, vk);
-      put_k(RA, rr, c8, va);
-    }
-    load_block(I + 1);
-    __syncthreads();
-    const int t0 = SB * (I + 1);
-#pragma unroll 2
-    for (int x = tid; x < (Cs - t0) * (DK / 8); x += NT) {
-      const int t = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-      float kv[8], qv[8], pr[8];
-      rows.k(s.tok0 + t, c8, kv);
-      rows.qt(s.tok0 + t, c8, qv);
-      ld8f(pre + t * DK + c8, pr);
-      const float4* mp = reinterpret_cast<const float4*>(midtab + (t / SB) * DK + c8);
-      const float4 m0 = mp[0], m1 = mp[1];
-      const float md[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float f = pr[j] * md[j];
-        kv[j] *= f;
-        qv[j] *= f;
+      for (int u = 0; u < BT; ++u) {
+        const int x = x0 + u * NT;
+        if (x < Cs * (DK / 8)) {
+          int t, c8;
+          tok_c8(x, t, c8);
+          const bool upper = (t >> lb) & 1;
+          const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DK) + c8;
+          pk[u].ld(static_cast<const T*>(p.k) + o);
+          p1[u].ld(static_cast<const T*>(upper ? p.q : p.e) + o);
+          p2[u].ld(static_cast<const T*>(upper ? p.g : p.k) + o);
+          ps[u].ld((upper ? pre : suf) + t * DK + c8);
+        }
       }
-      put_k(LK, t, c8, kv);
-      put_k(LQ, t, c8, qv);
+#pragma unroll
+      for (int u = 0; u < BT; ++u) {
+        const int x = x0 + u * NT;
+        if (x < Cs * (DK / 8)) {
+          int t, c8;
+          tok_c8(x, t, c8);
+          const bool upper = (t >> lb) & 1;
+          const int pv = t >> (lb + 1), r = t & (b - 1);
+          float kk[8], s1[8], s2[8], sc[8], fj[8];
+          pk[u].get(kk);
+          p1[u].get(s1);
+          p2[u].get(s2);
+          ps[u].get(sc);
+          Elt<float>::ld8g(ft + (t >> 4) * DK + c8, fj);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float f = sc[j] * fj[j];
+            s1[j] *= s2[j] * (upper ? rv[j] : 1.f) * f;  // r g q or e k
+            kk[j] *= f;
+          }
+          const Tile& dst = upper ? XL : YL;
+          put_k(dst, (pv << (lb + 1)) + r, c8, kk);
+          put_k(dst, (pv << (lb + 1)) + b + r, c8, s1);
+        }
+      }
     }
-    const uint32_t c0 = SB * I;
+    const int J0 = lev * nb / nlev, J1 = (lev + 1) * nb / nlev;
     drv.run_overlap(
+        [&] { mma_tiles(cta.tmem + 128 * lev, XL, YL, DK / 16, id, NS, false); },
         [&] {
-          mma_tiles(cta.tmem + c0, LK, RK, DK / 16, id, NS, false);
-          mma_tiles(cta.tmem + c0 + Cs, LK, RA, DK / 16, id, NS, false);
-          mma_tiles(cta.tmem + c0 + 2 * Cs, LQ, RK, DK / 16, id, NS, false);
-          mma_tiles(cta.tmem + c0 + 3 * Cs, LQ, RA, DK / 16, id, NS, false);
-        },
-        [&] { diag_block(I + 1); });
+          for (int J = J0; J < J1; ++J) {
+            __syncthreads();  // drow is free
+            store_block();
+            __syncthreads();
+            if (J + 1 < nb) fetch_block(J + 1);
+            diag_block(J);
+          }
+          if (lev == nlev - 1) zero_upper();
+        });
   }
-  if (drv.ok) {
-    load_block(0);
-    __syncthreads();
-    diag_block(0);
-  }
-  // Epilogue: row t = TMEM lane; the two warpgroups take alternate 16-column chunks.
-  const int t = tid & 127, wg = tid >> 7;
-  const int J = t / SB;
-  for (int gidx = 0; gidx < 4; ++gidx) {
-    for (int c0 = wg * 16; c0 < Cs; c0 += 32) {
+  // Epilogue: lane = row p*2b + X*b + r of level b; the valid columns are the
+  // 2b of column block p (Y = K first, then Y = A).
+  const int rho = tid & 127, wg = tid >> 7;
+  for (int lev = 0; lev < nlev; ++lev) {
+    const int lb = lcs - 1 - lev, b = 1 << lb;
+    const int pv = ((warp & 3) * 32) >> (lb + 1);  // warp-uniform: 2b >= 32
+    const int X = (rho >> lb) & 1, r = rho & (b - 1);
+    const int t = (2 * pv + 1) * b + r;
+    for (int c0 = wg * 16; c0 < 2 * b; c0 += 32) {
       float v[16];
-      tmem_ld16(cta.tmem + tmem_lane_base(warp) + gidx * Cs + c0, v);
-      const int I = c0 / SB;
-      if (t < Cs && I != J && drv.ok) {
+      tmem_ld16(cta.tmem + tmem_lane_base(warp) + 128 * lev + pv * 2 * b + c0, v);
+      if (rho < Cs && drv.ok) {
+        const int Y = c0 >> lb, s0 = 2 * pv * b + (c0 & (b - 1));
+        uint8_t* img = out + (2 * X + Y) * sq_bytes(Cs);
         float a8[8], b8[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          a8[j] = I < J ? v[j] : 0.f;
-          b8[j] = I < J ? v[8 + j] : 0.f;
-        }
-        sq_put(out + gidx * sq_bytes(Cs), Cs, t, c0, a8);
-        sq_put(out + gidx * sq_bytes(Cs), Cs, t, c0 + 8, b8);
+        for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
+        sq_put(img, Cs, t, s0, a8);
+        sq_put(img, Cs, t, s0 + 8, b8);
       }
     }
   }
