@@ -71,7 +71,7 @@ def kernel_model(C, dk, dv, es):
                    3 * C * C * f4 + 2 * C * dv * es + dk * dv * f4 + 2 * C * dk * es + 2 * C * dv * f4)
     m["bwd_grads"] = (2 * (4 * C * dk * dv + 4 * tri * dv),
                       4 * C * dv * f4 + 2 * dk * dv * f4 + 2 * C * dv * es + 4 * C * dk * f4 + 4 * C * C * f4)
-    m["bwd_gram_off"] = (4 * 2 * 2 * (tri - C * 8) * dk + 4 * 2 * 2 * C * 8.5 * dk, 4 * C * C * f4 + 4 * C * dk * es + 2 * C * dk * f4 + 4 * C * dk * f4)
+    m["bwd_gram"] = (4 * 2 * 2 * (tri - C * 8) * dk + 4 * 2 * 2 * C * 8.5 * dk, 4 * C * C * f4 + 4 * C * dk * es + 2 * C * dk * f4 + 4 * C * dk * f4)
     m["bwd_final"] = (0.0, 14 * C * dk * f4 + 6 * C * dk * es + C * dv * f4 + 4 * C * dv * es)
     return m
 

@@ -282,6 +282,100 @@ __global__ void __launch_bounds__(128) decay_kernel(ChunkParams p) {
 }
 
 // ---------------------------------------------------------------------------
+// Levels of the binary tree over a unit's 16-token blocks (shared by the Gram
+// kernel and its backward). Level lev has half-length b = Cs >> (lev + 1)
+// (64, 32, 16 for Cs = 128) and pivots P = (2p+1) b; tokens t with (t / b) odd
+// are "upper" (t >= P), the others "lower" (t < P).
+// ---------------------------------------------------------------------------
+constexpr int kMaxLev = 3;
+__device__ __forceinline__ int tree_levels(int Cs) { return Cs == 128 ? 3 : 2; }
+__device__ __forceinline__ int log2_cs(int Cs) { return Cs == 128 ? 7 : 6; }
+
+// ftab[lev][J][i] = F^b_J: product of the block totals between block J and its
+// pivot (upper blocks: pivot block .. J-1; lower blocks: J+1 .. pivot block - 1).
+// pre is the unit's in-block prefix product (pre[16 J + 15] = total of block J).
+template <int DK>
+__device__ __forceinline__ void tree_tables(const float* pre, float* ftab, int Cs) {
+  const int nb = Cs / SB, nlev = tree_levels(Cs), i = threadIdx.x;
+  if (i < DK) {
+    float tot[8];
+#pragma unroll
+    for (int J = 0; J < 8; ++J) tot[J] = J < nb ? pre[(SB * J + SB - 1) * DK + i] : 1.f;
+    for (int lev = 0; lev < nlev; ++lev) {
+      const int hb = (Cs >> (lev + 1)) / SB;  // blocks per half
+      for (int J0 = 0; J0 < nb; J0 += 2 * hb) {
+        float run = 1.f;
+        for (int J = J0 + hb; J < J0 + 2 * hb; ++J) {  // upper half: from the pivot forward
+          ftab[(lev * nb + J) * DK + i] = run;
+          run *= tot[J];
+        }
+        run = 1.f;
+        for (int J = J0 + hb - 1; J >= J0; --J) {  // lower half: from the pivot backward
+          ftab[(lev * nb + J) * DK + i] = run;
+          run *= tot[J];
+        }
+      }
+    }
+  }
+}
+
+// Operands of level lev (b = 2^lb):
+//   XL row p*2b + X*b + r = [k; r g q]_t * pre_t * F_J(t)   upper t = (2p+1)b + r
+//   YL row p*2b + Y*b + r = [k; e k]_s  * suf_s * F_J(s)    lower s = 2pb + r
+// Staged for the halves asked for; 256 threads, BT tokens per thread per batch
+// with all loads of a batch issued before any is used.
+template <int DK, typename T>
+__device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& s, const float* pre,
+                                            const float* suf, const float* ft, const float (&rv)[8], int Cs,
+                                            int lb, bool want_upper, bool want_lower, const Tile& XL,
+                                            const Tile& YL) {
+  constexpr int NT = 256;
+  constexpr int BT = sizeof(T) == 2 ? 4 : 2;
+  const int b = 1 << lb;
+  for (int x0 = threadIdx.x; x0 < Cs * (DK / 8); x0 += BT * NT) {
+    Pack8<T> pk[BT], p1[BT], p2[BT];
+    Pack8<float> ps[BT];
+#pragma unroll
+    for (int u = 0; u < BT; ++u) {
+      const int x = x0 + u * NT;
+      const int t = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      const bool upper = (t >> lb) & 1;
+      if (x < Cs * (DK / 8) && (upper ? want_upper : want_lower)) {
+        const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DK) + c8;
+        pk[u].ld(static_cast<const T*>(p.k) + o);
+        p1[u].ld(static_cast<const T*>(upper ? p.q : p.e) + o);
+        p2[u].ld(static_cast<const T*>(upper ? p.g : p.k) + o);
+        ps[u].ld((upper ? pre : suf) + t * DK + c8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < BT; ++u) {
+      const int x = x0 + u * NT;
+      const int t = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      const bool upper = (t >> lb) & 1;
+      if (x < Cs * (DK / 8) && (upper ? want_upper : want_lower)) {
+        const int pv = t >> (lb + 1), r = t & (b - 1);
+        float kk[8], s1[8], s2[8], sc[8], fj[8];
+        pk[u].get(kk);
+        p1[u].get(s1);
+        p2[u].get(s2);
+        ps[u].get(sc);
+        Elt<float>::ld8g(ft + (t >> 4) * DK + c8, fj);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float f = sc[j] * fj[j];
+          s1[j] *= s2[j] * (upper ? rv[j] : 1.f) * f;  // r g q or e k
+          kk[j] *= f;
+        }
+        const Tile& dst = upper ? XL : YL;
+        put_k(dst, (pv << (lb + 1)) + r, c8, kk);
+        put_k(dst, (pv << (lb + 1)) + b + r, c8, s1);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // gram_kernel: the four decayed Grams M^kk, M^ka (strictly lower), N^qk, N^qa
 // (lower, diagonal included) of one unit, written as bf16 hi/lo images.
 //
@@ -309,17 +403,16 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
   __shared__ uint32_t tslot;
   constexpr int NT = 256;
   constexpr int CH = DK / 16;  // channels per thread in the diagonal blocks
-  constexpr int MAXLEV = 3;
   const int Cs = p.Cs, nb = Cs / SB;
-  const int nlev = Cs == 128 ? 3 : 2;  // b = Cs/2, ..., 16
+  const int nlev = tree_levels(Cs);
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   const int tid = threadIdx.x, warp = tid >> 5;
   constexpr uint32_t LB = 128u * DK * 2u;
   const uint32_t base = smem_u32(sm);
   const Tile XL{base, base + LB, 128u, DK * 16u};
   const Tile YL{base + 2 * LB, base + 3 * LB, 128u, DK * 16u};
-  float* ftab = reinterpret_cast<float*>(sm + 4 * LB);  // [MAXLEV][nb][DK]
-  float* drow = ftab + MAXLEV * nb * DK;                 // [4][16][DK]: k, qt, a, alpha of one block
+  float* ftab = reinterpret_cast<float*>(sm + 4 * LB);  // [kMaxLev][nb][DK]
+  float* drow = ftab + kMaxLev * nb * DK;                // [4][16][DK]: k, qt, a, alpha of one block
   zero_smem(base, 4 * LB);
   TcCta cta;
   cta.init(&tslot, &bar, tmem_cols_for(128 * nlev));
@@ -330,27 +423,7 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
   MmaSync drv{&bar, 0u, true};
   const uint32_t id = idesc_bf16(128, Cs, 0, 0);
 
-  // F^b_J per level and channel: products of block totals toward the pivot.
-  if (tid < DK) {
-    float tot[8];
-#pragma unroll
-    for (int J = 0; J < 8; ++J) tot[J] = J < nb ? pre[(SB * J + SB - 1) * DK + tid] : 1.f;
-    for (int lev = 0; lev < nlev; ++lev) {
-      const int hb = (Cs >> (lev + 1)) / SB;  // blocks per half at this level
-      for (int J0 = 0; J0 < nb; J0 += 2 * hb) {
-        float run = 1.f;
-        for (int J = J0 + hb; J < J0 + 2 * hb; ++J) {  // upper half: from the pivot forward
-          ftab[(lev * nb + J) * DK + tid] = run;
-          run *= tot[J];
-        }
-        run = 1.f;
-        for (int J = J0 + hb - 1; J >= J0; --J) {  // lower half: from the pivot backward
-          ftab[(lev * nb + J) * DK + tid] = run;
-          run *= tot[J];
-        }
-      }
-    }
-  }
+  tree_tables<DK>(pre, ftab, Cs);
   __syncthreads();
 
   // Rows of block J for its exact diagonal block: fetched into registers one
@@ -454,7 +527,7 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
     gput_k4(out + g * sq_bytes(Cs), sq_half(Cs), (uint32_t)Cs * 16u, SB * J + t, SB * J + c4, w4);
   };
   // Zeros above the diagonal blocks of the four images.
-  const int lcs = Cs == 128 ? 7 : 6;  // log2(Cs)
+  const int lcs = log2_cs(Cs);
   // In the image an 8-row group is Cs 16-byte chunks; chunk c holds columns
   // 8 (c >> 3) .. + 7, so its part right of the diagonal block is contiguous.
   auto zero_upper = [&] {
@@ -472,59 +545,8 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
   ld8f(p.r + (int64_t)s.h * DK + (tid % (DK / 8)) * 8, rv);
   for (int lev = 0; lev < nlev && drv.ok; ++lev) {
     const int lb = lcs - 1 - lev;  // b = 2^lb
-    const int b = 1 << lb;
     const float* ft = ftab + lev * nb * DK;
-    // Stage XL / YL: four tokens per thread per batch, loads first. Upper tokens
-    // take (k, r g q, pre), lower ones (k, e k, suf); the sources are selected by
-    // pointer so that every load of the batch is issued before any is used.
-    constexpr int BT = sizeof(T) == 2 ? 4 : 2;  // tokens per thread per batch
-    auto tok_c8 = [&](int x, int& t, int& c8) {
-      t = x / (DK / 8);
-      c8 = (x % (DK / 8)) * 8;
-    };
-    for (int x0 = tid; x0 < Cs * (DK / 8); x0 += BT * NT) {
-      Pack8<T> pk[BT], p1[BT], p2[BT];
-      Pack8<float> ps[BT];
-#pragma unroll
-      for (int u = 0; u < BT; ++u) {
-        const int x = x0 + u * NT;
-        if (x < Cs * (DK / 8)) {
-          int t, c8;
-          tok_c8(x, t, c8);
-          const bool upper = (t >> lb) & 1;
-          const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DK) + c8;
-          pk[u].ld(static_cast<const T*>(p.k) + o);
-          p1[u].ld(static_cast<const T*>(upper ? p.q : p.e) + o);
-          p2[u].ld(static_cast<const T*>(upper ? p.g : p.k) + o);
-          ps[u].ld((upper ? pre : suf) + t * DK + c8);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < BT; ++u) {
-        const int x = x0 + u * NT;
-        if (x < Cs * (DK / 8)) {
-          int t, c8;
-          tok_c8(x, t, c8);
-          const bool upper = (t >> lb) & 1;
-          const int pv = t >> (lb + 1), r = t & (b - 1);
-          float kk[8], s1[8], s2[8], sc[8], fj[8];
-          pk[u].get(kk);
-          p1[u].get(s1);
-          p2[u].get(s2);
-          ps[u].get(sc);
-          Elt<float>::ld8g(ft + (t >> 4) * DK + c8, fj);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float f = sc[j] * fj[j];
-            s1[j] *= s2[j] * (upper ? rv[j] : 1.f) * f;  // r g q or e k
-            kk[j] *= f;
-          }
-          const Tile& dst = upper ? XL : YL;
-          put_k(dst, (pv << (lb + 1)) + r, c8, kk);
-          put_k(dst, (pv << (lb + 1)) + b + r, c8, s1);
-        }
-      }
-    }
+    stage_level<DK, T>(p, s, pre, suf, ft, rv, Cs, lb, true, true, XL, YL);
     const int J0 = lev * nb / nlev, J1 = (lev + 1) * nb / nlev;
     drv.run_overlap(
         [&] { mma_tiles(cta.tmem + 128 * lev, XL, YL, DK / 16, id, NS, false); },

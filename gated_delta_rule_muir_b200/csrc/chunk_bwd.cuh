@@ -24,9 +24,8 @@
 //                      dS <- Phi^T dS + E (the adjoint of the state map)
 //   bwd_dz_kernel      dP, dZ, dU
 //   bwd_grads_kernel   dQp, dKp, dKs, dAs, dGam_C and the four Gram cotangents
-//   bwd_gram_off_kernel  off-diagonal blocks of the Gram backward (tcgen05):
-//                      dX with the pivot at the start of the row block,
-//                      dY with the pivot at the end of the column block
+//   bwd_gram_kernel    the Gram backward: tree levels on tcgen05 (left and
+//                      right phases), exact diagonal blocks on the CUDA cores
 //   bwd_final_kernel   decay cotangents, reverse cumsum, chain rule to inputs
 #pragma once
 
@@ -526,192 +525,181 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
 }
 
 // ---------------------------------------------------------------------------
-// bwd_gram_off_kernel: off-diagonal blocks of the Gram backward. Results are
-// accumulated transposed in TMEM (lane = key channel, column = token):
-//   left  (rows t of block J, pivot = last token of block J-1):
-//     dX_t = pre_t * sum_{s < start(J)} dG_ts (Y_s * suf_s * mid(I(s), J))
-//     A = (Y*suf*mid)^T (MN-major over s), B = dG[J rows, s]^T (K-major, N = 16)
-//   right (columns s of block I, pivot = last token of block I):
-//     dY_s = suf_s * sum_{t > end(I)} dG_ts (X_t * pre_t * mid(I, J(t)))
-//     A = (X*pre*mid)^T (MN-major over t), B = dG[t, I cols] (MN-major, N = 16)
-// Region columns: dK_left 0, dQ_left Cs, dK_right 2Cs, dA_right 3Cs.
+// bwd_gram_kernel: the Gram cotangents dG pushed to the Gram factors, per unit
+// (sums over the Gram pairs s < t, s <= t for N, channel by channel):
+//   dK_left_t  = sum_s (dM^kk_ts k_s + dM^ka_ts a_s) Gam_{t<-s}
+//   dQ_left_t  = sum_s (dN^qk_ts k_s + dN^qa_ts a_s) Gam_{t<-s}
+//   dK_right_s = sum_t (dM^kk_ts k_t + dN^qk_ts qt_t) Gam_{t<-s}
+//   dA_right_s = sum_t (dM^ka_ts k_t + dN^qa_ts qt_t) Gam_{t<-s}
+// Pairs across 16-token blocks go level by level as in gram_kernel. With G_b
+// the level's tile of dG (row p*2b + X*b + r = (X, t) upper, column
+// p*2b + Y*b + r' = (Y, s) lower, zero across pivots):
+//   left  phase: D^T = YL^T G_b^T (lane = key channel, column (X, t)), then
+//                dX_left_t  += pre16_t F_J(t) D^T[., (X, t)]
+//   right phase: D^T = XL^T G_b   (lane = key channel, column (Y, s)), then
+//                dY_right_s += suf16_s F_J(s) D^T[., (Y, s)]
+// Each phase keeps its levels in TMEM (128 columns each), so every output is
+// formed once in the epilogue together with its exact diagonal-block part
+// (CUDA cores, running products) and written once.
 // ---------------------------------------------------------------------------
 template <int DK, typename T, int NS>
-__global__ void __launch_bounds__(256, 1) bwd_gram_off_kernel(ChunkParams p, BwdBufs q) {
+__global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
-  const int Cs = p.Cs, nb = Cs / SB;
-  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   constexpr int NT = 256;
+  const int Cs = p.Cs, nb = Cs / SB, nlev = tree_levels(Cs), lcs = log2_cs(Cs);
+  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
   const uint32_t base = smem_u32(sm);
-  const uint32_t AB = 128u * (uint32_t)Cs * 2u;  // M = 128 channels (padded) x K = Cs tokens
-  const uint32_t BB = (uint32_t)SB * Cs * 2u;    // N = 16 x K = Cs
-  const Tile A1{base, base + AB, 128u, (uint32_t)Cs * 16u};
-  const Tile A2{base + 2 * AB, base + 3 * AB, 128u, (uint32_t)Cs * 16u};
-  Tile Bk[4], Bm[4];
-  for (int g = 0; g < 4; ++g) {
-    const uint32_t b0 = base + 4 * AB + g * 2 * BB;
-    Bk[g] = Tile{b0, b0 + BB, 128u, (uint32_t)Cs * 16u};  // K-major: row = t (N), K = s
-    Bm[g] = Tile{b0, b0 + BB, 128u, (uint32_t)Cs * 16u};  // MN-major: row = t (K), N = s (16)
-  }
-  float* midtab = reinterpret_cast<float*>(sm + 4 * AB + 8 * BB);  // [nb][DK]
-  zero_smem(base, 4 * AB + 8 * BB);
+  constexpr uint32_t OB = 128u * DK * 2u;        // operand tile (128 token rows x dk), one half
+  const uint32_t GB = 128u * (uint32_t)Cs * 2u;  // dG tile (128 rows x Cs), one half
+  const Tile OP{base, base + OB, 128u, DK * 16u};  // YL (left phase) or XL (right phase)
+  const Tile GT{base + 2 * OB, base + 2 * OB + GB, 128u, (uint32_t)Cs * 16u};
+  float4* dgd = reinterpret_cast<float4*>(sm + 2 * OB + 2 * GB);  // [nb][16 t][16 s]: mkk, mka, nqk, nqa
+  float* ftab = reinterpret_cast<float*>(sm + 2 * OB + 2 * GB + (size_t)nb * SB * SB * 16);  // [kMaxLev][nb][DK]
   TcCta cta;
-  cta.init(&tslot, &bar, tmem_cols_for(4 * Cs));
+  cta.init(&tslot, &bar, tmem_cols_for(128 * nlev));
   MmaSync drv{&bar, 0u, true};
   const float* pre = p.dec + u * 4 * Cs * DK;
   const float* suf = pre + Cs * DK;
   const float* dG = q.dG + u * 4 * Cs * Cs;
-  const Rows<T> rows{p, s.b, s.h};
-  const uint32_t id16 = idesc_bf16(128, SB, 1, 0), id16m = idesc_bf16(128, SB, 1, 1);
-  // ---- left gradients: J ascending, mid(I, J) for I < J
-  for (int J = 1; J < nb && drv.ok; ++J) {
-    #pragma unroll 4
-    for (int x = tid; x < nb * DK; x += NT) {
-      const int I = x / DK, i = x % DK;
-      if (I == J - 1) midtab[x] = 1.f;
-      else if (I < J - 1) midtab[x] *= pre[(SB * (J - 1) + SB - 1) * DK + i];  // tot_{J-1}
-    }
-    __syncthreads();
-    #pragma unroll 4
-    for (int x = tid; x < SB * J * (DK / 8); x += NT) {
-      const int ss = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-      float kk[8], aa[8], sf[8];
-      rows.k(s.tok0 + ss, c8, kk);
-      rows.a(s.tok0 + ss, c8, aa);
-      ld8f(suf + ss * DK + c8, sf);
-      const float* mp = midtab + (ss / SB) * DK + c8;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { const float f = sf[j] * mp[j]; kk[j] *= f; aa[j] *= f; }
-      put_mn(A1, ss, c8, kk);
-      put_mn(A2, ss, c8, aa);
-    }
-    #pragma unroll 4
-    for (int x = tid; x < 4 * SB * (SB * J / 8); x += NT) {
-      const int g = x / (SB * (SB * J / 8)), rem = x % (SB * (SB * J / 8));
-      const int rr = rem / (SB * J / 8), c8 = (rem % (SB * J / 8)) * 8;
-      float v[8];
-      ld8f(dG + ((int64_t)g * Cs + SB * J + rr) * Cs + c8, v);
-      put_k(Bk[g], rr, c8, v);
-    }
-    drv.run([&] {
-      const uint32_t c = SB * J;
-      mma_tiles(cta.tmem + 0 * Cs + c, A1, Bk[0], J, id16, NS, false);  // dM^kk . K
-      mma_tiles(cta.tmem + 0 * Cs + c, A2, Bk[1], J, id16, NS, true);   // dM^ka . A
-      mma_tiles(cta.tmem + 1 * Cs + c, A1, Bk[2], J, id16, NS, false);  // dN^qk . K
-      mma_tiles(cta.tmem + 1 * Cs + c, A2, Bk[3], J, id16, NS, true);   // dN^qa . A
-    });
+  const int64_t gsz = (int64_t)Cs * Cs;
+  tree_tables<DK>(pre, ftab, Cs);
+  for (int x = tid; x < nb * SB * SB; x += NT) {  // diagonal blocks of the four cotangents
+    const int J = x >> 8, tt = (x >> 4) & 15, ss = x & 15;
+    const int64_t o = (int64_t)(SB * J + tt) * Cs + SB * J + ss;
+    dgd[x] = make_float4(dG[o], dG[gsz + o], dG[2 * gsz + o], dG[3 * gsz + o]);
   }
-  // ---- right gradients: I descending, mid(I, J) for J > I
-  for (int I = nb - 2; I >= 0 && drv.ok; --I) {
-    #pragma unroll 4
-    for (int x = tid; x < nb * DK; x += NT) {
-      const int J = x / DK, i = x % DK;
-      if (J == I + 1) midtab[x] = 1.f;
-      else if (J > I + 1) midtab[x] *= pre[(SB * (I + 1) + SB - 1) * DK + i];
-    }
-    __syncthreads();
-    const int t0 = SB * (I + 1);
-    #pragma unroll 4
-    for (int x = tid; x < (Cs - t0) * (DK / 8); x += NT) {
-      const int tt = t0 + x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-      float kk[8], qq[8], pr[8];
-      rows.k(s.tok0 + tt, c8, kk);
-      rows.qt(s.tok0 + tt, c8, qq);
-      ld8f(pre + tt * DK + c8, pr);
-      const float* mp = midtab + (tt / SB) * DK + c8;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { const float f = pr[j] * mp[j]; kk[j] *= f; qq[j] *= f; }
-      put_mn(A1, tt, c8, kk);
-      put_mn(A2, tt, c8, qq);
-    }
-    #pragma unroll 4
-    for (int x = tid; x < 4 * (Cs - t0) * 2; x += NT) {
-      const int g = x / ((Cs - t0) * 2), rem = x % ((Cs - t0) * 2);
-      const int tt = t0 + rem / 2, c8 = (rem % 2) * 8;
-      float v[8];
-      ld8f(dG + ((int64_t)g * Cs + tt) * Cs + SB * I + c8, v);
-      put_mn(Bm[g], tt, c8, v);
-    }
-    drv.run([&] {
-      const uint32_t c = SB * I;
-      const int k0 = t0, ks = (Cs - t0) / 16;
-      mma_tiles(cta.tmem + 2 * Cs + c, sub_tile(A1, k0, 0), sub_tile(Bm[0], k0, 0), ks, id16m, NS, false);
-      mma_tiles(cta.tmem + 2 * Cs + c, sub_tile(A2, k0, 0), sub_tile(Bm[2], k0, 0), ks, id16m, NS, true);
-      mma_tiles(cta.tmem + 3 * Cs + c, sub_tile(A1, k0, 0), sub_tile(Bm[1], k0, 0), ks, id16m, NS, false);
-      mma_tiles(cta.tmem + 3 * Cs + c, sub_tile(A2, k0, 0), sub_tile(Bm[3], k0, 0), ks, id16m, NS, true);
-    });
-  }
-  // ---- epilogue, one 16-token block at a time; lane = key channel i.
-  // Off-diagonal parts come from TMEM, scaled by pre (left) or suf (right);
-  // blocks without them (J = 0 left, J = nb-1 right) contribute zero. The
-  // block's own 16x16 diagonal part is added exactly on the CUDA cores with
-  // running products: for s <= t in the block, Gam_{t<-s} = prod_{u=s+1..t} alpha_u,
-  //   dK_left_t  += (dM^kk_ts k_s + dM^ka_ts a_s) Gam      dQ_left_t += (dN^qk_ts k_s + dN^qa_ts a_s) Gam
-  //   dK_right_s += (dM^kk_ts k_t + dN^qk_ts qt_t) Gam     dA_right_s += (dM^ka_ts k_t + dN^qa_ts qt_t) Gam
-  const int i = tid & 127, wg = tid >> 7;  // TMEM lane = key channel; warpgroups take alternate blocks
-  float* dgd = reinterpret_cast<float*>(sm + 4 * AB + 8 * BB + nb * DK * 4);  // [nb][4][16][16]
-#pragma unroll 4
-  for (int x = tid; x < nb * 4 * SB * SB; x += NT) {
-    const int J = x / (4 * SB * SB), g = (x / (SB * SB)) % 4, tt = (x / SB) % SB, ss = x % SB;
-    dgd[x] = dG[((int64_t)g * Cs + SB * J + tt) * Cs + SB * J + ss];
-  }
+  float rv[8];
+  ld8f(p.r + (int64_t)s.h * DK + (tid % (DK / 8)) * 8, rv);
   __syncthreads();
-  float* gl = q.gl + u * 4 * Cs * DK;
-  const int ic = i < DK ? i : DK - 1;
-  const float rr = p.r[(int64_t)s.h * DK + ic];
-  const int64_t kstride = (int64_t)p.H * DK;
-  for (int J = wg; J < nb; J += 2) {
-    float raw[4][SB];
+
+  // G_b, K-major: row (p, X, r) -> t = (2p+1) b + r, column (p', Y, r') -> s = 2p'b + r';
+  // dG_{2X+Y}[t][s] when p == p', else 0. Four pieces per thread per batch.
+  auto stage_g = [&](int lb) {
+    const int b = 1 << lb;
+    constexpr int BG = 4;
+    for (int x0 = tid; x0 < Cs << (lcs - 3); x0 += BG * NT) {
+      Pack8<float> gv[BG];
 #pragma unroll
-    for (int reg = 0; reg < 4; ++reg) tmem_ld16(cta.tmem + tmem_lane_base(warp) + reg * Cs + SB * J, raw[reg]);
-    if (i >= DK || !drv.ok) continue;
-    float K[SB], Av[SB], Q[SB], al[SB];
-    const int64_t o0 = toff(p, s.b, s.tok0 + SB * J, s.h, DK) + i;
+      for (int m = 0; m < BG; ++m) {
+        const int x = x0 + m * NT;
+        const int row = x >> (lcs - 3), c8 = (x & ((Cs >> 3) - 1)) << 3;
+        const int pv = row >> (lb + 1), pc = c8 >> (lb + 1);
+        if (x < Cs << (lcs - 3) && pv == pc) {
+          const int X = (row >> lb) & 1, Y = (c8 >> lb) & 1;
+          const int t = (2 * pv + 1) * b + (row & (b - 1)), s0 = 2 * pc * b + (c8 & (b - 1));
+          gv[m].ld(dG + (2 * X + Y) * gsz + (int64_t)t * Cs + s0);
+        }
+      }
 #pragma unroll
-    for (int tt = 0; tt < SB; ++tt) {
-      const int64_t o = o0 + tt * kstride;
-      const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
-      K[tt] = kk;
-      Av[tt] = Elt<T>::ld(static_cast<const T*>(p.e) + o) * kk;
-      Q[tt] = rr * Elt<T>::ld(static_cast<const T*>(p.g) + o) * Elt<T>::ld(static_cast<const T*>(p.q) + o);
-      al[tt] = expf(__ldg(p.la + o));
-    }
-    float dKl[SB], dQl[SB], dKr[SB], dAr[SB];
+      for (int m = 0; m < BG; ++m) {
+        const int x = x0 + m * NT;
+        if (x < Cs << (lcs - 3)) {
+          const int row = x >> (lcs - 3), c8 = (x & ((Cs >> 3) - 1)) << 3;
+          float v[8];
+          if ((row >> (lb + 1)) == (c8 >> (lb + 1))) {
+            gv[m].get(v);
+          } else {
 #pragma unroll
-    for (int tt = 0; tt < SB; ++tt) {
-      const int t = SB * J + tt;
-      const float pr = pre[t * DK + i], sf = suf[t * DK + i];
-      dKl[tt] = J == 0 ? 0.f : raw[0][tt] * pr;
-      dQl[tt] = J == 0 ? 0.f : raw[1][tt] * pr;
-      dKr[tt] = J == nb - 1 ? 0.f : raw[2][tt] * sf;
-      dAr[tt] = J == nb - 1 ? 0.f : raw[3][tt] * sf;
-    }
-    const float* dg = dgd + J * 4 * SB * SB;
-#pragma unroll
-    for (int ss = 0; ss < SB; ++ss) {
-      float gm = 1.f;
-#pragma unroll
-      for (int tt = ss; tt < SB; ++tt) {
-        if (tt > ss) gm *= al[tt];
-        const float mkk = dg[(0 * SB + tt) * SB + ss], mka = dg[(1 * SB + tt) * SB + ss];
-        const float nqk = dg[(2 * SB + tt) * SB + ss], nqa = dg[(3 * SB + tt) * SB + ss];
-        dKl[tt] += (mkk * K[ss] + mka * Av[ss]) * gm;
-        dQl[tt] += (nqk * K[ss] + nqa * Av[ss]) * gm;
-        dKr[ss] += (mkk * K[tt] + nqk * Q[tt]) * gm;
-        dAr[ss] += (mka * K[tt] + nqa * Q[tt]) * gm;
+            for (int j = 0; j < 8; ++j) v[j] = 0.f;
+          }
+          put_k(GT, row, c8, v);
+        }
       }
     }
+  };
+
+  const int i = tid & 127, wg = tid >> 7;  // epilogue: TMEM lane = key channel; warpgroups take alternate blocks
+  const int ic = i < DK ? i : DK - 1;
+  const int64_t kstride = (int64_t)p.H * DK;
+  float* gl = q.gl + u * 4 * Cs * DK;
+  for (int side = 0; side < 2 && drv.ok; ++side) {  // 0: left (dK_left, dQ_left), 1: right (dK_right, dA_right)
+    const uint32_t id = idesc_bf16(128, Cs, 1, side);
+    for (int lev = 0; lev < nlev && drv.ok; ++lev) {
+      const int lb = lcs - 1 - lev;
+      stage_g(lb);
+      stage_level<DK, T>(p, s, pre, suf, ftab + lev * nb * DK, rv, Cs, lb, side == 1, side == 0, OP, OP);
+      drv.run([&] {
+        mma_tiles(cta.tmem + 128 * lev, transposed(OP), side == 0 ? GT : transposed(GT), Cs / 16, id, NS, false);
+      });
+    }
+    if (!drv.ok) break;
+    for (int J = wg; J < nb; J += 2) {
+      float acc[2][SB];
 #pragma unroll
-    for (int tt = 0; tt < SB; ++tt) {
-      const int64_t o = (int64_t)(SB * J + tt) * DK + i;
-      gl[0 * Cs * DK + o] = dKl[tt];
-      gl[1 * Cs * DK + o] = dQl[tt];
-      gl[2 * Cs * DK + o] = dKr[tt];
-      gl[3 * Cs * DK + o] = dAr[tt];
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int tt = 0; tt < SB; ++tt) acc[c][tt] = 0.f;
+      for (int lev = 0; lev < nlev; ++lev) {
+        const int lb = lcs - 1 - lev, b = 1 << lb;
+        const bool upper = ((SB * J) >> lb) & 1;
+        if (upper != (side == 0)) continue;  // warp-uniform
+        const int pv = (SB * J) >> (lb + 1);
+        const int r0 = SB * J - (upper ? (2 * pv + 1) * b : 2 * pv * b);
+        const float f = ftab[(lev * nb + J) * DK + ic];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float v[16];
+          tmem_ld16(cta.tmem + tmem_lane_base(warp) + 128 * lev + pv * 2 * b + c * b + r0, v);
+#pragma unroll
+          for (int tt = 0; tt < SB; ++tt) acc[c][tt] += f * v[tt];
+        }
+      }
+      if (i >= DK) continue;
+      float K[SB], Z[SB], al[SB];  // Z = a (left) or qt (right)
+      const float rr = p.r[(int64_t)s.h * DK + i];
+      const int64_t o0 = toff(p, s.b, s.tok0 + SB * J, s.h, DK) + i;
+#pragma unroll
+      for (int tt = 0; tt < SB; ++tt) {
+        const int64_t o = o0 + tt * kstride;
+        const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
+        K[tt] = kk;
+        Z[tt] = side == 0 ? Elt<T>::ld(static_cast<const T*>(p.e) + o) * kk
+                          : rr * Elt<T>::ld(static_cast<const T*>(p.g) + o) * Elt<T>::ld(static_cast<const T*>(p.q) + o);
+        al[tt] = expf(__ldg(p.la + o));
+      }
+      const float* sc = side == 0 ? pre : suf;
+#pragma unroll
+      for (int tt = 0; tt < SB; ++tt) {
+        const float f = sc[(SB * J + tt) * DK + i];
+        acc[0][tt] *= f;
+        acc[1][tt] *= f;
+      }
+      const float4* dg = dgd + J * SB * SB;
+      if (side == 0) {
+#pragma unroll
+        for (int ss = 0; ss < SB; ++ss) {
+          float gm = 1.f;
+#pragma unroll
+          for (int tt = ss; tt < SB; ++tt) {
+            if (tt > ss) gm *= al[tt];
+            const float4 g = dg[tt * SB + ss];
+            acc[0][tt] += (g.x * K[ss] + g.y * Z[ss]) * gm;  // dK_left
+            acc[1][tt] += (g.z * K[ss] + g.w * Z[ss]) * gm;  // dQ_left
+          }
+        }
+      } else {
+#pragma unroll
+        for (int ss = 0; ss < SB; ++ss) {
+          float gm = 1.f;
+#pragma unroll
+          for (int tt = ss; tt < SB; ++tt) {
+            if (tt > ss) gm *= al[tt];
+            const float4 g = dg[tt * SB + ss];
+            acc[0][ss] += (g.x * K[tt] + g.z * Z[tt]) * gm;  // dK_right
+            acc[1][ss] += (g.y * K[tt] + g.w * Z[tt]) * gm;  // dA_right
+          }
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < SB; ++tt) {
+        const int64_t o = (int64_t)(SB * J + tt) * DK + i;
+        gl[(2 * side + 0) * Cs * DK + o] = acc[0][tt];
+        gl[(2 * side + 1) * Cs * DK + o] = acc[1][tt];
+      }
     }
   }
   cta.finish();
