@@ -76,6 +76,12 @@ def kernel_model(C, dk, dv, es):
     return m
 
 
+# DRAM bytes (read + write) per unit of the dominant kernel, from the ncu capture summarised in
+# profiles/gram_and_bwd_gram_B1_T16384_H16_d128_C128.md (2,048 units; traffic scales with units).
+# Only valid for the kernel version that capture measured: clear an entry when its kernel changes.
+NCU_TRAFFIC_PER_UNIT = {"bwd_gram": 1641.9e6 / 2048, "gram": 1129.1e6 / 2048}
+
+
 def algorithmic_step():
     """Work of one fwd+bwd step of the whole path (per head-token figures of the
     survey's measurement section, at C = 128, d = 128): flops and bytes."""
@@ -403,7 +409,8 @@ def main():
         ach = by_l / t_s / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s"}
     roof["frac"] = round(ach / roof["peak"], 4)
-    roof["traffic"] = None
+    tr = NCU_TRAFFIC_PER_UNIT.get(base)
+    roof["traffic"] = round(tr * units / launches_per_step) if tr is not None else None
     roof["kernel"] = name
     roof["peak_source"] = pk["src"]
     line["roofline"] = roof
