@@ -540,12 +540,27 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
 //                dY_right_s += suf16_s F_J(s) D^T[., (Y, s)]
 // Each phase keeps its levels in TMEM (128 columns each), so every output is
 // formed once in the epilogue together with its exact diagonal-block part
-// (CUDA cores, running products) and written once.
+// (CUDA cores; the same tree inside the block, down to single tokens) and
+// written once.
 // ---------------------------------------------------------------------------
+// Shared memory of bwd_gram_kernel: the operand and dG tiles, which the
+// epilogue reuses for the raw rows of its diagonal blocks (bf16 inputs: k and
+// e, or k, g and q, plus log alpha), then the dG diagonal blocks and the tables.
+template <int DK>
+__host__ __device__ constexpr size_t bwd_gram_front_bytes() {
+  constexpr size_t tiles = 2u * 128u * DK * 2u + 2u * 128u * 128u * 2u;
+  constexpr size_t rows = 3u * 128u * DK * 2u + 128u * DK * 4u;
+  return tiles > rows ? tiles : rows;
+}
+template <int DK>
+__host__ __device__ constexpr size_t bwd_gram_smem_bytes() {
+  return bwd_gram_front_bytes<DK>() + 8u * SB * SB * 16u + (size_t)kMaxLev * 8u * DK * 4u;
+}
+
 template <int DK, typename T, int NS>
 __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
   constexpr int NT = 256;
   const int Cs = p.Cs, nb = Cs / SB, nlev = tree_levels(Cs), lcs = log2_cs(Cs);
@@ -557,8 +572,17 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
   const uint32_t GB = 128u * (uint32_t)Cs * 2u;  // dG tile (128 rows x Cs), one half
   const Tile OP{base, base + OB, 128u, DK * 16u};  // YL (left phase) or XL (right phase)
   const Tile GT{base + 2 * OB, base + 2 * OB + GB, 128u, (uint32_t)Cs * 16u};
-  float4* dgd = reinterpret_cast<float4*>(sm + 2 * OB + 2 * GB);  // [nb][16 t][16 s]: mkk, mka, nqk, nqa
-  float* ftab = reinterpret_cast<float*>(sm + 2 * OB + 2 * GB + (size_t)nb * SB * SB * 16);  // [kMaxLev][nb][DK]
+  constexpr size_t FB = bwd_gram_front_bytes<DK>();
+  float4* dgd = reinterpret_cast<float4*>(sm + FB);  // [nb][16 t][16 s]: mkk, mka, nqk, nqa
+  float* ftab = reinterpret_cast<float*>(sm + FB + 8 * SB * SB * 16);  // [kMaxLev][nb][DK]
+  constexpr bool kRowsInSmem = sizeof(T) == 2;
+  constexpr uint32_t RB = 128u * DK * 2u;  // one bf16 [128][DK] array of raw rows
+  const T* rk = reinterpret_cast<const T*>(sm);
+  const T* rz1 = reinterpret_cast<const T*>(sm + RB);
+  const T* rz2 = reinterpret_cast<const T*>(sm + 2 * RB);
+  const float* rla = reinterpret_cast<const float*>(sm + 3 * RB);
+  uint32_t cp_phase = 0;
+  if (tid == 0) mbar_init(&bar_cp, 1);
   TcCta cta;
   cta.init(&tslot, &bar, tmem_cols_for(128 * nlev));
   MmaSync drv{&bar, 0u, true};
@@ -627,6 +651,28 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
       });
     }
     if (!drv.ok) break;
+    if constexpr (kRowsInSmem) {
+      // raw rows of the unit for the diagonal blocks, one bulk copy per (array, token):
+      // left k, e (, -), log alpha; right k, g, q, log alpha
+      const int na = side == 0 ? 2 : 3;
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0) mbar_expect_tx(&bar_cp, (uint32_t)Cs * DK * (2u * na + 4u));
+      for (int x = tid; x < Cs * 4; x += NT) {
+        const int a = x / Cs, tok = x % Cs;
+        const int64_t o = toff(p, s.b, s.tok0 + tok, s.h, DK);
+        if (a < na) {
+          const void* src = a == 0 ? p.k : (side == 0 ? p.e : (a == 1 ? p.g : p.q));
+          bulk_g2s(base + a * RB + tok * DK * 2, static_cast<const T*>(src) + o, DK * 2, &bar_cp);
+        } else if (a == 3) {
+          bulk_g2s(base + 3 * RB + tok * DK * 4, p.la + o, DK * 4, &bar_cp);
+        }
+      }
+      const bool ok = mbar_wait(&bar_cp, cp_phase);
+      cp_phase ^= 1u;
+      if (!__syncthreads_and(ok ? 1 : 0)) drv.ok = false;
+      if (!drv.ok) break;
+    }
     for (int J = wg; J < nb; J += 2) {
       float acc[2][SB];
 #pragma unroll
@@ -651,15 +697,26 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
       if (i >= DK) continue;
       float K[SB], Z[SB], al[SB];  // Z = a (left) or qt (right)
       const float rr = p.r[(int64_t)s.h * DK + i];
-      const int64_t o0 = toff(p, s.b, s.tok0 + SB * J, s.h, DK) + i;
+      if constexpr (kRowsInSmem) {
 #pragma unroll
-      for (int tt = 0; tt < SB; ++tt) {
-        const int64_t o = o0 + tt * kstride;
-        const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
-        K[tt] = kk;
-        Z[tt] = side == 0 ? Elt<T>::ld(static_cast<const T*>(p.e) + o) * kk
-                          : rr * Elt<T>::ld(static_cast<const T*>(p.g) + o) * Elt<T>::ld(static_cast<const T*>(p.q) + o);
-        al[tt] = expf(__ldg(p.la + o));
+        for (int tt = 0; tt < SB; ++tt) {
+          const int ro = (SB * J + tt) * DK + i;
+          const float kk = __bfloat162float(rk[ro]);
+          K[tt] = kk;
+          Z[tt] = side == 0 ? __bfloat162float(rz1[ro]) * kk : rr * __bfloat162float(rz1[ro]) * __bfloat162float(rz2[ro]);
+          al[tt] = expf(rla[ro]);
+        }
+      } else {
+        const int64_t o0 = toff(p, s.b, s.tok0 + SB * J, s.h, DK) + i;
+#pragma unroll
+        for (int tt = 0; tt < SB; ++tt) {
+          const int64_t o = o0 + tt * kstride;
+          const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
+          K[tt] = kk;
+          Z[tt] = side == 0 ? Elt<T>::ld(static_cast<const T*>(p.e) + o) * kk
+                            : rr * Elt<T>::ld(static_cast<const T*>(p.g) + o) * Elt<T>::ld(static_cast<const T*>(p.q) + o);
+          al[tt] = expf(__ldg(p.la + o));
+        }
       }
       const float* sc = side == 0 ? pre : suf;
 #pragma unroll
@@ -668,29 +725,74 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
         acc[0][tt] *= f;
         acc[1][tt] *= f;
       }
+      // Diagonal block, exact: pairs ss < tt inside the block go by sub-pivots
+      // (halves of 8, 4, 2, 1 tokens), where Gam_{tt<-ss} = fac_tt * fac_ss with
+      // fac the running product from the sub-pivot forward (upper tt) or backward
+      // (lower ss); the pairs tt == ss have Gam = 1.
       const float4* dg = dgd + J * SB * SB;
-      if (side == 0) {
 #pragma unroll
-        for (int ss = 0; ss < SB; ++ss) {
-          float gm = 1.f;
+      for (int tt = 0; tt < SB; ++tt) {  // tt == ss
+        const float4 g = dg[tt * SB + tt];
+        if (side == 0) {
+          acc[0][tt] += g.x * K[tt] + g.y * Z[tt];
+          acc[1][tt] += g.z * K[tt] + g.w * Z[tt];
+        } else {
+          acc[0][tt] += g.x * K[tt] + g.z * Z[tt];
+          acc[1][tt] += g.y * K[tt] + g.w * Z[tt];
+        }
+      }
 #pragma unroll
-          for (int tt = ss; tt < SB; ++tt) {
-            if (tt > ss) gm *= al[tt];
-            const float4 g = dg[tt * SB + ss];
-            acc[0][tt] += (g.x * K[ss] + g.y * Z[ss]) * gm;  // dK_left
-            acc[1][tt] += (g.z * K[ss] + g.w * Z[ss]) * gm;  // dQ_left
+      for (int sl = 0; sl < 4; ++sl) {
+        const int hb = 8 >> sl;  // half-length of this sub-level
+        float fac[SB], sk[SB], sz[SB];
+#pragma unroll
+        for (int b0 = 0; b0 < SB; b0 += 2 * hb) {
+          float run = 1.f;
+#pragma unroll
+          for (int uu = b0 + hb; uu < b0 + 2 * hb; ++uu) {  // upper: from the sub-pivot forward
+            run *= al[uu];
+            fac[uu] = run;
+          }
+          run = 1.f;
+#pragma unroll
+          for (int uu = b0 + hb - 1; uu >= b0; --uu) {  // lower: from the sub-pivot backward
+            fac[uu] = run;
+            run *= al[uu];
           }
         }
-      } else {
 #pragma unroll
-        for (int ss = 0; ss < SB; ++ss) {
-          float gm = 1.f;
+        for (int uu = 0; uu < SB; ++uu) {
+          sk[uu] = K[uu] * fac[uu];
+          sz[uu] = Z[uu] * fac[uu];
+        }
 #pragma unroll
-          for (int tt = ss; tt < SB; ++tt) {
-            if (tt > ss) gm *= al[tt];
-            const float4 g = dg[tt * SB + ss];
-            acc[0][ss] += (g.x * K[tt] + g.z * Z[tt]) * gm;  // dK_right
-            acc[1][ss] += (g.y * K[tt] + g.w * Z[tt]) * gm;  // dA_right
+        for (int b0 = 0; b0 < SB; b0 += 2 * hb) {
+          if (side == 0) {
+#pragma unroll
+            for (int tt = b0 + hb; tt < b0 + 2 * hb; ++tt) {
+              float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+              for (int ss = b0; ss < b0 + hb; ++ss) {
+                const float4 g = dg[tt * SB + ss];
+                a0 += g.x * sk[ss] + g.y * sz[ss];  // dK_left
+                a1 += g.z * sk[ss] + g.w * sz[ss];  // dQ_left
+              }
+              acc[0][tt] += fac[tt] * a0;
+              acc[1][tt] += fac[tt] * a1;
+            }
+          } else {
+#pragma unroll
+            for (int ss = b0; ss < b0 + hb; ++ss) {
+              float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+              for (int tt = b0 + hb; tt < b0 + 2 * hb; ++tt) {
+                const float4 g = dg[tt * SB + ss];
+                a0 += g.x * sk[tt] + g.z * sz[tt];  // dK_right
+                a1 += g.y * sk[tt] + g.w * sz[tt];  // dA_right
+              }
+              acc[0][ss] += fac[ss] * a0;
+              acc[1][ss] += fac[ss] * a1;
+            }
           }
         }
       }
@@ -701,6 +803,7 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
         gl[(2 * side + 1) * Cs * DK + o] = acc[1][tt];
       }
     }
+    __syncthreads();  // the raw rows are read; the next phase restages over them
   }
   cta.finish();
 }
