@@ -187,6 +187,53 @@ __device__ __forceinline__ void bulk_g2s_big(uint32_t dst, const uint8_t* src, u
   }
 }
 
+// Stage a contiguous fp32 matrix src[rows][cols] (rows, cols multiples of 8,
+// rows * cols <= 128 * 128) times `sign` as a bf16 hi/lo operand tile: K-major
+// over cols (put_k, row = MN index) or, with MN, MN-major over rows (put_mn,
+// row = K index). The raw matrix arrives by bulk copy into the tile's own
+// shared memory (hi and lo halves contiguous, at least 4 bytes per element),
+// every thread takes its pieces into registers, and after a barrier writes them
+// back converted. 256 threads, all of which call it; no MMA may be reading the
+// tile. Returns false if the copy's bounded wait ran out.
+template <bool MN>
+__device__ __forceinline__ bool stage_raw(const Tile& t, const float* src, int rows, int cols, float sign,
+                                          uint64_t* bar, uint32_t& phase) {
+  constexpr int NT = 256, MAXP = 128 * 128 / 8 / NT;
+  const uint32_t bytes = (uint32_t)rows * (uint32_t)cols * 4u;
+  fence_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(bar, bytes);
+    bulk_g2s_big(t.hi, reinterpret_cast<const uint8_t*>(src), bytes, bar);
+  }
+  const bool ok = __syncthreads_and(mbar_wait(bar, phase) ? 1 : 0) != 0;
+  phase ^= 1u;
+  const float4* raw = reinterpret_cast<const float4*>(__cvta_shared_to_generic(t.hi));
+  const int np = rows * cols / 8;
+  float v[MAXP][8];
+#pragma unroll
+  for (int k = 0; k < MAXP; ++k) {
+    const int x = threadIdx.x + k * NT;
+    if (x < np) {
+      const float4 a = raw[2 * x], b = raw[2 * x + 1];
+      v[k][0] = sign * a.x; v[k][1] = sign * a.y; v[k][2] = sign * a.z; v[k][3] = sign * a.w;
+      v[k][4] = sign * b.x; v[k][5] = sign * b.y; v[k][6] = sign * b.z; v[k][7] = sign * b.w;
+    }
+  }
+  __syncthreads();
+  const int g = cols / 8;
+#pragma unroll
+  for (int k = 0; k < MAXP; ++k) {
+    const int x = threadIdx.x + k * NT;
+    if (x < np) {
+      const int r = x / g, c8 = (x % g) * 8;
+      if (MN) put_mn(t, r, c8, v[k]);
+      else put_k(t, r, c8, v[k]);
+    }
+  }
+  return ok;
+}
+
 // CTA prologue shared by the tensor-core kernels: TMEM allocation + mbarrier.
 struct TcCta {
   uint32_t tmem;

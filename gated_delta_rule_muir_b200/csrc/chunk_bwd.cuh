@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
 template <int DK, int DV, typename T, int NS>
 __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
+  __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
@@ -424,6 +424,8 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   const Tile R1{base + 2 * TB, base + 3 * TB, 128u, DV * 16u};
   const Tile R2{base + 4 * TB, base + 5 * TB, 128u, DV * 16u};
   zero_smem(base, 6 * TB);
+  if (tid == 0) mbar_init(&bar_cp, 1);
+  uint32_t cph = 0;
   TcCta cta;
   cta.init(&tslot, &bar, 512);
   MmaSync drv{&bar, 0u, true};
@@ -456,18 +458,18 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   };
   // Row t of a [Cs][N] TMEM result -> dst (fp32, row-major, row stride ld), optional mask.
   auto drain = [&](uint32_t col, int n, float* dst, int64_t ld, int mask) {
-    for (int c = wg * 16; c < n; c += 32) {
-      float v[16];
-      tmem_ld16(cta.tmem + lane + col + c, v);
+    for (int c = wg * 32; c < n; c += 64) {
+      float v[32];
+      tmem_ld32(cta.tmem + lane + col + c, v);
       if (t < Cs && drv.ok) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 32; ++j) {
           const int sidx = c + j;
           if (mask == 1 && sidx >= t) v[j] = 0.f;  // strictly lower
           if (mask == 2 && sidx > t) v[j] = 0.f;   // lower incl. diagonal
         }
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
+        for (int j = 0; j < 32; j += 4)
           *reinterpret_cast<float4*>(dst + t * ld + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       }
     }
@@ -487,9 +489,9 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   }
   float* dG = q.dG + u * 4 * Cs * Cs;
   // pass 1
-  stage_rows_k(R0, q.dSC + u * DK * DV, DK, DV, DV, 1.f);
+  if (!stage_raw<false>(R0, q.dSC + u * DK * DV, DK, DV, 1.f, &bar_cp, cph)) drv.ok = false;
   stage_U(R1);
-  stage_rows_k(R2, q.P + u * Cs * DV, Cs, DV, DV, -1.f);
+  if (!stage_raw<false>(R2, q.P + u * Cs * DV, Cs, DV, -1.f, &bar_cp, cph)) drv.ok = false;
   drv.run([&] {
     mma_tiles(cta.tmem + 0, R1, R0, DV / 16, idK, NS, false);
     mma_tiles(cta.tmem + 128, R2, R0, DV / 16, idK, NS, false);
@@ -502,7 +504,7 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
     mma_tiles(cta.tmem + 0, R0, R1, DV / 16, idC, NS, false);    // dN^qk
     mma_tiles(cta.tmem + 128, R0, R2, DV / 16, idC, NS, false);  // dN^qa
   });
-  stage_rows_k(R0, q.dZ + u * Cs * DV, Cs, DV, DV, 1.f);
+  if (!stage_raw<false>(R0, q.dZ + u * Cs * DV, Cs, DV, 1.f, &bar_cp, cph)) drv.ok = false;
   drv.run([&] {
     mma_tiles(cta.tmem + 256, R0, R1, DV / 16, idC, NS, false);  // dM^kk
     mma_tiles(cta.tmem + 384, R0, R2, DV / 16, idC, NS, false);  // dM^ka
@@ -512,9 +514,9 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   drain(256, Cs, dG + 0 * Cs * Cs, Cs, 1);
   drain(384, Cs, dG + 1 * Cs * Cs, Cs, 1);
   // pass 3: R1 = S0, R0 = dO, R2 = dZ
-  stage_rows_k(R1, q.S_chunks + u * DK * DV, DK, DV, DV, 1.f);
+  if (!stage_raw<false>(R1, q.S_chunks + u * DK * DV, DK, DV, 1.f, &bar_cp, cph)) drv.ok = false;
   stage_dO(R0);
-  stage_rows_k(R2, q.dZ + u * Cs * DV, Cs, DV, DV, 1.f);
+  if (!stage_raw<false>(R2, q.dZ + u * Cs * DV, Cs, DV, 1.f, &bar_cp, cph)) drv.ok = false;
   drv.run([&] {
     mma_tiles(cta.tmem + 0, R0, R1, DV / 16, idK, NS, false);    // dQp
     mma_tiles(cta.tmem + 128, R2, R1, DV / 16, idK, NS, false);  // dKp
