@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(128) decay_kernel(ChunkParams p) {
   const float* la = p.la + toff(p, s.b, s.tok0, s.h, dk) + i;
   const int64_t stride = (int64_t)p.H * dk;
   float run = 1.f, before = 1.f;
+#pragma unroll 16
   for (int t = 0; t < Cs; ++t) {
     const float a = expf(__ldg(la + t * stride));
     if ((t & (SB - 1)) == 0) {
@@ -317,6 +318,7 @@ __global__ void __launch_bounds__(128) decay_kernel(ChunkParams p) {
     gam[t * dk + i] = before * run;
   }
   float after = 1.f, srun = 1.f;
+#pragma unroll 16
   for (int t = Cs - 1; t >= 0; --t) {
     if ((t & (SB - 1)) == SB - 1) {
       srun = 1.f;

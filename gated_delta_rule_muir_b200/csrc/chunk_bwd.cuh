@@ -834,15 +834,17 @@ __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q
     const int64_t o0 = toff(p, s.b, s.tok0, s.h, DK) + i;
     // The terms that land on the last token's cumulative log-decay enter every
     // dlog_alpha of the unit: gather them first.
-    float E = gam[(Cs - 1) * DK + i] * q.dgc[u * DK + i];
+    float E = __ldg(gam + (Cs - 1) * DK + i) * __ldg(q.dgc + u * DK + i);
+#pragma unroll 8
     for (int tt = 0; tt < Cs; ++tt) {
       const int64_t o = o0 + tt * stride_k;
       const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
       const float ee = Elt<T>::ld(static_cast<const T*>(p.e) + o);
       const int ti = tt * DK + i;
-      E += kk * gsuf[ti] * (g4[2 * Cs * DK + ti] + ee * g4[3 * Cs * DK + ti]);
+      E += kk * __ldg(gsuf + ti) * (__ldg(g4 + 2 * Cs * DK + ti) + ee * __ldg(g4 + 3 * Cs * DK + ti));
     }
     float run = E, dr_acc = 0.f;
+#pragma unroll 8
     for (int tt = Cs - 1; tt >= 0; --tt) {
       const int64_t o = o0 + tt * stride_k;
       const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
@@ -851,11 +853,11 @@ __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q
       const float qq = Elt<T>::ld(static_cast<const T*>(p.q) + o);
       const float a = ee * kk, qt = rr * gg * qq;
       const int ti = tt * DK + i;
-      const float G = gam[ti], Gs = gsuf[ti];
-      const float dQp = g4[0 * Cs * DK + ti], dKp = g4[1 * Cs * DK + ti];
-      const float dKs = g4[2 * Cs * DK + ti], dAs = g4[3 * Cs * DK + ti];
-      const float dKl = gl[0 * Cs * DK + ti], dQl = gl[1 * Cs * DK + ti];
-      const float dKr = gl[2 * Cs * DK + ti], dAr = gl[3 * Cs * DK + ti];
+      const float G = __ldg(gam + ti), Gs = __ldg(gsuf + ti);
+      const float dQp = __ldg(g4 + 0 * Cs * DK + ti), dKp = __ldg(g4 + 1 * Cs * DK + ti);
+      const float dKs = __ldg(g4 + 2 * Cs * DK + ti), dAs = __ldg(g4 + 3 * Cs * DK + ti);
+      const float dKl = __ldg(gl + 0 * Cs * DK + ti), dQl = __ldg(gl + 1 * Cs * DK + ti);
+      const float dKr = __ldg(gl + 2 * Cs * DK + ti), dAr = __ldg(gl + 3 * Cs * DK + ti);
       run += kk * dKl + qt * dQl - kk * dKr - a * dAr + kk * G * dKp + qt * G * dQp - kk * Gs * dKs - a * Gs * dAs;
       q.dla[o] = run;
       const float dqt = dQl + G * dQp;
@@ -872,9 +874,10 @@ __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q
   if (i < DV) {
     const float* dU = q.dU + u * Cs * DV;
     const int64_t o0 = toff(p, s.b, s.tok0, s.h, DV) + i;
+#pragma unroll 8
     for (int tt = 0; tt < Cs; ++tt) {
       const int64_t o = o0 + tt * stride_v;
-      const float du = dU[tt * DV + i];
+      const float du = __ldg(dU + tt * DV + i);
       Elt<T>::st(static_cast<T*>(q.dv) + o, Elt<T>::ld(static_cast<const T*>(p.w) + o) * du);
       Elt<T>::st(static_cast<T*>(q.dw) + o, Elt<T>::ld(static_cast<const T*>(p.v) + o) * du);
     }

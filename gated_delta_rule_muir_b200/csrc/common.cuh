@@ -51,7 +51,7 @@ template <> struct Elt<float> {
 
 template <> struct Elt<__nv_bfloat16> {
   using T = __nv_bfloat16;
-  static __device__ __forceinline__ float ld(const T* p) { return __bfloat162float(p[0]); }
+  static __device__ __forceinline__ float ld(const T* p) { return __bfloat162float(__ldg(p)); }
   static __device__ __forceinline__ void ld8g(const T* p, float (&o)[8]) {
     const uint4 u = *reinterpret_cast<const uint4*>(p);
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
