@@ -469,8 +469,12 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
           if (mask == 2 && sidx > t) v[j] = 0.f;   // lower incl. diagonal
         }
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + t * ld + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int j = 0; j < 32; j += 8) {
+          float w8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w8[e] = v[j + e];
+          stg256(dst + t * ld + c + j, w8);  // whole 32-byte sectors
+        }
       }
     }
   };
