@@ -859,17 +859,13 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
       float v[16];
       tmem_ld16(cta.tmem + lane + cW + c, v);
       if (t < Cs)
-#pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(wo + t * DK + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        stg_row16(wo + t * DK + c, v);
     }
     for (int c = wg * 16; c < DV; c += 32) {
       float v[16];
       tmem_ld16(cta.tmem + lane + cUt + c, v);
       if (t < Cs)
-#pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(uo + t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        stg_row16(uo + t * DV + c, v);
     }
   }
   // ---- phase 2 with W in B1: Phi = Diag(Gam_C) - (A*Gsuf)^T W, N^qa W (Q' = Qt*Gam - N^qa W in the epilogue)
@@ -912,8 +908,7 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
     tmem_ld16(cta.tmem + lane + cPsi + c, v);
     if (t < DK && drv.ok) {
       float* o = psi + ((int64_t)(c >> 5) * DK + t) * 32 + (c & 31);
-#pragma unroll
-      for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      stg_row16(o, v);
     }
   }
   for (int c = wg * 16; c < DK; c += 32) {
@@ -939,9 +934,7 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cOl + c, v);
     if (t < Cs && drv.ok) {
-#pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(ol + (int64_t)t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      stg_row16(ol + (int64_t)t * DV + c, v);
     }
   }
   cta.finish();

@@ -241,11 +241,13 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
     tmem_ld16(cta.tmem + lane + c, v);
     tmem_ld16(cta.tmem + lane + 128 + c, w);
     if (t < Cs && drv.ok) {
+      float pv[16];
 #pragma unroll
       for (int j = 0; j < 16; j += 4) {
         const float4 a = *reinterpret_cast<const float4*>(Ut + t * DV + c + j);
-        *reinterpret_cast<float4*>(P + t * DV + c + j) = make_float4(v[j] + a.x, v[j + 1] + a.y, v[j + 2] + a.z, v[j + 3] + a.w);
+        pv[j] = v[j] + a.x; pv[j + 1] = v[j + 1] + a.y; pv[j + 2] = v[j + 2] + a.z; pv[j + 3] = v[j + 3] + a.w;
       }
+      stg_row16(P + t * DV + c, pv);
       if (p.dz && p.z) {
         const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DV) + c;
 #pragma unroll
@@ -266,8 +268,7 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
     tmem_ld16(cta.tmem + lane + 256 + c, v);
     if (t < DK && drv.ok) {
       float* o = E + ((int64_t)(c >> 5) * DK + t) * 32 + (c & 31);
-#pragma unroll
-      for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      stg_row16(o, v);
     }
   }
   (void)rows;
@@ -382,9 +383,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
       put_mn(B3, t, c, a8);
       put_mn(B3, t, c + 8, b8);
       if (drv.ok)
-#pragma unroll
-        for (int j = 0; j < 16; j += 4)
-          *reinterpret_cast<float4*>(dZo + t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        stg_row16(dZo + t * DV + c, v);
     }
   }
   load_img(G + 0 * sq_bytes(Cs));  // M^kk^T
@@ -394,9 +393,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
     float v[16];
     tmem_ld16(cta.tmem + lane + cU + c, v);
     if (t < Cs && drv.ok)
-#pragma unroll
-      for (int j = 0; j < 16; j += 4)
-        *reinterpret_cast<float4*>(dUo + t * DV + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      stg_row16(dUo + t * DV + c, v);
   }
   cta.finish();
 }

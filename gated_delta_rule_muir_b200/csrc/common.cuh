@@ -127,6 +127,15 @@ __device__ __forceinline__ void stg256(float* p, const float (&v)[8]) {
                : "memory");
 }
 
+// 16 floats (p 32-byte aligned) in two 32-byte stores.
+__device__ __forceinline__ void stg_row16(float* p, const float (&v)[16]) {
+  float a[8], b[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) { a[j] = v[j]; b[j] = v[8 + j]; }
+  stg256(p, a);
+  stg256(p + 8, b);
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
