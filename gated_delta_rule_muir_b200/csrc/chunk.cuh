@@ -1102,7 +1102,7 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
       if (p.S_chunks) {
         float* o = p.S_chunks + ((uid_of(n) * DK) + tid) * dv + slab * NW;
 #pragma unroll
-        for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(st[j], st[j + 1], st[j + 2], st[j + 3]);
+        for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&st[j]));
       }
 #pragma unroll
       for (int j = 0; j < NW; j += 8) {
@@ -1118,8 +1118,7 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
     drv.run([&] { mma_tiles(cta.tmem, Phi, Sb, DK / 16, id, NS, false); });
     if (!drv.ok) break;
     float v[NW];
-    tmem_ld16(cta.tmem + lane, *reinterpret_cast<float(*)[16]>(&v[0]));
-    tmem_ld16(cta.tmem + lane + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+    tmem_ld32(cta.tmem + lane, v);
     if (tid < DK) {
       const float* add = psi_s + buf * (PS / 4) + tid * NW;
 #pragma unroll
@@ -1134,7 +1133,7 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
   if (p.S_T && tid < DK && drv.ok) {
     float* o = p.S_T + (((int64_t)b * p.H + h) * DK + tid) * dv + slab * NW;
 #pragma unroll
-    for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(st[j], st[j + 1], st[j + 2], st[j + 3]);
+    for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&st[j]));
   }
   cta.finish();
 }

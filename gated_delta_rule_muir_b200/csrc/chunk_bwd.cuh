@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
     if (tid < DK) {
       float* o = q.dSC + (uid_of(n) * DK + tid) * dv + slab * NW;
 #pragma unroll
-      for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(ds[j], ds[j + 1], ds[j + 2], ds[j + 3]);
+      for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&ds[j]));
 #pragma unroll
       for (int j = 0; j < NW; j += 8) {
         float v[8];
@@ -123,8 +123,7 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
     drv.run([&] { mma_tiles(cta.tmem, PhiT, Bt, DK / 16, id, NS, false); });
     if (!drv.ok) break;
     float v[NW];
-    tmem_ld16(cta.tmem + lane, *reinterpret_cast<float(*)[16]>(&v[0]));
-    tmem_ld16(cta.tmem + lane + 16, *reinterpret_cast<float(*)[16]>(&v[16]));
+    tmem_ld32(cta.tmem + lane, v);
     if (tid < DK) {
       const float* add = e_s + buf * (ES / 4) + tid * NW;
 #pragma unroll
@@ -139,7 +138,7 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
   if (q.dS0 && tid < DK && drv.ok) {
     float* o = q.dS0 + (((int64_t)b * p.H + h) * DK + tid) * dv + slab * NW;
 #pragma unroll
-    for (int j = 0; j < NW; j += 4) *reinterpret_cast<float4*>(o + j) = make_float4(ds[j], ds[j + 1], ds[j + 2], ds[j + 3]);
+    for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&ds[j]));
   }
   cta.finish();
 }
