@@ -187,6 +187,22 @@ class Step:
                                 use_saved=True)
 
 
+def max_over_ranks(ms, device):
+    """The slowest rank's time: every rank contributes its own device time and
+    gets back the maximum (the whole job is done when the last replica is)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_rank, ms_per_step):
+    """Whole-job tokens/s of `world` replicas that each process `tokens_per_rank`
+    tokens per step, timed by the slowest rank."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def time_steps(fn, steps, dist_on):
     import torch
     import torch.distributed as dist
@@ -201,9 +217,7 @@ def time_steps(fn, steps, dist_on):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     if dist_on:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, "cuda")
         dist.barrier()
     return ms
 
@@ -372,7 +386,7 @@ def main():
         ms = time_steps(step, args.steps, dist_on) / args.steps
         launches = (muir.launch_count() - n0)
     tok = WL["B"] * WL["T"]
-    value = world * tok / (ms * 1e-3)
+    value = job_throughput(world, tok, ms)
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
