@@ -66,7 +66,8 @@ def kernel_model(C, dk, dv, es):
     m["scan"] = (2 * (dk + C) * dk * dv, (dk + C) * (dk + dv) * f4 + 2 * C * dv * es)
     m["scan_recompute"] = (2 * (dk + C) * dk * dv, (dk + C) * (dk + dv) * f4 + dk * dv * f4 + 2 * C * dv * es)
     m["rscan"] = (2 * (dk + C) * dk * dv, (dk + C) * dk * f4 + 2 * dk * dv * f4 + 2 * C * dv * es)
-    m["bwd_p"] = (2 * C * dk * dv, C * dk * f4 + 2 * dk * dv * f4 + 2 * C * dv * f4)
+    m["out"] = (2 * C * dk * dv, C * dk * f4 + dk * dv * f4 + C * dv * f4 + 2 * C * dv * es)
+    m["bwd_pe"] = (3 * 2 * C * dk * dv, 2 * C * dk * f4 + 2 * dk * dv * f4 + 3 * C * dv * f4 + 3 * C * dv * es)
     m["bwd_dz"] = (2 * (tri * dv + C * dk * dv + tri * dv + tri * dv + C * dk * dv + tri * dv),
                    3 * C * C * f4 + 2 * C * dv * es + dk * dv * f4 + 2 * C * dk * es + 2 * C * dv * f4)
     m["bwd_grads"] = (2 * (4 * C * dk * dv + 4 * tri * dv),
@@ -80,6 +81,18 @@ def kernel_model(C, dk, dv, es):
 # profiles/gram_and_bwd_gram_B1_T16384_H16_d128_C128.md (2,048 units; traffic scales with units).
 # Only valid for the kernel version that capture measured: clear an entry when its kernel changes.
 NCU_TRAFFIC_PER_UNIT = {"gram": 1129.1e6 / 2048}
+
+
+def flop_split(C, dk, dv):
+    """Share of the step's modelled flops issued on the tensor cores; the rest (the
+    exact 16x16 diagonal Gram blocks, forward and backward) runs on the CUDA cores."""
+    m = kernel_model(C, dk, dv, 2)
+    alu = 4 * 2 * C * 8.5 * dk + 4 * 2 * 2 * C * 8.5 * dk
+    fwd = ("decay", "gram", "solve", "maps", "scan", "out")
+    bwd = ("bwd_pe", "rscan", "bwd_dz", "bwd_grads", "bwd_gram", "bwd_final")
+    total = sum(m[k][0] for k in fwd + bwd if k in m)
+    return {"mma_share": round(1.0 - alu / total, 4), "alu_share": round(alu / total, 4),
+            "note": "per unit of the step's kernels as modelled; the pages report 98% on matrix units"}
 
 
 def algorithmic_step():
@@ -223,7 +236,8 @@ def time_steps(fn, steps, dist_on):
 
 
 def bench_decode(dev, steps, warmup, pk):
-    """Decode GB/s: one launch over all 24 layers x batch rows (per-row readout scale)."""
+    """Decode GB/s of one token through all 24 layers: one launch over the 24 x batch
+    rows (per-row readout scale), and a CUDA graph of 24 per-layer launches."""
     import torch
     import gated_delta_rule_muir_b200 as muir
     out = {}
@@ -247,10 +261,28 @@ def bench_decode(dev, steps, warmup, pk):
             fn()
         reps = max(steps, 20)
         ms = time_steps(fn, reps, False) / reps
+        # the same token as a CUDA graph of 24 per-layer launches (batch rows each)
+        sl = [slice(l * nb, (l + 1) * nb) for l in range(L)]
+        layer_calls = lambda: [muir.decode_step(S[i], q[i], k[i], v[i], e[i], w[i], gg[i], z[i], la[i], r[i], y=y[i])
+                               for i in sl]
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            layer_calls()  # warm-up outside the capture
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer_calls()
+        for _ in range(max(warmup, 3)):
+            graph.replay()
+        ms_g = time_steps(graph.replay, reps, False) / reps
+        del graph
         state_bytes = 2.0 * n * H * dk * dv * 4
         io_bytes = n * H * (5 * dk * 2 + dk * 4 + dk * 4 + 3 * dv * 2 + dv * 2)
         gbs = (state_bytes + io_bytes) / (ms * 1e-3) / 1e9
+        gbs_g = (state_bytes + io_bytes) / (ms_g * 1e-3) / 1e9
         out[f"batch{nb}"] = {"ms_per_token": round(ms, 4), "GB_s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 3),
+                             "graph24_ms_per_token": round(ms_g, 4), "graph24_GB_s": round(gbs_g, 1),
                              "state_MB": round(n * H * dk * dv * 4 / 1e6, 1),
                              "note": "state fits in L2: effective bandwidth" if n * H * dk * dv * 4 < 100e6 else "HBM"}
         del S, q, k, v, e, gg, w, z, la, r, y
@@ -313,13 +345,46 @@ def blas_threads():
         return 1
 
 
+def oracle_forward_sample(T_sample):
+    """Forward only of the fp64 oracle on all heads of the first T_sample tokens."""
+    from gated_delta_rule_muir_b200.inputs import make_inputs
+    from oracle import muir_oracle as orc
+    d = make_inputs(WL["B"], T_sample, WL["H"], WL["dk"], WL["dv"], dtype=WL["dtype"], rate_lo=WL["rate_lo"],
+                    rate_hi=WL["rate_hi"], seed=WL["seed"])
+    t0 = time.perf_counter()
+    orc.forward(*[d[n] for n in NAMES])
+    return time.perf_counter() - t0
+
+
+def oracle_decode_sample(steps):
+    """Decode steps of the fp64 oracle for one sequence through all 24 layers (384 heads)."""
+    from gated_delta_rule_muir_b200.inputs import make_inputs
+    from oracle import muir_oracle as orc
+    L, H = DECODE["layers"], DECODE["H"]
+    d = make_inputs(L, steps, H, DECODE["dk"], DECODE["dv"], dtype="bf16", rate_lo=1e-4, rate_hi=0.7, seed=3,
+                    with_state=True)
+    S = d["S0"]
+    t0 = time.perf_counter()
+    for t in range(steps):
+        tok = [d[n][:, t] if d[n] is not None else None for n in NAMES[:8]]
+        _, S = orc.decode_step(S, *tok, d["r"])
+    return time.perf_counter() - t0
+
+
 def cpu_baseline():
     sec = oracle_sample(CPU_SAMPLE_T)
     tok = WL["B"] * CPU_SAMPLE_T
+    sec_f = oracle_forward_sample(CPU_SAMPLE_T)
+    dec_steps = 32
+    sec_d = oracle_decode_sample(dec_steps)
     return {"value": round(tok / sec, 2), "unit": "tokens/s", "cores": blas_threads(), "host_cpus": os.cpu_count(),
             "kind": "oracle",
             "sample": f"fp64 numpy oracle fwd+bwd, all {WL['H']} heads, first {CPU_SAMPLE_T} of {WL['T']} tokens "
-                      f"({sec:.1f} s)"}
+                      f"({sec:.1f} s)",
+            "forward_tokens_s": round(tok / sec_f, 2),
+            "decode_tokens_s": round(dec_steps / sec_d, 2),
+            "detail": f"forward only on the same sample ({sec_f:.1f} s); decode: one sequence, 24 layers x "
+                      f"{DECODE['H']} heads, {dec_steps} tokens ({sec_d:.1f} s)"}
 
 
 def run_reference(args, rank):
@@ -428,6 +493,7 @@ def main():
     roof["kernel"] = name
     roof["peak_source"] = pk["src"]
     line["roofline"] = roof
+    line["flop_split"] = flop_split(C, dk, dv)
     sfl, sby = algorithmic_step()
     t_step = ms * 1e-3
     line["step_roofline"] = {"algorithmic_TFLOP_s": round(sfl / t_step / 1e12, 2),
