@@ -49,8 +49,10 @@ def _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, S0, flags=0):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
-    for n, t, d in (("q", q, dk), ("k", k, dk), ("e", e, dk), ("g", g, dk), ("v", v, dv), ("w", w, dv)):
+    for n, t, d in (("q", q, dk), ("k", k, dk), ("e", e, dk), ("v", v, dv), ("w", w, dv)):
         _need(t, n, (B, T, H, d), dt)
+    if g is not None:  # g = None: static-only readout (g = 1)
+        _need(g, "g", (B, T, H, dk), dt)
     if z is not None:
         _need(z, "z", (B, T, H, dv), dt)
     _need(log_alpha, "log_alpha", (B, T, H, dk), torch.float32)
@@ -127,6 +129,8 @@ def chunk_bwd(q, k, v, e, w, g, z, log_alpha, r, dy, *, chunk=128, S0=None, dS_T
         N.check(lib.muir_chunk_bwd(C.byref(a), C.byref(gr), _ptr(ws), nbytes, _stream(stream)), "muir_chunk_bwd")
         return out
     out = {n: torch.empty(B, T, H, dk, dtype=dt, device=dev) for n in ("dq", "dk", "de", "dg")}
+    if g is None:
+        out["dg"] = None
     out.update({n: torch.empty(B, T, H, dv, dtype=dt, device=dev) for n in ("dv", "dw")})
     out["dz"] = torch.empty(B, T, H, dv, dtype=dt, device=dev) if z is not None else None
     out["dlog_alpha"] = torch.empty(B, T, H, dk, dtype=torch.float32, device=dev)
@@ -148,8 +152,10 @@ def decode_step(S, q, k, v, e, w, g, z, log_alpha, r, *, y=None, stream=None):
     n, H, dk, dv = S.shape
     dt = q.dtype
     _need(S, "S", (n, H, dk, dv), torch.float32)
-    for nm, t, d in (("q", q, dk), ("k", k, dk), ("e", e, dk), ("g", g, dk), ("v", v, dv), ("w", w, dv)):
+    for nm, t, d in (("q", q, dk), ("k", k, dk), ("e", e, dk), ("v", v, dv), ("w", w, dv)):
         _need(t, nm, (n, H, d), dt)
+    if g is not None:
+        _need(g, "g", (n, H, dk), dt)
     if z is not None:
         _need(z, "z", (n, H, dv), dt)
     _need(log_alpha, "log_alpha", (n, H, dk), torch.float32)

@@ -272,7 +272,12 @@ struct Rows {
   __device__ __forceinline__ void qt(int64_t tok, int c8, float (&o)[8]) const {
     float qq[8], gg[8], rr[8];
     Elt<T>::ld8(static_cast<const T*>(p.q) + toff(p, b, tok, h, p.dk) + c8, qq);
-    Elt<T>::ld8(static_cast<const T*>(p.g) + toff(p, b, tok, h, p.dk) + c8, gg);
+    if (p.g) {
+      Elt<T>::ld8(static_cast<const T*>(p.g) + toff(p, b, tok, h, p.dk) + c8, gg);
+    } else {  // static-only readout: g = 1
+#pragma unroll
+      for (int i = 0; i < 8; ++i) gg[i] = 1.f;
+    }
     ld8f(p.r + (int64_t)h * p.dk + c8, rr);
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i] = rr[i] * gg[i] * qq[i];
@@ -393,7 +398,8 @@ __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& 
         const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DK) + c8;
         pk[u].ld(static_cast<const T*>(p.k) + o);
         p1[u].ld(static_cast<const T*>(upper ? p.q : p.e) + o);
-        p2[u].ld(static_cast<const T*>(upper ? p.g : p.k) + o);
+        if (upper) p2[u].ld_or_one(p.g ? static_cast<const T*>(p.g) + o : nullptr);
+        else p2[u].ld(static_cast<const T*>(p.k) + o);
         ps[u].ld((upper ? pre : suf) + t * DK + c8);
       }
     }
@@ -491,7 +497,7 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
         fk[f].ld(static_cast<const T*>(p.k) + o);
         fe[f].ld(static_cast<const T*>(p.e) + o);
         fq[f].ld(static_cast<const T*>(p.q) + o);
-        fg[f].ld(static_cast<const T*>(p.g) + o);
+        fg[f].ld_or_one(p.g ? static_cast<const T*>(p.g) + o : nullptr);
         fl[f].ld(p.la + o);
       }
     }

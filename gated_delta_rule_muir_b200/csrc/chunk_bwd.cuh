@@ -659,11 +659,12 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
       const int na = side == 0 ? 2 : 3;
       fence_async_smem();
       __syncthreads();
-      if (tid == 0) mbar_expect_tx(&bar_cp, (uint32_t)Cs * DK * (2u * na + 4u));
+      const bool no_g = side == 1 && !p.g;  // static-only readout: g = 1 is not copied
+      if (tid == 0) mbar_expect_tx(&bar_cp, (uint32_t)Cs * DK * (2u * (na - (no_g ? 1 : 0)) + 4u));
       for (int x = tid; x < Cs * 4; x += NT) {
         const int a = x / Cs, tok = x % Cs;
         const int64_t o = toff(p, s.b, s.tok0 + tok, s.h, DK);
-        if (a < na) {
+        if (a < na && !(no_g && a == 1)) {
           const void* src = a == 0 ? p.k : (side == 0 ? p.e : (a == 1 ? p.g : p.q));
           bulk_g2s(base + a * RB + tok * DK * 2, static_cast<const T*>(src) + o, DK * 2, &bar_cp);
         } else if (a == 3) {
@@ -705,7 +706,8 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
           const int ro = (SB * J + tt) * DK + i;
           const float kk = __bfloat162float(rk[ro]);
           K[tt] = kk;
-          Z[tt] = side == 0 ? __bfloat162float(rz1[ro]) * kk : rr * __bfloat162float(rz1[ro]) * __bfloat162float(rz2[ro]);
+          Z[tt] = side == 0 ? __bfloat162float(rz1[ro]) * kk
+                            : rr * (p.g ? __bfloat162float(rz1[ro]) : 1.f) * __bfloat162float(rz2[ro]);
           al[tt] = expf(rla[ro]);
         }
       } else {
@@ -716,7 +718,8 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
           const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
           K[tt] = kk;
           Z[tt] = side == 0 ? Elt<T>::ld(static_cast<const T*>(p.e) + o) * kk
-                            : rr * Elt<T>::ld(static_cast<const T*>(p.g) + o) * Elt<T>::ld(static_cast<const T*>(p.q) + o);
+                            : rr * Elt<T>::ld_or_one(p.g ? static_cast<const T*>(p.g) + o : nullptr) *
+                                  Elt<T>::ld(static_cast<const T*>(p.q) + o);
           al[tt] = expf(__ldg(p.la + o));
         }
       }
@@ -849,7 +852,7 @@ __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q
       const int64_t o = o0 + tt * stride_k;
       const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
       const float ee = Elt<T>::ld(static_cast<const T*>(p.e) + o);
-      const float gg = Elt<T>::ld(static_cast<const T*>(p.g) + o);
+      const float gg = Elt<T>::ld_or_one(p.g ? static_cast<const T*>(p.g) + o : nullptr);
       const float qq = Elt<T>::ld(static_cast<const T*>(p.q) + o);
       const float a = ee * kk, qt = rr * gg * qq;
       const int ti = tt * DK + i;
@@ -864,7 +867,7 @@ __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q
       const float da = dAr + Gs * dAs;
       const float dkt = dKl + dKr + G * dKp + Gs * dKs + ee * da;
       Elt<T>::st(static_cast<T*>(q.dq) + o, rr * gg * dqt);
-      Elt<T>::st(static_cast<T*>(q.dg) + o, rr * qq * dqt);
+      if (q.dg) Elt<T>::st(static_cast<T*>(q.dg) + o, rr * qq * dqt);
       Elt<T>::st(static_cast<T*>(q.dk) + o, dkt);
       Elt<T>::st(static_cast<T*>(q.de) + o, kk * da);
       dr_acc += gg * qq * dqt;

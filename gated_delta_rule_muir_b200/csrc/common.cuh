@@ -22,6 +22,7 @@ template <typename T> struct Elt;
 
 template <> struct Elt<float> {
   static __device__ __forceinline__ float ld(const float* p) { return __ldg(p); }
+  static __device__ __forceinline__ float ld_or_one(const float* p) { return p ? __ldg(p) : 1.f; }
   // 8 consecutive elements through a generic pointer (e.g. shared memory).
   static __device__ __forceinline__ void ld8g(const float* p, float (&o)[8]) {
     const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
@@ -52,6 +53,7 @@ template <> struct Elt<float> {
 template <> struct Elt<__nv_bfloat16> {
   using T = __nv_bfloat16;
   static __device__ __forceinline__ float ld(const T* p) { return __bfloat162float(__ldg(p)); }
+  static __device__ __forceinline__ float ld_or_one(const T* p) { return p ? __bfloat162float(__ldg(p)) : 1.f; }
   static __device__ __forceinline__ void ld8g(const T* p, float (&o)[8]) {
     const uint4 u = *reinterpret_cast<const uint4*>(p);
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -102,6 +104,9 @@ template <> struct Pack8<float> {
     a = __ldg(reinterpret_cast<const float4*>(p));
     b = __ldg(reinterpret_cast<const float4*>(p) + 1);
   }
+  __device__ __forceinline__ void set_one() { a = b = make_float4(1.f, 1.f, 1.f, 1.f); }
+  // load, or all ones when p is null (an absent gate)
+  __device__ __forceinline__ void ld_or_one(const float* p) { if (p) ld(p); else set_one(); }
   __device__ __forceinline__ void get(float (&o)[8]) const {
     o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
     o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
@@ -110,6 +115,8 @@ template <> struct Pack8<float> {
 template <> struct Pack8<__nv_bfloat16> {
   uint4 u;
   __device__ __forceinline__ void ld(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void set_one() { u = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u); }
+  __device__ __forceinline__ void ld_or_one(const __nv_bfloat16* p) { if (p) ld(p); else set_one(); }
   __device__ __forceinline__ void get(float (&o)[8]) const {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll

@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(128) decode_step_kernel(DecodeParams p) {
   for (int i = tid; i < DK; i += 128) {
     const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + vo + i);
     const float ee = Elt<T>::ld(static_cast<const T*>(p.e) + vo + i);
-    const float gg = Elt<T>::ld(static_cast<const T*>(p.g) + vo + i);
+    const float gg = Elt<T>::ld_or_one(p.g ? static_cast<const T*>(p.g) + vo + i : nullptr);
     const float qq = Elt<T>::ld(static_cast<const T*>(p.q) + vo + i);
     const float rr = __ldg(p.r + n * p.r_stride + (int64_t)h * DK + i);
     const float al = expf(__ldg(p.la + vo + i));

@@ -125,7 +125,7 @@ int muir_decode_step(const muir_decode_args* a, void* stream) {
   g_err.clear();
   if (!a) return fail(MUIR_ERR_INVALID_ARG, "decode: args is NULL");
   if (a->n_seq == 0) return MUIR_OK;  // nothing to do (empty tensors may carry NULL pointers)
-  if (!a->S || !a->q || !a->k || !a->v || !a->e || !a->w || !a->g || !a->log_alpha || !a->r || !a->y)
+  if (!a->S || !a->q || !a->k || !a->v || !a->e || !a->w || !a->log_alpha || !a->r || !a->y)
     return fail(MUIR_ERR_INVALID_ARG, "decode: a required pointer is NULL");
   if (a->n_seq < 0 || a->H <= 0 || !dim_ok(a->dk) || !dim_ok(a->dv))
     return fail(MUIR_ERR_UNSUPPORTED, "decode: unsupported sizes H=%d dk=%d dv=%d", a->H, a->dk, a->dv);

@@ -77,7 +77,9 @@ typedef struct muir_chunk_args {
   const void* v;  /* [B,T,H,dv] value */
   const void* e;  /* [B,T,H,dk] erase gate, acts on key rows */
   const void* w;  /* [B,T,H,dv] write gate, acts on value columns */
-  const void* g;  /* [B,T,H,dk] dynamic query (read) gate */
+  const void* g;  /* [B,T,H,dk] dynamic query (read) gate, or NULL for the static-only
+                     readout (g = 1: the query is scaled by r alone; openai-hub article,
+                     matched-filter section, compares static and dynamic readouts) */
   const void* z;  /* [B,T,H,dv] output gate, or NULL for none */
   const float* log_alpha; /* [B,T,H,dk] log of the channel decay, <= 0 */
   const float* r; /* [H,dk] static matched-filter row scale */
@@ -122,7 +124,7 @@ typedef struct muir_chunk_grads {
   void* dv;            /* [B,T,H,dv] (dtype) */
   void* de;            /* [B,T,H,dk] (dtype) */
   void* dw;            /* [B,T,H,dv] (dtype) */
-  void* dg;            /* [B,T,H,dk] (dtype) */
+  void* dg;            /* [B,T,H,dk] (dtype); may be NULL (and is ignored) when g is NULL */
   void* dz;            /* [B,T,H,dv] (dtype), or NULL; ignored when z is NULL */
   float* dlog_alpha;   /* [B,T,H,dk]; d/d(alpha) = dlog_alpha / alpha */
   float* dS0;          /* [B,H,dk,dv], or NULL */
@@ -177,7 +179,7 @@ typedef struct muir_decode_args {
   const void* v;       /* [n_seq,H,dv] */
   const void* e;       /* [n_seq,H,dk] */
   const void* w;       /* [n_seq,H,dv] */
-  const void* g;       /* [n_seq,H,dk] */
+  const void* g;       /* [n_seq,H,dk], or NULL for the static-only readout (g = 1) */
   const void* z;       /* [n_seq,H,dv] or NULL */
   const float* log_alpha; /* [n_seq,H,dk] */
   const float* r;      /* [H,dk] when r_seq_stride == 0, else row n at r + n*r_seq_stride */

@@ -47,6 +47,7 @@ def _f(x):
 def _prep(q, k, v, e, w, g, z, log_alpha, r):
     q, k, v, e, w, g, log_alpha, r = map(_f, (q, k, v, e, w, g, log_alpha, r))
     z = np.ones_like(v) if z is None else _f(z)
+    g = np.ones_like(q) if g is None else g  # [mf]: the static-only readout has no dynamic gate (g = 1)
     alpha = np.exp(log_alpha)
     qt = r[None, None] * g * q          # [mf]: static row scale times dynamic query gate
     a = e * k                           # erase direction: erase gate on key rows
@@ -100,7 +101,7 @@ def backward(q, k, v, e, w, g, z, log_alpha, r, dy, S0=None, dS_T=None, checkpoi
 
     States are re-created from checkpoints saved every `checkpoint_every` tokens.
     Returns a dict with dq, dk, dv, de, dw, dg, dz, dlog_alpha ([B,T,H,*]), dS0
-    [B,H,dk,dv] and dr [H,dk].
+    [B,H,dk,dv] and dr [H,dk]; dg is None when g is None (the static-only readout).
 
     With G the cotangent of S_t and do = z * dy_t:
         dz = o * dy,   G += qt do^T,   dqt = S_t do
@@ -113,6 +114,7 @@ def backward(q, k, v, e, w, g, z, log_alpha, r, dy, S0=None, dS_T=None, checkpoi
         from x = alpha*S_{t-1}: dalpha_i = sum_j dx_ij S_{t-1,ij}, G <- alpha*dx
         dlog_alpha = alpha * dalpha.
     """
+    has_g = g is not None
     q, k, v, e, w, g, z, alpha, qt, a, u, r = _prep(q, k, v, e, w, g, z, log_alpha, r)
     dy = _f(dy)
     B, T, H, dk = q.shape
@@ -161,6 +163,8 @@ def backward(q, k, v, e, w, g, z, log_alpha, r, dy, S0=None, dS_T=None, checkpoi
             G = alpha[:, t][..., :, None] * dx
     grads["dS0"] = G
     grads["dr"] = dr
+    if not has_g:
+        grads["dg"] = None
     return grads
 
 

@@ -131,3 +131,17 @@ def test_noalloc_rejects_flags(lib):
     a = _chunk_args(flags=N.MUIR_SAVE_FOR_BWD)
     assert lib.muir_chunk_fwd_noalloc(C.byref(a), C.c_void_p(1 << 20), None, None) == N.MUIR_ERR_INVALID_ARG
     assert b"flags" in lib.muir_last_error()
+
+
+def test_static_readout_needs_no_query_gate_or_its_gradient(lib):
+    """g = NULL selects the static-only readout: dg may then be NULL too; with g
+    present, dg is required."""
+    fake = C.c_void_p(1 << 20)
+    g_full = N.ChunkGrads(dy=fake, dq=fake, dk=fake, dv=fake, de=fake, dw=fake, dg=None, dlog_alpha=fake)
+    a = _chunk_args()
+    assert lib.muir_chunk_bwd(C.byref(a), C.byref(g_full), fake, 1 << 40, None) == N.MUIR_ERR_INVALID_ARG
+    a = _chunk_args(g=None)
+    assert lib.muir_chunk_fwd_workspace(C.byref(a)) > 0
+    # argument validation passes and the call stops at the (deliberately too small)
+    # workspace, before anything is launched
+    assert lib.muir_chunk_bwd(C.byref(a), C.byref(g_full), fake, 1, None) == N.MUIR_ERR_WORKSPACE
