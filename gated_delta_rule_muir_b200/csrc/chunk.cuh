@@ -398,8 +398,7 @@ __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& 
         const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DK) + c8;
         pk[u].ld(static_cast<const T*>(p.k) + o);
         p1[u].ld(static_cast<const T*>(upper ? p.q : p.e) + o);
-        if (upper) p2[u].ld_or_one(p.g ? static_cast<const T*>(p.g) + o : nullptr);
-        else p2[u].ld(static_cast<const T*>(p.k) + o);
+        p2[u].ld(static_cast<const T*>(upper && p.g ? p.g : p.k) + o);
         ps[u].ld((upper ? pre : suf) + t * DK + c8);
       }
     }
@@ -415,6 +414,10 @@ __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& 
         p1[u].get(s1);
         p2[u].get(s2);
         ps[u].get(sc);
+        if (upper && !p.g) {  // static-only readout: g = 1 (p2 held k as a stand-in)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) s2[j] = 1.f;
+        }
         Elt<float>::ld8g(ft + (t >> 4) * DK + c8, fj);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {

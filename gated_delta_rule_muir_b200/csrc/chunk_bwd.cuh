@@ -671,6 +671,10 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
           bulk_g2s(base + 3 * RB + tok * DK * 4, p.la + o, DK * 4, &bar_cp);
         }
       }
+      if (no_g) {  // the g rows are ones
+        const uint4 one = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+        for (uint32_t o = tid * 16u; o < (uint32_t)Cs * DK * 2u; o += NT * 16u) sts128(base + RB + o, one);
+      }
       const bool ok = mbar_wait(&bar_cp, cp_phase);
       cp_phase ^= 1u;
       if (!__syncthreads_and(ok ? 1 : 0)) drv.ok = false;
@@ -706,8 +710,7 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
           const int ro = (SB * J + tt) * DK + i;
           const float kk = __bfloat162float(rk[ro]);
           K[tt] = kk;
-          Z[tt] = side == 0 ? __bfloat162float(rz1[ro]) * kk
-                            : rr * (p.g ? __bfloat162float(rz1[ro]) : 1.f) * __bfloat162float(rz2[ro]);
+          Z[tt] = side == 0 ? __bfloat162float(rz1[ro]) * kk : rr * __bfloat162float(rz1[ro]) * __bfloat162float(rz2[ro]);
           al[tt] = expf(rla[ro]);
         }
       } else {
