@@ -185,6 +185,20 @@ def state_init(S, S_src=None, *, stream=None):
     return S
 
 
+def row_scale(S, *, exponent=0.5, eps=1e-12, r=None, stream=None):
+    """Static matched-filter row scale from measured row energies of states
+    S [n,H,dk,dv] fp32: r[h,i] = (mean_{n,j} S[n,h,i,j]^2 + eps)^(-exponent), [H,dk]."""
+    lib = N.load()
+    n, H, dk, dv = S.shape
+    _need(S, "S", (n, H, dk, dv), torch.float32)
+    if r is None:
+        r = torch.empty(H, dk, dtype=torch.float32, device=S.device)
+    _need(r, "r", (H, dk), torch.float32)
+    N.check(lib.muir_row_scale(_ptr(S), n, H, dk, dv, float(exponent), float(eps), _ptr(r), _stream(stream)),
+            "muir_row_scale")
+    return r
+
+
 def launch_count() -> int:
     """Number of kernels libmuir has launched in this process."""
     return int(N.load().muir_launch_count())

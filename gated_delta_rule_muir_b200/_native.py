@@ -44,6 +44,7 @@ SIGNATURES = {
     "muir_chunk_bwd": (C.c_int, [C.POINTER(ChunkArgs), C.POINTER(ChunkGrads), vp, C.c_size_t, vp]),
     "muir_decode_step": (C.c_int, [C.POINTER(DecodeArgs), vp]),
     "muir_state_init": (C.c_int, [vp, vp, C.c_int64, C.c_int32, C.c_int32, C.c_int32, vp]),
+    "muir_row_scale": (C.c_int, [vp, C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_float, C.c_float, vp, vp]),
     "muir_device_status": (C.c_int, [vp]),
     "muir_last_error": (C.c_char_p, []),
     "muir_version": (C.c_int, []),

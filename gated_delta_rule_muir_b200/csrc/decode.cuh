@@ -137,6 +137,30 @@ __global__ void __launch_bounds__(128) decode_step_kernel(DecodeParams p) {
   }
 }
 
+// Row energies of states S [n,H,dk,dv] -> r[h,i] = (mean_{n,j} S[n,h,i,j]^2 + eps)^(-exponent).
+// One CTA per (h, i); the sum of squares is accumulated in fp64.
+__global__ void row_scale_kernel(const float* __restrict__ S, int64_t n, int H, int dk, int dv, float exponent,
+                                 float eps, float* __restrict__ r) {
+  const int h = blockIdx.x / dk, i = blockIdx.x % dk;
+  double acc = 0.0;
+  const int64_t per = n * dv;
+  for (int64_t x = threadIdx.x; x < per; x += blockDim.x) {
+    const int64_t m = x / dv, j = x % dv;
+    const float v = __ldg(S + (((m * H + h) * dk + i) * dv + j));
+    acc += (double)v * v;
+  }
+  __shared__ double part[32];
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += part[w];
+    const double e = tot / (double)per + (double)eps;
+    r[(int64_t)h * dk + i] = (float)pow(e, -(double)exponent);
+  }
+}
+
 __global__ void state_init_kernel(float4* __restrict__ S, const float4* __restrict__ src, int64_t n4) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x)
     S[i] = src ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);

@@ -121,6 +121,20 @@ int muir_state_init(float* S, const float* S_src, int64_t n_seq, int32_t H, int3
   return cuda_check("state_init launch");
 }
 
+int muir_row_scale(const float* S, int64_t n_seq, int32_t H, int32_t dk, int32_t dv, float exponent, float eps, float* r,
+                   void* stream) {
+  g_err.clear();
+  if (!S || !r) return fail(MUIR_ERR_INVALID_ARG, "row_scale: S or r is NULL");
+  if (n_seq <= 0 || H <= 0 || !dim_ok(dk) || !dim_ok(dv))
+    return fail(MUIR_ERR_UNSUPPORTED, "row_scale: unsupported sizes n_seq=%lld H=%d dk=%d dv=%d", (long long)n_seq, H,
+                dk, dv);
+  if (!(exponent >= 0.f) || !(eps >= 0.f)) return fail(MUIR_ERR_INVALID_ARG, "row_scale: exponent and eps must be >= 0");
+  Launch L_("row_scale", static_cast<cudaStream_t>(stream));
+  muir::row_scale_kernel<<<(unsigned)(H * dk), 256, 0, static_cast<cudaStream_t>(stream)>>>(S, n_seq, H, dk, dv,
+                                                                                            exponent, eps, r);
+  return cuda_check("row_scale launch");
+}
+
 int muir_decode_step(const muir_decode_args* a, void* stream) {
   g_err.clear();
   if (!a) return fail(MUIR_ERR_INVALID_ARG, "decode: args is NULL");

@@ -194,6 +194,17 @@ int muir_decode_step(const muir_decode_args* a, void* stream);
 int muir_state_init(float* S, const float* S_src, int64_t n_seq, int32_t H, int32_t dk, int32_t dv,
                     void* stream);
 
+/* Static matched-filter row scale from measured row energies (openai-hub
+ * article, matched-filter section: the static readout weights each state row
+ * by an inverse fractional power of its expected energy; 0.5 is the inverse
+ * square root). For states S [n_seq,H,dk,dv] fp32 (device), e.g. collected
+ * along a calibration stream, with E[h,i] = mean over (n, j) of S[n,h,i,j]^2:
+ *     r[h,i] = (E[h,i] + eps)^(-exponent)          r [H,dk] fp32 (device)
+ * The sums are accumulated in fp64. exponent, eps >= 0. The scale is returned
+ * as is (no normalisation), for the caller to rescale if wanted. */
+int muir_row_scale(const float* S, int64_t n_seq, int32_t H, int32_t dk, int32_t dv, float exponent, float eps, float* r,
+                   void* stream);
+
 /* Synchronises `stream`, then returns and clears the device-side status word:
  * MUIR_OK, or MUIR_ERR_TIMEOUT if a kernel's bounded wait expired since the
  * last call (that kernel's outputs are then invalid), or MUIR_ERR_CUDA. */

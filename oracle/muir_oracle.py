@@ -96,6 +96,14 @@ def decode_step(S, q, k, v, e, w, g, z, log_alpha, r):
     return y[:, 0], S_new
 
 
+def row_scale(S, exponent=0.5, eps=1e-12):
+    """[mf]: the static readout weights state row i by an inverse fractional power
+    of its expected energy. Measured over states S [N,H,dk,dv]:
+    r[h,i] = (mean_{n,j} S[n,h,i,j]^2 + eps)^(-exponent)."""
+    S = _f(S)
+    return (np.mean(S * S, axis=(0, 3)) + eps) ** (-exponent)
+
+
 def backward(q, k, v, e, w, g, z, log_alpha, r, dy, S0=None, dS_T=None, checkpoint_every=64):
     """Reverse-mode of forward(), written out by hand, token by token.
 

@@ -145,3 +145,10 @@ def test_static_readout_needs_no_query_gate_or_its_gradient(lib):
     # argument validation passes and the call stops at the (deliberately too small)
     # workspace, before anything is launched
     assert lib.muir_chunk_bwd(C.byref(a), C.byref(g_full), fake, 1, None) == N.MUIR_ERR_WORKSPACE
+
+
+def test_row_scale_rejects_bad_args(lib):
+    fake = C.c_void_p(1 << 20)
+    assert lib.muir_row_scale(None, 1, 1, 32, 32, 0.5, 0.0, fake, None) == N.MUIR_ERR_INVALID_ARG
+    assert lib.muir_row_scale(fake, 1, 1, 48, 32, 0.5, 0.0, fake, None) == N.MUIR_ERR_UNSUPPORTED
+    assert lib.muir_row_scale(fake, 1, 1, 32, 32, -1.0, 0.0, fake, None) == N.MUIR_ERR_INVALID_ARG

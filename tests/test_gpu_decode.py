@@ -70,3 +70,13 @@ def test_decode_empty(cuda_ok):
     z = torch.zeros(0, 2, 32, device="cuda")
     y = muir.decode_step(S, z, z, z, z, z, z, z, z, torch.zeros(2, 32, device="cuda"))
     assert y.shape == (0, 2, 32)
+
+
+def test_row_scale_matches_oracle(cuda_ok):
+    """Static row scale from measured energies: states of a decode run, all rows."""
+    g = torch.Generator().manual_seed(9)
+    S = (torch.randn(6, 3, 64, 32, generator=g, dtype=torch.float64) *
+         torch.rand(1, 3, 64, 1, generator=g, dtype=torch.float64) * 3)
+    r = muir.row_scale(S.float().cuda(), exponent=0.5, eps=1e-6)
+    r_ref = orc.row_scale(S.float().double().numpy(), exponent=0.5, eps=1e-6)
+    assert rel_err(r, r_ref) < 1e-5

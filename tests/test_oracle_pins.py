@@ -246,3 +246,26 @@ def test_state_size_matches_pages():
     assert nbytes == 25_165_824 and round(nbytes / 1e6) == vals["approx_total_MB"]
     assert (DECODE.extra["layers"], DECODE.H, DECODE.dk, DECODE.dv) == \
         (vals["layers"], vals["heads"], vals["dk"], vals["dv"])
+
+
+def test_row_scale_matches_the_stationary_energy_of_a_decaying_row():
+    """A row that decays by abar per token and receives unit-variance writes has
+    stationary energy 1 / (1 - abar^2); with exponent 0.5 the measured scale is
+    its inverse square root, sqrt(1 - abar^2), the static scale the input recipe
+    uses up to the constant (1 + abar)^0.5. Rows of constant magnitude c give c^-1
+    exactly."""
+    rng = np.random.default_rng(7)
+    abar = np.array([0.5, 0.9, 0.99])
+    n_chain, T = 256, 3000
+    s = np.zeros((n_chain, abar.size))
+    samples = []
+    for t in range(T):
+        s = abar * s + rng.standard_normal(s.shape)
+        if t >= 1000 and t % 10 == 0:
+            samples.append(s.copy())
+    S = np.stack(samples)[:, None, :, :].transpose(0, 1, 3, 2)  # [N, H=1, dk=3, dv=n_chain]
+    r = orc.row_scale(S, exponent=0.5)[0]
+    np.testing.assert_allclose(r, np.sqrt(1 - abar ** 2), rtol=0.08)
+    c = np.array([0.5, 2.0, 3.0])
+    S2 = np.broadcast_to(c[None, None, :, None], (4, 1, 3, 5)) * np.where(np.arange(5) % 2, 1.0, -1.0)
+    np.testing.assert_allclose(orc.row_scale(S2, exponent=0.5, eps=0.0)[0], 1.0 / c, rtol=1e-12)
