@@ -185,6 +185,36 @@ def state_init(S, S_src=None, *, stream=None):
     return S
 
 
+def chunk_segment_map(q, k, v, e, w, g, z, log_alpha, r, *, chunk=128, workspace=None, stream=None):
+    """The segment's chunkwise forward as an affine map of its start state,
+    S_end = Phi S0 + Psi: returns (Phi [B,H,dk,dk], Psi [B,H,dk,dv]) fp32."""
+    lib = N.load()
+    a, (B, T, H, dk, dv, dt) = _chunk_args(q, k, v, e, w, g, z, log_alpha, r, chunk, None)
+    Phi = torch.empty(B, H, dk, dk, dtype=torch.float32, device=q.device)
+    Psi = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    nbytes = int(lib.muir_chunk_segment_map_workspace(C.byref(a)))
+    ws = _workspace(nbytes, q.device, workspace)
+    N.check(lib.muir_chunk_segment_map(C.byref(a), _ptr(Phi), _ptr(Psi), _ptr(ws), nbytes, _stream(stream)),
+            "muir_chunk_segment_map")
+    return Phi, Psi
+
+
+def apply_map(Phi, Psi, S_in=None, *, S_out=None, stream=None):
+    """S_out = Phi S_in + Psi for [n,H] maps (S_in None: S_out = Psi), fp32."""
+    lib = N.load()
+    n, H, dk, _ = Phi.shape
+    dv = Psi.shape[-1]
+    _need(Phi, "Phi", (n, H, dk, dk), torch.float32)
+    _need(Psi, "Psi", (n, H, dk, dv), torch.float32)
+    if S_in is not None:
+        _need(S_in, "S_in", (n, H, dk, dv), torch.float32)
+    if S_out is None:
+        S_out = torch.empty_like(Psi)
+    N.check(lib.muir_apply_map(_ptr(Phi), _ptr(Psi), _ptr(S_in), _ptr(S_out), n, H, dk, dv, _stream(stream)),
+            "muir_apply_map")
+    return S_out
+
+
 def row_scale(S, *, exponent=0.5, eps=1e-12, r=None, stream=None):
     """Static matched-filter row scale from measured row energies of states
     S [n,H,dk,dv] fp32: r[h,i] = (mean_{n,j} S[n,h,i,j]^2 + eps)^(-exponent), [H,dk]."""

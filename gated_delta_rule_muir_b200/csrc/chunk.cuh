@@ -1148,6 +1148,131 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
 }
 
 // ---------------------------------------------------------------------------
+// segmap_kernel: the affine map of a whole sequence segment, S_end = Phi_seg S0
+// + Psi_seg, as the composition of its chunk maps (the exchange step of a scan
+// split along T across ranks: each rank composes its segment, the maps are
+// gathered, and each rank starts from its predecessors' composed maps). The
+// composition is the scan run on the augmented state X = [Phi_acc | Psi_acc]
+// (dk x (dk + dv)): X <- Phi_n X + [0 | Psi_n] from X = [I | 0]. One CTA per
+// (batch, head, 32-column slab of X), with the same double-buffered bulk copies
+// of Phi_n (and of the Psi_n slab for the Psi columns) as scan_kernel.
+// ---------------------------------------------------------------------------
+template <int DK, int NS>
+__global__ void __launch_bounds__(128, 1) segmap_kernel(ChunkParams p, const uint8_t* ma, const float* psi, int units,
+                                                        int ulen, float* Phi_seg, float* Psi_seg) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  __shared__ uint64_t bar, bar_c[2];
+  __shared__ uint32_t tslot;
+  constexpr int NW = 32;
+  const int dv = p.dv, vslabs = dv / NW, slabs = DK / NW + vslabs;
+  const int slab = blockIdx.x % slabs;
+  const int bh = blockIdx.x / slabs;
+  const bool phi_part = slab < DK / NW;
+  const int vs = slab - DK / NW;  // Psi slab index (Psi columns)
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const MapGeom g = map_geom(DK, ulen);
+  const uint32_t PS = DK * NW * 4u;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t psi_off = 2 * g.tile;
+  const uint32_t s_off = psi_off + 2 * PS;
+  const Tile Sb{base + s_off, base + s_off + NW * DK * 2u, 128u, DK * 16u};
+  if (tid == 0) {
+    mbar_init(&bar_c[0], 1);
+    mbar_init(&bar_c[1], 1);
+  }
+  TcCta cta;
+  cta.init(&tslot, &bar, 32);
+  MmaSync drv{&bar, 0u, true};
+  const uint32_t lane = tmem_lane_base(warp);
+  const float* psi_s = reinterpret_cast<const float*>(static_cast<const uint8_t*>(sm) + psi_off);
+  auto issue = [&](int n, int buf) {
+    if (tid == 0) {
+      const int64_t uid = (int64_t)bh * units + n;
+      mbar_expect_tx(&bar_c[buf], g.tile + (phi_part ? 0u : PS));
+      bulk_g2s_big(base + buf * g.tile, ma + uid * g.unit, g.tile, &bar_c[buf]);
+      if (!phi_part)
+        bulk_g2s_big(base + psi_off + buf * PS, reinterpret_cast<const uint8_t*>(psi + (uid * vslabs + vs) * DK * NW),
+                     PS, &bar_c[buf]);
+    }
+  };
+  float st[NW];
+#pragma unroll
+  for (int j = 0; j < NW; ++j) st[j] = (phi_part && tid == slab * NW + j) ? 1.f : 0.f;
+  issue(0, 0);
+  if (units > 1) issue(1, 1);
+  const uint32_t id = idesc_bf16(128, NW, 0, 1);
+  for (int n = 0; n < units && drv.ok; ++n) {
+    const int buf = n & 1;
+    if (tid < DK) {
+#pragma unroll
+      for (int j = 0; j < NW; j += 8) {
+        float v[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) v[e2] = st[j + e2];
+        put_mn(Sb, tid, j, v);
+      }
+    }
+    const bool c_ok = mbar_wait(&bar_c[buf], (uint32_t)(n >> 1) & 1u);
+    if (!__syncthreads_and(c_ok ? 1 : 0)) { drv.ok = false; break; }
+    const Tile Phi{base + buf * g.tile, base + buf * g.tile + g.half, 128u, DK * 16u};
+    drv.run([&] { mma_tiles(cta.tmem, Phi, Sb, DK / 16, id, NS, false); });
+    if (!drv.ok) break;
+    float v[NW];
+    tmem_ld32(cta.tmem + lane, v);
+    if (tid < DK) {
+      if (phi_part) {
+#pragma unroll
+        for (int j = 0; j < NW; ++j) st[j] = v[j];
+      } else {
+        const float* add = psi_s + buf * (PS / 4) + tid * NW;
+#pragma unroll
+        for (int j = 0; j < NW; j += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(add + j);
+          st[j] = v[j] + a4.x; st[j + 1] = v[j + 1] + a4.y; st[j + 2] = v[j + 2] + a4.z; st[j + 3] = v[j + 3] + a4.w;
+        }
+      }
+    }
+    __syncthreads();  // buffer `buf` is free again
+    if (n + 2 < units) issue(n + 2, buf);
+  }
+  if (tid < DK && drv.ok) {
+    float* o = phi_part ? Phi_seg + ((int64_t)bh * DK + tid) * DK + slab * NW
+                        : Psi_seg + ((int64_t)bh * DK + tid) * dv + vs * NW;
+#pragma unroll
+    for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&st[j]));
+  }
+  cta.finish();
+}
+
+// The identity map of an empty segment: Phi = I, Psi = 0 ([nh][dk][dk], [nh][dk][dv]).
+__global__ void identity_map_kernel(float* __restrict__ Phi, float* __restrict__ Psi, int64_t nh, int dk, int dv) {
+  const int64_t np = nh * dk * dk, ns = nh * dk * dv;
+  for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < np + ns; x += (int64_t)gridDim.x * blockDim.x) {
+    if (x < np) Phi[x] = ((x / dk) % dk) == (x % dk) ? 1.f : 0.f;
+    else Psi[x - np] = 0.f;
+  }
+}
+
+// apply_map_kernel: S_out = Phi S_in + Psi per (sequence, head), fp32 on the CUDA
+// cores (S_in NULL: S_out = Psi). Thread = one output element; rows of Phi and
+// columns of S_in are read through the cache.
+__global__ void apply_map_kernel(const float* __restrict__ Phi, const float* __restrict__ Psi,
+                                 const float* __restrict__ S_in, float* __restrict__ S_out, int64_t nh, int dk, int dv) {
+  const int64_t total = nh * dk * dv;
+  for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < total; x += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = x / ((int64_t)dk * dv);
+    const int i = (int)((x / dv) % dk), j = (int)(x % dv);
+    float acc = __ldg(Psi + x);
+    if (S_in) {
+      const float* ph = Phi + (m * dk + i) * dk;
+      const float* sc = S_in + m * dk * dv + j;
+      for (int c = 0; c < dk; ++c) acc = fmaf(__ldg(ph + c), __ldg(sc + (int64_t)c * dv), acc);
+    }
+    S_out[x] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // out_kernel: outputs of one chunk from its start state, all chunks in
 // parallel:  y = z * (Q' S0 + Oloc).
 // A = Q' tiles of the map image (bulk copy, K-major over key channels),

@@ -135,6 +135,24 @@ int muir_row_scale(const float* S, int64_t n_seq, int32_t H, int32_t dk, int32_t
   return cuda_check("row_scale launch");
 }
 
+int muir_apply_map(const float* Phi, const float* Psi, const float* S_in, float* S_out, int64_t n_seq, int32_t H,
+                   int32_t dk, int32_t dv, void* stream) {
+  g_err.clear();
+  if (!Phi || !Psi || !S_out) return fail(MUIR_ERR_INVALID_ARG, "apply_map: Phi, Psi or S_out is NULL");
+  if (n_seq < 0 || H <= 0 || !dim_ok(dk) || !dim_ok(dv))
+    return fail(MUIR_ERR_UNSUPPORTED, "apply_map: unsupported sizes n_seq=%lld H=%d dk=%d dv=%d", (long long)n_seq, H,
+                dk, dv);
+  if (S_in && S_in == S_out) return fail(MUIR_ERR_INVALID_ARG, "apply_map: S_in and S_out must differ");
+  const int64_t total = n_seq * H * (int64_t)dk * dv;
+  if (total == 0) return MUIR_OK;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  Launch L_("apply_map", static_cast<cudaStream_t>(stream));
+  muir::apply_map_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(Phi, Psi, S_in, S_out,
+                                                                                         n_seq * H, dk, dv);
+  return cuda_check("apply_map launch");
+}
+
 int muir_decode_step(const muir_decode_args* a, void* stream) {
   g_err.clear();
   if (!a) return fail(MUIR_ERR_INVALID_ARG, "decode: args is NULL");

@@ -167,6 +167,23 @@ int muir_chunk_bwd(const muir_chunk_args* a, const muir_chunk_grads* gr, void* w
  */
 int muir_chunk_fwd_noalloc(const muir_chunk_args* a, void* y, float* S_T, void* stream);
 
+/*
+ * Sequence segments (a scan split along T; the pages have no counterpart). The
+ * chunkwise forward is an affine map of its start state, S_T = Phi S0 + Psi.
+ * muir_chunk_segment_map returns that map for a whole segment (the chunk maps
+ * of its units of min(chunk, 128) tokens, composed in order on the tensor
+ * cores): Phi [B,H,dk,dk] and Psi [B,H,dk,dv] fp32 (device, caller-owned), so
+ * that ranks holding consecutive segments can exchange maps, and each one
+ * start from its predecessors' maps applied to the initial state. a->S0 is
+ * ignored; a->flags must be 0. Workspace: muir_chunk_segment_map_workspace(a).
+ * muir_apply_map computes S_out = Phi S_in + Psi (S_in NULL: S_out = Psi) in
+ * fp32 on [n_seq,H] maps; S_in and S_out must not alias.
+ */
+size_t muir_chunk_segment_map_workspace(const muir_chunk_args* a);
+int muir_chunk_segment_map(const muir_chunk_args* a, float* Phi, float* Psi, void* ws, size_t ws_bytes, void* stream);
+int muir_apply_map(const float* Phi, const float* Psi, const float* S_in, float* S_out, int64_t n_seq, int32_t H,
+                   int32_t dk, int32_t dv, void* stream);
+
 /* One recurrent step for n_seq independent sequences (streaming decode,
  * openai-hub article, section on 10M-token streaming). */
 typedef struct muir_decode_args {
