@@ -761,7 +761,8 @@ __global__ void __launch_bounds__(256, 1) solve_kernel(ChunkParams p) {
 // ---------------------------------------------------------------------------
 // maps_kernel: the chunk's affine map. TMEM column bases (fp32, 128 lanes):
 //   phase 1: W -> 0, Z = M^kk U -> 128, Ut = T Z -> 256
-//   phase 2: Phi -> 0, Q' -> 384, Oloc -> 256 (after Ut left TMEM), Psi -> 128
+//   phase 2: Phi -> 384, Psi -> 128 (Z consumed)
+//   phase 3: Oloc -> 256 (Ut consumed), Q' -> 0 (W consumed)
 // Shared memory: one A tile and two MN-major B tiles (128 x 128 bf16 hi+lo
 // each). Negated operands are staged negated.
 // ---------------------------------------------------------------------------
@@ -794,7 +795,8 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
   const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups take alternate 16-column chunks
-  constexpr uint32_t cW = 0, cZ = 128, cUt = 256, cPhi = 0, cPsi = 128, cOl = 256, cQ = 384;
+  // W stays in TMEM until its second use; Z's and Ut's columns are reused once they are consumed
+  constexpr uint32_t cW = 0, cZ = 128, cUt = 256, cPhi = 384, cPsi = 128, cOl = 256, cQ = 0;
   uint32_t cp_phase = 0;
   // A <- a Gram or T image (one bulk copy); the MMA that last read A has completed.
   auto load_img = [&](const uint8_t* img) {
@@ -877,21 +879,22 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
         stg_row16(uo + t * DV + c, v);
     }
   }
-  // ---- phase 2 with W in B1: Phi = Diag(Gam_C) - (A*Gsuf)^T W, N^qa W (Q' = Qt*Gam - N^qa W in the epilogue)
+  // ---- phase 2, A = (A*Gsuf)^T staged once for both of its products:
+  //   D_Phi = (A*Gsuf)^T W (Phi = Diag(Gam_C) - D_Phi in the epilogue), Psi = (A*Gsuf)^T (-Ut) + (K*Gsuf)^T U
   tmem_to_b(B1, cW, DK, 1.f);
-  stage_suffixed(true, -1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cPhi, A, B1, Cs / 16, idKt, NS, false); });
-  load_img(G + 3 * sq_bytes(Cs));  // N^qa
-  drv.run([&] { mma_tiles(cta.tmem + cQ, A, B1, Cs / 16, idK, NS, false); });
-  // ---- phase 3 with -Ut in B1, U in B2: Oloc = N^qa (-Ut) + N^qk U, Psi = (K*Gsuf)^T U + (A*Gsuf)^T (-Ut)
-  tmem_to_b(B1, cUt, DV, -1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cOl, A, B1, Cs / 16, idV, NS, false); });  // A still holds N^qa
-  load_img(G + 2 * sq_bytes(Cs));                                                 // N^qk
-  drv.run([&] { mma_tiles(cta.tmem + cOl, A, B2, Cs / 16, idV, NS, true); });
-  stage_suffixed(false, 1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B2, Cs / 16, idVt, NS, false); });
   stage_suffixed(true, 1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B1, Cs / 16, idVt, NS, true); });
+  drv.run([&] { mma_tiles(cta.tmem + cPhi, A, B1, Cs / 16, idKt, NS, false); });
+  tmem_to_b(B1, cUt, DV, -1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B1, Cs / 16, idVt, NS, false); });
+  stage_suffixed(false, 1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B2, Cs / 16, idVt, NS, true); });
+  // ---- phase 3: Oloc = N^qa (-Ut) + N^qk U, and N^qa W (Q' = Qt*Gam - N^qa W in the epilogue)
+  load_img(G + 3 * sq_bytes(Cs));  // N^qa
+  drv.run([&] { mma_tiles(cta.tmem + cOl, A, B1, Cs / 16, idV, NS, false); });  // B1 holds -Ut
+  tmem_to_b(B1, cW, DK, 1.f);
+  drv.run([&] { mma_tiles(cta.tmem + cQ, A, B1, Cs / 16, idK, NS, false); });
+  load_img(G + 2 * sq_bytes(Cs));  // N^qk
+  drv.run([&] { mma_tiles(cta.tmem + cOl, A, B2, Cs / 16, idV, NS, true); });
   // ---- epilogue: Phi, Q' -> map image (bf16 hi/lo tiles); Psi -> 32-column slabs; Oloc -> row-major
   const MapGeom mg = map_geom(DK, Cs);
   uint8_t* ma = p.ma + (int64_t)blockIdx.x * mg.unit;
@@ -903,8 +906,10 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
     tmem_ld16(cta.tmem + lane + cPhi + c, v);
     if (t < DK && drv.ok) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
+      for (int j = 0; j < 16; ++j) {
+        v[j] = -v[j];
         if (c + j == t) v[j] += gC[t];
+      }
       float a8[8], b8[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
