@@ -234,6 +234,56 @@ __device__ __forceinline__ bool stage_raw(const Tile& t, const float* src, int r
   return ok;
 }
 
+// Stage the elementwise product a * b * f * sign over the unit's `rows` tokens as
+// a bf16 hi/lo operand tile (rows = tokens): K-major over the COLS channels
+// (put_k) or, with MN, MN-major with K = token (put_mn). a, b are [B,T,H,COLS]
+// inputs (b may be null), f a contiguous fp32 [rows][COLS] matrix (may be
+// null). 256 threads; BT tokens per thread per batch with every load of a batch
+// issued before any is used.
+template <typename T, bool MN, int COLS>
+__device__ __forceinline__ void stage_prod(const Tile& t, const ChunkParams& p, const SubIdx& s, int rows, const T* a,
+                                           const T* b, const float* f, float sign) {
+  constexpr int NT = 256, BT = sizeof(T) == 2 ? 4 : 2, G = COLS / 8;
+  for (int x0 = threadIdx.x; x0 < rows * G; x0 += BT * NT) {
+    Pack8<T> pa[BT], pb[BT];
+    Pack8<float> pf[BT];
+#pragma unroll
+    for (int u = 0; u < BT; ++u) {
+      const int x = x0 + u * NT;
+      if (x < rows * G) {
+        const int r = x / G, c8 = (x % G) * 8;
+        const int64_t o = toff(p, s.b, s.tok0 + r, s.h, COLS) + c8;
+        pa[u].ld(a + o);
+        if (b) pb[u].ld(b + o);
+        if (f) pf[u].ld(f + r * COLS + c8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < BT; ++u) {
+      const int x = x0 + u * NT;
+      if (x < rows * G) {
+        const int r = x / G, c8 = (x % G) * 8;
+        float va[8], vb[8];
+        pa[u].get(va);
+        if (b) {
+          pb[u].get(vb);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) va[j] *= vb[j];
+        }
+        if (f) {
+          pf[u].get(vb);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) va[j] *= vb[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) va[j] *= sign;
+        if (MN) put_mn(t, r, c8, va);
+        else put_k(t, r, c8, va);
+      }
+    }
+  }
+}
+
 // CTA prologue shared by the tensor-core kernels: TMEM allocation + mbarrier.
 struct TcCta {
   uint32_t tmem;
@@ -822,40 +872,16 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
       }
     }
   };
-  // (X * Gsuf)^T as an MN-major A operand (M = channel, K = token), scaled by sign.
+  // (X * Gsuf)^T as an MN-major A operand (M = channel, K = token), X = k or e k, scaled by sign.
   auto stage_suffixed = [&](bool erase, float sign) {
-#pragma unroll 4
-    for (int x = tid; x < Cs * (DK / 8); x += NT) {
-      const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-      float xx[8], gs[8];
-      if (erase) rows.a(s.tok0 + r, c8, xx);
-      else rows.k(s.tok0 + r, c8, xx);
-      ld8f(gsuf + r * DK + c8, gs);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xx[j] *= sign * gs[j];
-      put_mn(A, r, c8, xx);
-    }
+    stage_prod<T, true, DK>(A, p, s, Cs, static_cast<const T*>(p.k), erase ? static_cast<const T*>(p.e) : nullptr,
+                            gsuf, sign);
   };
   const uint32_t idK = idesc_bf16(128, DK, 0, 1), idV = idesc_bf16(128, DV, 0, 1);
   const uint32_t idKt = idesc_bf16(128, DK, 1, 1), idVt = idesc_bf16(128, DV, 1, 1);
   // ---- phase 1: W = T (K*Gam), Z = M^kk U, Ut = T Z
-#pragma unroll 4
-  for (int x = tid; x < Cs * (DK / 8); x += NT) {  // B1 = K*Gam (K = token, N = channel)
-    const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-    float kk[8], gm[8];
-    rows.k(s.tok0 + r, c8, kk);
-    ld8f(gam + r * DK + c8, gm);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) kk[j] *= gm[j];
-    put_mn(B1, r, c8, kk);
-  }
-#pragma unroll 4
-  for (int x = tid; x < Cs * (DV / 8); x += NT) {  // B2 = U
-    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
-    float uu[8];
-    rows.u(s.tok0 + r, c8, uu);
-    put_mn(B2, r, c8, uu);
-  }
+  stage_prod<T, true, DK>(B1, p, s, Cs, static_cast<const T*>(p.k), nullptr, gam, 1.f);  // K*Gam (K = token)
+  stage_prod<T, true, DV>(B2, p, s, Cs, static_cast<const T*>(p.v), static_cast<const T*>(p.w), nullptr, 1.f);  // U
   load_img(Tm);
   drv.run([&] { mma_tiles(cta.tmem + cW, A, B1, Cs / 16, idK, NS, false); });
   load_img(G + 0 * sq_bytes(Cs));  // M^kk

@@ -319,20 +319,8 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
     cp_phase ^= 1u;
     if (!ok) drv.ok = false;
   };
-  // B1 = dO (K = token, N = value column)
-#pragma unroll 4
-  for (int x = tid; x < Cs * (DV / 8); x += NT) {
-    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
-    const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
-    float dd[8], zz[8];
-    Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
-    if (p.z) {
-      Elt<T>::ld8(static_cast<const T*>(p.z) + o, zz);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dd[j] *= zz[j];
-    }
-    put_mn(B1, r, c8, dd);
-  }
+  // B1 = dO = z * dy (K = token, N = value column)
+  stage_prod<T, true, DV>(B1, p, s, Cs, static_cast<const T*>(p.dy), static_cast<const T*>(p.z), nullptr, 1.f);
   stage_rows_mn(B2, q.dSC + u * DK * DV, DK, DV, DV, 1.f);  // dS_C (K = channel)
   const uint32_t idT = idesc_bf16(128, DV, 1, 1), idK = idesc_bf16(128, DV, 0, 1);
   load_img(G + 3 * sq_bytes(Cs));  // N^qa -> -dP (partial): N^qa^T dO
@@ -427,30 +415,11 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
   const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
-  auto stage_dO = [&](const Tile& dst) {
-    #pragma unroll 4
-    for (int x = tid; x < Cs * (DV / 8); x += NT) {
-      const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
-      const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
-      float dd[8], zz[8];
-      Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
-      if (p.z) {
-        Elt<T>::ld8(static_cast<const T*>(p.z) + o, zz);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) dd[j] *= zz[j];
-      }
-      put_k(dst, r, c8, dd);
-    }
+  auto stage_dO = [&](const Tile& dst) {  // z * dy (dy alone without z)
+    stage_prod<T, false, DV>(dst, p, s, Cs, static_cast<const T*>(p.dy), static_cast<const T*>(p.z), nullptr, 1.f);
   };
-  auto stage_U = [&](const Tile& dst) {
-    const Rows<T> rows{p, s.b, s.h};
-    #pragma unroll 4
-    for (int x = tid; x < Cs * (DV / 8); x += NT) {
-      const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
-      float uu[8];
-      rows.u(s.tok0 + r, c8, uu);
-      put_k(dst, r, c8, uu);
-    }
+  auto stage_U = [&](const Tile& dst) {  // w * v
+    stage_prod<T, false, DV>(dst, p, s, Cs, static_cast<const T*>(p.v), static_cast<const T*>(p.w), nullptr, 1.f);
   };
   // Row t of a [Cs][N] TMEM result -> dst (fp32, row-major, row stride ld), optional mask.
   auto drain = [&](uint32_t col, int n, float* dst, int64_t ld, int mask) {
