@@ -562,6 +562,7 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
   const float* dG = q.dG + u * 4 * Cs * Cs;
   const int64_t gsz = (int64_t)Cs * Cs;
   tree_tables<DK>(pre, ftab, Cs);
+#pragma unroll 8
   for (int x = tid; x < nb * SB * SB; x += NT) {  // diagonal blocks of the four cotangents
     const int J = x >> 8, tt = (x >> 4) & 15, ss = x & 15;
     const int64_t o = (int64_t)(SB * J + tt) * Cs + SB * J + ss;
