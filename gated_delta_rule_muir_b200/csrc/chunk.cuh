@@ -1139,11 +1139,6 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
   for (int n = 0; n < units && drv.ok; ++n) {
     const int buf = n & 1;
     if (tid < DK) {
-      if (p.S_chunks) {
-        float* o = p.S_chunks + ((uid_of(n) * DK) + tid) * dv + slab * NW;
-#pragma unroll
-        for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&st[j]));
-      }
 #pragma unroll
       for (int j = 0; j < NW; j += 8) {
         float v[8];
@@ -1155,7 +1150,14 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
     const bool c_ok = mbar_wait(&bar_c[buf], (uint32_t)(n >> 1) & 1u);
     if (!__syncthreads_and(c_ok ? 1 : 0)) { drv.ok = false; break; }
     const Tile Phi{base + buf * g.tile, base + buf * g.tile + g.half, 128u, DK * 16u};
-    drv.run([&] { mma_tiles(cta.tmem, Phi, Sb, DK / 16, id, NS, false); });
+    drv.run_overlap([&] { mma_tiles(cta.tmem, Phi, Sb, DK / 16, id, NS, false); },
+                    [&] {  // the chunk-start state leaves while the tensor core works
+                      if (tid < DK && p.S_chunks) {
+                        float* o = p.S_chunks + ((uid_of(n) * DK) + tid) * dv + slab * NW;
+#pragma unroll
+                        for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&st[j]));
+                      }
+                    });
     if (!drv.ok) break;
     float v[NW];
     tmem_ld32(cta.tmem + lane, v);

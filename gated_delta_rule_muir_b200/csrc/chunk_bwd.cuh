@@ -106,9 +106,6 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
     const int n = p.nsub - 1 - k;
     const int buf = k & 1;
     if (tid < DK) {
-      float* o = q.dSC + (uid_of(n) * DK + tid) * dv + slab * NW;
-#pragma unroll
-      for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&ds[j]));
 #pragma unroll
       for (int j = 0; j < NW; j += 8) {
         float v[8];
@@ -120,7 +117,14 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
     const bool c_ok = mbar_wait(&bar_c[buf], (uint32_t)(k >> 1) & 1u);
     if (!__syncthreads_and(c_ok ? 1 : 0)) { drv.ok = false; break; }
     const Tile PhiT{base + buf * g.tile, base + buf * g.tile + g.half, DK * 16u, 128u};
-    drv.run([&] { mma_tiles(cta.tmem, PhiT, Bt, DK / 16, id, NS, false); });
+    drv.run_overlap([&] { mma_tiles(cta.tmem, PhiT, Bt, DK / 16, id, NS, false); },
+                    [&] {  // the unit's state cotangent leaves while the tensor core works
+                      if (tid < DK) {
+                        float* o = q.dSC + (uid_of(n) * DK + tid) * dv + slab * NW;
+#pragma unroll
+                        for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&ds[j]));
+                      }
+                    });
     if (!drv.ok) break;
     float v[NW];
     tmem_ld32(cta.tmem + lane, v);
