@@ -1147,10 +1147,12 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
         put_mn(Sb, tid, j, v);
       }
     }
+    fence_async_smem();  // the state operand is visible to the tensor core after the barrier below
+    tc_fence_before();
     const bool c_ok = mbar_wait(&bar_c[buf], (uint32_t)(n >> 1) & 1u);
     if (!__syncthreads_and(c_ok ? 1 : 0)) { drv.ok = false; break; }
     const Tile Phi{base + buf * g.tile, base + buf * g.tile + g.half, 128u, DK * 16u};
-    drv.run_overlap([&] { mma_tiles(cta.tmem, Phi, Sb, DK / 16, id, NS, false); },
+    drv.run_synced([&] { mma_tiles(cta.tmem, Phi, Sb, DK / 16, id, NS, false); },
                     [&] {  // the chunk-start state leaves while the tensor core works
                       if (tid < DK && p.S_chunks) {
                         float* o = p.S_chunks + ((uid_of(n) * DK) + tid) * dv + slab * NW;

@@ -114,10 +114,12 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
         put_mn(Bt, tid, j, v);
       }
     }
+    fence_async_smem();  // the cotangent operand is visible to the tensor core after the barrier below
+    tc_fence_before();
     const bool c_ok = mbar_wait(&bar_c[buf], (uint32_t)(k >> 1) & 1u);
     if (!__syncthreads_and(c_ok ? 1 : 0)) { drv.ok = false; break; }
     const Tile PhiT{base + buf * g.tile, base + buf * g.tile + g.half, DK * 16u, 128u};
-    drv.run_overlap([&] { mma_tiles(cta.tmem, PhiT, Bt, DK / 16, id, NS, false); },
+    drv.run_synced([&] { mma_tiles(cta.tmem, PhiT, Bt, DK / 16, id, NS, false); },
                     [&] {  // the unit's state cotangent leaves while the tensor core works
                       if (tid < DK) {
                         float* o = q.dSC + (uid_of(n) * DK + tid) * dv + slab * NW;

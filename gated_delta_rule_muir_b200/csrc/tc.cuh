@@ -310,6 +310,24 @@ struct MmaSync {
     return done;
   }
 
+  // As run_overlap, for callers that have already made their operand writes
+  // visible (fence_async_smem + tc_fence_before by every thread, then a CTA
+  // barrier): saves that barrier.
+  template <typename F, typename W>
+  __device__ __forceinline__ bool run_synced(F issue, W work) {
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue();
+      mma_commit(bar);
+    }
+    work();
+    const bool done = __syncthreads_and(mbar_wait(bar, phase) ? 1 : 0) != 0;
+    phase ^= 1u;
+    tc_fence_after();
+    ok = ok && done;
+    return done;
+  }
+
   // Same, but all threads run `work` (which must not touch the staged operands
   // or the accumulators of these MMAs) while the tensor core executes.
   template <typename F, typename W>
