@@ -187,8 +187,8 @@ __device__ __forceinline__ void bulk_g2s_big(uint32_t dst, const uint8_t* src, u
   }
 }
 
-// Stage a contiguous fp32 matrix src[rows][cols] (rows, cols multiples of 8,
-// rows * cols <= 128 * 128) times `sign` as a bf16 hi/lo operand tile: K-major
+// Stage a contiguous fp32 matrix src[rows][cols] (rows a multiple of 8, cols / 8
+// a power of two, rows * cols <= 128 * 128) times `sign` as a bf16 hi/lo operand tile: K-major
 // over cols (put_k, row = MN index) or, with MN, MN-major over rows (put_mn,
 // row = K index). The raw matrix arrives by bulk copy into the tile's own
 // shared memory (hi and lo halves contiguous, at least 4 bytes per element),
@@ -210,23 +210,27 @@ __device__ __forceinline__ bool stage_raw(const Tile& t, const float* src, int r
   phase ^= 1u;
   const float4* raw = reinterpret_cast<const float4*>(__cvta_shared_to_generic(t.hi));
   const int np = rows * cols / 8;
+  const int g = cols / 8;
   float v[MAXP][8];
 #pragma unroll
   for (int k = 0; k < MAXP; ++k) {
     const int x = threadIdx.x + k * NT;
     if (x < np) {
-      const float4 a = raw[2 * x], b = raw[2 * x + 1];
+      int r, c8;
+      piece_of_rot(x, g, r, c8);
+      const int e = r * g + (c8 >> 3);
+      const float4 a = raw[2 * e], b = raw[2 * e + 1];
       v[k][0] = sign * a.x; v[k][1] = sign * a.y; v[k][2] = sign * a.z; v[k][3] = sign * a.w;
       v[k][4] = sign * b.x; v[k][5] = sign * b.y; v[k][6] = sign * b.z; v[k][7] = sign * b.w;
     }
   }
   __syncthreads();
-  const int g = cols / 8;
 #pragma unroll
   for (int k = 0; k < MAXP; ++k) {
     const int x = threadIdx.x + k * NT;
     if (x < np) {
-      const int r = x / g, c8 = (x % g) * 8;
+      int r, c8;
+      piece_of_rot(x, g, r, c8);
       if (MN) put_mn(t, r, c8, v[k]);
       else put_k(t, r, c8, v[k]);
     }
@@ -251,7 +255,8 @@ __device__ __forceinline__ void stage_prod(const Tile& t, const ChunkParams& p, 
     for (int u = 0; u < BT; ++u) {
       const int x = x0 + u * NT;
       if (x < rows * G) {
-        const int r = x / G, c8 = (x % G) * 8;
+        int r, c8;
+        row_piece<T, G>(x, r, c8);
         const int64_t o = toff(p, s.b, s.tok0 + r, s.h, COLS) + c8;
         pa[u].ld(a + o);
         if (b) pb[u].ld(b + o);
@@ -262,7 +267,8 @@ __device__ __forceinline__ void stage_prod(const Tile& t, const ChunkParams& p, 
     for (int u = 0; u < BT; ++u) {
       const int x = x0 + u * NT;
       if (x < rows * G) {
-        const int r = x / G, c8 = (x % G) * 8;
+        int r, c8;
+        row_piece<T, G>(x, r, c8);
         float va[8], vb[8];
         pa[u].get(va);
         if (b) {
@@ -427,7 +433,8 @@ __device__ __forceinline__ void tree_tables(const float* pre, float* ftab, int C
 //   XL row p*2b + X*b + r = [k; r g q]_t * pre_t * F_J(t)   upper t = (2p+1)b + r
 //   YL row p*2b + Y*b + r = [k; e k]_s  * suf_s * F_J(s)    lower s = 2pb + r
 // Staged for the halves asked for; 256 threads, BT tokens per thread per batch
-// with all loads of a batch issued before any is used.
+// with all loads of a batch issued before any is used. Pieces go by row_piece,
+// which keeps a thread on the same 8 channels throughout: rv holds r there.
 template <int DK, typename T>
 __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& s, const float* pre,
                                             const float* suf, const float* ft, const float (&rv)[8], int Cs,
@@ -442,7 +449,8 @@ __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& 
 #pragma unroll
     for (int u = 0; u < BT; ++u) {
       const int x = x0 + u * NT;
-      const int t = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      int t, c8;
+      row_piece<T, DK / 8>(x, t, c8);
       const bool upper = (t >> lb) & 1;
       if (x < Cs * (DK / 8) && (upper ? want_upper : want_lower)) {
         const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DK) + c8;
@@ -455,7 +463,8 @@ __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& 
 #pragma unroll
     for (int u = 0; u < BT; ++u) {
       const int x = x0 + u * NT;
-      const int t = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      int t, c8;
+      row_piece<T, DK / 8>(x, t, c8);
       const bool upper = (t >> lb) & 1;
       if (x < Cs * (DK / 8) && (upper ? want_upper : want_lower)) {
         const int pv = t >> (lb + 1), r = t & (b - 1);
@@ -649,8 +658,12 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
   };
 
   fetch_block(0);
-  float rv[8];  // r for this thread's 8 channels (fixed: NT is a multiple of DK / 8)
-  ld8f(p.r + (int64_t)s.h * DK + (tid % (DK / 8)) * 8, rv);
+  float rv[8];  // r for this thread's 8 channels in stage_level (fixed: 256 pieces per sweep)
+  {
+    int r_, c8_;
+    row_piece<T, DK / 8>(tid, r_, c8_);
+    ld8f(p.r + (int64_t)s.h * DK + c8_, rv);
+  }
   for (int lev = 0; lev < nlev && drv.ok; ++lev) {
     const int lb = lcs - 1 - lev;  // b = 2^lb
     const float* ft = ftab + lev * nb * DK;
@@ -1026,7 +1039,8 @@ __global__ void __launch_bounds__(128, 1) compose_kernel(ChunkParams p) {
   const float* psi0 = p.psi + u0 * DK * DV;
 #pragma unroll 4
   for (int x = tid; x < DK * (DV / 8); x += 128) {
-    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+    int r, c8;
+    piece_of<DV / 8>(x, r, c8);
     float v[8];
     ld8f(psi0 + ((int64_t)(c8 >> 5) * DK + r) * 32 + (c8 & 31), v);
     put_mn(Bpsi, r, c8, v);
@@ -1339,7 +1353,8 @@ __global__ void __launch_bounds__(128, 1) out_kernel(ChunkParams p, const uint8_
   const float* S0 = p.S_chunks + uid * DK * DV;
 #pragma unroll 4
   for (int x = tid; x < DK * (DV / 8); x += 128) {
-    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+    int r, c8;
+    piece_of<DV / 8>(x, r, c8);
     float v[8];
     ld8f(S0 + (int64_t)r * DV + c8, v);
     put_mn(Sb, r, c8, v);

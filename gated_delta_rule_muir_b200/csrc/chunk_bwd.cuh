@@ -150,12 +150,14 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
 }
 
 // Stage a row-major fp32 matrix src[rows][cols] (row stride ld) as a K-major
-// operand contracting over cols (put_k), values scaled by sign. rows <= 128.
+// operand contracting over cols (put_k), values scaled by sign. rows <= 128 and a
+// multiple of 8, cols / 8 a power of two.
 __device__ __forceinline__ void stage_rows_k(const Tile& t, const float* src, int rows, int cols, int64_t ld,
                                              float sign) {
   #pragma unroll 4
   for (int x = threadIdx.x; x < rows * (cols / 8); x += blockDim.x) {
-    const int r = x / (cols / 8), c8 = (x % (cols / 8)) * 8;
+    int r, c8;
+    piece_of_rt(x, cols / 8, r, c8);
     float v[8];
     ld8f(src + r * ld + c8, v);
 #pragma unroll
@@ -168,7 +170,8 @@ __device__ __forceinline__ void stage_rows_mn(const Tile& t, const float* src, i
                                               float sign) {
   #pragma unroll 4
   for (int x = threadIdx.x; x < rows * (cols / 8); x += blockDim.x) {
-    const int r = x / (cols / 8), c8 = (x % (cols / 8)) * 8;
+    int r, c8;
+    piece_of_rt(x, cols / 8, r, c8);
     float v[8];
     ld8f(src + r * ld + c8, v);
 #pragma unroll
@@ -226,7 +229,8 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
   // dO = z * dy (B region is free: both MMAs above have completed)
 #pragma unroll 4
   for (int x = tid; x < Cs * (DV / 8); x += NT) {
-    const int r = x / (DV / 8), c8 = (x % (DV / 8)) * 8;
+    int r, c8;
+    row_piece<T, DV / 8>(x, r, c8);
     const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
     float dd[8], zz[8];
     Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
@@ -337,7 +341,8 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   auto stage_suf = [&](bool erase) {
 #pragma unroll 4
     for (int x = tid; x < Cs * (DK / 8); x += NT) {
-      const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+      int r, c8;
+      row_piece<T, DK / 8>(x, r, c8);
       float xx[8], gs[8];
       if (erase) rows.a(s.tok0 + r, c8, xx);
       else rows.k(s.tok0 + r, c8, xx);
@@ -574,8 +579,12 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
     const int64_t o = (int64_t)(SB * J + tt) * Cs + SB * J + ss;
     dgd[x] = make_float4(dG[o], dG[gsz + o], dG[2 * gsz + o], dG[3 * gsz + o]);
   }
-  float rv[8];
-  ld8f(p.r + (int64_t)s.h * DK + (tid % (DK / 8)) * 8, rv);
+  float rv[8];  // r for this thread's 8 channels in stage_level (fixed: 256 pieces per sweep)
+  {
+    int r_, c8_;
+    row_piece<T, DK / 8>(tid, r_, c8_);
+    ld8f(p.r + (int64_t)s.h * DK + c8_, rv);
+  }
   __syncthreads();
 
   // G_b, K-major: row (p, X, r) -> t = (2p+1) b + r, column (p', Y, r') -> s = 2p'b + r';
@@ -588,7 +597,8 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
 #pragma unroll
       for (int m = 0; m < BG; ++m) {
         const int x = x0 + m * NT;
-        const int row = x >> (lcs - 3), c8 = (x & ((Cs >> 3) - 1)) << 3;
+        int row, c8;
+        piece_of_rt(x, Cs >> 3, row, c8);
         const int pv = row >> (lb + 1), pc = c8 >> (lb + 1);
         if (x < Cs << (lcs - 3) && pv == pc) {
           const int X = (row >> lb) & 1, Y = (c8 >> lb) & 1;
@@ -600,7 +610,8 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
       for (int m = 0; m < BG; ++m) {
         const int x = x0 + m * NT;
         if (x < Cs << (lcs - 3)) {
-          const int row = x >> (lcs - 3), c8 = (x & ((Cs >> 3) - 1)) << 3;
+          int row, c8;
+          piece_of_rt(x, Cs >> 3, row, c8);
           float v[8];
           if ((row >> (lb + 1)) == (c8 >> (lb + 1))) {
             gv[m].get(v);

@@ -200,6 +200,51 @@ __device__ __forceinline__ void put_k(const Tile& t, int m, int k8, const float 
   sts128(t.lo + off, lo);
 }
 
+// Staging sweeps over a rows x (8 G) matrix in 8-element pieces (G a power of
+// two, rows a multiple of 8). put_k and put_mn store a piece to the bank group
+// given by its row & 7, and a 128-bit shared-memory access serves a warp in four
+// phases of 8 consecutive threads, so piece x goes to row ((x / 8G) * 8 + x % 8),
+// column block (x / 8) % G: the 8 threads of a phase take 8 consecutive rows of
+// one column block and store without bank conflicts (taking one row's 8 column
+// blocks would put all 8 in one bank group). In global memory a warp then reads
+// 8 rows x 4 pieces, the same number of sectors as 2 rows x 16 pieces.
+template <int G>
+__device__ __forceinline__ void piece_of(int x, int& r, int& c8) {
+  static_assert(G > 0 && (G & (G - 1)) == 0, "G must be a power of two");
+  constexpr int lg = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : G == 16 ? 4 : G == 32 ? 5 : 6;
+  static_assert((1 << lg) == G, "G out of range");
+  r = ((x >> (3 + lg)) << 3) | (x & 7);
+  c8 = ((x >> 3) & (G - 1)) << 3;
+}
+// Piece order for a sweep reading rows of element type T from global memory:
+// piece_of for fp32 rows (a warp reads 8 rows x 128 bytes, whole lines); for
+// bf16 rows plain row-major order (a warp reads 2 rows x 256 bytes) keeps the
+// loads in whole lines, at the price of bank conflicts on the stores.
+template <typename T, int G>
+__device__ __forceinline__ void row_piece(int x, int& r, int& c8) {
+  if constexpr (sizeof(T) == 4) {
+    piece_of<G>(x, r, c8);
+  } else {
+    r = x / G;
+    c8 = (x % G) * 8;
+  }
+}
+
+// The same for a G known only at run time (a power of two).
+__device__ __forceinline__ void piece_of_rt(int x, int G, int& r, int& c8) {
+  const int lg = 31 - __clz(G);
+  r = ((x >> (3 + lg)) << 3) | (x & 7);
+  c8 = ((x >> 3) & (G - 1)) << 3;
+}
+// For a source read back from row-major shared memory: the column block is also
+// rotated by the row within the phase, so that the phase's reads spread over
+// the bank groups as well.
+__device__ __forceinline__ void piece_of_rot(int x, int G, int& r, int& c8) {
+  const int lg = 31 - __clz(G);
+  r = ((x >> (3 + lg)) << 3) | (x & 7);
+  c8 = (((x >> 3) + (x & 7)) & (G - 1)) << 3;
+}
+
 // MN-major (natural view, lbo = 128): 8 consecutive MN indices m8..m8+7 of contraction row k.
 __device__ __forceinline__ void put_mn(const Tile& t, int k, int m8, const float (&x)[8]) {
   uint4 hi, lo;
