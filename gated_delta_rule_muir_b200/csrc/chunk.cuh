@@ -171,6 +171,12 @@ __host__ __device__ inline uint32_t sq_bytes(int Cs) { return 2u * sq_half(Cs); 
 __device__ __forceinline__ void sq_put(uint8_t* img, int Cs, int r, int c8, const float (&x)[8]) {
   gput_k(img, sq_half(Cs), (uint32_t)Cs * 16u, r, c8, x);
 }
+// An image is lower block-triangular: in row group rg (rows 8 rg .. + 7) only
+// the columns up to the end of the diagonal 16-block, 16 (rg / 2 + 1), can be
+// nonzero, and they are the first sq_prefix(rg) bytes of the group's Cs * 16.
+__host__ __device__ inline uint32_t sq_prefix(int rg) { return (uint32_t)(2 * (rg >> 1) + 2) * 128u; }
+// zeroed shared-memory source of the bulk stores that clear the rest (>= Cs * 16 - 256)
+constexpr uint32_t kZeroBuf = 2048u;
 __device__ __forceinline__ float sq_get(const uint8_t* img, int Cs, int r, int c) {
   const uint32_t off = (uint32_t)(r >> 3) * (uint32_t)Cs * 16u + (uint32_t)(c >> 3) * 128u + (uint32_t)(r & 7) * 16u +
                        (uint32_t)(c & 7) * 2u;
@@ -510,8 +516,8 @@ __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& 
 //   D = XL YL^T (M = 128, N = Cs, K = dk): row block p, column block p holds
 //   the four Gram blocks of pivot p; the other blocks of D are not used.
 // The 16x16 diagonal blocks are computed exactly on the CUDA cores with
-// running products while the tensor core runs; entries above the diagonal
-// blocks are written as zeros.
+// running products while the tensor core runs; the zeros right of the diagonal
+// blocks are written by bulk stores from shared memory.
 // ---------------------------------------------------------------------------
 template <int DK, typename T, int NS>
 __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
@@ -643,20 +649,22 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
     }
     gput_k4(out + g * sq_bytes(Cs), sq_half(Cs), (uint32_t)Cs * 16u, SB * J + t, SB * J + c4, w4);
   };
-  // Zeros above the diagonal blocks of the four images.
+  // Zeros right of the diagonal blocks of the four images, written by the
+  // bulk-copy engine from a zeroed buffer while the threads compute.
   const int lcs = log2_cs(Cs);
-  // In the image an 8-row group is Cs 16-byte chunks; chunk c holds columns
-  // 8 (c >> 3) .. + 7, so its part right of the diagonal block is contiguous.
-  auto zero_upper = [&] {
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int x = tid; x < 8 << (2 * lcs - 3); x += NT) {  // (image, hi/lo, row group, chunk)
-      const int c = x & (Cs - 1), rg = (x >> lcs) & ((Cs >> 3) - 1), gh = x >> (2 * lcs - 3);
-      if ((c >> 4) <= (rg >> 1)) continue;
-      uint8_t* img = out + (gh >> 1) * sq_bytes(Cs) + (gh & 1) * sq_half(Cs);
-      *reinterpret_cast<uint4*>(img + (uint32_t)rg * (uint32_t)Cs * 16u + (uint32_t)c * 16u) = z;
+  if (warp == 0) {
+    const int lane = tid & 31, ng = Cs >> 3;
+    const uint32_t zbuf = base + 4 * LB + (uint32_t)(kMaxLev * 8 * DK + 4 * SB * DK) * 4u, gb = (uint32_t)Cs * 16u;
+    for (uint32_t o = lane * 16u; o < kZeroBuf; o += 512u) sts128(zbuf + o, make_uint4(0, 0, 0, 0));
+    fence_async_smem();
+    __syncwarp();
+    for (int x = lane; x < 8 * ng; x += 32) {  // (image, hi/lo, row group)
+      const int rg = x & (ng - 1), gh = x / ng;
+      const uint32_t pb = sq_prefix(rg);
+      if (pb < gb) bulk_s2g(out + (gh >> 1) * sq_bytes(Cs) + (gh & 1) * sq_half(Cs) + rg * gb + pb, zbuf, gb - pb);
     }
-  };
-
+    bulk_commit();
+  }
   fetch_block(0);
   float rv[8];  // r for this thread's 8 channels in stage_level (fixed: 256 pieces per sweep)
   {
@@ -679,7 +687,6 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
             if (J + 1 < nb) fetch_block(J + 1);
             diag_block(J);
           }
-          if (lev == nlev - 1) zero_upper();
         });
   }
   // Epilogue: lane = row p*2b + X*b + r of level b; the valid columns are the
@@ -704,6 +711,7 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
       }
     }
   }
+  if (warp == 0) bulk_wait_all();  // the zero stores have read their source
   cta.finish();
 }
 

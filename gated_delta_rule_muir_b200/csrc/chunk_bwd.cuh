@@ -225,22 +225,8 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
       mma_tiles(cta.tmem + 128, Qt, B, DK / 16, id, NS, false);
     });
   const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
-  const Rows<T> rows{p, s.b, s.h};
   // dO = z * dy (B region is free: both MMAs above have completed)
-#pragma unroll 4
-  for (int x = tid; x < Cs * (DV / 8); x += NT) {
-    int r, c8;
-    row_piece<T, DV / 8>(x, r, c8);
-    const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DV) + c8;
-    float dd[8], zz[8];
-    Elt<T>::ld8(static_cast<const T*>(p.dy) + o, dd);
-    if (p.z) {
-      Elt<T>::ld8(static_cast<const T*>(p.z) + o, zz);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dd[j] *= zz[j];
-    }
-    put_mn(Bo, r, c8, dd);
-  }
+  stage_prod<T, true, DV>(Bo, p, s, Cs, static_cast<const T*>(p.dy), static_cast<const T*>(p.z), nullptr, 1.f);
   if (drv.ok) drv.run([&] { mma_tiles(cta.tmem + 256, QtT, Bo, Cs / 16, idesc_bf16(128, DV, 1, 1), NS, false); });
   const float* Ut = p.usave + u * Cs * DV;
   const float* olu = p.ol + u * Cs * DV;
@@ -280,7 +266,6 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
       stg_row16(o, v);
     }
   }
-  (void)rows;
   cta.finish();
 }
 
@@ -314,7 +299,6 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   cta.init(&tslot, &bar, 512);
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
-  const Rows<T> rows{p, s.b, s.h};
   const uint8_t* G = p.gr + u * 4 * sq_bytes(Cs);
   const float* gsuf = p.dec + (u * 4 + 3) * Cs * DK;
   const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
@@ -339,18 +323,8 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   drv.run([&] { mma_tiles(cta.tmem + cU, AT, B1, Cs / 16, idT, NS, false); });
   // (A*Gsuf) and (K*Gsuf): rows s, K = channel (K-major)
   auto stage_suf = [&](bool erase) {
-#pragma unroll 4
-    for (int x = tid; x < Cs * (DK / 8); x += NT) {
-      int r, c8;
-      row_piece<T, DK / 8>(x, r, c8);
-      float xx[8], gs[8];
-      if (erase) rows.a(s.tok0 + r, c8, xx);
-      else rows.k(s.tok0 + r, c8, xx);
-      ld8f(gsuf + r * DK + c8, gs);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xx[j] *= gs[j];
-      put_k(Ak, r, c8, xx);
-    }
+    stage_prod<T, false, DK>(Ak, p, s, Cs, static_cast<const T*>(p.k), erase ? static_cast<const T*>(p.e) : nullptr,
+                             gsuf, 1.f);
   };
   stage_suf(true);
   drv.run([&] { mma_tiles(cta.tmem + cP, Ak, B2, DK / 16, idK, NS, true); });  // -dP = N^qa^T dO + (A*Gsuf) dS_C
