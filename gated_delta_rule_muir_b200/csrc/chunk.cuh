@@ -818,13 +818,14 @@ __global__ void __launch_bounds__(256, 1) solve_kernel(ChunkParams p) {
       }
     }
   }
+  fence_async_smem();
   __syncthreads();
-  // the K-major tile of T is exactly its workspace image
-  if (drv.ok) {
-    uint4* out = reinterpret_cast<uint4*>(p.tt + (int64_t)blockIdx.x * sq_bytes(Cs));
-    const uint4* src = reinterpret_cast<const uint4*>(sm + 2 * H);
-#pragma unroll 4
-    for (int x = tid; x < (int)(2 * H / 16); x += NT) out[x] = src[x];
+  // the K-major tile of T is exactly its workspace image: one bulk store
+  if (drv.ok && tid == 0) {
+    uint8_t* out = p.tt + (int64_t)blockIdx.x * sq_bytes(Cs);
+    for (uint32_t o = 0; o < 2 * H; o += 32768u) bulk_s2g(out + o, base + 2 * H + o, 2 * H - o < 32768u ? 2 * H - o : 32768u);
+    bulk_commit();
+    bulk_wait_all();
   }
   cta.finish();
 }
@@ -870,14 +871,22 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   constexpr uint32_t cW = 0, cZ = 128, cUt = 256, cPhi = 384, cPsi = 128, cOl = 256, cQ = 0;
   uint32_t cp_phase = 0;
   // A <- a Gram or T image (one bulk copy); the MMA that last read A has completed.
-  auto load_img = [&](const uint8_t* img) {
+  // issue_img starts the copy, wait_img waits for it: work that does not touch A
+  // can run in between.
+  auto issue_img = [&](const uint8_t* img) {
     if (tid == 0) {
       mbar_expect_tx(&bar_cp, 2 * H);
       bulk_g2s_big(base, img, 2 * H, &bar_cp);
     }
+  };
+  auto wait_img = [&] {
     const bool ok = mbar_wait(&bar_cp, cp_phase);
     cp_phase ^= 1u;
     if (!ok) drv.ok = false;
+  };
+  auto load_img = [&](const uint8_t* img) {
+    issue_img(img);
+    wait_img();
   };
   // TMEM columns [col, col+n) of this thread's row (times sign) -> MN-major B tile row t.
   auto tmem_to_b = [&](const Tile& dst, uint32_t col, int n, float sign) {
@@ -901,14 +910,16 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   const uint32_t idK = idesc_bf16(128, DK, 0, 1), idV = idesc_bf16(128, DV, 0, 1);
   const uint32_t idKt = idesc_bf16(128, DK, 1, 1), idVt = idesc_bf16(128, DV, 1, 1);
   // ---- phase 1: W = T (K*Gam), Z = M^kk U, Ut = T Z
+  issue_img(Tm);
   stage_prod<T, true, DK>(B1, p, s, Cs, static_cast<const T*>(p.k), nullptr, gam, 1.f);  // K*Gam (K = token)
   stage_prod<T, true, DV>(B2, p, s, Cs, static_cast<const T*>(p.v), static_cast<const T*>(p.w), nullptr, 1.f);  // U
-  load_img(Tm);
+  wait_img();
   drv.run([&] { mma_tiles(cta.tmem + cW, A, B1, Cs / 16, idK, NS, false); });
   load_img(G + 0 * sq_bytes(Cs));  // M^kk
   drv.run([&] { mma_tiles(cta.tmem + cZ, A, B2, Cs / 16, idV, NS, false); });
+  issue_img(Tm);
   tmem_to_b(B1, cZ, DV, 1.f);
-  load_img(Tm);
+  wait_img();
   drv.run([&] { mma_tiles(cta.tmem + cUt, A, B1, Cs / 16, idV, NS, false); });
   if (p.wsave) {  // the backward pass reuses W and Ut
     float* wo = p.wsave + (int64_t)blockIdx.x * Cs * DK;

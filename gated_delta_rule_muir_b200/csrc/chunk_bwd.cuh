@@ -304,20 +304,29 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
   constexpr uint32_t cP = 0, cU = 128, cZ = 256;
   uint32_t cp_phase = 0;
-  auto load_img = [&](const uint8_t* img) {
+  // image copies into the A region: issue_img starts one (no MMA may be reading
+  // the region), wait_img waits for it; work that does not touch A runs between
+  auto issue_img = [&](const uint8_t* img) {
     if (tid == 0) {
       mbar_expect_tx(&bar_cp, 2 * H);
       bulk_g2s_big(base, img, 2 * H, &bar_cp);
     }
+  };
+  auto wait_img = [&] {
     const bool ok = mbar_wait(&bar_cp, cp_phase);
     cp_phase ^= 1u;
     if (!ok) drv.ok = false;
   };
+  auto load_img = [&](const uint8_t* img) {
+    issue_img(img);
+    wait_img();
+  };
+  issue_img(G + 3 * sq_bytes(Cs));  // N^qa -> -dP (partial): N^qa^T dO
   // B1 = dO = z * dy (K = token, N = value column)
   stage_prod<T, true, DV>(B1, p, s, Cs, static_cast<const T*>(p.dy), static_cast<const T*>(p.z), nullptr, 1.f);
   stage_rows_mn(B2, q.dSC + u * DK * DV, DK, DV, DV, 1.f);  // dS_C (K = channel)
   const uint32_t idT = idesc_bf16(128, DV, 1, 1), idK = idesc_bf16(128, DV, 0, 1);
-  load_img(G + 3 * sq_bytes(Cs));  // N^qa -> -dP (partial): N^qa^T dO
+  wait_img();
   drv.run([&] { mma_tiles(cta.tmem + cP, AT, B1, Cs / 16, idT, NS, false); });
   load_img(G + 2 * sq_bytes(Cs));  // N^qk -> dU: N^qk^T dO
   drv.run([&] { mma_tiles(cta.tmem + cU, AT, B1, Cs / 16, idT, NS, false); });
@@ -331,6 +340,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   stage_suf(false);
   drv.run([&] { mma_tiles(cta.tmem + cU, Ak, B2, DK / 16, idK, NS, true); });  // + (K*Gsuf) dS_C
   // dP (TMEM, negated) -> B3 (K = token), then dZ = T^T dP
+  issue_img(p.tt + u * sq_bytes(Cs));  // T^T
   for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cP + c, v);
@@ -342,7 +352,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
       put_mn(B3, t, c + 8, b8);
     }
   }
-  load_img(p.tt + u * sq_bytes(Cs));  // T^T
+  wait_img();
   drv.run([&] { mma_tiles(cta.tmem + cZ, AT, B3, Cs / 16, idT, NS, false); });
   float* dZo = q.dZ + u * Cs * DV;
   for (int c = wg * 16; c < DV; c += 32) {
