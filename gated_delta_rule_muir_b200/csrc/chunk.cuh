@@ -1344,13 +1344,16 @@ __global__ void apply_map_kernel(const float* __restrict__ Phi, const float* __r
 // out_kernel: outputs of one chunk from its start state, all chunks in
 // parallel:  y = z * (Q' S0 + Oloc).
 // A = Q' tiles of the map image (bulk copy, K-major over key channels),
-// B = S0 (MN-major: K = key channel, N = value column), staged by the threads.
+// B = S0 (MN-major: K = key channel, N = value column), bulk-copied raw and
+// converted in place (stage_raw). 256 threads: TMEM row t = tid % 128, the two
+// warpgroups take alternate 16-column chunks; every load of a row's Oloc and z
+// is issued before the accumulator is read.
 // ---------------------------------------------------------------------------
 template <int DK, int DV, typename T, int NS>
-__global__ void __launch_bounds__(128, 1) out_kernel(ChunkParams p, const uint8_t* ma, const float* ol, int units,
+__global__ void __launch_bounds__(256, 1) out_kernel(ChunkParams p, const uint8_t* ma, const float* ol, int units,
                                                      int ulen) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar, bar_cp;
+  __shared__ uint64_t bar, bar_cp, bar_s0;
   __shared__ uint32_t tslot;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t uid = blockIdx.x;
@@ -1362,24 +1365,20 @@ __global__ void __launch_bounds__(128, 1) out_kernel(ChunkParams p, const uint8_
   const uint32_t base = smem_u32(sm);
   const uint32_t s_off = (uint32_t)nq * g.tile;
   const Tile Sb{base + s_off, base + s_off + DK * DV * 2u, 128u, DK * 16u};
-  if (tid == 0) mbar_init(&bar_cp, 1);
+  if (tid == 0) {
+    mbar_init(&bar_cp, 1);
+    mbar_init(&bar_s0, 1);
+  }
   TcCta cta;
   cta.init(&tslot, &bar, tmem_cols_for(nq * DV));
   if (tid == 0) {
     mbar_expect_tx(&bar_cp, nq * g.tile);
     bulk_g2s_big(base, ma + uid * g.unit + g.tile, nq * g.tile, &bar_cp);
   }
-  const float* S0 = p.S_chunks + uid * DK * DV;
-#pragma unroll 4
-  for (int x = tid; x < DK * (DV / 8); x += 128) {
-    int r, c8;
-    piece_of<DV / 8>(x, r, c8);
-    float v[8];
-    ld8f(S0 + (int64_t)r * DV + c8, v);
-    put_mn(Sb, r, c8, v);
-  }
+  uint32_t ph_s0 = 0;
+  const bool s0_ok = stage_raw<true>(Sb, p.S_chunks + uid * DK * DV, DK, DV, 1.f, &bar_s0, ph_s0);
   MmaSync drv{&bar, 0u, true};
-  drv.ok = __syncthreads_and(mbar_wait(&bar_cp, 0) ? 1 : 0) != 0;
+  drv.ok = __syncthreads_and((mbar_wait(&bar_cp, 0) && s0_ok) ? 1 : 0) != 0;
   const uint32_t id = idesc_bf16(128, DV, 0, 1);
   if (drv.ok)
     drv.run([&] {
@@ -1389,28 +1388,40 @@ __global__ void __launch_bounds__(128, 1) out_kernel(ChunkParams p, const uint8_
       }
     });
   const uint32_t lane = tmem_lane_base(warp);
+  const int t = tid & 127, wg = tid >> 7;
+  constexpr int NC = DV / 32;  // 16-column chunks per thread
   const float* olu = ol + uid * ulen * DV;
+  const T* zp = static_cast<const T*>(p.z);
   for (int j = 0; j < nq; ++j) {
-    const int tt = j * 128 + tid;
+    const int tt = j * 128 + t;
     const bool on = tt < ulen && drv.ok;
     const int64_t yo = toff(p, b, (int64_t)n * ulen + tt, h, DV);
-    for (int c = 0; c < DV; c += 16) {
+    Pack8<float> pa[NC][2];
+    Pack8<T> pz[NC][2];
+    if (on) {
+#pragma unroll
+      for (int k = 0; k < NC; ++k)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          const int c = wg * 16 + 32 * k + 8 * h8;
+          pa[k][h8].ld(olu + (int64_t)tt * DV + c);
+          pz[k][h8].ld_or_one(zp ? zp + yo + c : nullptr);  // y = o when z is absent
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = wg * 16 + 32 * k;
       float v[16];
       tmem_ld16(cta.tmem + lane + j * DV + c, v);
       if (!on) continue;
 #pragma unroll
-      for (int h8 = 0; h8 < 16; h8 += 8) {
-        float o8[8], a8[8];
-        ld8f(olu + (int64_t)tt * DV + c + h8, a8);
+      for (int h8 = 0; h8 < 2; ++h8) {
+        float a8[8], z8[8], o8[8];
+        pa[k][h8].get(a8);
+        pz[k][h8].get(z8);
 #pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) o8[e2] = v[h8 + e2] + a8[e2];
-        if (p.z) {
-          float zz[8];
-          Elt<T>::ld8(static_cast<const T*>(p.z) + yo + c + h8, zz);
-#pragma unroll
-          for (int e2 = 0; e2 < 8; ++e2) o8[e2] *= zz[e2];
-        }
-        Elt<T>::st8(static_cast<T*>(p.y) + yo + c + h8, o8);
+        for (int e2 = 0; e2 < 8; ++e2) o8[e2] = (v[8 * h8 + e2] + a8[e2]) * z8[e2];
+        Elt<T>::st8(static_cast<T*>(p.y) + yo + c + 8 * h8, o8);
       }
     }
   }
