@@ -194,26 +194,21 @@ __device__ __forceinline__ void bulk_g2s_big(uint32_t dst, const uint8_t* src, u
 }
 
 // Stage a contiguous fp32 matrix src[rows][cols] (rows a multiple of 8, cols / 8
-// a power of two, rows * cols <= 128 * 128) times `sign` as a bf16 hi/lo operand tile: K-major
-// over cols (put_k, row = MN index) or, with MN, MN-major over rows (put_mn,
-// row = K index). The raw matrix arrives by bulk copy into the tile's own
-// shared memory (hi and lo halves contiguous, at least 4 bytes per element),
+// a power of two, rows * cols <= 128 * 128) times `sign` as a bf16 hi/lo operand
+// tile: K-major over cols (put_k, row = MN index) or, with MN, MN-major over rows
+// (put_mn, row = K index). The raw matrix arrives by bulk copy into the tile's
+// own shared memory (hi and lo halves contiguous, at least 4 bytes per element),
 // every thread takes its pieces into registers, and after a barrier writes them
-// back converted. 256 threads, all of which call it; no MMA may be reading the
-// tile. Returns false if the copy's bounded wait ran out.
+// back converted. In two steps: raw_issue (thread 0 starts the copy on `bar`,
+// whose transaction count the caller has set) and, once the copy has landed,
+// raw_convert (every thread; ends without a barrier). stage_raw does both.
+__device__ __forceinline__ void raw_issue(const Tile& t, const float* src, int rows, int cols, uint64_t* bar) {
+  if (threadIdx.x == 0)
+    bulk_g2s_big(t.hi, reinterpret_cast<const uint8_t*>(src), (uint32_t)rows * (uint32_t)cols * 4u, bar);
+}
 template <bool MN>
-__device__ __forceinline__ bool stage_raw(const Tile& t, const float* src, int rows, int cols, float sign,
-                                          uint64_t* bar, uint32_t& phase) {
+__device__ __forceinline__ void raw_convert(const Tile& t, int rows, int cols, float sign) {
   constexpr int NT = 256, MAXP = 128 * 128 / 8 / NT;
-  const uint32_t bytes = (uint32_t)rows * (uint32_t)cols * 4u;
-  fence_async_smem();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_expect_tx(bar, bytes);
-    bulk_g2s_big(t.hi, reinterpret_cast<const uint8_t*>(src), bytes, bar);
-  }
-  const bool ok = __syncthreads_and(mbar_wait(bar, phase) ? 1 : 0) != 0;
-  phase ^= 1u;
   const float4* raw = reinterpret_cast<const float4*>(__cvta_shared_to_generic(t.hi));
   const int np = rows * cols / 8;
   const int g = cols / 8;
@@ -241,6 +236,19 @@ __device__ __forceinline__ bool stage_raw(const Tile& t, const float* src, int r
       else put_k(t, r, c8, v[k]);
     }
   }
+}
+// 256 threads, all of which call it; no MMA may be reading the tile. Returns
+// false if the copy's bounded wait ran out.
+template <bool MN>
+__device__ __forceinline__ bool stage_raw(const Tile& t, const float* src, int rows, int cols, float sign,
+                                          uint64_t* bar, uint32_t& phase) {
+  fence_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_expect_tx(bar, (uint32_t)rows * (uint32_t)cols * 4u);
+  raw_issue(t, src, rows, cols, bar);
+  const bool ok = __syncthreads_and(mbar_wait(bar, phase) ? 1 : 0) != 0;
+  phase ^= 1u;
+  raw_convert<MN>(t, rows, cols, sign);
   return ok;
 }
 

@@ -190,7 +190,7 @@ __device__ __forceinline__ void stage_rows_mn(const Tile& t, const float* src, i
 template <int DK, int DV, typename T, int NS>
 __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar, bar_cp;
+  __shared__ uint64_t bar, bar_cp, bar_s;
   __shared__ uint32_t tslot;
   const int Cs = p.Cs;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
@@ -205,7 +205,10 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
   const Tile A{base + 2 * TB, base + 3 * TB, 128u, DK * 16u};  // W: rows = tokens, K = key channel
   const Tile B{base + 4 * TB, base + 5 * TB, 128u, DK * 16u};  // S0: K = key channel, N = value column
   const Tile Bo{base + 4 * TB, base + 5 * TB, 128u, (uint32_t)Cs * 16u};  // dO: K = token, N = value column
-  if (tid == 0) mbar_init(&bar_cp, 1);
+  if (tid == 0) {
+    mbar_init(&bar_cp, 1);
+    mbar_init(&bar_s, 1);
+  }
   TcCta cta;
   cta.init(&tslot, &bar, 512);
   if (tid == 0) {
@@ -215,9 +218,10 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
   const float* S0 = q.S_chunks + u * DK * DV;
-  stage_rows_k(A, p.wsave + u * Cs * DK, Cs, DK, DK, 1.f);
-  stage_rows_mn(B, S0, DK, DV, DV, 1.f);
-  drv.ok = __syncthreads_and(mbar_wait(&bar_cp, 0) ? 1 : 0) != 0;
+  uint32_t ph_s = 0;
+  bool st_ok = stage_raw<false>(A, p.wsave + u * Cs * DK, Cs, DK, 1.f, &bar_s, ph_s);
+  st_ok = stage_raw<true>(B, S0, DK, DV, 1.f, &bar_s, ph_s) && st_ok;
+  drv.ok = __syncthreads_and((mbar_wait(&bar_cp, 0) && st_ok) ? 1 : 0) != 0;
   const uint32_t id = idesc_bf16(128, DV, 0, 1);
   if (drv.ok)
     drv.run([&] {
@@ -231,28 +235,51 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
   const float* Ut = p.usave + u * Cs * DV;
   const float* olu = p.ol + u * Cs * DV;
   float* P = q.P + u * Cs * DV;
-  for (int c = wg * 16; c < DV; c += 32) {
-    float v[16], w[16];
-    tmem_ld16(cta.tmem + lane + c, v);
-    tmem_ld16(cta.tmem + lane + 128 + c, w);
-    if (t < Cs && drv.ok) {
+  {
+    // every load of the row is issued before the accumulators are read
+    constexpr int NC = DV / 32;  // 16-column chunks per thread
+    const bool on = t < Cs && drv.ok, wdz = p.dz && p.z;
+    const int64_t o = toff(p, s.b, s.tok0 + (t < Cs ? t : 0), s.h, DV);
+    Pack8<float> pu[NC][2], po[NC][2];
+    Pack8<T> pd[NC][2];
+    if (on) {
+#pragma unroll
+      for (int k = 0; k < NC; ++k)
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          const int c = wg * 16 + 32 * k + 8 * h8;
+          pu[k][h8].ld(Ut + t * DV + c);
+          if (wdz) {
+            pd[k][h8].ld(static_cast<const T*>(p.dy) + o + c);
+            po[k][h8].ld(olu + (int64_t)t * DV + c);
+          }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = wg * 16 + 32 * k;
+      float v[16], w[16];
+      tmem_ld16(cta.tmem + lane + c, v);
+      tmem_ld16(cta.tmem + lane + 128 + c, w);
+      if (!on) continue;
       float pv[16];
 #pragma unroll
-      for (int j = 0; j < 16; j += 4) {
-        const float4 a = *reinterpret_cast<const float4*>(Ut + t * DV + c + j);
-        pv[j] = v[j] + a.x; pv[j + 1] = v[j + 1] + a.y; pv[j + 2] = v[j + 2] + a.z; pv[j + 3] = v[j + 3] + a.w;
+      for (int h8 = 0; h8 < 2; ++h8) {
+        float a8[8];
+        pu[k][h8].get(a8);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) pv[8 * h8 + j] = v[8 * h8 + j] + a8[j];
       }
       stg_row16(P + t * DV + c, pv);
-      if (p.dz && p.z) {
-        const int64_t o = toff(p, s.b, s.tok0 + t, s.h, DV) + c;
+      if (wdz) {
 #pragma unroll
-        for (int h8 = 0; h8 < 16; h8 += 8) {
+        for (int h8 = 0; h8 < 2; ++h8) {
           float dd[8], ol8[8], out[8];
-          Elt<T>::ld8(static_cast<const T*>(p.dy) + o + h8, dd);
-          ld8f(olu + (int64_t)t * DV + c + h8, ol8);
+          pd[k][h8].get(dd);
+          po[k][h8].get(ol8);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) out[j] = dd[j] * (w[h8 + j] + ol8[j]);
-          Elt<T>::st8(static_cast<T*>(p.dz) + o + h8, out);
+          for (int j = 0; j < 8; ++j) out[j] = dd[j] * (w[8 * h8 + j] + ol8[j]);
+          Elt<T>::st8(static_cast<T*>(p.dz) + o + c + 8 * h8, out);
         }
       }
     }
@@ -440,6 +467,20 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   };
   const uint32_t idK = idesc_bf16(128, DK, 0, 0), idC = idesc_bf16(128, Cs, 0, 0);
   float* g4 = q.g4 + u * 4 * Cs * DK;
+  float* dG = q.dG + u * 4 * Cs * Cs;
+  const uint32_t mat_dkdv = (uint32_t)DK * DV * 4u, mat_csdv = (uint32_t)Cs * DV * 4u;
+  // Each raw fp32 operand is bulk-copied into its tile (raw_issue) while other
+  // work runs, and converted once it has landed.
+  auto raw_wait = [&] {
+    if (!__syncthreads_and(mbar_wait(&bar_cp, cph) ? 1 : 0)) drv.ok = false;
+    cph ^= 1u;
+  };
+  // pass 1: R0 = dS_C, R1 = U, R2 = -P
+  fence_async_smem();
+  __syncthreads();
+  if (tid == 0) mbar_expect_tx(&bar_cp, mat_dkdv + mat_csdv);
+  raw_issue(R0, q.dSC + u * DK * DV, DK, DV, &bar_cp);
+  raw_issue(R2, q.P + u * Cs * DV, Cs, DV, &bar_cp);
   if (tid < DK) {  // dGam_C[i] = sum_j dS_C[i][j] S0[i][j]
     const float* d = q.dSC + u * DK * DV + tid * DV;
     const float* s0 = q.S_chunks + u * DK * DV + tid * DV;
@@ -451,39 +492,43 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
     }
     q.dgc[u * DK + tid] = acc;
   }
-  float* dG = q.dG + u * 4 * Cs * Cs;
-  // pass 1
-  if (!stage_raw<false>(R0, q.dSC + u * DK * DV, DK, DV, 1.f, &bar_cp, cph)) drv.ok = false;
   stage_U(R1);
-  if (!stage_raw<false>(R2, q.P + u * Cs * DV, Cs, DV, -1.f, &bar_cp, cph)) drv.ok = false;
+  raw_wait();
+  raw_convert<false>(R0, DK, DV, 1.f);
+  raw_convert<false>(R2, Cs, DV, -1.f);
   drv.run([&] {
     mma_tiles(cta.tmem + 0, R1, R0, DV / 16, idK, NS, false);
     mma_tiles(cta.tmem + 128, R2, R0, DV / 16, idK, NS, false);
   });
   drain(0, DK, g4 + 2 * Cs * DK, DK, 0);    // dKs
   drain(128, DK, g4 + 3 * Cs * DK, DK, 0);  // dAs
-  // pass 2: R1 = U, R2 = -P stay
+  // pass 2: R1 = U, R2 = -P stay; R0 = dO, then dZ
   stage_dO(R0);
   drv.run([&] {
     mma_tiles(cta.tmem + 0, R0, R1, DV / 16, idC, NS, false);    // dN^qk
     mma_tiles(cta.tmem + 128, R0, R2, DV / 16, idC, NS, false);  // dN^qa
   });
-  if (!stage_raw<false>(R0, q.dZ + u * Cs * DV, Cs, DV, 1.f, &bar_cp, cph)) drv.ok = false;
+  if (tid == 0) mbar_expect_tx(&bar_cp, mat_csdv);
+  raw_issue(R0, q.dZ + u * Cs * DV, Cs, DV, &bar_cp);
+  drain(0, Cs, dG + 2 * Cs * Cs, Cs, 2);
+  drain(128, Cs, dG + 3 * Cs * Cs, Cs, 2);
+  raw_wait();
+  raw_convert<false>(R0, Cs, DV, 1.f);
   drv.run([&] {
     mma_tiles(cta.tmem + 256, R0, R1, DV / 16, idC, NS, false);  // dM^kk
     mma_tiles(cta.tmem + 384, R0, R2, DV / 16, idC, NS, false);  // dM^ka
   });
-  drain(0, Cs, dG + 2 * Cs * Cs, Cs, 2);
-  drain(128, Cs, dG + 3 * Cs * Cs, Cs, 2);
+  // pass 3: R0 = dZ stays, R1 = S0, R2 = dO
+  if (tid == 0) mbar_expect_tx(&bar_cp, mat_dkdv);
+  raw_issue(R1, q.S_chunks + u * DK * DV, DK, DV, &bar_cp);
+  stage_dO(R2);
   drain(256, Cs, dG + 0 * Cs * Cs, Cs, 1);
   drain(384, Cs, dG + 1 * Cs * Cs, Cs, 1);
-  // pass 3: R1 = S0, R0 = dO, R2 = dZ
-  if (!stage_raw<false>(R1, q.S_chunks + u * DK * DV, DK, DV, 1.f, &bar_cp, cph)) drv.ok = false;
-  stage_dO(R0);
-  if (!stage_raw<false>(R2, q.dZ + u * Cs * DV, Cs, DV, 1.f, &bar_cp, cph)) drv.ok = false;
+  raw_wait();
+  raw_convert<false>(R1, DK, DV, 1.f);
   drv.run([&] {
-    mma_tiles(cta.tmem + 0, R0, R1, DV / 16, idK, NS, false);    // dQp
-    mma_tiles(cta.tmem + 128, R2, R1, DV / 16, idK, NS, false);  // dKp
+    mma_tiles(cta.tmem + 0, R2, R1, DV / 16, idK, NS, false);    // dQp
+    mma_tiles(cta.tmem + 128, R0, R1, DV / 16, idK, NS, false);  // dKp
   });
   drain(0, DK, g4 + 0 * Cs * DK, DK, 0);
   drain(128, DK, g4 + 1 * Cs * DK, DK, 0);
