@@ -549,7 +549,6 @@ __global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
   cta.init(&tslot, &bar, tmem_cols_for(128 * nlev));
   const float* pre = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
   const float* suf = pre + Cs * DK;
-  const Rows<T> rows{p, s.b, s.h};
   uint8_t* out = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
   MmaSync drv{&bar, 0u, true};
   const uint32_t id = idesc_bf16(128, Cs, 0, 0);
@@ -871,7 +870,6 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   const float* gsuf = dec + 3 * Cs * DK;
   const uint8_t* G = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
   const uint8_t* Tm = p.tt + (int64_t)blockIdx.x * sq_bytes(Cs);
-  const Rows<T> rows{p, s.b, s.h};
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
   const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups take alternate 16-column chunks
@@ -991,17 +989,40 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
       stg_row16(o, v);
     }
   }
-  for (int c = wg * 16; c < DK; c += 32) {
-    float v[16];
-    tmem_ld16(cta.tmem + lane + cQ + c, v);
-    if (t < Cs && drv.ok) {
-      float qq[8], gm[8];
+  {
+    // Q' = Qt * Gam - N^qa W, Qt = r g q: every load of the row is issued first
+    constexpr int NC = DK / 32;  // 16-column chunks per thread
+    const bool on = t < Cs && drv.ok;
+    const int64_t o = toff(p, s.b, s.tok0 + (t < Cs ? t : 0), s.h, DK);
+    const T* gp = static_cast<const T*>(p.g);
+    Pack8<T> pq[NC][2], pg[NC][2];
+    Pack8<float> pm[NC][2];
+    if (on) {
 #pragma unroll
-      for (int h8 = 0; h8 < 16; h8 += 8) {
-        rows.qt(s.tok0 + t, c + h8, qq);
-        ld8f(gam + t * DK + c + h8, gm);
+      for (int k = 0; k < NC; ++k)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[h8 + j] = qq[j] * gm[j] - v[h8 + j];
+        for (int h8 = 0; h8 < 2; ++h8) {
+          const int c = wg * 16 + 32 * k + 8 * h8;
+          pq[k][h8].ld(static_cast<const T*>(p.q) + o + c);
+          pg[k][h8].ld_or_one(gp ? gp + o + c : nullptr);  // static-only readout: g = 1
+          pm[k][h8].ld(gam + t * DK + c);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = wg * 16 + 32 * k;
+      float v[16];
+      tmem_ld16(cta.tmem + lane + cQ + c, v);
+      if (!on) continue;
+#pragma unroll
+      for (int h8 = 0; h8 < 2; ++h8) {
+        float qq[8], gg[8], gm[8], rr[8];
+        pq[k][h8].get(qq);
+        pg[k][h8].get(gg);
+        pm[k][h8].get(gm);
+        ld8f(p.r + (int64_t)s.h * DK + c + 8 * h8, rr);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[8 * h8 + j] = (rr[j] * gg[j] * qq[j]) * gm[j] - v[8 * h8 + j];
       }
       float a8[8], b8[8];
 #pragma unroll

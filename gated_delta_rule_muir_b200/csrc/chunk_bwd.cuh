@@ -382,6 +382,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   wait_img();
   drv.run([&] { mma_tiles(cta.tmem + cZ, AT, B3, Cs / 16, idT, NS, false); });
   float* dZo = q.dZ + u * Cs * DV;
+  issue_img(G + 0 * sq_bytes(Cs));  // M^kk^T (A is free: the T^T product has completed)
   for (int c = wg * 16; c < DV; c += 32) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cZ + c, v);
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
         stg_row16(dZo + t * DV + c, v);
     }
   }
-  load_img(G + 0 * sq_bytes(Cs));  // M^kk^T
+  wait_img();
   drv.run([&] { mma_tiles(cta.tmem + cU, AT, B3, Cs / 16, idT, NS, true); });
   float* dUo = q.dU + u * Cs * DV;
   for (int c = wg * 16; c < DV; c += 32) {
