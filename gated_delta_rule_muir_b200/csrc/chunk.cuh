@@ -957,7 +957,50 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   drv.run([&] { mma_tiles(cta.tmem + cOl, A, B1, Cs / 16, idV, NS, false); });  // B1 holds -Ut
   tmem_to_b(B1, cW, DK, 1.f);
   drv.run([&] { mma_tiles(cta.tmem + cQ, A, B1, Cs / 16, idK, NS, false); });
-  load_img(G + 2 * sq_bytes(Cs));  // N^qk
+  issue_img(G + 2 * sq_bytes(Cs));  // N^qk (A is free: the Q product has completed)
+  // Qt * Gam (Qt = r g q) as fp32 rows in B1's shared memory (B1 is free), read
+  // back by the epilogue's TMEM rows. The 16-byte chunk j of row t is stored at
+  // chunk j ^ (t & 7), so that 8 consecutive rows reading the same chunk hit 8
+  // distinct bank groups.
+  float* qgam = reinterpret_cast<float*>(sm + 2 * TBY);
+  {
+    constexpr int BT = 4;
+    const T* gp = static_cast<const T*>(p.g);
+    for (int x0 = tid; x0 < Cs * (DK / 8); x0 += BT * NT) {
+      Pack8<T> pq[BT], pg[BT];
+      Pack8<float> pm[BT];
+#pragma unroll
+      for (int u = 0; u < BT; ++u) {
+        const int x = x0 + u * NT;
+        if (x < Cs * (DK / 8)) {
+          const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+          const int64_t o = toff(p, s.b, s.tok0 + r, s.h, DK) + c8;
+          pq[u].ld(static_cast<const T*>(p.q) + o);
+          pg[u].ld_or_one(gp ? gp + o : nullptr);  // static-only readout: g = 1
+          pm[u].ld(gam + r * DK + c8);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < BT; ++u) {
+        const int x = x0 + u * NT;
+        if (x < Cs * (DK / 8)) {
+          const int r = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
+          float qq[8], gg[8], gm[8], rr[8];
+          pq[u].get(qq);
+          pg[u].get(gg);
+          pm[u].get(gm);
+          ld8f(p.r + (int64_t)s.h * DK + c8, rr);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) qq[j] = (rr[j] * gg[j] * qq[j]) * gm[j];
+          const int j0 = c8 >> 2;
+          *reinterpret_cast<float4*>(qgam + r * DK + ((j0 ^ (r & 7)) << 2)) = make_float4(qq[0], qq[1], qq[2], qq[3]);
+          *reinterpret_cast<float4*>(qgam + r * DK + (((j0 + 1) ^ (r & 7)) << 2)) =
+              make_float4(qq[4], qq[5], qq[6], qq[7]);
+        }
+      }
+    }
+  }
+  wait_img();
   drv.run([&] { mma_tiles(cta.tmem + cOl, A, B2, Cs / 16, idV, NS, true); });
   // ---- epilogue: Phi, Q' -> map image (bf16 hi/lo tiles); Psi -> 32-column slabs; Oloc -> row-major
   const MapGeom mg = map_geom(DK, Cs);
@@ -989,40 +1032,18 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
       stg_row16(o, v);
     }
   }
-  {
-    // Q' = Qt * Gam - N^qa W, Qt = r g q: every load of the row is issued first
-    constexpr int NC = DK / 32;  // 16-column chunks per thread
-    const bool on = t < Cs && drv.ok;
-    const int64_t o = toff(p, s.b, s.tok0 + (t < Cs ? t : 0), s.h, DK);
-    const T* gp = static_cast<const T*>(p.g);
-    Pack8<T> pq[NC][2], pg[NC][2];
-    Pack8<float> pm[NC][2];
-    if (on) {
+  // Q' = Qt * Gam - N^qa W, Qt * Gam from shared memory (staged above)
+  for (int c = wg * 16; c < DK; c += 32) {
+    float v[16];
+    tmem_ld16(cta.tmem + lane + cQ + c, v);
+    if (t < Cs && drv.ok) {
 #pragma unroll
-      for (int k = 0; k < NC; ++k)
-#pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          const int c = wg * 16 + 32 * k + 8 * h8;
-          pq[k][h8].ld(static_cast<const T*>(p.q) + o + c);
-          pg[k][h8].ld_or_one(gp ? gp + o + c : nullptr);  // static-only readout: g = 1
-          pm[k][h8].ld(gam + t * DK + c);
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      const int c = wg * 16 + 32 * k;
-      float v[16];
-      tmem_ld16(cta.tmem + lane + cQ + c, v);
-      if (!on) continue;
-#pragma unroll
-      for (int h8 = 0; h8 < 2; ++h8) {
-        float qq[8], gg[8], gm[8], rr[8];
-        pq[k][h8].get(qq);
-        pg[k][h8].get(gg);
-        pm[k][h8].get(gm);
-        ld8f(p.r + (int64_t)s.h * DK + c + 8 * h8, rr);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[8 * h8 + j] = (rr[j] * gg[j] * qq[j]) * gm[j] - v[8 * h8 + j];
+      for (int jj = 0; jj < 4; ++jj) {
+        const float4 a = *reinterpret_cast<const float4*>(qgam + t * DK + ((((c >> 2) + jj) ^ (t & 7)) << 2));
+        v[4 * jj] = a.x - v[4 * jj];
+        v[4 * jj + 1] = a.y - v[4 * jj + 1];
+        v[4 * jj + 2] = a.z - v[4 * jj + 2];
+        v[4 * jj + 3] = a.w - v[4 * jj + 3];
       }
       float a8[8], b8[8];
 #pragma unroll
