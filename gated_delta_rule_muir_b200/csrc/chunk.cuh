@@ -304,6 +304,42 @@ __device__ __forceinline__ void stage_prod(const Tile& t, const ChunkParams& p, 
   }
 }
 
+// Bytes of shared scratch drain_rows needs: 32 x 32 floats for each of 8 warps.
+constexpr uint32_t kDrainScratch = 8u * 32u * 32u * 4u;
+
+// Drain TMEM columns [col, col + n) (n a multiple of 32) of this warp's 32 rows
+// (TMEM lanes 32 (w % 4) ..; the two warpgroups take alternate 32-column chunks)
+// to the row-major fp32 matrix dst (row stride ld floats, rows 16-byte aligned).
+// A row-per-lane store would touch 32 lines per instruction; instead each chunk
+// goes through this warp's 4 KB of `scratch` (16-byte piece j of row r at piece
+// j ^ (r & 7), conflict-free both ways) and out as 4 rows x 128 bytes per
+// store. mask(row, c, v) may edit the 32 values first. Rows >= nrows, and all
+// rows when !on, are not stored. Every thread calls it.
+template <typename F>
+__device__ __forceinline__ void drain_rows(uint32_t tmem_lane_addr, uint32_t col, int n, float* dst, int64_t ld,
+                                           int nrows, float* scratch, bool on, F mask) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, wg = w >> 2;
+  const int row0 = (w & 3) * 32;
+  float* sc = scratch + w * 32 * 32;
+  for (int c = wg * 32; c < n; c += 64) {
+    float v[32];
+    tmem_ld32(tmem_lane_addr + col + c, v);
+    mask(row0 + lane, c, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(sc + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+          make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = (lane >> 3) + 4 * i, j = lane & 7;
+      const float4 a = *reinterpret_cast<const float4*>(sc + r * 32 + ((j ^ (r & 7)) << 2));
+      if (on && row0 + r < nrows) *reinterpret_cast<float4*>(dst + (int64_t)(row0 + r) * ld + c + 4 * j) = a;
+    }
+    __syncwarp();
+  }
+}
+
 // CTA prologue shared by the tensor-core kernels: TMEM allocation + mbarrier.
 struct TcCta {
   uint32_t tmem;

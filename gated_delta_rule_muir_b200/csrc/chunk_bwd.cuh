@@ -444,27 +444,17 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   auto stage_U = [&](const Tile& dst) {  // w * v
     stage_prod<T, false, DV>(dst, p, s, Cs, static_cast<const T*>(p.v), static_cast<const T*>(p.w), nullptr, 1.f);
   };
-  // Row t of a [Cs][N] TMEM result -> dst (fp32, row-major, row stride ld), optional mask.
+  // Rows of a [Cs][N] TMEM result -> dst (fp32, row-major, row stride ld), optional mask.
+  float* scratch = reinterpret_cast<float*>(sm + 6 * TB);
   auto drain = [&](uint32_t col, int n, float* dst, int64_t ld, int mask) {
-    for (int c = wg * 32; c < n; c += 64) {
-      float v[32];
-      tmem_ld32(cta.tmem + lane + col + c, v);
-      if (t < Cs && drv.ok) {
+    drain_rows(cta.tmem + lane + 0u, col, n, dst, ld, Cs, scratch, drv.ok, [&](int row, int c, float(&v)[32]) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int sidx = c + j;
-          if (mask == 1 && sidx >= t) v[j] = 0.f;  // strictly lower
-          if (mask == 2 && sidx > t) v[j] = 0.f;   // lower incl. diagonal
-        }
-#pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          float w8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w8[e] = v[j + e];
-          stg256(dst + t * ld + c + j, w8);  // whole 32-byte sectors
-        }
+      for (int j = 0; j < 32; ++j) {
+        const int sidx = c + j;
+        if (mask == 1 && sidx >= row) v[j] = 0.f;  // strictly lower
+        if (mask == 2 && sidx > row) v[j] = 0.f;   // lower incl. diagonal
       }
-    }
+    });
   };
   const uint32_t idK = idesc_bf16(128, DK, 0, 0), idC = idesc_bf16(128, Cs, 0, 0);
   float* g4 = q.g4 + u * 4 * Cs * DK;
