@@ -80,7 +80,7 @@ def kernel_model(C, dk, dv, es):
 # DRAM bytes (read + write) per unit of the dominant kernel, from the ncu capture summarised in
 # profiles/gram_and_bwd_gram_B1_T16384_H16_d128_C128.md (2,048 units; traffic scales with units).
 # Only valid for the kernel version that capture measured: clear an entry when its kernel changes.
-NCU_TRAFFIC_PER_UNIT = {}  # gram, bwd_gram: changed since the last capture
+NCU_TRAFFIC_PER_UNIT = {"bwd_gram": 1649.1e6 / 2048, "gram": 1139.2e6 / 2048}
 
 
 def flop_split(C, dk, dv):
