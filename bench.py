@@ -235,6 +235,39 @@ def time_steps(fn, steps, dist_on):
     return ms
 
 
+GATE_WL = {"N": 32768, "D": 2048, "Ok": 2048, "Ov": 2048}  # tokens of the fwd+bwd workload, d_model = H*d
+
+
+def bench_gate_proj(dev, steps, warmup, pk):
+    """The fused gate projection (muir_gate_proj) over the fwd+bwd workload's tokens:
+    x [32768, 2048] bf16 -> log_alpha (fp32), e, z, w, g (bf16). Inputs and outputs
+    exceed L2. Algorithmic work: 2N(512 D + 64 Ok + 64 Ok + 128 Ov + 128 Ov + 128 Ok)
+    flops; bytes = x + weights + outputs."""
+    import torch
+    import gated_delta_rule_muir_b200 as muir
+    N, D, Ok, Ov = GATE_WL["N"], GATE_WL["D"], GATE_WL["Ok"], GATE_WL["Ov"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    x = torch.randn(N, D, device=dev, generator=g).bfloat16()
+    wd = (torch.randn(D, 512, device=dev, generator=g) / D ** 0.5).bfloat16()
+    ups = [(torch.randn(r, o, device=dev, generator=g) / r ** 0.5).bfloat16()
+           for r, o in zip(muir.GATE_RANKS, (Ok, Ok, Ov, Ov, Ok))]
+    out = muir.gate_proj(x, wd, *ups)
+    fn = lambda: muir.gate_proj(x, wd, *ups, out=out)
+    for _ in range(max(warmup, 3)):
+        fn()
+    reps = max(steps, 10)
+    ms = time_steps(fn, reps, False) / reps
+    flops = 2.0 * N * (512 * D + 64 * Ok * 2 + 128 * Ov * 2 + 128 * Ok)
+    byts = 2.0 * (N * D + D * 512 + sum(u.numel() for u in ups)) + N * Ok * 4 + 2.0 * N * (Ok + 2 * Ov + Ok)
+    t = ms * 1e-3
+    roof_ms = 1e3 * max(flops / (pk["bf16"] * 1e12), byts / (pk["hbm"] * 1e9))
+    return {"workload": f"gate_proj_bf16_N{N}_D{D}_Ok{Ok}_Ov{Ov}", "ms": round(ms, 4), "tokens_s": round(N / t, 1),
+            "algorithmic_TFLOP_s": round(flops / t / 1e12, 2), "frac_tc_peak": round(flops / t / 1e12 / pk["bf16"], 4),
+            "algorithmic_GB_s": round(byts / t / 1e9, 1), "frac_hbm": round(byts / t / 1e9 / pk["hbm"], 4),
+            "roofline_ms": round(roof_ms, 4), "frac_roofline": round(roof_ms / ms, 4), "gpu_launches": reps}
+
+
 def bench_decode(dev, steps, warmup, pk):
     """Decode GB/s of one token through all 24 layers: one launch over the 24 x batch
     rows (per-row readout scale), and a CUDA graph of 24 per-layer launches."""
@@ -418,6 +451,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true", help="only the timed step (for profiling)")
     ap.add_argument("--T", type=int, default=None, help="override the sequence length (profiling runs)")
     ap.add_argument("--fwd-only", action="store_true", help="time the forward pass only (profiling runs)")
+    ap.add_argument("--gate-only", action="store_true", help="only the gate projection's measurement (profiling runs)")
     args = ap.parse_args()
     if args.T:
         WL["T"] = args.T
@@ -441,6 +475,10 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     pk = peaks()
+    if args.gate_only:
+        if rank == 0:
+            print(json.dumps(bench_gate_proj(dev, args.steps, args.warmup, pk)))
+        return
     Step.fwd_only = args.fwd_only
     d = make_workload(dev)
     step = Step(d)
@@ -503,6 +541,7 @@ def main():
                              "roofline_ms": round(1e3 * max(sfl / (pk["bf16_sus"] * 1e12), sby / (pk["hbm"] * 1e9)), 3)}
     if not args.skip_extras and rank == 0:
         line["decode"] = bench_decode(dev, args.steps, args.warmup, pk)
+        line["gate_proj"] = bench_gate_proj(dev, args.steps, args.warmup, pk)
         line["e2e"] = e2e_pass(d, max(2, min(args.steps, 5)), 1)
         if world == 1:
             line["cpu_baseline"] = cpu_baseline()

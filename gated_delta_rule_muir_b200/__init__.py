@@ -14,7 +14,7 @@ import torch
 from . import _native as N
 
 __all__ = ["chunk_fwd", "chunk_bwd", "decode_step", "state_init", "device_status", "chunk_fwd_workspace_bytes",
-           "chunk_bwd_workspace_bytes", "MuirError", "KernelTimer", "launch_count"]
+           "chunk_bwd_workspace_bytes", "MuirError", "KernelTimer", "launch_count", "gate_proj", "GATE_RANKS"]
 
 MuirError = N.MuirError
 
@@ -227,6 +227,37 @@ def row_scale(S, *, exponent=0.5, eps=1e-12, r=None, stream=None):
     N.check(lib.muir_row_scale(_ptr(S), n, H, dk, dv, float(exponent), float(eps), _ptr(r), _stream(stream)),
             "muir_row_scale")
     return r
+
+
+GATE_RANKS = (64, 64, 128, 128, 128)  # decay, erase, output, write, read (total rank 512)
+
+
+def gate_proj(x, w_down, u_decay, u_erase, u_out, u_write, u_read, *, out=None, stream=None):
+    """Fused low-rank gate projection (muir_gate_proj): x [N, D] and weights of x's
+    dtype (w_down [D, 512], u_decay / u_erase [64, Ok], u_out / u_write [128, Ov],
+    u_read [128, Ok]) -> dict of log_alpha [N, Ok] fp32 and e, z, w, g in x's dtype
+    (e, g [N, Ok]; z, w [N, Ov]). `out` may hold preallocated outputs."""
+    lib = N.load()
+    n, D = x.shape
+    Ok, Ov = u_decay.shape[1], u_out.shape[1]
+    dt = x.dtype
+    _need(x, "x", (n, D), dt)
+    _need(w_down, "w_down", (D, 512), dt)
+    for name, t, shape in (("u_decay", u_decay, (64, Ok)), ("u_erase", u_erase, (64, Ok)),
+                           ("u_out", u_out, (128, Ov)), ("u_write", u_write, (128, Ov)),
+                           ("u_read", u_read, (128, Ok))):
+        _need(t, name, shape, dt)
+    out = dict(out or {})
+    shapes = {"log_alpha": ((n, Ok), torch.float32), "e": ((n, Ok), dt), "z": ((n, Ov), dt),
+              "w": ((n, Ov), dt), "g": ((n, Ok), dt)}
+    for name, (shape, odt) in shapes.items():
+        if name not in out:
+            out[name] = torch.empty(shape, dtype=odt, device=x.device)
+        _need(out[name], name, shape, odt)
+    N.check(lib.muir_gate_proj(_ptr(x), _ptr(w_down), _ptr(u_decay), _ptr(u_erase), _ptr(u_out), _ptr(u_write),
+                               _ptr(u_read), _ptr(out["log_alpha"]), _ptr(out["e"]), _ptr(out["z"]), _ptr(out["w"]),
+                               _ptr(out["g"]), n, D, Ok, Ov, _dtype_code(dt), _stream(stream)), "muir_gate_proj")
+    return out
 
 
 def launch_count() -> int:

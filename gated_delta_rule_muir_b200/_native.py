@@ -48,6 +48,8 @@ SIGNATURES = {
     "muir_chunk_segment_map_workspace": (C.c_size_t, [C.POINTER(ChunkArgs)]),
     "muir_chunk_segment_map": (C.c_int, [C.POINTER(ChunkArgs), vp, vp, vp, C.c_size_t, vp]),
     "muir_apply_map": (C.c_int, [vp, vp, vp, vp, C.c_int64, C.c_int32, C.c_int32, C.c_int32, vp]),
+    "muir_gate_proj": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, C.c_int64, C.c_int32, C.c_int32,
+                                 C.c_int32, C.c_int32, vp]),
     "muir_device_status": (C.c_int, [vp]),
     "muir_last_error": (C.c_char_p, []),
     "muir_version": (C.c_int, []),

@@ -15,6 +15,7 @@
 #include "selftest.cuh"
 #include "chunk.cuh"
 #include "chunk_bwd.cuh"
+#include "gate_proj.cuh"
 
 namespace {
 
@@ -89,7 +90,7 @@ bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 
 extern "C" {
 
-int muir_version(void) { return 101; }
+int muir_version(void) { return 102; }
 
 const char* muir_last_error(void) { return g_err.c_str(); }
 
@@ -256,6 +257,7 @@ int64_t muir_launch_count(void) { return g_prof.launches; }
 }  // extern "C"
 
 #include "api_chunk.inc"
+#include "api_gate.inc"
 
 // ---------------------------------------------------------------------------
 // Allocation-free chunkwise forward.

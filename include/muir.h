@@ -222,6 +222,31 @@ int muir_state_init(float* S, const float* S_src, int64_t n_seq, int32_t H, int3
 int muir_row_scale(const float* S, int64_t n_seq, int32_t H, int32_t dk, int32_t dv, float exponent, float eps, float* r,
                    void* stream);
 
+/* Fused low-rank gate projection (openai-hub article, section "五套门控被压进一个
+ * 低秩投影" and its table; liuch.name post, second bullet): the five gate
+ * tensors of the operator from the layer input x with one shared down-projection
+ * of total rank 512, sliced 64 / 64 / 128 / 128 / 128 for the decay, erase,
+ * output, write and dynamic-read gates, each slice with its own up-projection:
+ *     h = x W_down,   u_j = h[:, slice_j] U_j
+ *     log_alpha = log sigmoid(u_decay)   e = sigmoid(u_erase)   z = sigmoid(u_out)
+ *     w = sigmoid(u_write)               g = sigmoid(u_read)
+ * Arguments (device pointers, row-major, every pointer 16-byte aligned; the
+ * element type of every array but log_alpha is `dtype`, log_alpha is float):
+ *     x        [n_tokens][d_model]          w_down  [d_model][512]
+ *     u_decay, u_erase [64][ok]             u_out, u_write [128][ov]
+ *     u_read   [128][ok]
+ *     log_alpha, e, g  [n_tokens][ok]  (out)   z, w  [n_tokens][ov]  (out)
+ * ok = H*d_k and ov = H*d_v, so the outputs are in the operator's [B,T,H,d]
+ * layout with the tokens flattened. d_model must be a multiple of 64, ok and ov
+ * multiples of 256 (else MUIR_ERR_UNSUPPORTED). n_tokens may be 0 (no launch;
+ * the pointers are not read and may be NULL) or any size (a ragged last tile is
+ * masked). Otherwise a NULL or misaligned pointer gives MUIR_ERR_INVALID_ARG. h is accumulated in fp32 and kept
+ * at fp32 accuracy into the up-projections; the activations are evaluated in
+ * fp32. Enqueued on `stream`; the caller owns every buffer. */
+int muir_gate_proj(const void* x, const void* w_down, const void* u_decay, const void* u_erase, const void* u_out,
+                   const void* u_write, const void* u_read, float* log_alpha, void* e, void* z, void* w, void* g,
+                   int64_t n_tokens, int32_t d_model, int32_t ok, int32_t ov, int32_t dtype, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device-side status word:
  * MUIR_OK, or MUIR_ERR_TIMEOUT if a kernel's bounded wait expired since the
  * last call (that kernel's outputs are then invalid), or MUIR_ERR_CUDA. */

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version(lib):
-    assert lib.muir_version() == 101
+    assert lib.muir_version() == 102
 
 
 def test_decode_rejects_null_and_bad_sizes(lib):
@@ -152,3 +152,23 @@ def test_row_scale_rejects_bad_args(lib):
     assert lib.muir_row_scale(None, 1, 1, 32, 32, 0.5, 0.0, fake, None) == N.MUIR_ERR_INVALID_ARG
     assert lib.muir_row_scale(fake, 1, 1, 48, 32, 0.5, 0.0, fake, None) == N.MUIR_ERR_UNSUPPORTED
     assert lib.muir_row_scale(fake, 1, 1, 32, 32, -1.0, 0.0, fake, None) == N.MUIR_ERR_INVALID_ARG
+
+
+def test_gate_proj_validates_before_launching(lib):
+    """Every rejection (and the empty batch) returns before any CUDA call."""
+    fake = C.c_void_p(1 << 20)
+    ptrs = [fake] * 12
+
+    def call(p=ptrs, n=256, d=2048, ok=2048, ov=2048, dtype=N.MUIR_BF16):
+        return lib.muir_gate_proj(*p, n, d, ok, ov, dtype, None)
+
+    assert call(p=[None] + ptrs[1:]) == N.MUIR_ERR_INVALID_ARG
+    assert call(p=ptrs[:7] + [None] + ptrs[8:]) == N.MUIR_ERR_INVALID_ARG  # log_alpha
+    assert call(p=ptrs[:3] + [C.c_void_p((1 << 20) + 8)] + ptrs[4:]) == N.MUIR_ERR_INVALID_ARG  # misaligned
+    assert call(dtype=7) == N.MUIR_ERR_INVALID_ARG
+    assert call(n=-1) == N.MUIR_ERR_INVALID_ARG
+    assert call(d=96) == N.MUIR_ERR_UNSUPPORTED
+    assert call(ok=384) == N.MUIR_ERR_UNSUPPORTED
+    assert call(ov=0) == N.MUIR_ERR_UNSUPPORTED
+    assert call(n=0) == N.MUIR_OK
+    assert call(p=[None] * 12, n=0) == N.MUIR_OK  # an empty batch reads no pointer
