@@ -99,6 +99,8 @@ __global__ void __launch_bounds__(256, 1) gate_proj_kernel(GateParams p) {
   const uint32_t lane = tmem_lane_base(warp);
   const int t = tid & 127, wg = tid >> 7;  // TMEM row (token); warpgroups take alternate 16-column chunks
   const bool on = row0 + t < p.n;
+  constexpr int UP = 128 * (256 / 8) / NT;  // U pieces per thread at most (r = 128, nch = 256)
+  Pack8<T> pu[UP];
   for (int j = 0; j < 5 && drv.ok; ++j) {
     const int r = gate_rank(j), off = gate_off(j);
     const int O = (j == 2 || j == 3) ? p.ov : p.ok;
@@ -113,17 +115,38 @@ __global__ void __launch_bounds__(256, 1) gate_proj_kernel(GateParams p) {
       put_k(Ah, t, c, a8);
       put_k(Ah, t, c + 8, b8);
     }
+    // U_j chunk n0: all of a thread's loads go out at once (into pu), the next
+    // chunk's while the current chunk's MMA runs
     const T* U = static_cast<const T*>(p.up[j]);
-    for (int n0 = 0; n0 < O && drv.ok; n0 += nch) {
-#pragma unroll 4
-      for (int x = tid; x < r * (nch / 8); x += NT) {
-        int k, n8;
-        piece_of_rt(x, nch / 8, k, n8);
-        float v[8];
-        Elt<T>::ld8(U + (int64_t)k * O + n0 + n8, v);
-        put_mn(Ub, k, n8, v);
+    const int np = r * (nch / 8);
+    auto load_u = [&](int n0) {
+#pragma unroll
+      for (int m = 0; m < UP; ++m) {
+        const int x = tid + m * NT;
+        if (x < np) {
+          int k, n8;
+          piece_of_rt(x, nch / 8, k, n8);
+          pu[m].ld(U + (int64_t)k * O + n0 + n8);
+        }
       }
-      drv.run([&] { mma_tiles(cta.tmem, Ah, Ub, r / 16, idesc_bf16(128, nch, 0, 1), 3, false); });
+    };
+    load_u(0);
+    for (int n0 = 0; n0 < O && drv.ok; n0 += nch) {
+#pragma unroll
+      for (int m = 0; m < UP; ++m) {
+        const int x = tid + m * NT;
+        if (x < np) {
+          int k, n8;
+          piece_of_rt(x, nch / 8, k, n8);
+          float v[8];
+          pu[m].get(v);
+          put_mn(Ub, k, n8, v);
+        }
+      }
+      drv.run_overlap([&] { mma_tiles(cta.tmem, Ah, Ub, r / 16, idesc_bf16(128, nch, 0, 1), 3, false); },
+                      [&] {
+                        if (n0 + nch < O) load_u(n0 + nch);
+                      });
       for (int c = wg * 16; c < nch; c += 32) {
         float v[16];
         tmem_ld16(cta.tmem + lane + c, v);
