@@ -64,33 +64,57 @@ __global__ void __launch_bounds__(256, 1) gate_proj_kernel(GateParams p) {
   const Tile Wt{base + 32768u, base + 32768u + 65536u, 128u, KC * 16u};  // 64 (K) x 512 (N), MN-major
   const T* xp = static_cast<const T*>(p.x);
   const T* wd = static_cast<const T*>(p.wd);
-  for (int k0 = 0; k0 < p.d && drv.ok; k0 += KC) {
-    for (int x = tid; x < 128 * (KC / 8); x += NT) {
+  // A K step's loads go out at once (into px, pw); the next step's while the
+  // current step's MMAs run.
+  constexpr int XP = 128 * (KC / 8) / NT, WP = KC * (512 / 8) / NT;  // pieces per thread
+  Pack8<T> px[XP], pw[WP];
+  auto load_xw = [&](int k0) {
+#pragma unroll
+    for (int m = 0; m < XP; ++m) {
       int r, c8;
-      piece_of<KC / 8>(x, r, c8);
+      piece_of<KC / 8>(tid + m * NT, r, c8);
+      if (row0 + r < p.n) px[m].ld(xp + (row0 + r) * p.d + k0 + c8);
+    }
+#pragma unroll
+    for (int m = 0; m < WP; ++m) {
+      int k, n8;
+      piece_of<512 / 8>(tid + m * NT, k, n8);
+      pw[m].ld(wd + (int64_t)(k0 + k) * 512 + n8);
+    }
+  };
+  load_xw(0);
+  for (int k0 = 0; k0 < p.d && drv.ok; k0 += KC) {
+#pragma unroll
+    for (int m = 0; m < XP; ++m) {
+      int r, c8;
+      piece_of<KC / 8>(tid + m * NT, r, c8);
       float v[8];
       if (row0 + r < p.n) {
-        Elt<T>::ld8(xp + (row0 + r) * p.d + k0 + c8, v);
-      } else {
+        px[m].get(v);
+      } else {  // rows past the last token
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] = 0.f;
       }
       put_k(X, r, c8, v);
     }
-#pragma unroll 4
-    for (int x = tid; x < KC * (512 / 8); x += NT) {
+#pragma unroll
+    for (int m = 0; m < WP; ++m) {
       int k, n8;
-      piece_of<512 / 8>(x, k, n8);
+      piece_of<512 / 8>(tid + m * NT, k, n8);
       float v[8];
-      Elt<T>::ld8(wd + (int64_t)(k0 + k) * 512 + n8, v);
+      pw[m].get(v);
       put_mn(Wt, k, n8, v);
     }
-    drv.run([&] {
-      const uint32_t id = idesc_bf16(128, 256, 0, 1);
-      mma_tiles(cta.tmem + 0, X, Wt, KC / 16, id, NS1, k0 > 0);
-      const Tile W2{Wt.hi + 32u * Wt.sbo, Wt.lo + 32u * Wt.sbo, Wt.lbo, Wt.sbo};  // columns 256..511
-      mma_tiles(cta.tmem + 256, X, W2, KC / 16, id, NS1, k0 > 0);
-    });
+    drv.run_overlap(
+        [&] {
+          const uint32_t id = idesc_bf16(128, 256, 0, 1);
+          mma_tiles(cta.tmem + 0, X, Wt, KC / 16, id, NS1, k0 > 0);
+          const Tile W2{Wt.hi + 32u * Wt.sbo, Wt.lo + 32u * Wt.sbo, Wt.lbo, Wt.sbo};  // columns 256..511
+          mma_tiles(cta.tmem + 256, X, W2, KC / 16, id, NS1, k0 > 0);
+        },
+        [&] {
+          if (k0 + KC < p.d) load_xw(k0 + KC);
+        });
   }
 
   // ---- gate by gate: u_j = h_j U_j, activated
