@@ -42,9 +42,14 @@ __host__ __device__ constexpr int gate_rank(int j) { return j < 2 ? 64 : 128; }
 __host__ __device__ constexpr int gate_off(int j) { return j == 0 ? 0 : j == 1 ? 64 : 128 * (j - 1); }
 constexpr uint32_t kGateSmem = 192u * 1024u;
 
-__device__ __forceinline__ float gate_sigmoid(float u) { return 1.f / (1.f + expf(-u)); }
-// log(sigmoid(u)) = min(u, 0) - log(1 + exp(-|u|)), finite for every finite u
-__device__ __forceinline__ float gate_log_sigmoid(float u) { return fminf(u, 0.f) - log1pf(expf(-fabsf(u))); }
+// The fast exponential and division intrinsics (a few ulp): the epilogue applies
+// one activation per output element, which dominates the kernel's instruction
+// count with the correctly rounded forms. For u << 0 the denominator overflows
+// to +inf and the quotient is 0.
+__device__ __forceinline__ float gate_sigmoid(float u) { return __fdividef(1.f, 1.f + __expf(-u)); }
+// log(sigmoid(u)) = min(u, 0) - log(1 + exp(-|u|)), finite for every finite u;
+// log1pf keeps its accuracy near 0 (slow-decay rows)
+__device__ __forceinline__ float gate_log_sigmoid(float u) { return fminf(u, 0.f) - log1pf(__expf(-fabsf(u))); }
 
 template <typename T, int NS1>
 __global__ void __launch_bounds__(256, 1) gate_proj_kernel(GateParams p) {
