@@ -149,23 +149,9 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
   cta.finish();
 }
 
-// Stage a row-major fp32 matrix src[rows][cols] (row stride ld) as a K-major
-// operand contracting over cols (put_k), values scaled by sign. rows <= 128 and a
-// multiple of 8, cols / 8 a power of two.
-__device__ __forceinline__ void stage_rows_k(const Tile& t, const float* src, int rows, int cols, int64_t ld,
-                                             float sign) {
-  #pragma unroll 4
-  for (int x = threadIdx.x; x < rows * (cols / 8); x += blockDim.x) {
-    int r, c8;
-    piece_of_rt(x, cols / 8, r, c8);
-    float v[8];
-    ld8f(src + r * ld + c8, v);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] *= sign;
-    put_k(t, r, c8, v);
-  }
-}
-// Same matrix as an MN-major operand contracting over rows (put_mn).
+// Stage a row-major fp32 matrix src[rows][cols] (row stride ld) as an MN-major
+// operand contracting over rows (put_mn), values scaled by sign. rows <= 128 and
+// a multiple of 8, cols / 8 a power of two.
 __device__ __forceinline__ void stage_rows_mn(const Tile& t, const float* src, int rows, int cols, int64_t ld,
                                               float sign) {
   #pragma unroll 4
