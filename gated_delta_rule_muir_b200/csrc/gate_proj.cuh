@@ -15,11 +15,12 @@
 // One CTA of 256 threads per 128-token tile. h stays on chip: its 128 x 512
 // fp32 tile fills TMEM. The down-projection runs over D in 64-wide K steps (x
 // tile K-major, W_down tile MN-major, two N = 256 MMAs per step; one bf16 pass
-// for bf16 inputs, whose products are exact, three hi/lo passes for fp32). Then
-// gate by gate the rank slice of h is drained to shared memory as a bf16 hi/lo
-// K-major operand and multiplied by column chunks of U_j (3 passes, so h keeps
-// fp32 accuracy) into TMEM columns whose slices have already been drained; the
-// activation is applied on the way out.
+// for bf16 inputs, whose products are exact and whose packed values are stored
+// as they are, three hi/lo passes for fp32). Then gate by gate the rank slice of
+// h is drained to shared memory as a bf16 hi/lo K-major operand and multiplied
+// by column chunks of U_j (h's hi and lo parts, so h keeps fp32 accuracy: 2
+// passes against an exact bf16 U, 3 against fp32) into TMEM columns whose
+// slices have already been drained; the activation is applied on the way out.
 #pragma once
 
 #include "chunk.cuh"
@@ -93,22 +94,30 @@ __global__ void __launch_bounds__(256, 1) gate_proj_kernel(GateParams p) {
     for (int m = 0; m < XP; ++m) {
       int r, c8;
       piece_of<KC / 8>(tid + m * NT, r, c8);
-      float v[8];
-      if (row0 + r < p.n) {
-        px[m].get(v);
-      } else {  // rows past the last token
+      if constexpr (sizeof(T) == 2) {  // exact in bf16: the packed values are the hi plane
+        put_k_raw(X, r, c8, row0 + r < p.n ? px[m].u : make_uint4(0, 0, 0, 0));
+      } else {
+        float v[8];
+        if (row0 + r < p.n) {
+          px[m].get(v);
+        } else {  // rows past the last token
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = 0.f;
+          for (int j = 0; j < 8; ++j) v[j] = 0.f;
+        }
+        put_k(X, r, c8, v);
       }
-      put_k(X, r, c8, v);
     }
 #pragma unroll
     for (int m = 0; m < WP; ++m) {
       int k, n8;
       piece_of<512 / 8>(tid + m * NT, k, n8);
-      float v[8];
-      pw[m].get(v);
-      put_mn(Wt, k, n8, v);
+      if constexpr (sizeof(T) == 2) {
+        put_mn_raw(Wt, k, n8, pw[m].u);
+      } else {
+        float v[8];
+        pw[m].get(v);
+        put_mn(Wt, k, n8, v);
+      }
     }
     drv.run_overlap(
         [&] {
@@ -129,6 +138,7 @@ __global__ void __launch_bounds__(256, 1) gate_proj_kernel(GateParams p) {
   const int t = tid & 127, wg = tid >> 7;  // TMEM row (token); warpgroups take alternate 16-column chunks
   const bool on = row0 + t < p.n;
   constexpr int UP = 128 * (256 / 8) / NT;  // U pieces per thread at most (r = 128, nch = 256)
+  constexpr int kUpPasses = sizeof(T) == 2 ? 2 : 3;
   Pack8<T> pu[UP];
   for (int j = 0; j < 5 && drv.ok; ++j) {
     const int r = gate_rank(j), off = gate_off(j);
@@ -167,12 +177,17 @@ __global__ void __launch_bounds__(256, 1) gate_proj_kernel(GateParams p) {
         if (x < np) {
           int k, n8;
           piece_of_rt(x, nch / 8, k, n8);
-          float v[8];
-          pu[m].get(v);
-          put_mn(Ub, k, n8, v);
+          if constexpr (sizeof(T) == 2) {
+            put_mn_raw(Ub, k, n8, pu[m].u);
+          } else {
+            float v[8];
+            pu[m].get(v);
+            put_mn(Ub, k, n8, v);
+          }
         }
       }
-      drv.run_overlap([&] { mma_tiles(cta.tmem, Ah, Ub, r / 16, idesc_bf16(128, nch, 0, 1), 3, false); },
+      // bf16 U is exact: h's hi and lo parts times U's hi plane (2 passes); fp32 U: 3 passes
+      drv.run_overlap([&] { mma_tiles(cta.tmem, Ah, Ub, r / 16, idesc_bf16(128, nch, 0, 1), kUpPasses, false); },
                       [&] {
                         if (n0 + nch < O) load_u(n0 + nch);
                       });

@@ -163,7 +163,8 @@ struct Tile {
 __device__ __forceinline__ Tile transposed(const Tile& t) { return Tile{t.hi, t.lo, t.sbo, t.lbo}; }
 
 // D[tmem] (+)= A * B for one tile pair covering `ksteps` MMA steps of K = 16.
-// M = 128 rows of A (lanes of D), N columns of B. nsplit = 1 (hi*hi) or 3.
+// M = 128 rows of A (lanes of D), N columns of B. nsplit = 1 (hi*hi), 3
+// (hi*hi + hi*lo + lo*hi), or 2 (hi*hi + A.lo*B.hi, for a B exact in bf16).
 __device__ __forceinline__ void mma_tiles(uint32_t d_tmem, const Tile& A, const Tile& B, int ksteps, uint32_t idesc,
                                           int nsplit, bool accumulate) {
   for (int j = 0; j < ksteps; ++j) {
@@ -174,6 +175,8 @@ __device__ __forceinline__ void mma_tiles(uint32_t d_tmem, const Tile& A, const 
       const uint64_t al = sdesc(A.lo + oa, A.lbo, A.sbo), bl = sdesc(B.lo + ob, B.lbo, B.sbo);
       mma_bf16(d_tmem, ah, bl, idesc, 1u);
       mma_bf16(d_tmem, al, bh, idesc, 1u);
+    } else if (nsplit == 2) {
+      mma_bf16(d_tmem, sdesc(A.lo + oa, A.lbo, A.sbo), bh, idesc, 1u);
     }
   }
 }
@@ -253,6 +256,16 @@ __device__ __forceinline__ void piece_of_rot(int x, int G, int& r, int& c8) {
   const int lg = 31 - __clz(G);
   r = ((x >> (3 + lg)) << 3) | (x & 7);
   c8 = (((x >> 3) + (x & 7)) & (G - 1)) << 3;
+}
+
+// 8 values that are exact in bf16, already packed (uint4 of 8 bf16): the hi
+// plane only (their lo part is zero and is never read: 1-pass, or 2-pass with
+// this tile as the exact B operand). K-major and MN-major offsets as put_k / put_mn.
+__device__ __forceinline__ void put_k_raw(const Tile& t, int m, int k8, const uint4& v) {
+  sts128(t.hi + (uint32_t)(m >> 3) * t.sbo + (uint32_t)(k8 >> 3) * 128u + (uint32_t)(m & 7) * 16u, v);
+}
+__device__ __forceinline__ void put_mn_raw(const Tile& t, int k, int m8, const uint4& v) {
+  sts128(t.hi + (uint32_t)(m8 >> 3) * t.sbo + (uint32_t)(k >> 3) * 128u + (uint32_t)(k & 7) * 16u, v);
 }
 
 // MN-major (natural view, lbo = 128): 8 consecutive MN indices m8..m8+7 of contraction row k.
