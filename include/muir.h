@@ -98,6 +98,17 @@ typedef struct muir_chunk_args {
  *   ws  workspace of at least muir_chunk_fwd_workspace(a) bytes, 256-byte
  *       aligned; contents on entry are ignored.
  */
+/*
+ * muir_chunk_fwd_workspace: bytes of device scratch that muir_chunk_fwd needs
+ * for these arguments (openai-hub article, section "为 TPU 重写长序列并行算法":
+ * the chunkwise algorithm keeps per-chunk intermediates, which the pages' XLA
+ * version wrote to HBM; here they are the per-unit decay products, Gram and T
+ * images, chunk maps and chunk-start states). Only the sizes, chunk, dtype and
+ * flags of *a are read; with MUIR_SAVE_FOR_BWD it returns the size that also
+ * holds what the backward pass reuses. Returns 0 when the arguments are
+ * invalid (muir_last_error() says why) and for empty problems (B = 0 or T = 0),
+ * which need no workspace. The caller allocates and owns the workspace.
+ */
 size_t muir_chunk_fwd_workspace(const muir_chunk_args* a);
 int muir_chunk_fwd(const muir_chunk_args* a, void* y, float* S_T, void* ws, size_t ws_bytes,
                    void* stream);
@@ -140,6 +151,15 @@ typedef struct muir_chunk_grads {
  *       MUIR_USE_SAVED in a->flags, the workspace a forward pass with
  *       MUIR_SAVE_FOR_BWD filled (see above).
  */
+/*
+ * muir_chunk_bwd_workspace: bytes of device scratch muir_chunk_bwd needs (the
+ * same section of the openai-hub article: the backward pass recomputes the
+ * per-chunk states and keeps the cotangents of the chunk quantities between
+ * its kernels). Only the sizes, chunk and dtype of *a are read. Returns 0 when
+ * the arguments are invalid and for empty problems. The caller allocates and
+ * owns the workspace; it equals muir_chunk_fwd_workspace() of the same
+ * arguments with MUIR_SAVE_FOR_BWD.
+ */
 size_t muir_chunk_bwd_workspace(const muir_chunk_args* a);
 int muir_chunk_bwd(const muir_chunk_args* a, const muir_chunk_grads* gr, void* ws, size_t ws_bytes,
                    void* stream);
@@ -160,6 +180,9 @@ int muir_chunk_bwd(const muir_chunk_args* a, const muir_chunk_grads* gr, void* w
  *   - The first call on a device looks up the scratch address with
  *     cudaGetSymbolAddress (once per device, with that device current); make
  *     that first call before any stream capture on the device.
+ *   - The scratch address is cached per device for the life of the process:
+ *     do not keep using the library on a device after cudaDeviceReset (or any
+ *     other teardown of its primary context), which may move the area.
  *   - All calls on a device share the one scratch area and it keeps the last
  *     call's contents; the kernels write every scratch byte they read within
  *     the same call, so nothing needs clearing. Calls that overlap on the GPU
@@ -207,7 +230,15 @@ typedef struct muir_decode_args {
 /* Reads and writes each state element exactly once (memory-bound). */
 int muir_decode_step(const muir_decode_args* a, void* stream);
 
-/* S [n_seq,H,dk,dv] := S_src, or zeros when S_src is NULL. In-place safe. */
+/* Set up the recurrent state (openai-hub article, section "1000 万 Token，KV
+ * Cache 已经装不下了": the model carries a fixed-size fp32 state per head, about
+ * 25 MB over 24 layers of 16 heads of 128 x 128, in place of a KV cache):
+ * S [n_seq,H,dk,dv] fp32 := S_src, or zeros when S_src is NULL. Both are device
+ * pointers owned by the caller, 16-byte aligned; S == S_src is allowed (a no-op
+ * copy), other overlaps are not. dk, dv in {32, 64, 128}. n_seq = 0 launches
+ * nothing. Returns MUIR_ERR_INVALID_ARG for a NULL S or a misaligned pointer,
+ * MUIR_ERR_UNSUPPORTED for n_seq < 0, H <= 0 or dk, dv outside {32, 64, 128},
+ * and MUIR_ERR_CUDA if the launch fails. */
 int muir_state_init(float* S, const float* S_src, int64_t n_seq, int32_t H, int32_t dk, int32_t dv,
                     void* stream);
 

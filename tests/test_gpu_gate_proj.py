@@ -50,6 +50,9 @@ def _check(got, ref, dtype):
 
 @pytest.mark.parametrize("dtype,N,D,Ok,Ov", [
     (torch.float32, 300, 128, 256, 256),
+    # fp32 with several K steps and several U chunks per gate (the prefetch of
+    # the next chunk and the reuse of the staged h), and a ragged last tile
+    (torch.float32, 389, 256, 512, 768),
     (torch.bfloat16, 333, 256, 512, 256),
     (torch.bfloat16, 5, 64, 256, 512),
 ])
