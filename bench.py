@@ -77,32 +77,54 @@ def kernel_model(C, dk, dv, es):
     return m
 
 
-# DRAM bytes (read + write) per unit of the dominant kernel, from the ncu capture summarised in
-# profiles/gram_and_bwd_gram_B1_T16384_H16_d128_C128.md (2,048 units; traffic scales with units).
-# Only valid for the kernel version that capture measured: clear an entry when its kernel changes.
-NCU_TRAFFIC_PER_UNIT = {"bwd_gram": 1649.1e6 / 2048, "gram": 1139.2e6 / 2048}
-
-
 def flop_split(C, dk, dv):
-    """Share of the step's modelled flops issued on the tensor cores; the rest (the
-    exact 16x16 diagonal Gram blocks, forward and backward) runs on the CUDA cores."""
+    """Modelled share of the step's flops issued on the tensor cores. The CUDA-core
+    share counts every vector step of the kernels per unit (one chunk of one head):
+    the exact 16x16 diagonal Gram blocks (forward and backward), the 16x16 leaves of
+    the triangular solve, the decay products, the elementwise decay scaling of the
+    staged operands and epilogues, the state additions of the scans, the output
+    gate, and the chain rule of the final backward kernel (an exponential counts as
+    one flop). The tensor-core share is the algorithmic MMA work of the model (each
+    multiply-add 2 flops, math counted once). The instruction counts behind the
+    measured split are in the ncu summary of the step's kernels."""
     m = kernel_model(C, dk, dv, 2)
-    alu = 4 * 2 * C * 8.5 * dk + 4 * 2 * 2 * C * 8.5 * dk
-    fwd = ("decay", "gram", "solve", "maps", "scan", "out")
-    bwd = ("bwd_pe", "rscan", "bwd_dz", "bwd_grads", "bwd_gram", "bwd_final")
-    total = sum(m[k][0] for k in fwd + bwd if k in m)
-    return {"mma_share": round(1.0 - alu / total, 4), "alu_share": round(alu / total, 4),
-            "note": "per unit of the step's kernels as modelled; the pages report 98% on matrix units"}
+    nb = C // 16
+    alu = {
+        "diag_blocks": 4 * 2 * C * 8.5 * dk + 4 * 2 * 2 * C * 8.5 * dk,
+        "solve_leaves": nb * 16 * (16 * 15 / 2) * 2,
+        "decay": 4 * C * dk,
+        "operand_scaling": (12 + 8 + 3) * C * dk + 2.5 * (12 + 8 + 3) * C * dk,
+        "scan_adds": 2 * dk * dv,
+        "output_gate": 2 * C * dv,
+        "final_chain_rule": 35 * C * dk + 4 * C * dv,
+    }
+    fwd = ("gram", "solve", "maps", "scan", "out")
+    bwd = ("bwd_pe", "rscan", "bwd_dz", "bwd_grads", "bwd_gram")
+    mma = sum(m[k][0] for k in fwd + bwd) - alu["diag_blocks"] - alu["solve_leaves"]
+    tot_alu = sum(alu.values())
+    return {"mma_share": round(mma / (mma + tot_alu), 4), "alu_share": round(tot_alu / (mma + tot_alu), 4),
+            "alu_terms_per_unit": {k: round(v) for k, v in alu.items()},
+            "note": "modelled per unit of the step's kernels; the pages report 98% on matrix units"}
+
+
+def pass_work(C, d, es):
+    """Algorithmic work per head-token of the forward and the backward pass (the
+    survey's measurement section): flops count a multiply-add as 2, triangles once
+    and no zero tile; bytes are the compulsory HBM traffic of the pass's inputs and
+    outputs (es = bytes per input element; log_alpha and the state are fp32).
+    Returns (fwd_flops, fwd_bytes, bwd_flops, bwd_bytes)."""
+    fwd_fl = 8 * C * d + C * C / 3 + 8 * d * d
+    bwd_fl = 22 * C * d + C * C / 3 + 22 * d * d
+    fwd_by = 7 * d * es + 4 * d + d * es          # q k v e w g z, log_alpha, y
+    bwd_by = (7 * d * es + 4 * d) + d * es + 7 * d * es + 4 * d + 2 * 4 * d  # inputs, dy, grads, dlog_alpha, states
+    return fwd_fl, fwd_by, bwd_fl, bwd_by
 
 
 def algorithmic_step():
-    """Work of one fwd+bwd step of the whole path (per head-token figures of the
-    survey's measurement section, at C = 128, d = 128): flops and bytes."""
-    C, d = WL["chunk"], WL["dk"]
+    """Work of one fwd+bwd step of the whole path at the benchmark's shape: flops and bytes."""
     ht = WL["B"] * WL["T"] * WL["H"]
-    fwd_fl = 8 * C * d + C * C / 3 + 8 * d * d
-    bwd_fl = 22 * C * d + C * C / 3 + 22 * d * d
-    return ht * (fwd_fl + bwd_fl), ht * (2560 + 5888)
+    ff, fb, bf, bb = pass_work(WL["chunk"], WL["dk"], 2)
+    return ht * (ff + bf), ht * (fb + bb)
 
 
 class ClockSampler:
@@ -191,13 +213,18 @@ class Step:
             muir.chunk_fwd(*self.args, chunk=C, y=self.y, S_T=self.S, workspace=self.ws, save_for_bwd=True)
             self.grads = muir.chunk_bwd(*self.args, d["dy"], chunk=C, workspace=self.ws, use_saved=True)
 
-    def __call__(self):
-        C = WL["chunk"]
-        save = not self.fwd_only
-        self.muir.chunk_fwd(*self.args, chunk=C, y=self.y, S_T=self.S, workspace=self.ws, save_for_bwd=save)
-        if save:
-            self.muir.chunk_bwd(*self.args, self.d["dy"], chunk=C, workspace=self.ws, outputs=self.grads,
+    def fwd(self):
+        self.muir.chunk_fwd(*self.args, chunk=WL["chunk"], y=self.y, S_T=self.S, workspace=self.ws,
+                            save_for_bwd=not self.fwd_only)
+
+    def bwd(self):
+        if not self.fwd_only:
+            self.muir.chunk_bwd(*self.args, self.d["dy"], chunk=WL["chunk"], workspace=self.ws, outputs=self.grads,
                                 use_saved=True)
+
+    def __call__(self):
+        self.fwd()
+        self.bwd()
 
 
 def max_over_ranks(ms, device):
@@ -214,6 +241,34 @@ def job_throughput(world, tokens_per_rank, ms_per_step):
     """Whole-job tokens/s of `world` replicas that each process `tokens_per_rank`
     tokens per step, timed by the slowest rank."""
     return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
+def time_step_passes(step, steps, dist_on):
+    """Time `steps` calls of step() as time_steps does, and also each call's forward
+    and backward pass with CUDA events recorded between them on the launching
+    stream. Returns (total ms, mean forward ms, mean backward ms)."""
+    import torch
+    import torch.distributed as dist
+    if dist_on:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in ev:
+        e[0].record()
+        step.fwd()
+        e[1].record()
+        step.bwd()
+        e[2].record()
+    torch.cuda.synchronize()
+    ms = ev[0][0].elapsed_time(ev[-1][2])
+    f = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    b = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    if dist_on:
+        ms = max_over_ranks(ms, "cuda")
+        f = max_over_ranks(f, "cuda")
+        b = max_over_ranks(b, "cuda")
+        dist.barrier()
+    return ms, f, b
 
 
 def time_steps(fn, steps, dist_on):
@@ -266,6 +321,64 @@ def bench_gate_proj(dev, steps, warmup, pk):
             "algorithmic_TFLOP_s": round(flops / t / 1e12, 2), "frac_tc_peak": round(flops / t / 1e12 / pk["bf16"], 4),
             "algorithmic_GB_s": round(byts / t / 1e9, 1), "frac_hbm": round(byts / t / 1e9 / pk["hbm"], 4),
             "roofline_ms": round(roof_ms, 4), "frac_roofline": round(roof_ms / ms, 4), "gpu_launches": reps}
+
+
+FWD_WORKLOADS = [
+    # the training shape's forward alone (no saving), then the training-forward workload at every chunk
+    # size, then the fp32 stress workload
+    dict(name="fwd_bf16_B1_T32768_H16_d128_C128", B=1, T=32768, C=128, dtype="bf16", lo=1e-4, hi=0.7, bimodal=False,
+         seed=2),
+    dict(name="train_fwd_bf16_B8_T4096_H16_d128_C64", B=8, T=4096, C=64, dtype="bf16", lo=1e-4, hi=0.7,
+         bimodal=False, seed=1),
+    dict(name="train_fwd_bf16_B8_T4096_H16_d128_C128", B=8, T=4096, C=128, dtype="bf16", lo=1e-4, hi=0.7,
+         bimodal=False, seed=1),
+    dict(name="train_fwd_bf16_B8_T4096_H16_d128_C256", B=8, T=4096, C=256, dtype="bf16", lo=1e-4, hi=0.7,
+         bimodal=False, seed=1),
+    dict(name="stress_fwd_f32_B2_T32768_H16_d128_C256", B=2, T=32768, C=256, dtype="f32", lo=0, hi=0, bimodal=True,
+         seed=4),
+]
+
+
+def bench_forwards(dev, steps, warmup, pk):
+    """Forward-only throughput (muir_chunk_fwd, nothing saved) on each forward
+    workload, against the survey's per-head-token forward work: % of the measured
+    bf16 tensor peak (burst and sustained; for the fp32 workload also against the
+    tf32 peak, taken as half the bf16 figure, the nominal ratio), % of the measured
+    HBM bandwidth, and the fraction of the max(flops, bytes) roofline."""
+    import torch
+    import gated_delta_rule_muir_b200 as muir
+    from gated_delta_rule_muir_b200.inputs import device_inputs
+    H, d = WL["H"], WL["dk"]
+    out = {}
+    for wl in FWD_WORKLOADS:
+        x = device_inputs(wl["B"], wl["T"], H, d, d, dtype=wl["dtype"], rate_lo=wl["lo"], rate_hi=wl["hi"],
+                          bimodal=wl["bimodal"], seed=wl["seed"], device=dev)
+        a = [x[n] for n in NAMES]
+        y = torch.empty_like(x["v"])
+        S = torch.empty(wl["B"], H, d, d, device=dev)
+        ws = torch.empty(muir.chunk_fwd_workspace_bytes(*a, wl["C"]), dtype=torch.uint8, device=dev)
+        fn = lambda: muir.chunk_fwd(*a, chunk=wl["C"], y=y, S_T=S, workspace=ws)
+        for _ in range(max(warmup, 3)):
+            fn()
+        reps = max(steps, 10)
+        ms = time_steps(fn, reps, False) / reps
+        es = 2 if wl["dtype"] == "bf16" else 4
+        ff, fb, _, _ = pass_work(wl["C"], d, es)
+        ht = wl["B"] * wl["T"] * H
+        t = ms * 1e-3
+        tf, gb = ht * ff / t / 1e12, ht * fb / t / 1e9
+        roof_ms = 1e3 * max(ht * ff / (pk["bf16"] * 1e12), ht * fb / (pk["hbm"] * 1e9))
+        r = {"ms": round(ms, 4), "tokens_s": round(wl["B"] * wl["T"] / t, 1), "algorithmic_TFLOP_s": round(tf, 2),
+             "frac_tc_peak": round(tf / pk["bf16"], 4), "frac_tc_peak_sustained": round(tf / pk["bf16_sus"], 4),
+             "algorithmic_GB_s": round(gb, 1), "frac_hbm": round(gb / pk["hbm"], 4),
+             "roofline_ms": round(roof_ms, 4), "frac_roofline": round(roof_ms / ms, 4),
+             "per_head_token": {"flops": round(ff), "bytes": fb}}
+        if es == 4:
+            r["frac_tf32_peak"] = round(tf / (pk["bf16"] / 2), 4)
+        out[wl["name"]] = r
+        del x, a, y, S, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def bench_decode(dev, steps, warmup, pk):
@@ -486,7 +599,8 @@ def main():
         for _ in range(args.warmup):
             step()
         n0 = muir.launch_count()
-        ms = time_steps(step, args.steps, dist_on) / args.steps
+        ms_tot, ms_f, ms_b = time_step_passes(step, args.steps, dist_on)
+        ms = ms_tot / args.steps
         launches = (muir.launch_count() - n0)
     tok = WL["B"] * WL["T"]
     value = job_throughput(world, tok, ms)
@@ -501,36 +615,48 @@ def main():
                        "step": "forward only" if Step.fwd_only else
                        "forward (saving its chunk maps) + backward (using them)"},
             "gpu_launches": int(launches), "clocks": clk.summary()}
+    # Roofline of the dominant pass against the survey's algorithmic work per head-token
+    # (fwd 2,560 B, bwd 5,888 B at bf16, d = 128): both passes are HBM-bound by that model
+    # (flops / bytes below the bf16 ridge). Each pass is one C-ABI call of several kernel
+    # launches, timed live by the events around it on the launching stream.
+    C, dk, dv = WL["chunk"], WL["dk"], WL["dv"]
+    ht = WL["B"] * WL["T"] * WL["H"]
+    ff, fb, bf, bb = pass_work(C, dk, 2)
+    passes = {"muir_chunk_fwd": (ms_f, ff, fb), "muir_chunk_bwd": (ms_b, bf, bb)}
+    if Step.fwd_only:
+        passes.pop("muir_chunk_bwd")
+    pname, (p_ms, p_fl, p_by) = max(passes.items(), key=lambda kv: kv[1][0])
+    t_p = p_ms * 1e-3
+    ach = ht * p_by / t_p / 1e9
+    roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s",
+            "frac": round(ach / pk["hbm"], 4), "traffic": None, "kernel": pname,
+            "ms_per_launch": round(p_ms, 4), "algorithmic_bytes_per_head_token": p_by,
+            "head_tokens_per_launch": ht, "frac_tc_peak": round(ht * p_fl / t_p / 1e12 / pk["bf16_sus"], 4),
+            "peak_source": pk["src"]}
+    line["roofline"] = roof
+    line["passes_ms"] = {k: round(v[0], 4) for k, v in passes.items()}
     # per-kernel device times (library events on the launch stream), same workload
     with muir.KernelTimer() as kt:
         for _ in range(args.steps):
             step()
     kern = {k: {"launches": c, "ms_per_step": round(t / args.steps, 4)} for k, (c, t) in kt.result.items()}
     line["kernels"] = kern
-    C, dk, dv = WL["chunk"], WL["dk"], WL["dv"]
+    # the slowest single kernel, with its modelled algorithmic flops (vs the tensor peak) and its
+    # interface bytes (the intermediates it exchanges with the other kernels, vs HBM)
     model = kernel_model(C, dk, dv, 2)
     units = WL["B"] * WL["H"] * (WL["T"] // C)
-    top = max(kt.result.items(), key=lambda kv: kv[1][1])
-    name, (cnt, tot) = top
+    name, (cnt, tot) = max(kt.result.items(), key=lambda kv: kv[1][1])
     base = name.split(":")[-1]
-    fl, by = model[base]
-    per_launch_ms = tot / cnt
-    launches_per_step = cnt / args.steps
-    fl_l, by_l = fl * units / launches_per_step, by * units / launches_per_step
-    t_s = per_launch_ms * 1e-3
-    tc_bound, hbm_bound = fl_l / (pk["bf16_sus"] * 1e12), by_l / (pk["hbm"] * 1e9)
-    if tc_bound >= hbm_bound:
-        ach = fl_l / t_s / 1e12
-        roof = {"bound": "tensor", "achieved": round(ach, 2), "peak": pk["bf16_sus"], "unit": "TFLOP/s"}
-    else:
-        ach = by_l / t_s / 1e9
-        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s"}
-    roof["frac"] = round(ach / roof["peak"], 4)
-    tr = NCU_TRAFFIC_PER_UNIT.get(base)
-    roof["traffic"] = round(tr * units / launches_per_step) if tr is not None else None
-    roof["kernel"] = name
-    roof["peak_source"] = pk["src"]
-    line["roofline"] = roof
+    if base in model:
+        fl, by = model[base]
+        t_k = tot / cnt * 1e-3
+        lps = cnt / args.steps
+        line["slowest_kernel"] = {
+            "kernel": name, "ms_per_launch": round(tot / cnt, 4),
+            "algorithmic_TFLOP_s": round(fl * units / lps / t_k / 1e12, 2),
+            "frac_tc_peak": round(fl * units / lps / t_k / 1e12 / pk["bf16_sus"], 4),
+            "interface_GB_s": round(by * units / lps / t_k / 1e9, 1),
+            "frac_hbm_interface": round(by * units / lps / t_k / 1e9 / pk["hbm"], 4)}
     line["flop_split"] = flop_split(C, dk, dv)
     sfl, sby = algorithmic_step()
     t_step = ms * 1e-3
@@ -540,6 +666,7 @@ def main():
                              "frac_hbm_peak": round(sby / t_step / 1e9 / pk["hbm"], 4),
                              "roofline_ms": round(1e3 * max(sfl / (pk["bf16_sus"] * 1e12), sby / (pk["hbm"] * 1e9)), 3)}
     if not args.skip_extras and rank == 0:
+        line["forward"] = bench_forwards(dev, args.steps, args.warmup, pk)
         line["decode"] = bench_decode(dev, args.steps, args.warmup, pk)
         line["gate_proj"] = bench_gate_proj(dev, args.steps, args.warmup, pk)
         line["e2e"] = e2e_pass(d, max(2, min(args.steps, 5)), 1)

@@ -207,6 +207,20 @@ int muir_selftest_gemm(const float* A, const float* B, float* D, int32_t N, int3
   return cuda_check("selftest launch");
 }
 
+// Diagnostic entry point: one bounded wait on an mbarrier that completes
+// (arrive != 0) or that nothing ever completes (arrive == 0), given up after
+// limit_ns. out (device int) receives 1 if the wait saw the phase complete.
+int muir_selftest_wait(uint64_t limit_ns, int32_t arrive, int32_t* out, void* stream) {
+  g_err.clear();
+  if (!out) return fail(MUIR_ERR_INVALID_ARG, "selftest_wait: out is NULL");
+  if (limit_ns > muir::kWaitLimitNs)
+    return fail(MUIR_ERR_INVALID_ARG, "selftest_wait: limit %llu ns above the library's %llu ns",
+                (unsigned long long)limit_ns, (unsigned long long)muir::kWaitLimitNs);
+  Launch L_("selftest_wait", static_cast<cudaStream_t>(stream));
+  muir::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, arrive, out);
+  return cuda_check("selftest_wait launch");
+}
+
 void muir_profile_begin(void) {
   for (auto& r : g_prof.recs) {
     g_prof.pool.push_back(r.a);

@@ -83,4 +83,20 @@ __global__ void __launch_bounds__(128) selftest_gemm_kernel(const float* __restr
   if (warp == 0) tmem_dealloc(tmem, N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256)));
 }
 
+// Exercises the give-up path of the bounded wait. One warp initialises an
+// mbarrier (count 1) in its own shared memory; with `arrive` set, thread 0
+// arrives first so the phase completes, otherwise nothing ever arrives. Thread
+// 0 then waits for phase 0 through mbar_wait_for with limit_ns. No copy or MMA
+// is in flight at any time, so the kernel ends cleanly either way; a wait that
+// ran out is recorded in the status word. out[0] = 1 if the wait saw the phase
+// complete, 0 if it gave up.
+__global__ void __launch_bounds__(32) selftest_wait_kernel(uint64_t limit_ns, int arrive, int* out) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    if (arrive) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bar)) : "memory");
+    out[0] = mbar_wait_for(&bar, 0u, limit_ns) ? 1 : 0;
+  }
+}
+
 }  // namespace muir

@@ -44,10 +44,10 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Wait for the phase with the given parity to complete. Bounded: gives up after
-// about one second, records the timeout in the device status word and returns
-// false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete. Bounded: gives up once
+// limit_ns of global time have passed since the first check, records the
+// timeout in the device status word and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
@@ -63,9 +63,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if ((it & 63) == 0) {
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) t0 = now;
-      else if (now - t0 > 1000000000ull) { flag_timeout(); return false; }
+      else if (now - t0 > limit_ns) { flag_timeout(); return false; }
     }
   }
+}
+
+// The library's waits: about one second.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // ---- bulk asynchronous copies (global -> shared, completion on an mbarrier) --

@@ -162,3 +162,46 @@ def device_inputs(B: int, T: int, H: int, dk: int, dv: int, *, dtype: str, rate_
         out["dy"] = normal(B, T, H, dv).to(tdt)
         out["dS_T"] = 0.1 * normal(B, H, dk, dv)
     return out
+
+
+def stream_inputs(rows: int, T: int, H: int, dk: int, dv: int, *, c: torch.Tensor, dtype: str, seed: int,
+                  device, token_major: bool = True, out: dict | None = None) -> dict:
+    """One window of a decode stream with fixed per-(head, key row) base decay
+    rates c [H, dk] (fp32, on `device`): the same distributions as device_inputs,
+    with only the per-token jitter redrawn. token_major=True gives [T, rows, H, d]
+    (token t of every row is one contiguous slice, as a decode step takes it);
+    otherwise [rows, T, H, d]. With `out`, the tensors are written into those
+    buffers (same shapes and dtypes) instead of new ones."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed * 1000003 + 11)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    shape = (lambda d: (T, rows, H, d)) if token_major else (lambda d: (rows, T, H, d))
+
+    def normal(d):
+        return torch.randn(*shape(d), generator=gen, device=device, dtype=torch.float32)
+
+    def unit_silu(x):
+        s = torch.nn.functional.silu(x)
+        return s / s.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+
+    vals = {
+        "q": lambda: unit_silu(normal(dk)).to(tdt),
+        "k": lambda: unit_silu(normal(dk)).to(tdt),
+        "v": lambda: normal(dv).to(tdt),
+        "e": lambda: torch.sigmoid(normal(dk)).to(tdt),
+        "w": lambda: torch.sigmoid(normal(dv)).to(tdt),
+        "g": lambda: torch.sigmoid(normal(dk)).to(tdt),
+        "z": lambda: torch.sigmoid(normal(dv)).to(tdt),
+        "log_alpha": lambda: -(c * torch.exp(0.1 * normal(dk))),
+    }
+    res = {}
+    for n, f in vals.items():
+        x = f()
+        if out is not None:
+            out[n].copy_(x)
+            res[n] = out[n]
+        else:
+            res[n] = x
+        del x
+    res["r"] = torch.sqrt(1.0 - torch.exp(-c)).contiguous()
+    return res

@@ -14,6 +14,16 @@
  * buffers) through the tensor-core operand layouts the chunk kernels use;
  * a_mode/b_mode bit 0 = MN-major operand, bit 1 = read through the transposed
  * view of a tile written in the other arrangement; nsplit 1 or 3 bf16 passes.
+ *
+ * muir_selftest_wait(): the give-up path of the library's bounded device
+ * waits. One warp waits for phase 0 of an mbarrier in its own shared memory,
+ * through the same wait routine the kernels use but with a limit of limit_ns
+ * (at most the library's one second). With arrive != 0 the phase completes
+ * before the wait; with arrive == 0 nothing ever completes it, so the wait runs
+ * out, sets the status word that muir_device_status() reports as
+ * MUIR_ERR_TIMEOUT, and the kernel returns. No copy or tensor-core operation is
+ * in flight, so the give-up leaves nothing behind. *out (a device int32)
+ * receives 1 if the wait saw the phase complete, else 0.
  */
 #ifndef MUIR_PROFILE_H
 #define MUIR_PROFILE_H
@@ -33,6 +43,7 @@ int muir_profile_end(char* names_buf, size_t names_cap, float* ms, int64_t* laun
 int64_t muir_launch_count(void);
 int muir_selftest_gemm(const float* A, const float* B, float* D, int32_t N, int32_t K, int32_t a_mode,
                        int32_t b_mode, int32_t nsplit, void* stream);
+int muir_selftest_wait(uint64_t limit_ns, int32_t arrive, int32_t* out, void* stream);
 
 #ifdef __cplusplus
 }

@@ -172,3 +172,11 @@ def test_gate_proj_validates_before_launching(lib):
     assert call(ov=0) == N.MUIR_ERR_UNSUPPORTED
     assert call(n=0) == N.MUIR_OK
     assert call(p=[None] * 12, n=0) == N.MUIR_OK  # an empty batch reads no pointer
+
+
+def test_selftest_wait_rejects_bad_arguments(lib):
+    # the diagnostic bounded-wait kernel takes limits up to the library's own (1 s)
+    fake = C.c_void_p(1 << 20)
+    assert lib.muir_selftest_wait(C.c_uint64(10 ** 10), 0, fake, None) == N.MUIR_ERR_INVALID_ARG
+    assert b"limit" in lib.muir_last_error()
+    assert lib.muir_selftest_wait(C.c_uint64(1000), 0, None, None) == N.MUIR_ERR_INVALID_ARG

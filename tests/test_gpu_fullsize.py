@@ -1,11 +1,10 @@
 """Full-size workloads: the GPU computes every head; the fp64 oracle recomputes
 sampled (batch, head) chains, which are independent of all other chains."""
-import numpy as np
 import pytest
 import torch
 
 import gated_delta_rule_muir_b200 as muir
-from gated_delta_rule_muir_b200.inputs import TRAIN_FWD, TRAIN_FWD_BWD, STRESS, DECODE, device_inputs
+from gated_delta_rule_muir_b200.inputs import TRAIN_FWD, TRAIN_FWD_BWD, STRESS, device_inputs
 from oracle import muir_oracle as orc
 from tests.gpu_util import INPUT_NAMES, rel_err
 
@@ -86,42 +85,3 @@ def test_stress_forward_full_size(cuda_ok):
     assert rel_err(y[1:2, :, 3:4], y_ref) < 1e-4
     assert rel_err(S[1:2, 3:4], S_ref) < 1e-4
 
-
-def test_decode_stream_drift_against_chunked_recompute(cuda_ok):
-    """24 layers x 16 heads x 128x128 fp32 state (25 MB), batch 1: prefill 4096 tokens
-    with the chunked forward, decode 65,536 tokens one at a time, and compare the
-    decoded state and outputs with a chunked recompute of the same window from the
-    same start state (final state 1e-3, outputs 2e-2). The 24 layers act as 24
-    independent rows of the decode call; one (layer, head) chain of the last window
-    is also checked against the oracle."""
-    dev = torch.device("cuda")
-    L = DECODE.extra["layers"]
-    H, dk, dv = DECODE.H, DECODE.dk, DECODE.dv
-    pre = _gen(DECODE, dev, B=L, T=DECODE.extra["prefill"])
-    r = pre["r"]
-    _, S = muir.chunk_fwd(*[pre[n] for n in INPUT_NAMES], chunk=128)
-    del pre
-    Tw, win = 65536, 4096
-    S_dec = S.clone()
-    S_chk = S.clone()
-    ys_err = []
-    for w0 in range(0, Tw, win):
-        S_start = S_chk
-        d = device_inputs(L, win, H, dk, dv, dtype="bf16", rate_lo=1e-4, rate_hi=0.7, bimodal=False,
-                          seed=3 + w0, device=dev)
-        d["r"] = r
-        y_c, S_chk = muir.chunk_fwd(*[d[n] for n in INPUT_NAMES], chunk=128, S0=S_chk)
-        ys = []
-        for t in range(win):
-            ys.append(muir.decode_step(S_dec, *[d[n][:, t].contiguous() for n in INPUT_NAMES[:8]], r))
-        y_d = torch.stack(ys, 1)
-        ys_err.append(rel_err(y_d, y_c.double().cpu().numpy()))
-    assert muir.device_status() == 0
-    assert max(ys_err) < 2e-2
-    assert rel_err(S_dec, S_chk.double().cpu().numpy()) < 1e-3
-    # oracle spot check of the last window on one (layer, head)
-    c = _chain(d, 0, 7)
-    y_ref, S_ref = orc.forward(*[c[n] for n in INPUT_NAMES], S0=S_start[0:1, 7:8].double().cpu().numpy())
-    assert rel_err(y_d[0:1, :, 7:8], y_ref) < 2e-2
-    assert rel_err(S_dec[0:1, 7:8], S_ref) < 1e-3
-    assert np.isfinite(S_dec.cpu().numpy()).all()
