@@ -29,9 +29,9 @@
 //
 // Kernels (one CTA per (batch, head, unit of Cs = min(chunk, 128) tokens) unless noted):
 //   decay_kernel      pre, suf, Gam_t, Gsuf_t            -> workspace
-//   gram_kernel       the 4 Grams: blocks across the binary tree of 16-token
-//                     blocks on tcgen05 (one product per level), the exact
-//                     16x16 diagonal blocks on the CUDA cores meanwhile
+//   gram_kernel       the 4 Grams (gram.cuh): blocks across the binary tree of
+//                     8-token blocks on tcgen05 (one product per level), the
+//                     exact 8x8 diagonal blocks on the CUDA cores meanwhile
 //   solve_kernel      T: exact 16x16 leaves, then recursive 2x2 block merges
 //                     T21 = -T22 M21 T11 on tcgen05 (block-Neumann recursion)
 //   maps_kernel       W, Ut, Phi, Psi, Q', Oloc (tcgen05)  -> workspace
@@ -46,6 +46,14 @@
 namespace muir {
 
 constexpr int SB = 16;  // pivot block length (tokens)
+
+// Column slab width of the sequential scans: Psi (and the backward's E) are
+// stored per unit as [dv / kSlab][dk][kSlab], and every scan CTA carries one
+// kSlab-column slab of the state, so that B * H * dv / kSlab CTAs run the scan.
+constexpr int kSlab = 16;
+__host__ __device__ inline int64_t slab_off(int c, int row, int dk) {
+  return ((int64_t)(c / kSlab) * dk + row) * kSlab + (c % kSlab);
+}
 
 struct ChunkParams {
   int B;
@@ -63,7 +71,7 @@ struct ChunkParams {
   uint8_t* gr; // [nsubtot][4] images of M^kk, M^ka, N^qk, N^qa (see sq_put)
   uint8_t* tt; // [nsubtot] image of T
   uint8_t* ma;  // [nunits] images of Phi and Q' (see MapGeom)
-  float* psi;   // [nunits][dv/32][dk][32]: Psi in 32-column slabs
+  float* psi;   // [nunits][dv/kSlab][dk][kSlab]: Psi in column slabs (slab_off)
   float* ol;    // [nunits][Cs][dv]: Oloc
   uint8_t* ma2; // the same three for chunk-256 maps composed from two 128-token units
   float* psi2;
@@ -110,6 +118,8 @@ __device__ __forceinline__ void lds_vec(const float* p, float (&o)[N]) {
       const float4 a = reinterpret_cast<const float4*>(p)[i];
       o[4 * i] = a.x; o[4 * i + 1] = a.y; o[4 * i + 2] = a.z; o[4 * i + 3] = a.w;
     }
+  } else if constexpr (N == 1) {
+    o[0] = *p;
   } else {
     static_assert(N % 2 == 0, "even length");
 #pragma unroll
@@ -543,222 +553,6 @@ __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& 
 }
 
 // ---------------------------------------------------------------------------
-// gram_kernel: the four decayed Grams M^kk, M^ka (strictly lower), N^qk, N^qa
-// (lower, diagonal included) of one unit, written as bf16 hi/lo images.
-//
-// Pairs (t, s) in different 16-token blocks are taken level by level over the
-// binary tree of the unit's blocks: at level b (64, 32, 16 for Cs = 128) the
-// pivots are P = (2p+1) b, and every t in [P, P+b) meets every s in [P-b, P):
-//   Gam_{t<-s} = pre^b_t * suf^b_s,  pre^b_t = prod_{u=P..t} alpha_u,
-//                                    suf^b_s = prod_{u=s+1..P-1} alpha_u,
-// both products of alphas in [0, 1] (no division). With pre16 / suf16 the
-// in-block products and tot_J the block totals, pre^b_t = pre16_t F^b_J(t) and
-// suf^b_s = suf16_s F^b_J(s), where F^b_J is the product of the block totals
-// between block J and the pivot. One tcgen05 product per level:
-//   XL rows p*2b + X*b + r = [K; Qt]_t pre^b_t   (t = (2p+1)b + r, X = K, Qt)
-//   YL rows p*2b + Y*b + r = [K; A]_s  suf^b_s   (s = 2pb + r,     Y = K, A)
-//   D = XL YL^T (M = 128, N = Cs, K = dk): row block p, column block p holds
-//   the four Gram blocks of pivot p; the other blocks of D are not used.
-// The 16x16 diagonal blocks are computed exactly on the CUDA cores with
-// running products while the tensor core runs; the zeros right of the diagonal
-// blocks are written by bulk stores from shared memory.
-// ---------------------------------------------------------------------------
-template <int DK, typename T, int NS>
-__global__ void __launch_bounds__(256, 1) gram_kernel(ChunkParams p) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ uint64_t bar;
-  __shared__ uint32_t tslot;
-  constexpr int NT = 256;
-  constexpr int CH = DK / 16;  // channels per thread in the diagonal blocks
-  const int Cs = p.Cs, nb = Cs / SB;
-  const int nlev = tree_levels(Cs);
-  const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  constexpr uint32_t LB = 128u * DK * 2u;
-  const uint32_t base = smem_u32(sm);
-  const Tile XL{base, base + LB, 128u, DK * 16u};
-  const Tile YL{base + 2 * LB, base + 3 * LB, 128u, DK * 16u};
-  float* ftab = reinterpret_cast<float*>(sm + 4 * LB);  // [kMaxLev][nb][DK]
-  float* drow = ftab + kMaxLev * nb * DK;                // [4][16][DK]: k, qt, a, alpha of one block
-  zero_smem(base, 4 * LB);
-  TcCta cta;
-  cta.init(&tslot, &bar, tmem_cols_for(128 * nlev));
-  const float* pre = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
-  const float* suf = pre + Cs * DK;
-  uint8_t* out = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
-  MmaSync drv{&bar, 0u, true};
-  const uint32_t id = idesc_bf16(128, Cs, 0, 0);
-
-  tree_tables<DK>(pre, ftab, Cs);
-  __syncthreads();
-
-  // Rows of block J for its exact diagonal block: fetched into registers one
-  // block ahead (the loads fly while the previous block is computed), then
-  // stored to drow as k, qt, a, alpha.
-  constexpr int FPT = (SB * (DK / 8) + NT - 1) / NT;  // 8-channel pieces per thread
-  Pack8<T> fk[FPT], fe[FPT], fq[FPT], fg[FPT];
-  Pack8<float> fl[FPT];
-  auto fetch_block = [&](int J) {
-#pragma unroll
-    for (int f = 0; f < FPT; ++f) {
-      const int x = tid + f * NT;
-      if (x < SB * (DK / 8)) {
-        const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-        const int64_t o = toff(p, s.b, s.tok0 + SB * J + rr, s.h, DK) + c8;
-        fk[f].ld(static_cast<const T*>(p.k) + o);
-        fe[f].ld(static_cast<const T*>(p.e) + o);
-        fq[f].ld(static_cast<const T*>(p.q) + o);
-        fg[f].ld_or_one(p.g ? static_cast<const T*>(p.g) + o : nullptr);
-        fl[f].ld(p.la + o);
-      }
-    }
-  };
-  auto store_block = [&] {
-#pragma unroll
-    for (int f = 0; f < FPT; ++f) {
-      const int x = tid + f * NT;
-      if (x < SB * (DK / 8)) {
-        const int rr = x / (DK / 8), c8 = (x % (DK / 8)) * 8;
-        float kk[8], ee[8], qq[8], gg[8], la[8], rr8[8];
-        fk[f].get(kk);
-        fe[f].get(ee);
-        fq[f].get(qq);
-        fg[f].get(gg);
-        fl[f].get(la);
-        ld8f(p.r + (int64_t)s.h * DK + c8, rr8);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          la[j] = expf(la[j]);
-          ee[j] *= kk[j];               // a = e k
-          qq[j] = rr8[j] * gg[j] * qq[j];  // qt = r g q
-        }
-        Elt<float>::st8(drow + (0 * SB + rr) * DK + c8, kk);
-        Elt<float>::st8(drow + (1 * SB + rr) * DK + c8, qq);
-        Elt<float>::st8(drow + (2 * SB + rr) * DK + c8, ee);
-        Elt<float>::st8(drow + (3 * SB + rr) * DK + c8, la);
-      }
-    }
-  };
-  // thread = (row t, channel group cg of CH channels); for s = t, t-1, ... the
-  // running product Gam_{t<-s} = Gam_{t<-s+1} alpha_{s+1} scales both right
-  // operands; the 64 partial sums are reduced over the 16 lanes of the row by
-  // recursive halving, after which lane cg holds Gram cg/4, columns 4(cg%4)..+3.
-  // Warps w and w + 4 share a scheduler: rows (2w, 2w+1) go with (14-2w, 15-2w)
-  // so that every scheduler runs 18 row steps.
-  auto diag_block = [&](int J) {
-    const int pair = warp < 4 ? warp : 11 - warp;
-    const int t = 2 * pair + ((tid >> 4) & 1), cg = tid & 15, c0 = cg * CH;
-    float xk[CH], xq[CH], gm[CH];
-    lds_vec(drow + (0 * SB + t) * DK + c0, xk);
-    lds_vec(drow + (1 * SB + t) * DK + c0, xq);
-#pragma unroll
-    for (int j = 0; j < CH; ++j) gm[j] = 1.f;
-    float v[64];
-#pragma unroll
-    for (int ss = SB - 1; ss >= 0; --ss) {
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      if (ss <= t) {
-        float yk[CH], ya[CH], al[CH];
-        lds_vec(drow + (0 * SB + ss) * DK + c0, yk);
-        lds_vec(drow + (2 * SB + ss) * DK + c0, ya);
-        lds_vec(drow + (3 * SB + ss) * DK + c0, al);
-#pragma unroll
-        for (int j = 0; j < CH; ++j) {
-          yk[j] *= gm[j];
-          ya[j] *= gm[j];
-          a0 += xk[j] * yk[j]; a1 += xk[j] * ya[j]; a2 += xq[j] * yk[j]; a3 += xq[j] * ya[j];
-          gm[j] *= al[j];
-        }
-      }
-      v[0 * 16 + ss] = a0; v[1 * 16 + ss] = a1; v[2 * 16 + ss] = a2; v[3 * 16 + ss] = a3;
-    }
-#pragma unroll
-    for (int m = 8, n = 32; m >= 1; m >>= 1, n >>= 1) {
-      const bool up = (cg & m) != 0;
-#pragma unroll
-      for (int j = 0; j < n; ++j) {
-        const float send = up ? v[j] : v[j + n];
-        const float keep = up ? v[j + n] : v[j];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-      }
-    }
-    const int g = cg >> 2, c4 = (cg & 3) * 4;
-    const bool strict = g < 2;  // M^kk, M^ka exclude the diagonal
-    float w4[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int ss = c4 + j;
-      w4[j] = (ss < t || (!strict && ss == t)) ? v[j] : 0.f;
-    }
-    gput_k4(out + g * sq_bytes(Cs), sq_half(Cs), (uint32_t)Cs * 16u, SB * J + t, SB * J + c4, w4);
-  };
-  // Zeros right of the diagonal blocks of the four images, written by the
-  // bulk-copy engine from a zeroed buffer while the threads compute.
-  const int lcs = log2_cs(Cs);
-  if (warp == 0) {
-    const int lane = tid & 31, ng = Cs >> 3;
-    const uint32_t zbuf = base + 4 * LB + (uint32_t)(kMaxLev * 8 * DK + 4 * SB * DK) * 4u, gb = (uint32_t)Cs * 16u;
-    for (uint32_t o = lane * 16u; o < kZeroBuf; o += 512u) sts128(zbuf + o, make_uint4(0, 0, 0, 0));
-    fence_async_smem();
-    __syncwarp();
-    for (int x = lane; x < 8 * ng; x += 32) {  // (image, hi/lo, row group)
-      const int rg = x & (ng - 1), gh = x / ng;
-      const uint32_t pb = sq_prefix(rg);
-      if (pb < gb) bulk_s2g(out + (gh >> 1) * sq_bytes(Cs) + (gh & 1) * sq_half(Cs) + rg * gb + pb, zbuf, gb - pb);
-    }
-    bulk_commit();
-  }
-  fetch_block(0);
-  float rv[8];  // r for this thread's 8 channels in stage_level (fixed: 256 pieces per sweep)
-  {
-    int r_, c8_;
-    row_piece<T, DK / 8>(tid, r_, c8_);
-    ld8f(p.r + (int64_t)s.h * DK + c8_, rv);
-  }
-  for (int lev = 0; lev < nlev && drv.ok; ++lev) {
-    const int lb = lcs - 1 - lev;  // b = 2^lb
-    const float* ft = ftab + lev * nb * DK;
-    stage_level<DK, T>(p, s, pre, suf, ft, rv, Cs, lb, true, true, XL, YL);
-    const int J0 = lev * nb / nlev, J1 = (lev + 1) * nb / nlev;
-    drv.run_overlap(
-        [&] { mma_tiles(cta.tmem + 128 * lev, XL, YL, DK / 16, id, NS, false); },
-        [&] {
-          for (int J = J0; J < J1; ++J) {
-            __syncthreads();  // drow is free
-            store_block();
-            __syncthreads();
-            if (J + 1 < nb) fetch_block(J + 1);
-            diag_block(J);
-          }
-        });
-  }
-  // Epilogue: lane = row p*2b + X*b + r of level b; the valid columns are the
-  // 2b of column block p (Y = K first, then Y = A).
-  const int rho = tid & 127, wg = tid >> 7;
-  for (int lev = 0; lev < nlev; ++lev) {
-    const int lb = lcs - 1 - lev, b = 1 << lb;
-    const int pv = ((warp & 3) * 32) >> (lb + 1);  // warp-uniform: 2b >= 32
-    const int X = (rho >> lb) & 1, r = rho & (b - 1);
-    const int t = (2 * pv + 1) * b + r;
-    for (int c0 = wg * 16; c0 < 2 * b; c0 += 32) {
-      float v[16];
-      tmem_ld16(cta.tmem + tmem_lane_base(warp) + 128 * lev + pv * 2 * b + c0, v);
-      if (rho < Cs && drv.ok) {
-        const int Y = c0 >> lb, s0 = 2 * pv * b + (c0 & (b - 1));
-        uint8_t* img = out + (2 * X + Y) * sq_bytes(Cs);
-        float a8[8], b8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
-        sq_put(img, Cs, t, s0, a8);
-        sq_put(img, Cs, t, s0 + 8, b8);
-      }
-    }
-  }
-  if (warp == 0) bulk_wait_all();  // the zero stores have read their source
-  cta.finish();
-}
-
-// ---------------------------------------------------------------------------
 // solve_kernel: T = (I + M^ka)^-1 (unit lower triangular) by the recursive
 // block method: exact 16x16 leaves by forward substitution, then for block size
 // h = 16, 32, 64 every pair [[A,0],[B,D]] of adjacent h-blocks gets the lower
@@ -1064,7 +858,7 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
     float v[16];
     tmem_ld16(cta.tmem + lane + cPsi + c, v);
     if (t < DK && drv.ok) {
-      float* o = psi + ((int64_t)(c >> 5) * DK + t) * 32 + (c & 31);
+      float* o = psi + slab_off(c, t, DK);
       stg_row16(o, v);
     }
   }
@@ -1147,7 +941,7 @@ __global__ void __launch_bounds__(128, 1) compose_kernel(ChunkParams p) {
     int r, c8;
     piece_of<DV / 8>(x, r, c8);
     float v[8];
-    ld8f(psi0 + ((int64_t)(c8 >> 5) * DK + r) * 32 + (c8 & 31), v);
+    ld8f(psi0 + slab_off(c8, r, DK), v);
     put_mn(Bpsi, r, c8, v);
   }
   if (drv.ok)
@@ -1178,8 +972,8 @@ __global__ void __launch_bounds__(128, 1) compose_kernel(ChunkParams p) {
       float v[16];
       tmem_ld16(cta.tmem + lane + 256 + j * 128 + c, v);
       if (on) {
-        const float* a = j == 0 ? psi1 + ((int64_t)(c >> 5) * DK + tid) * 32 + (c & 31) : ol1 + (int64_t)tid * DV + c;
-        float* o = j == 0 ? psi + ((int64_t)(c >> 5) * DK + tid) * 32 + (c & 31) : ol + (int64_t)(Cs + tid) * DV + c;
+        const float* a = j == 0 ? psi1 + slab_off(c, tid, DK) : ol1 + (int64_t)tid * DV + c;
+        float* o = j == 0 ? psi + slab_off(c, tid, DK) : ol + (int64_t)(Cs + tid) * DV + c;
 #pragma unroll
         for (int e = 0; e < 16; e += 4)
           *reinterpret_cast<float4*>(o + e) = make_float4(v[e] + a[e], v[e + 1] + a[e + 1], v[e + 2] + a[e + 2],
@@ -1216,7 +1010,7 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar, bar_c[2];
   __shared__ uint32_t tslot;
-  constexpr int NW = 32;
+  constexpr int NW = kSlab;
   const int dv = p.dv, slabs = dv / NW;
   const int slab = blockIdx.x % slabs;
   const int bh = blockIdx.x / slabs;
@@ -1281,7 +1075,7 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
                     });
     if (!drv.ok) break;
     float v[NW];
-    tmem_ld32(cta.tmem + lane, v);
+    tmem_ld_slab(cta.tmem + lane, v);
     if (tid < DK) {
       const float* add = psi_s + buf * (PS / 4) + tid * NW;
 #pragma unroll
@@ -1317,7 +1111,7 @@ __global__ void __launch_bounds__(128, 1) segmap_kernel(ChunkParams p, const uin
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar, bar_c[2];
   __shared__ uint32_t tslot;
-  constexpr int NW = 32;
+  constexpr int NW = kSlab;
   const int dv = p.dv, vslabs = dv / NW, slabs = DK / NW + vslabs;
   const int slab = blockIdx.x % slabs;
   const int bh = blockIdx.x / slabs;
@@ -1372,7 +1166,7 @@ __global__ void __launch_bounds__(128, 1) segmap_kernel(ChunkParams p, const uin
     drv.run([&] { mma_tiles(cta.tmem, Phi, Sb, DK / 16, id, NS, false); });
     if (!drv.ok) break;
     float v[NW];
-    tmem_ld32(cta.tmem + lane, v);
+    tmem_ld_slab(cta.tmem + lane, v);
     if (tid < DK) {
       if (phi_part) {
 #pragma unroll

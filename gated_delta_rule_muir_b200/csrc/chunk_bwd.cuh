@@ -20,7 +20,7 @@
 //
 // Kernels:
 //   bwd_pe_kernel      P = W S0 + Ut, dz = dy * (Q' S0 + Oloc), E = Q'^T dO
-//   rscan_kernel       reverse sweep over units per (b, h, 32-column slab):
+//   rscan_kernel       reverse sweep over units per (b, h, kSlab-column slab):
 //                      dS <- Phi^T dS + E (the adjoint of the state map)
 //   bwd_dz_kernel      dP, dZ, dU
 //   bwd_grads_kernel   dQp, dKp, dKs, dAs, dGam_C and the four Gram cotangents
@@ -40,7 +40,7 @@ struct BwdBufs {
   float* dZ;        // [nst][Cs][dv]
   float* dU;        // [nst][Cs][dv]
   float* dgc;       // [nst][dk]
-  float* E;         // [nst][dv/32][dk][32]: Q'^T dO per unit, 32-column slabs
+  float* E;         // [nst][dv/kSlab][dk][kSlab]: Q'^T dO per unit, column slabs (slab_off)
   float* g4;        // [nst][4][Cs][dk]: dQp, dKp, dKs, dAs
   float* dG;        // [nst][4][Cs][Cs]: dM^kk, dM^ka, dN^qk, dN^qa
   float* gl;        // [nst][4][Cs][dk]: dK_left, dQ_left, dK_right, dA_right
@@ -55,7 +55,7 @@ struct BwdBufs {
 // rscan_kernel: the sequential part of the backward pass. For n = last..0:
 //   dSC[n] = dS;   dS <- Phi_n^T dS + E_n,   E_n = Q'_n^T dO_n (from bwd_pe)
 // A = Phi^T: tile 0 of the map image read through the transposed view; B = dS
-// (K = key row, N = 32 slab columns, MN-major) from registers. Phi_n and the
+// (K = key row, N = kSlab slab columns, MN-major) from registers. Phi_n and the
 // E_n slab arrive by bulk copies into two alternating buffers, two units ahead.
 // ---------------------------------------------------------------------------
 template <int DK, int NS>
@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar, bar_c[2];
   __shared__ uint32_t tslot;
-  constexpr int NW = 32;
+  constexpr int NW = kSlab;
   const int dv = p.dv, slabs = dv / NW;
   const int slab = blockIdx.x % slabs;
   const int bh = blockIdx.x / slabs;
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(128, 1) rscan_kernel(ChunkParams p, BwdBufs q)
                     });
     if (!drv.ok) break;
     float v[NW];
-    tmem_ld32(cta.tmem + lane, v);
+    tmem_ld_slab(cta.tmem + lane, v);
     if (tid < DK) {
       const float* add = e_s + buf * (ES / 4) + tid * NW;
 #pragma unroll
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
     float v[16];
     tmem_ld16(cta.tmem + lane + 256 + c, v);
     if (t < DK && drv.ok) {
-      float* o = E + ((int64_t)(c >> 5) * DK + t) * 32 + (c & 31);
+      float* o = E + slab_off(c, t, DK);
       stg_row16(o, v);
     }
   }

@@ -14,6 +14,7 @@
 #include "decode.cuh"
 #include "selftest.cuh"
 #include "chunk.cuh"
+#include "gram.cuh"
 #include "chunk_bwd.cuh"
 #include "gate_proj.cuh"
 

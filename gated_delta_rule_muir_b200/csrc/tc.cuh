@@ -355,6 +355,13 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+template <int N>
+__device__ __forceinline__ void tmem_ld_slab(uint32_t taddr, float (&v)[N]) {
+  static_assert(N == 16 || N == 32, "slab width");
+  if constexpr (N == 32) tmem_ld32(taddr, v);
+  else tmem_ld16(taddr, v);
+}
+
 // ---- a tiny synchronous MMA driver ----------------------------------------
 //
 // Holds the mbarrier phase. Usage (all threads of a 128-thread CTA):

@@ -42,18 +42,22 @@ def _run_stream(batch, windows, sub, seed0):
     win = DECODE.extra["drift_every"]
     assert win % sub == 0
     c = torch.from_numpy(base_rates(H, dk, DECODE.rate_lo, DECODE.rate_hi, False, DECODE.seed)).to(dev, torch.float32)
-    # prefill: chunked forward over 4096 tokens from a zero state
-    pre = stream_inputs(rows, DECODE.extra["prefill"], H, dk, dv, c=c, dtype="bf16", seed=seed0, device=dev,
-                        token_major=False)
-    r = pre["r"]
-    _, S_dec = muir.chunk_fwd(*[pre[n] for n in INPUT_NAMES], chunk=128)
-    del pre
-    # token-major stretch buffers and the decode graph over them
+    # token-major stretch buffers, and the same stretches row-major for the chunked forward
     tdt = torch.bfloat16
     buf = {n: torch.empty(sub, rows, H, dk if n in ("q", "k", "e", "g", "log_alpha") else dv,
                           dtype=torch.float32 if n == "log_alpha" else tdt, device=dev) for n in STEP_NAMES}
+    rm = {n: torch.empty_like(buf[n].transpose(0, 1), memory_format=torch.contiguous_format) for n in STEP_NAMES}
+    r = torch.sqrt(1.0 - torch.exp(-c)).contiguous()
+    ws = torch.empty(muir.chunk_fwd_workspace_bytes(*[rm[n] for n in STEP_NAMES], r, 128), dtype=torch.uint8,
+                     device=dev)
+    # prefill: the chunked forward over 4096 tokens from a zero state, one stretch at a time
+    S_dec = None
+    for j in range(DECODE.extra["prefill"] // sub):
+        stream_inputs(rows, sub, H, dk, dv, c=c, dtype="bf16", seed=seed0 + 500000 + j, device=dev,
+                      token_major=False, out=rm)
+        _, S_dec = muir.chunk_fwd(*[rm[n] for n in STEP_NAMES], r, chunk=128, S0=S_dec, workspace=ws)
     ybuf = torch.empty(sub, rows, H, dv, dtype=tdt, device=dev)
-    stream_inputs(sub, rows, H, dk, dv, c=c, dtype="bf16", seed=seed0 + 1, device=dev, out=buf)
+    stream_inputs(rows, sub, H, dk, dv, c=c, dtype="bf16", seed=seed0 + 1, device=dev, out=buf)
     S_warm = S_dec.clone()
     calls = lambda S: [muir.decode_step(S, *[buf[n][t] for n in STEP_NAMES], r, y=ybuf[t]) for t in range(sub)]
     side = torch.cuda.Stream()
@@ -65,9 +69,6 @@ def _run_stream(batch, windows, sub, seed0):
     with torch.cuda.graph(graph):
         calls(S_dec)
     del S_warm
-    rm = {n: torch.empty_like(buf[n].transpose(0, 1), memory_format=torch.contiguous_format) for n in STEP_NAMES}
-    ws = torch.empty(muir.chunk_fwd_workspace_bytes(*[rm[n] for n in STEP_NAMES], r, 128), dtype=torch.uint8,
-                     device=dev)
     report = []
     for w in range(windows):
         S_chk = S_dec.clone()  # the recompute starts from the decoded state (D12)
@@ -75,7 +76,7 @@ def _run_stream(batch, windows, sub, seed0):
         nsub = win // sub
         for j in range(nsub):
             seed = seed0 + 2 + w * nsub + j
-            stream_inputs(sub, rows, H, dk, dv, c=c, dtype="bf16", seed=seed, device=dev, out=buf)
+            stream_inputs(rows, sub, H, dk, dv, c=c, dtype="bf16", seed=seed, device=dev, out=buf)
             for n in STEP_NAMES:  # [rows, sub, H, d] for the chunked recompute
                 rm[n].copy_(buf[n].transpose(0, 1))
             y_c, S_chk = muir.chunk_fwd(*[rm[n] for n in STEP_NAMES], r, chunk=128, S0=S_chk, workspace=ws)
