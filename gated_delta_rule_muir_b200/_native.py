@@ -59,6 +59,7 @@ SIGNATURES = {
 EXTRA_SIGNATURES = {
     "muir_selftest_gemm": (C.c_int, [vp, vp, vp, C.c_int32, C.c_int32, C.c_int32, C.c_int32, C.c_int32, vp]),
     "muir_selftest_wait": (C.c_int, [C.c_uint64, C.c_int32, vp, vp]),
+    "muir_selftest_sw128": (C.c_int, [vp, vp, vp, C.c_int32, C.c_int32, C.c_int32, vp]),
     "muir_profile_begin": (None, []),
     "muir_profile_end": (C.c_int, [C.c_char_p, C.c_size_t, C.POINTER(C.c_float), C.POINTER(C.c_int64), C.c_int]),
     "muir_launch_count": (C.c_int64, []),

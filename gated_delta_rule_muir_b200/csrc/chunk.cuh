@@ -80,6 +80,7 @@ struct ChunkParams {
   void* y;
   float* S_T;
   float* S_chunks;  // optional [units][dk][dv]: state at the start of every unit
+  float* S_end;     // optional [B*H][dk][dv]: state after the last unit (kept for the backward)
   // backward
   float* wsave;     // optional [nsubtot][Cs][dk]: W
   float* usave;     // optional [nsubtot][Cs][dv]: Ut
@@ -1089,6 +1090,11 @@ __global__ void __launch_bounds__(128, 1) scan_kernel(ChunkParams p, const uint8
   }
   if (p.S_T && tid < DK && drv.ok) {
     float* o = p.S_T + (((int64_t)b * p.H + h) * DK + tid) * dv + slab * NW;
+#pragma unroll
+    for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&st[j]));
+  }
+  if (p.S_end && tid < DK && drv.ok) {
+    float* o = p.S_end + (((int64_t)b * p.H + h) * DK + tid) * dv + slab * NW;
 #pragma unroll
     for (int j = 0; j < NW; j += 8) stg256(o + j, *reinterpret_cast<const float(*)[8]>(&st[j]));
   }

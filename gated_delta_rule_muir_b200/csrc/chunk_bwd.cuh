@@ -22,7 +22,7 @@
 //   bwd_pe_kernel      P = W S0 + Ut, dz = dy * (Q' S0 + Oloc), E = Q'^T dO
 //   rscan_kernel       reverse sweep over units per (b, h, kSlab-column slab):
 //                      dS <- Phi^T dS + E (the adjoint of the state map)
-//   bwd_dz_kernel      dP, dZ, dU
+//   bwd_dz_kernel      dP, dZ, dU (written as dv = w dU, dw = v dU)
 //   bwd_grads_kernel   dQp, dKp, dKs, dAs, dGam_C and the four Gram cotangents
 //   bwd_gram_kernel    the Gram backward: tree levels on tcgen05 (left and
 //                      right phases), exact diagonal blocks on the CUDA cores
@@ -38,8 +38,7 @@ struct BwdBufs {
   float* dSC;       // [nst][dk][dv]   state cotangent at each unit's end
   float* P;         // [nst][Cs][dv]
   float* dZ;        // [nst][Cs][dv]
-  float* dU;        // [nst][Cs][dv]
-  float* dgc;       // [nst][dk]
+  float* eC;        // [nst][dk]: rowsum(dS_C * S_C), all that lands on the unit's last log-decay
   float* E;         // [nst][dv/kSlab][dk][kSlab]: Q'^T dO per unit, column slabs (slab_off)
   float* g4;        // [nst][4][Cs][dk]: dQp, dKp, dKs, dAs
   float* dG;        // [nst][4][Cs][Cs]: dM^kk, dM^ka, dN^qk, dN^qa
@@ -383,13 +382,44 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
     }
   }
   wait_img();
-  drv.run([&] { mma_tiles(cta.tmem + cU, AT, B3, Cs / 16, idT, NS, true); });
-  float* dUo = q.dU + u * Cs * DV;
-  for (int c = wg * 16; c < DV; c += 32) {
+  // dU -> dv = w dU and dw = v dU, straight into the gradients; this thread's w
+  // and v pieces are loaded while the last product runs
+  constexpr int NCH = DV / 32;  // 16-column chunks per thread
+  const int64_t vo = toff(p, s.b, s.tok0 + t, s.h, DV);
+  Pack8<T> pw[NCH][2], pv[NCH][2];
+  drv.run_overlap([&] { mma_tiles(cta.tmem + cU, AT, B3, Cs / 16, idT, NS, true); },
+                  [&] {
+                    if (t < Cs) {
+#pragma unroll
+                      for (int k = 0; k < NCH; ++k)
+#pragma unroll
+                        for (int h8 = 0; h8 < 2; ++h8) {
+                          const int c = wg * 16 + 32 * k + 8 * h8;
+                          pw[k][h8].ld(static_cast<const T*>(p.w) + vo + c);
+                          pv[k][h8].ld(static_cast<const T*>(p.v) + vo + c);
+                        }
+                    }
+                  });
+#pragma unroll
+  for (int k = 0; k < NCH; ++k) {
+    const int c = wg * 16 + 32 * k;
     float v[16];
     tmem_ld16(cta.tmem + lane + cU + c, v);
-    if (t < Cs && drv.ok)
-      stg_row16(dUo + t * DV + c, v);
+    if (t < Cs && drv.ok) {
+#pragma unroll
+      for (int h8 = 0; h8 < 2; ++h8) {
+        float ww[8], vv[8], a8[8], b8[8];
+        pw[k][h8].get(ww);
+        pv[k][h8].get(vv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          a8[j] = ww[j] * v[8 * h8 + j];
+          b8[j] = vv[j] * v[8 * h8 + j];
+        }
+        Elt<T>::st8(static_cast<T*>(q.dv) + vo + c + 8 * h8, a8);
+        Elt<T>::st8(static_cast<T*>(q.dw) + vo + c + 8 * h8, b8);
+      }
+    }
   }
   cta.finish();
 }
@@ -458,16 +488,23 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   if (tid == 0) mbar_expect_tx(&bar_cp, mat_dkdv + mat_csdv);
   raw_issue(R0, q.dSC + u * DK * DV, DK, DV, &bar_cp);
   raw_issue(R2, q.P + u * Cs * DV, Cs, DV, &bar_cp);
-  if (tid < DK) {  // dGam_C[i] = sum_j dS_C[i][j] S0[i][j]
+  if (tid < DK) {
+    // Everything that reaches the unit's last cumulative log-decay L_{C-1}: the
+    // decay of S0 (Gam_C dGam_C, dGam_C = rowsum(dS_C * S0)) plus the suffix
+    // factors of K_s and A_s (sum_s K_s dK_s + A_s dA_s, with dK_s = U dS_C^T and
+    // dA_s = -P dS_C^T). Since S_C = Diag(Gam_C) S0 + K_s^T U - A_s^T P, the sum
+    // is rowsum(dS_C * S_C), with S_C the next unit's start state (or the state
+    // after the sequence's last unit).
     const float* d = q.dSC + u * DK * DV + tid * DV;
-    const float* s0 = q.S_chunks + u * DK * DV + tid * DV;
+    const float* sc = (s.n + 1 < p.nsub ? q.S_chunks + (u + 1) * DK * DV
+                                        : p.S_end + ((int64_t)s.b * p.H + s.h) * DK * DV) + tid * DV;
     float acc = 0.f;
 #pragma unroll 4
     for (int j = 0; j < DV; j += 4) {
-      const float4 a = *reinterpret_cast<const float4*>(d + j), c = *reinterpret_cast<const float4*>(s0 + j);
+      const float4 a = *reinterpret_cast<const float4*>(d + j), c = *reinterpret_cast<const float4*>(sc + j);
       acc += a.x * c.x + a.y * c.y + a.z * c.z + a.w * c.w;
     }
-    q.dgc[u * DK + tid] = acc;
+    q.eC[u * DK + tid] = acc;
   }
   stage_U(R1);
   raw_wait();
@@ -812,10 +849,10 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
 // ---------------------------------------------------------------------------
 // bwd_final_kernel: per unit, thread = key channel i (then value channel j):
 //   dL_t = k dKl + qt dQl - k dKr - a dAr + Kp dKp + Qp dQp - Ks dKs - As dAs
-//   dL_{C-1} += sum_s (Ks dKs + As dAs) + Gam_C dGam_C
+//   dL_{C-1} += sum_s (Ks dKs + As dAs) + Gam_C dGam_C = rowsum(dS_C * S_C)
 //   dlog_alpha_t = sum_{u >= t} dL_u
 //   dqt = dQl + Gam dQp, da = dAr + Gsuf dAs, dk = dKl + dKr + Gam dKp + Gsuf dKs + e da
-//   dq = r g dqt, dg = r q dqt, dr += g q dqt, de = k da, dv = w dU, dw = v dU
+//   dq = r g dqt, dg = r q dqt, dr += g q dqt, de = k da  (dv, dw come from bwd_dz)
 // ---------------------------------------------------------------------------
 template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q) {
@@ -823,7 +860,7 @@ __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q
   const int64_t u = blockIdx.x;
   const SubIdx s = sub_of(p, (int)u, p.nsub, Cs);
   const int i = threadIdx.x;
-  const int64_t stride_k = (int64_t)p.H * DK, stride_v = (int64_t)p.H * DV;
+  const int64_t stride_k = (int64_t)p.H * DK;
   if (i < DK) {
     const float* gam = p.dec + (u * 4 + 2) * Cs * DK;
     const float* gsuf = p.dec + (u * 4 + 3) * Cs * DK;
@@ -831,17 +868,9 @@ __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q
     const float* gl = q.gl + u * 4 * Cs * DK;
     const float rr = p.r[(int64_t)s.h * DK + i];
     const int64_t o0 = toff(p, s.b, s.tok0, s.h, DK) + i;
-    // The terms that land on the last token's cumulative log-decay enter every
-    // dlog_alpha of the unit: gather them first.
-    float E = __ldg(gam + (Cs - 1) * DK + i) * __ldg(q.dgc + u * DK + i);
-#pragma unroll 8
-    for (int tt = 0; tt < Cs; ++tt) {
-      const int64_t o = o0 + tt * stride_k;
-      const float kk = Elt<T>::ld(static_cast<const T*>(p.k) + o);
-      const float ee = Elt<T>::ld(static_cast<const T*>(p.e) + o);
-      const int ti = tt * DK + i;
-      E += kk * __ldg(gsuf + ti) * (__ldg(g4 + 2 * Cs * DK + ti) + ee * __ldg(g4 + 3 * Cs * DK + ti));
-    }
+    // what lands on the last token's cumulative log-decay enters every dlog_alpha
+    // of the unit (gathered by bwd_grads)
+    const float E = __ldg(q.eC + u * DK + i);
     float run = E, dr_acc = 0.f;
 #pragma unroll 8
     for (int tt = Cs - 1; tt >= 0; --tt) {
@@ -869,17 +898,6 @@ __global__ void __launch_bounds__(128) bwd_final_kernel(ChunkParams p, BwdBufs q
       dr_acc += gg * qq * dqt;
     }
     if (q.dr) atomicAdd(q.dr + (int64_t)s.h * DK + i, dr_acc);
-  }
-  if (i < DV) {
-    const float* dU = q.dU + u * Cs * DV;
-    const int64_t o0 = toff(p, s.b, s.tok0, s.h, DV) + i;
-#pragma unroll 8
-    for (int tt = 0; tt < Cs; ++tt) {
-      const int64_t o = o0 + tt * stride_v;
-      const float du = __ldg(dU + tt * DV + i);
-      Elt<T>::st(static_cast<T*>(q.dv) + o, Elt<T>::ld(static_cast<const T*>(p.w) + o) * du);
-      Elt<T>::st(static_cast<T*>(q.dw) + o, Elt<T>::ld(static_cast<const T*>(p.v) + o) * du);
-    }
   }
 }
 

@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar;
   __shared__ uint32_t tslot;
-  constexpr int NT = 256, G = DK / 8, CH = DK / 16;
+  constexpr int G = DK / 8;
   constexpr uint32_t LB = 128u * DK * 2u;  // one bf16 plane of a 128-row operand tile
   constexpr uint32_t PL = NS > 1 ? 2u : 1u;  // planes per operand tile
   const int Cs = p.Cs, nb = Cs >> 3;
@@ -169,6 +169,9 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
     const T* x2p = upper && gp ? gp : kp;            // g, or a stand-in that is not used
     const bool use_g = upper && gp != nullptr;
     const Tile dst = upper ? XL : YL;
+    float rl[8];  // r (a register copy: the lambda captures rv by reference)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rl[j] = rv[j];
     float run[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) run[j] = 0.f;
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
           // pre_t includes alpha_t (upper); suf_s covers the alphas after s (lower)
           const float f = exp2_neg(run[j] + (upper ? l2 : 0.f) + off[j]);
           run[j] += l2;
-          const float m1 = upper ? rv[j] * (use_g ? x2[j] : 1.f) : kk[j];  // r g, or k
+          const float m1 = upper ? rl[j] * (use_g ? x2[j] : 1.f) : kk[j];  // r g, or k
           x1[j] = x1[j] * m1 * f;
           kk[j] *= f;
         }

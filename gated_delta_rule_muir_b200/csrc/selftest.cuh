@@ -4,6 +4,7 @@
 #pragma once
 
 #include "tc.cuh"
+#include "tma.cuh"
 
 namespace muir {
 
@@ -97,6 +98,78 @@ __global__ void __launch_bounds__(32) selftest_wait_kernel(uint64_t limit_ns, in
     if (arrive) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bar)) : "memory");
     out[0] = mbar_wait_for(&bar, 0u, limit_ns) ? 1 : 0;
   }
+}
+
+// D[128, N] = A[128, K] B[K, N], bf16 A (row-major: the K-major operand) and B
+// (row-major [K][N]: the MN-major operand), through 128-byte-swizzled shared
+// memory filled by TMA boxes (use_tma) or by the threads in the same layout.
+// K in {64, 128}; N in {64, 128, 256}. One CTA of 128 threads.
+__global__ void __launch_bounds__(128) selftest_sw128_kernel(const __grid_constant__ CUtensorMap ta,
+                                                             const __grid_constant__ CUtensorMap tb,
+                                                             const __nv_bfloat16* __restrict__ A,
+                                                             const __nv_bfloat16* __restrict__ B, float* __restrict__ D,
+                                                             int N, int K, int use_tma) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ uint64_t bar, bar_cp;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t base = (smem_u32(smem) + 1023u) & ~1023u;
+  const uint32_t bbase = base + (uint32_t)(K / 64) * 16384u;
+  const uint32_t ncols = N <= 32 ? 32u : N <= 64 ? 64u : N <= 128 ? 128u : 256u;
+  if (warp == 0) tmem_alloc(&tslot, ncols);
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    mbar_init(&bar_cp, 1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tslot;
+  bool ok = true;
+  if (use_tma) {
+    if (tid == 0) {
+      mbar_expect_tx(&bar_cp, (uint32_t)(K / 64) * 16384u + (uint32_t)(N / 64) * (uint32_t)K * 128u);
+      for (int a = 0; a < K / 64; ++a) tma_load_2d(base + a * 16384u, &ta, 64 * a, 0, &bar_cp);
+      for (int n = 0; n < N / 64; ++n) tma_load_2d(bbase + (uint32_t)n * K * 128u, &tb, 64 * n, 0, &bar_cp);
+    }
+    ok = __syncthreads_and(mbar_wait(&bar_cp, 0) ? 1 : 0) != 0;
+  } else {
+    for (int idx = tid; idx < 128 * (K / 8); idx += 128) {
+      const int m = idx / (K / 8), c = idx % (K / 8);
+      const uint4 v = *reinterpret_cast<const uint4*>(A + (int64_t)m * K + 8 * c);
+      sts128(base + (uint32_t)(c / 8) * 16384u + (uint32_t)m * 128u + (uint32_t)(((c % 8) ^ (m & 7)) * 16), v);
+    }
+    for (int idx = tid; idx < K * (N / 8); idx += 128) {
+      const int k = idx / (N / 8), c = idx % (N / 8);
+      const uint4 v = *reinterpret_cast<const uint4*>(B + (int64_t)k * N + 8 * c);
+      sts128(bbase + (uint32_t)(c / 8) * K * 128u + (uint32_t)k * 128u + (uint32_t)(((c % 8) ^ (k & 7)) * 16), v);
+    }
+    fence_async_smem();
+    __syncthreads();
+  }
+  if (ok && tid == 0) {
+    tc_fence_after();
+    const uint32_t id = idesc_bf16(128, N, 0, 1);
+    for (int ks = 0; ks < K / 16; ++ks) {
+      const uint64_t ad = sdesc_sw128(base + (uint32_t)(ks / 4) * 16384u + (uint32_t)(ks % 4) * 32u, 16u, 1024u);
+      const uint64_t bd = sdesc_sw128(bbase + (uint32_t)ks * 2048u, (uint32_t)K * 128u, 1024u);
+      mma_bf16(tmem, ad, bd, id, ks > 0 ? 1u : 0u);
+    }
+    mma_commit(&bar);
+  }
+  if (ok) ok = __syncthreads_and(mbar_wait(&bar, 0) ? 1 : 0) != 0;
+  tc_fence_after();
+  if (ok) {
+    for (int c = 0; c < N; c += 16) {
+      float v[16];
+      tmem_ld16(tmem + tmem_lane_base(warp) + c, v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) D[tid * N + c + i] = v[i];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, ncols);
 }
 
 }  // namespace muir

@@ -24,6 +24,12 @@
  * MUIR_ERR_TIMEOUT, and the kernel returns. No copy or tensor-core operation is
  * in flight, so the give-up leaves nothing behind. *out (a device int32)
  * receives 1 if the wait saw the phase complete, else 0.
+ *
+ * muir_selftest_sw128(): D[128,N] = A[128,K] * B[K,N] with bf16 A and B
+ * (row-major device buffers) and fp32 D, through the 128-byte-swizzled operand
+ * tiles of the TMA-fed kernels: A as the K-major operand, B as the MN-major
+ * one, loaded by TMA boxes (use_tma != 0) or written by the threads in the same
+ * layout. K in {64, 128}, N in {64, 128, 256}.
  */
 #ifndef MUIR_PROFILE_H
 #define MUIR_PROFILE_H
@@ -44,6 +50,7 @@ int64_t muir_launch_count(void);
 int muir_selftest_gemm(const float* A, const float* B, float* D, int32_t N, int32_t K, int32_t a_mode,
                        int32_t b_mode, int32_t nsplit, void* stream);
 int muir_selftest_wait(uint64_t limit_ns, int32_t arrive, int32_t* out, void* stream);
+int muir_selftest_sw128(const void* A, const void* B, float* D, int32_t N, int32_t K, int32_t use_tma, void* stream);
 
 #ifdef __cplusplus
 }

@@ -29,3 +29,26 @@ def test_selftest_gemm(cuda_ok, a_mn, b_mn, N_, K, nsplit):
     ref = (A.double() @ B.double()).numpy()
     err = np.max(np.abs(D.double().cpu().numpy() - ref)) / np.max(np.abs(ref))
     assert err < (1e-2 if nsplit == 1 else 5e-5), err
+
+
+@pytest.mark.parametrize("use_tma", [0, 1])
+@pytest.mark.parametrize("N_,K", [(64, 64), (128, 64), (256, 128), (64, 128)])
+def test_selftest_sw128(cuda_ok, use_tma, N_, K):
+    """128-byte-swizzled operands: A K-major, B MN-major, written by the threads or
+    loaded by TMA boxes. bf16 products are exact, so only the fp32 accumulation
+    order separates the result from the fp64 matmul of the same bf16 values."""
+    lib = N.load()
+    g = torch.Generator().manual_seed(7 * N_ + K + 1000 * use_tma)
+    A = torch.randn(128, K, generator=g).bfloat16()
+    B = torch.randn(K, N_, generator=g).bfloat16()
+    Ad, Bd = A.cuda(), B.cuda()
+    D = torch.full((128, N_), float("nan"), device="cuda")
+    N.check(lib.muir_selftest_sw128(C.c_void_p(Ad.data_ptr()), C.c_void_p(Bd.data_ptr()), C.c_void_p(D.data_ptr()),
+                                    N_, K, use_tma, C.c_void_p(torch.cuda.current_stream().cuda_stream)),
+            "selftest_sw128")
+    torch.cuda.synchronize()
+    from gated_delta_rule_muir_b200 import device_status
+    assert device_status() == 0
+    ref = (A.double() @ B.double()).numpy()
+    err = np.max(np.abs(D.double().cpu().numpy() - ref)) / np.max(np.abs(ref))
+    assert err < 1e-5, err
