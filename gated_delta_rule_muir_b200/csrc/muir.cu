@@ -17,6 +17,7 @@
 #include "gram.cuh"
 #include "chunk_bwd.cuh"
 #include "gate_proj.cuh"
+#include "gate_proj_tma.cuh"
 
 namespace {
 
