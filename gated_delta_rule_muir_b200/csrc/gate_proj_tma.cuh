@@ -55,11 +55,15 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
-// Two sigmoids, 1 / (1 + 2^(-u log2 e)), with the paired fp32 multiply and add.
+// Two sigmoids, 1 / d with d = 1 + 2^(-u log2 e), paired: one reciprocal serves
+// both, 1/d1 = d2 / (d1 d2) and 1/d2 = d1 / (d1 d2). The exponent is capped at
+// 57 so that d1 d2 stays finite; a sigmoid below 2^-57 comes out as 2^-57.
 __device__ __forceinline__ float2 sigmoid2(float2 u) {
   const float2 a = __fmul2_rn(u, make_float2(-kLog2e, -kLog2e));
-  const float2 d = __fadd2_rn(make_float2(ex2_approx(a.x), ex2_approx(a.y)), make_float2(1.f, 1.f));
-  return make_float2(__fdividef(1.f, d.x), __fdividef(1.f, d.y));
+  const float2 d = __fadd2_rn(make_float2(ex2_approx(fminf(a.x, 57.f)), ex2_approx(fminf(a.y, 57.f))),
+                              make_float2(1.f, 1.f));
+  const float r = __fdividef(1.f, d.x * d.y);
+  return __fmul2_rn(make_float2(d.y, d.x), make_float2(r, r));
 }
 
 // Activation and store of W consecutive output columns of one token row: log

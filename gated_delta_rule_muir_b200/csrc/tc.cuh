@@ -46,7 +46,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Wait for the phase with the given parity to complete. Bounded: gives up once
 // limit_ns of global time have passed since the first check, records the
-// timeout in the device status word and returns false.
+// timeout in the device status word and returns false. Each try may suspend the
+// thread in hardware for up to 20 us (it resumes as soon as the phase completes),
+// so a waiting warp does not spin on the issue slots other warps need.
 __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   uint64_t t0 = 0;
@@ -54,13 +56,13 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, ui
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(a), "r"(parity)
         : "memory");
     if (ok) return true;
-    if ((it & 63) == 0) {
+    if ((it & 3) == 0) {
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) t0 = now;
       else if (now - t0 > limit_ns) { flag_timeout(); return false; }
