@@ -67,9 +67,10 @@ __device__ __forceinline__ float2 sigmoid2(float2 u) {
 }
 
 // Activation and store of W consecutive output columns of one token row: log
-// sigmoid into log_alpha (gate 0, fp32), sigmoid into the bf16 gates.
+// sigmoid into log_alpha (gate 0, fp32), sigmoid into the bf16 gates. The values
+// come by reference to a fixed-size array so that they stay in registers.
 template <int W>
-__device__ __forceinline__ void emit_gate_w(const GateParams& p, int j, const float* v, int64_t o);
+__device__ __forceinline__ void emit_gate_w(const GateParams& p, int j, const float (&v)[W], int64_t o);
 
 // Two log sigmoids, log sigmoid(u) = min(u, 0) - log1p(exp(-|u|)), paired where
 // the operations allow; log1p(y) is formed as y * log(1 + y) / ((1 + y) - 1),
@@ -101,7 +102,7 @@ __device__ __forceinline__ float2 log_sigmoid2(float2 u) {
 //   acc_full[b]  output buffer b computed            (MMA commit -> epilogue)
 //   acc_empty[b] output buffer b read out            (16 epilogue warps -> MMA)
 template <int W>
-__device__ __forceinline__ void emit_gate_w(const GateParams& p, int j, const float* v, int64_t o) {
+__device__ __forceinline__ void emit_gate_w(const GateParams& p, int j, const float (&v)[W], int64_t o) {
   if (j == 0) {
     float* dst = p.log_alpha + o;
 #pragma unroll
@@ -124,10 +125,6 @@ __device__ __forceinline__ void emit_gate_w(const GateParams& p, int j, const fl
       *reinterpret_cast<uint4*>(dst + q8) = pk;
     }
   }
-}
-__device__ __forceinline__ void emit_gate(const GateParams& p, int j, const float* v, int W, int64_t o) {
-  if (W == 16) emit_gate_w<16>(p, j, v, o);
-  else emit_gate_w<32>(p, j, v, o);
 }
 
 constexpr int kGtEpiWarps = 16;
@@ -178,11 +175,16 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
   if (warp == 0) {
     // ---- TMA producer: the down-projection stages, then the U chunks -------
     if (lane_id == 0) {
-      int use[2] = {0, 0};
+      // phase bookkeeping in registers (bit s: parity of stage s's next wait;
+      // a dynamically indexed array would live in local memory)
+      uint32_t used = 0, eph = 0;  // used: bit s once stage s has been filled
       bool ok = true;
-      auto acquire = [&](int s) {  // wait until stage s is free, then announce its bytes
-        if (use[s] > 0) ok = mbar_wait(&empty[s], (uint32_t)(use[s] - 1) & 1u);
-        ++use[s];
+      auto acquire = [&](int s) {  // wait until stage s is free
+        if ((used >> s) & 1u) {
+          ok = mbar_wait(&empty[s], (eph >> s) & 1u);
+          eph ^= 1u << s;
+        }
+        used |= 1u << s;
         return ok;
       };
       int i = 0;  // stage counter
@@ -210,14 +212,15 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
   } else if (warp == 1) {
     // ---- MMA issuer ----------------------------------------------------------
     if (lane_id == 0) {
-      int fuse[2] = {0, 0};   // uses of each stage's full barrier
-      int buse[2] = {0, 0};   // uses of each TMEM output buffer
+      uint32_t fph = 0;               // bit s: parity of stage s's next full wait
+      uint32_t bused = 0, bph = 0;    // bit b: buffer b has been filled / parity of its next drain wait
       bool ok = true;
       int i = 0;
       const uint32_t id1 = idesc_bf16(128, 256, 0, 1);
       for (int ks = 0; ks < nk && ok; ++ks, ++i) {
         const int s = i & 1;
-        ok = mbar_wait(&full[s], (uint32_t)fuse[s]++ & 1u);
+        ok = mbar_wait(&full[s], (fph >> s) & 1u);
+        fph ^= 1u << s;
         if (!ok) break;
         tc_fence_after();
         const uint32_t st = base + (uint32_t)s * kGtStage;
@@ -232,9 +235,10 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
         mma_commit(&empty[s]);
       }
       if (ok) mma_commit(&h_full);
-      // wait until the given buffer's previous contents have been read out
+      // wait until the given buffer's last contents have been read out (a wait on
+      // a phase that has already completed returns at once, so asking twice is fine)
       auto buffer_free = [&](int b) {
-        if (buse[b] > 0) return mbar_wait(&acc_empty[b], (uint32_t)(buse[b] - 1) & 1u);
+        if ((bused >> b) & 1u) return mbar_wait(&acc_empty[b], (bph >> b) & 1u);
         return true;
       };
       int q = 0;  // output chunk counter (buffer q & 1)
@@ -250,7 +254,9 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
           ok = buffer_free(0) && buffer_free(1);
           for (int c = 0; c < nchunk && ok; ++c, ++i, ++q) {
             const int s = i & 1, b = q & 1;
-            ok = mbar_wait(&full[s], (uint32_t)fuse[s]++ & 1u) && buffer_free(b);
+            ok = mbar_wait(&full[s], (fph >> s) & 1u);
+            fph ^= 1u << s;
+            ok = ok && buffer_free(b);
             if (!ok) break;
             tc_fence_after();
             const uint32_t st = base + (uint32_t)s * kGtStage;
@@ -264,7 +270,9 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
             }
             mma_commit(&empty[s]);
             mma_commit(&acc_full[b]);
-            ++buse[b];
+            // bit b of bph: parity of the drain of b's latest fill (fill k is drained in phase k)
+            if ((bused >> b) & 1u) bph ^= 1u << b;
+            bused |= 1u << b;
           }
         }
         if (ok) mma_commit(&ah_empty);  // the group's MMAs done: the h tile may be rewritten
@@ -282,7 +290,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
     bool ok = mbar_wait(&h_full, 0u);
     tc_fence_after();
     int q = 0;
-    int afull[2] = {0, 0};
+    uint32_t aph = 0;  // bit b: parity of buffer b's next full wait
     for (int g = 0; g < 4 && ok; ++g) {
       if (g > 0) {
         ok = mbar_wait(&ah_empty, (uint32_t)(g - 1) & 1u);
@@ -316,7 +324,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
         const int nch = gt_nch(j), O = O_of(j), nchunk = O / nch, W = nch / 4;
         for (int c = 0; c < nchunk; ++c, ++q) {
           const int b = q & 1;
-          ok = mbar_wait(&acc_full[b], (uint32_t)afull[b]++ & 1u);
+          ok = mbar_wait(&acc_full[b], (aph >> b) & 1u);
+          aph ^= 1u << b;
           if (!ok) break;
           tc_fence_after();
           const uint32_t acc = tmem + lane + (uint32_t)(b * nch + grp * W);
@@ -327,7 +336,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
             tc_fence_before();
             __syncwarp();
             if (lane_id == 0) mbar_arrive(&acc_empty[b]);
-            if (on) emit_gate(p, j, v, 16, o);
+            if (on) emit_gate_w<16>(p, j, v, o);
           } else {
             for (int h32 = 0; h32 < W; h32 += 32) {
               float v[32];
@@ -337,7 +346,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gate_proj_tma_kernel(const __gr
                 __syncwarp();
                 if (lane_id == 0) mbar_arrive(&acc_empty[b]);
               }
-              if (on) emit_gate(p, j, v, 32, o + h32);
+              if (on) emit_gate_w<32>(p, j, v, o + h32);
             }
           }
         }
