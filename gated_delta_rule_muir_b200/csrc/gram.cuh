@@ -53,6 +53,23 @@ __device__ __forceinline__ void put_row(const Tile& t, int m, int k8, const floa
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// v[j] <- v[j ^ pm] for a run-time pm in [0, 8), by three stages of conditional
+// swaps with fixed indices (an index computed at run time would put v in local
+// memory).
+__device__ __forceinline__ void xor_permute8(float (&v)[8], int pm) {
+#pragma unroll
+  for (int bit = 1; bit < 8; bit <<= 1) {
+    const bool sw = (pm & bit) != 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j & bit) continue;
+      const float a = v[j], c = v[j | bit];
+      v[j] = sw ? c : a;
+      v[j | bit] = sw ? a : c;
+    }
+  }
+}
+
 // 2^x for x <= 0 with the hardware's approximate base-2 exponential (relative
 // error near 2^-22); results below the normal range flush to 0, the correct
 // limit of a product of decays that underflows.
@@ -117,9 +134,7 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
   const int sg = tid / nb, sJ = tid % nb;
   const bool stager = sg < G;
   const int c8 = sg * 8;
-  float rv[8];
   if (stager) {
-    ld8f(p.r + (int64_t)s.h * DK + c8, rv);
     // totals of the 8-block in log2 units
     float acc[8];
 #pragma unroll
@@ -169,9 +184,8 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
     const T* x2p = upper && gp ? gp : kp;            // g, or a stand-in that is not used
     const bool use_g = upper && gp != nullptr;
     const Tile dst = upper ? XL : YL;
-    float rl[8];  // r (a register copy: the lambda captures rv by reference)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) rl[j] = rv[j];
+    float rl[8];  // r of these channels (loaded here: an array captured by the lambda would live in local memory)
+    ld8f(p.r + (int64_t)s.h * DK + c8, rl);
     float run[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) run[j] = 0.f;
@@ -244,10 +258,8 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
       if (on) {
         const int Jl = ((P - b) >> 3) + (cq >> 3);  // the lower 8-block of these columns
         const int pm = (Jl & 7) ^ 7;                 // a lower block
-        float o8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) o8[j] = v[j ^ pm];
-        sq_put(out + (2 * X + wg) * sq_bytes(Cs), Cs, t, P - b + cq, o8);
+        xor_permute8(v, pm);  // v[j] <- v[j ^ pm]
+        sq_put(out + (2 * X + wg) * sq_bytes(Cs), Cs, t, P - b + cq, v);
       }
     }
   };
