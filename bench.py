@@ -381,9 +381,10 @@ def bench_forwards(dev, steps, warmup, pk):
     return out
 
 
-def bench_decode(dev, steps, warmup, pk):
+def bench_decode(dev, steps, warmup, pk, graph=True):
     """Decode GB/s of one token through all 24 layers: one launch over the 24 x batch
-    rows (per-row readout scale), and a CUDA graph of 24 per-layer launches."""
+    rows (per-row readout scale), and (graph=True) a CUDA graph of 24 per-layer
+    launches."""
     import torch
     import gated_delta_rule_muir_b200 as muir
     out = {}
@@ -405,8 +406,16 @@ def bench_decode(dev, steps, warmup, pk):
         fn = lambda: muir.decode_step(S, q, k, v, e, w, gg, z, la, r, y=y)
         for _ in range(max(warmup, 3)):
             fn()
-        reps = max(steps, 20)
+        reps = max(steps, 20) if graph else steps
         ms = time_steps(fn, reps, False) / reps
+        state_bytes = 2.0 * n * H * dk * dv * 4
+        io_bytes = n * H * (5 * dk * 2 + dk * 4 + dk * 4 + 3 * dv * 2 + dv * 2)
+        gbs = (state_bytes + io_bytes) / (ms * 1e-3) / 1e9
+        if not graph:
+            out[f"batch{nb}"] = {"ms_per_token": round(ms, 4), "GB_s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 3),
+                                 "state_MB": round(n * H * dk * dv * 4 / 1e6, 1)}
+            del S, q, k, v, e, gg, w, z, la, r, y
+            continue
         # the same token as a CUDA graph of 24 per-layer launches (batch rows each)
         sl = [slice(l * nb, (l + 1) * nb) for l in range(L)]
         layer_calls = lambda: [muir.decode_step(S[i], q[i], k[i], v[i], e[i], w[i], gg[i], z[i], la[i], r[i], y=y[i])
@@ -423,9 +432,6 @@ def bench_decode(dev, steps, warmup, pk):
             graph.replay()
         ms_g = time_steps(graph.replay, reps, False) / reps
         del graph
-        state_bytes = 2.0 * n * H * dk * dv * 4
-        io_bytes = n * H * (5 * dk * 2 + dk * 4 + dk * 4 + 3 * dv * 2 + dv * 2)
-        gbs = (state_bytes + io_bytes) / (ms * 1e-3) / 1e9
         gbs_g = (state_bytes + io_bytes) / (ms_g * 1e-3) / 1e9
         out[f"batch{nb}"] = {"ms_per_token": round(ms, 4), "GB_s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 3),
                              "graph24_ms_per_token": round(ms_g, 4), "graph24_GB_s": round(gbs_g, 1),
@@ -565,6 +571,9 @@ def main():
     ap.add_argument("--T", type=int, default=None, help="override the sequence length (profiling runs)")
     ap.add_argument("--fwd-only", action="store_true", help="time the forward pass only (profiling runs)")
     ap.add_argument("--gate-only", action="store_true", help="only the gate projection's measurement (profiling runs)")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="only the decode step at batch 1, 8, 64: W warm-up and K timed launches each, no graph "
+                         "(profiling runs)")
     args = ap.parse_args()
     if args.T:
         WL["T"] = args.T
@@ -591,6 +600,10 @@ def main():
     if args.gate_only:
         if rank == 0:
             print(json.dumps(bench_gate_proj(dev, args.steps, args.warmup, pk)))
+        return
+    if args.decode_only:
+        if rank == 0:
+            print(json.dumps(bench_decode(dev, args.steps, args.warmup, pk, graph=False)))
         return
     Step.fwd_only = args.fwd_only
     d = make_workload(dev)
