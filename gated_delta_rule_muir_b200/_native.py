@@ -5,14 +5,19 @@ import ctypes as C
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmuir.so")
+# MUIR_LIBRARY selects another in-tree build of the same library (the checking
+# build, libmuir_check.so, in its test); there is still no fallback.
+LIB_PATH = os.environ.get("MUIR_LIBRARY") or os.path.join(_PKG, "libmuir.so")
+CHECK_LIB_PATH = os.path.join(_PKG, "libmuir_check.so")
 
-MUIR_OK, MUIR_ERR_INVALID_ARG, MUIR_ERR_UNSUPPORTED, MUIR_ERR_WORKSPACE, MUIR_ERR_CUDA, MUIR_ERR_TIMEOUT = range(6)
+(MUIR_OK, MUIR_ERR_INVALID_ARG, MUIR_ERR_UNSUPPORTED, MUIR_ERR_WORKSPACE, MUIR_ERR_CUDA, MUIR_ERR_TIMEOUT,
+ MUIR_ERR_BOUNDS) = range(7)
 MUIR_F32, MUIR_BF16 = 0, 1
 MUIR_SAVE_FOR_BWD, MUIR_USE_SAVED = 1, 2
 
 ERROR_NAMES = {MUIR_ERR_INVALID_ARG: "invalid argument", MUIR_ERR_UNSUPPORTED: "unsupported",
-               MUIR_ERR_WORKSPACE: "workspace", MUIR_ERR_CUDA: "CUDA error", MUIR_ERR_TIMEOUT: "device timeout"}
+               MUIR_ERR_WORKSPACE: "workspace", MUIR_ERR_CUDA: "CUDA error", MUIR_ERR_TIMEOUT: "device timeout",
+               MUIR_ERR_BOUNDS: "bounds check"}
 
 vp = C.c_void_p
 

@@ -105,6 +105,9 @@ __device__ __forceinline__ SubIdx sub_of(const ChunkParams& p, int sid, int unit
 
 // Offset of element 0 of token `tok` of (b, h) in a [B,T,H,d] tensor.
 __device__ __forceinline__ int64_t toff(const ChunkParams& p, int b, int64_t tok, int h, int d) {
+#ifdef MUIR_CHECK
+  if (!check_bounds(b >= 0 && b < p.B && tok >= 0 && tok < p.T && h >= 0 && h < p.H, kStatusBoundsToken)) return 0;
+#endif
   return (((int64_t)b * p.T + tok) * p.H + h) * d;
 }
 
@@ -180,6 +183,9 @@ __device__ __forceinline__ void map_put_q(uint8_t* img, const MapGeom& g, int dk
 __host__ __device__ inline uint32_t sq_half(int Cs) { return 128u * (uint32_t)Cs * 2u; }
 __host__ __device__ inline uint32_t sq_bytes(int Cs) { return 2u * sq_half(Cs); }
 __device__ __forceinline__ void sq_put(uint8_t* img, int Cs, int r, int c8, const float (&x)[8]) {
+#ifdef MUIR_CHECK
+  if (!check_bounds(r >= 0 && r < Cs && c8 >= 0 && c8 + 8 <= Cs, kStatusBoundsImage)) return;
+#endif
   gput_k(img, sq_half(Cs), (uint32_t)Cs * 16u, r, c8, x);
 }
 // An image is lower block-triangular: in row group rg (rows 8 rg .. + 7) only
@@ -1281,7 +1287,7 @@ __global__ void __launch_bounds__(256, 1) out_kernel(ChunkParams p, const uint8_
   for (int j = 0; j < nq; ++j) {
     const int tt = j * 128 + t;
     const bool on = tt < ulen && drv.ok;
-    const int64_t yo = toff(p, b, (int64_t)n * ulen + tt, h, DV);
+    const int64_t yo = toff(p, b, (int64_t)n * ulen + (on ? tt : 0), h, DV);  // rows past the unit: unused
     Pack8<float> pa[NC][2];
     Pack8<T> pz[NC][2];
     if (on) {

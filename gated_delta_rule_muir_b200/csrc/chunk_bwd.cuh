@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   // dU -> dv = w dU and dw = v dU, straight into the gradients; this thread's w
   // and v pieces are loaded while the last product runs
   constexpr int NCH = DV / 32;  // 16-column chunks per thread
-  const int64_t vo = toff(p, s.b, s.tok0 + t, s.h, DV);
+  const int64_t vo = toff(p, s.b, s.tok0 + (t < Cs ? t : 0), s.h, DV);  // rows past the unit: unused
   Pack8<T> pw[NCH][2], pv[NCH][2];
   drv.run_overlap([&] { mma_tiles(cta.tmem + cU, AT, B3, Cs / 16, idT, NS, true); },
                   [&] {

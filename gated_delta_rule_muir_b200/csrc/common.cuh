@@ -13,8 +13,36 @@ namespace muir {
 __device__ unsigned int g_status;
 
 constexpr unsigned int kStatusTimeout = 1u;
+// a checking build found an index out of its bounds: a shared-memory address, a
+// (batch, token, head) index of an input or output tensor, a Gram image index
+constexpr unsigned int kStatusBoundsSmem = 2u, kStatusBoundsToken = 4u, kStatusBoundsImage = 8u;
+constexpr unsigned int kStatusBounds = kStatusBoundsSmem | kStatusBoundsToken | kStatusBoundsImage;
 
 __device__ __forceinline__ void flag_timeout() { atomicOr(&g_status, kStatusTimeout); }
+
+// Checking builds (-DMUIR_CHECK): the central access helpers test their indices,
+// and a failed test records kStatusBounds in the status word and skips (or
+// redirects to an in-bounds address) the access instead of trapping. Without
+// MUIR_CHECK the tests compile away.
+#ifdef MUIR_CHECK
+__device__ __forceinline__ bool check_bounds(bool ok, unsigned int what) {
+  if (!ok) atomicOr(&g_status, what);
+  return ok;
+}
+// Upper end of this CTA's shared-memory window, with 1 KB of slack for the
+// region the system reserves ahead of the kernel's own shared memory.
+__device__ __forceinline__ uint32_t smem_window_end() {
+  uint32_t n;
+  asm("mov.u32 %0, %%total_smem_size;" : "=r"(n));
+  return n + 1024u;
+}
+#define MUIR_SMEM_GUARD(addr, bytes) \
+  if (!::muir::check_bounds((uint32_t)(addr) + (uint32_t)(bytes) <= ::muir::smem_window_end(), \
+                            ::muir::kStatusBoundsSmem))                                          \
+  return
+#else
+#define MUIR_SMEM_GUARD(addr, bytes)
+#endif
 
 // ---- element access -----------------------------------------------------
 

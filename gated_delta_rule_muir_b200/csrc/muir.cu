@@ -92,7 +92,7 @@ bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 
 extern "C" {
 
-int muir_version(void) { return 102; }
+int muir_version(void) { return 103; }
 
 const char* muir_last_error(void) { return g_err.c_str(); }
 
@@ -104,6 +104,11 @@ int muir_device_status(void* stream) {
   if (cudaMemcpyFromSymbol(&host, muir::g_status, sizeof host) != cudaSuccess) return cuda_check("read status");
   if (cudaMemcpyToSymbol(muir::g_status, &zero, sizeof zero) != cudaSuccess) return cuda_check("clear status");
   if (host & muir::kStatusTimeout) return fail(MUIR_ERR_TIMEOUT, "a bounded device wait expired");
+  if (host & muir::kStatusBounds)
+    return fail(MUIR_ERR_BOUNDS, "an index failed its bounds check (checking build):%s%s%s",
+                (host & muir::kStatusBoundsSmem) ? " shared-memory address" : "",
+                (host & muir::kStatusBoundsToken) ? " tensor (batch, token, head) index" : "",
+                (host & muir::kStatusBoundsImage) ? " Gram image index" : "");
   return MUIR_OK;
 }
 

@@ -86,6 +86,7 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 // Copy `bytes` (multiple of 16, both addresses 16-byte aligned) from global to
 // shared memory; completes as transaction bytes on `bar`. No multicast.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  MUIR_SMEM_GUARD(dst, bytes);
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
@@ -209,6 +210,7 @@ __device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo
 // store with a memory clobber would serialise every staging loop). Ordering
 // with the tensor core is established by fence_async_smem() + a CTA barrier.
 __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
+  MUIR_SMEM_GUARD(addr, 16u);
   *reinterpret_cast<uint4*>(__cvta_shared_to_generic(addr)) = v;
 }
 

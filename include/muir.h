@@ -54,6 +54,8 @@ extern "C" {
 #define MUIR_ERR_WORKSPACE 3   /* workspace pointer NULL/misaligned or smaller than the query */
 #define MUIR_ERR_CUDA 4        /* a CUDA runtime call failed (launch, attribute) */
 #define MUIR_ERR_TIMEOUT 5     /* a bounded device wait expired (from muir_device_status) */
+#define MUIR_ERR_BOUNDS 6      /* checking builds (-DMUIR_CHECK) only: a device index failed its bounds
+                                  check; the access was skipped (from muir_device_status) */
 
 #define MUIR_F32 0
 #define MUIR_BF16 1
@@ -280,7 +282,8 @@ int muir_gate_proj(const void* x, const void* w_down, const void* u_decay, const
 
 /* Synchronises `stream`, then returns and clears the device-side status word:
  * MUIR_OK, or MUIR_ERR_TIMEOUT if a kernel's bounded wait expired since the
- * last call (that kernel's outputs are then invalid), or MUIR_ERR_CUDA. */
+ * last call (that kernel's outputs are then invalid), MUIR_ERR_BOUNDS (checking
+ * builds only) if an index failed its bounds check, or MUIR_ERR_CUDA. */
 int muir_device_status(void* stream);
 
 /* Message describing the last error on the calling thread ("" if none). */

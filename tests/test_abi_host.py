@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version(lib):
-    assert lib.muir_version() == 102
+    assert lib.muir_version() == 103
 
 
 def test_decode_rejects_null_and_bad_sizes(lib):
