@@ -57,8 +57,8 @@ def kernel_model(C, dk, dv, es):
     tri = C * C / 2
     m = {}
     m["decay"] = (0.0, C * dk * f4 + 4 * C * dk * f4)
-    # off-diagonal blocks (tensor cores) + the exact 16x16 diagonal blocks (CUDA cores)
-    m["gram"] = (4 * 2 * (tri - C * 8) * dk + 4 * 2 * C * 8.5 * dk,
+    # off-diagonal blocks (tensor cores) + the exact 8x8 diagonal blocks (CUDA cores)
+    m["gram"] = (4 * 2 * (tri - C * 4) * dk + 4 * 2 * C * 4.5 * dk,
                      4 * C * dk * es + 3 * C * dk * f4 + 4 * C * C * f4)
     m["solve"] = (C ** 3 / 3.0, 2 * C * C * f4)
     maps_fl = 2 * (tri * dk + tri * dv + tri * dv + C * dk * dk + tri * dk + 2 * tri * dv + 2 * C * dk * dv)
@@ -80,7 +80,7 @@ def kernel_model(C, dk, dv, es):
 def flop_split(C, dk, dv):
     """Modelled share of the step's flops issued on the tensor cores. The CUDA-core
     share counts every vector step of the kernels per unit (one chunk of one head):
-    the exact 16x16 diagonal Gram blocks (forward and backward), the 16x16 leaves of
+    the exact diagonal Gram blocks (8x8 forward, 16x16 backward), the 16x16 leaves of
     the triangular solve, the decay products, the elementwise decay scaling of the
     staged operands and epilogues, the state additions of the scans, the output
     gate, and the chain rule of the final backward kernel (an exponential counts as
@@ -90,7 +90,7 @@ def flop_split(C, dk, dv):
     m = kernel_model(C, dk, dv, 2)
     nb = C // 16
     alu = {
-        "diag_blocks": 4 * 2 * C * 8.5 * dk + 4 * 2 * 2 * C * 8.5 * dk,
+        "diag_blocks": 4 * 2 * C * 4.5 * dk + 4 * 2 * 2 * C * 8.5 * dk,
         "solve_leaves": nb * 16 * (16 * 15 / 2) * 2,
         "decay": 4 * C * dk,
         "operand_scaling": (12 + 8 + 3) * C * dk + 2.5 * (12 + 8 + 3) * C * dk,

@@ -502,11 +502,15 @@ __device__ __forceinline__ void tree_tables(const float* pre, float* ftab, int C
 // Staged for the halves asked for; 256 threads, BT tokens per thread per batch
 // with all loads of a batch issued before any is used. Pieces go by row_piece,
 // which keeps a thread on the same 8 channels throughout: rv holds r there.
-template <int DK, typename T>
+// The operand tiles are no-swizzle Tiles (put_k) or SwTiles (put_sw).
+__device__ __forceinline__ void put_op(const Tile& t, int r, int c8, const float (&x)[8]) { put_k(t, r, c8, x); }
+__device__ __forceinline__ void put_op(const SwTile& t, int r, int c8, const float (&x)[8]) { put_sw(t, r, c8, x); }
+
+template <int DK, typename T, typename OpTile>
 __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& s, const float* pre,
                                             const float* suf, const float* ft, const float (&rv)[8], int Cs,
-                                            int lb, bool want_upper, bool want_lower, const Tile& XL,
-                                            const Tile& YL) {
+                                            int lb, bool want_upper, bool want_lower, const OpTile& XL,
+                                            const OpTile& YL) {
   constexpr int NT = 256;
   constexpr int BT = sizeof(T) == 2 ? 4 : 2;
   const int b = 1 << lb;
@@ -551,9 +555,9 @@ __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& 
           s1[j] *= s2[j] * (upper ? rv[j] : 1.f) * f;  // r g q or e k
           kk[j] *= f;
         }
-        const Tile& dst = upper ? XL : YL;
-        put_k(dst, (pv << (lb + 1)) + r, c8, kk);
-        put_k(dst, (pv << (lb + 1)) + b + r, c8, s1);
+        const OpTile& dst = upper ? XL : YL;
+        put_op(dst, (pv << (lb + 1)) + r, c8, kk);
+        put_op(dst, (pv << (lb + 1)) + b + r, c8, s1);
       }
     }
   }

@@ -579,7 +579,7 @@ __host__ __device__ constexpr size_t bwd_gram_front_bytes() {
 }
 template <int DK>
 __host__ __device__ constexpr size_t bwd_gram_smem_bytes() {
-  return bwd_gram_front_bytes<DK>() + 8u * SB * SB * 16u + (size_t)kMaxLev * 8u * DK * 4u;
+  return 1024u + bwd_gram_front_bytes<DK>() + 8u * SB * SB * 16u + (size_t)kMaxLev * 8u * DK * 4u;
 }
 
 template <int DK, typename T, int NS>
@@ -592,20 +592,28 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
-  const uint32_t base = smem_u32(sm);
+  const uint32_t base = (smem_u32(sm) + 1023u) & ~1023u;  // swizzled tiles start on 1024-byte boundaries
+  uint8_t* const sma = sm + (base - smem_u32(sm));
   constexpr uint32_t OB = 128u * DK * 2u;        // operand tile (128 token rows x dk), one half
   const uint32_t GB = 128u * (uint32_t)Cs * 2u;  // dG tile (128 rows x Cs), one half
-  const Tile OP{base, base + OB, 128u, DK * 16u};  // YL (left phase) or XL (right phase)
+  // YL (left phase) or XL (right phase): token rows, read as the MN-major A
+  // operand (M = key channel, K = token). With dk a multiple of 64 the rows are
+  // 128-byte swizzled, so that the row-major staging sweep stores without bank
+  // conflicts; with dk = 32 (rows of 64 bytes) they stay in the no-swizzle layout.
+  using OpTile = std::conditional_t<(DK % 64 == 0), SwTile, Tile>;
+  OpTile OP;
+  if constexpr (DK % 64 == 0) OP = SwTile{base, base + OB, 128u * 128u};
+  else OP = Tile{base, base + OB, 128u, DK * 16u};
   const Tile GT{base + 2 * OB, base + 2 * OB + GB, 128u, (uint32_t)Cs * 16u};
   constexpr size_t FB = bwd_gram_front_bytes<DK>();
-  float4* dgd = reinterpret_cast<float4*>(sm + FB);  // [nb][16 t][16 s]: mkk, mka, nqk, nqa
-  float* ftab = reinterpret_cast<float*>(sm + FB + 8 * SB * SB * 16);  // [kMaxLev][nb][DK]
+  float4* dgd = reinterpret_cast<float4*>(sma + FB);  // [nb][16 t][16 s]: mkk, mka, nqk, nqa
+  float* ftab = reinterpret_cast<float*>(sma + FB + 8 * SB * SB * 16);  // [kMaxLev][nb][DK]
   constexpr bool kRowsInSmem = sizeof(T) == 2;
   constexpr uint32_t RB = 128u * DK * 2u;  // one bf16 [128][DK] array of raw rows
-  const T* rk = reinterpret_cast<const T*>(sm);
-  const T* rz1 = reinterpret_cast<const T*>(sm + RB);
-  const T* rz2 = reinterpret_cast<const T*>(sm + 2 * RB);
-  const float* rla = reinterpret_cast<const float*>(sm + 3 * RB);
+  const T* rk = reinterpret_cast<const T*>(sma);
+  const T* rz1 = reinterpret_cast<const T*>(sma + RB);
+  const T* rz2 = reinterpret_cast<const T*>(sma + 2 * RB);
+  const float* rla = reinterpret_cast<const float*>(sma + 3 * RB);
   uint32_t cp_phase = 0;
   if (tid == 0) mbar_init(&bar_cp, 1);
   TcCta cta;
@@ -679,7 +687,10 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
       stage_g(lb);
       stage_level<DK, T>(p, s, pre, suf, ftab + lev * nb * DK, rv, Cs, lb, side == 1, side == 0, OP, OP);
       drv.run([&] {
-        mma_tiles(cta.tmem + 128 * lev, transposed(OP), side == 0 ? GT : transposed(GT), Cs / 16, id, NS, false);
+        if constexpr (DK % 64 == 0)
+          mma_tiles_swa(cta.tmem + 128 * lev, OP, side == 0 ? GT : transposed(GT), Cs / 16, id, NS, false);
+        else
+          mma_tiles(cta.tmem + 128 * lev, transposed(OP), side == 0 ? GT : transposed(GT), Cs / 16, id, NS, false);
       });
     }
     if (!drv.ok) break;

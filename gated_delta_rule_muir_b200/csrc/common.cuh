@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace muir {
 
 // Device-side status word: bit 0 = a bounded wait expired. Read and cleared by

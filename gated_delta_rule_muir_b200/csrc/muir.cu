@@ -229,14 +229,17 @@ int muir_selftest_wait(uint64_t limit_ns, int32_t arrive, int32_t* out, void* st
 }
 
 // Diagnostic entry point: D[128,N] = A[128,K] B[K,N] (bf16 A and B row-major,
-// fp32 D) through 128-byte-swizzled operand tiles, loaded by TMA (use_tma) or
-// by the threads. K in {64, 128}, N in {64, 128, 256}.
-int muir_selftest_sw128(const void* A, const void* B, float* D, int32_t N, int32_t K, int32_t use_tma, void* stream) {
+// fp32 D) through 128-byte-swizzled operand tiles, loaded by TMA (mode 1) or by
+// the threads (mode 0; mode 2 with A stored as the MN-major operand). K in
+// {64, 128}, N in {64, 128, 256}.
+int muir_selftest_sw128(const void* A, const void* B, float* D, int32_t N, int32_t K, int32_t mode, void* stream) {
   g_err.clear();
   if (!A || !B || !D) return fail(MUIR_ERR_INVALID_ARG, "selftest_sw128: NULL pointer");
   if ((K != 64 && K != 128) || (N != 64 && N != 128 && N != 256))
     return fail(MUIR_ERR_UNSUPPORTED, "selftest_sw128: N=%d K=%d", N, K);
   if (!aligned16(A) || !aligned16(B)) return fail(MUIR_ERR_INVALID_ARG, "selftest_sw128: misaligned pointer");
+  if (mode < 0 || mode > 2) return fail(MUIR_ERR_INVALID_ARG, "selftest_sw128: mode %d", mode);
+  const bool use_tma = mode == 1;
   CUtensorMap ta{}, tb{};
   if (use_tma && (!muir_host::make_tmap_bf16(&ta, A, 128, K, K, 128) ||
                   !muir_host::make_tmap_bf16(&tb, B, K, N, N, (uint32_t)K)))
@@ -247,7 +250,7 @@ int muir_selftest_sw128(const void* A, const void* B, float* D, int32_t N, int32
     return cuda_check("selftest_sw128 attribute");
   Launch L_("selftest_sw128", static_cast<cudaStream_t>(stream));
   muir::selftest_sw128_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
-      ta, tb, static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), D, N, K, use_tma);
+      ta, tb, static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), D, N, K, mode);
   return cuda_check("selftest_sw128 launch");
 }
 

@@ -102,13 +102,16 @@ __global__ void __launch_bounds__(32) selftest_wait_kernel(uint64_t limit_ns, in
 
 // D[128, N] = A[128, K] B[K, N], bf16 A (row-major: the K-major operand) and B
 // (row-major [K][N]: the MN-major operand), through 128-byte-swizzled shared
-// memory filled by TMA boxes (use_tma) or by the threads in the same layout.
-// K in {64, 128}; N in {64, 128, 256}. One CTA of 128 threads.
+// memory filled by TMA boxes (mode 1) or by the threads in the same layout
+// (mode 0). Mode 2 has the threads store A transposed, as the MN-major operand:
+// rows = K, 64-column boxes along M (the layout of a token-major tile read as
+// the A operand of a product over tokens). K in {64, 128}; N in {64, 128, 256}.
+// One CTA of 128 threads.
 __global__ void __launch_bounds__(128) selftest_sw128_kernel(const __grid_constant__ CUtensorMap ta,
                                                              const __grid_constant__ CUtensorMap tb,
                                                              const __nv_bfloat16* __restrict__ A,
                                                              const __nv_bfloat16* __restrict__ B, float* __restrict__ D,
-                                                             int N, int K, int use_tma) {
+                                                             int N, int K, int mode) {
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ uint64_t bar, bar_cp;
   __shared__ uint32_t tslot;
@@ -126,7 +129,7 @@ __global__ void __launch_bounds__(128) selftest_sw128_kernel(const __grid_consta
   tc_fence_after();
   const uint32_t tmem = tslot;
   bool ok = true;
-  if (use_tma) {
+  if (mode == 1) {
     if (tid == 0) {
       mbar_expect_tx(&bar_cp, (uint32_t)(K / 64) * 16384u + (uint32_t)(N / 64) * (uint32_t)K * 128u);
       for (int a = 0; a < K / 64; ++a) tma_load_2d(base + a * 16384u, &ta, 64 * a, 0, &bar_cp);
@@ -134,10 +137,21 @@ __global__ void __launch_bounds__(128) selftest_sw128_kernel(const __grid_consta
     }
     ok = __syncthreads_and(mbar_wait(&bar_cp, 0) ? 1 : 0) != 0;
   } else {
-    for (int idx = tid; idx < 128 * (K / 8); idx += 128) {
-      const int m = idx / (K / 8), c = idx % (K / 8);
-      const uint4 v = *reinterpret_cast<const uint4*>(A + (int64_t)m * K + 8 * c);
-      sts128(base + (uint32_t)(c / 8) * 16384u + (uint32_t)m * 128u + (uint32_t)(((c % 8) ^ (m & 7)) * 16), v);
+    if (mode == 2) {
+      for (int idx = tid; idx < K * 16; idx += 128) {  // row k of A^T: 16 pieces of 8 values of m
+        const int k = idx / 16, c = idx % 16;
+        __align__(16) __nv_bfloat16 e[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) e[j] = A[(int64_t)(8 * c + j) * K + k];
+        sts128(base + (uint32_t)(c / 8) * K * 128u + (uint32_t)k * 128u + (uint32_t)(((c % 8) ^ (k & 7)) * 16),
+               *reinterpret_cast<const uint4*>(e));
+      }
+    } else {
+      for (int idx = tid; idx < 128 * (K / 8); idx += 128) {
+        const int m = idx / (K / 8), c = idx % (K / 8);
+        const uint4 v = *reinterpret_cast<const uint4*>(A + (int64_t)m * K + 8 * c);
+        sts128(base + (uint32_t)(c / 8) * 16384u + (uint32_t)m * 128u + (uint32_t)(((c % 8) ^ (m & 7)) * 16), v);
+      }
     }
     for (int idx = tid; idx < K * (N / 8); idx += 128) {
       const int k = idx / (N / 8), c = idx % (N / 8);
@@ -149,9 +163,10 @@ __global__ void __launch_bounds__(128) selftest_sw128_kernel(const __grid_consta
   }
   if (ok && tid == 0) {
     tc_fence_after();
-    const uint32_t id = idesc_bf16(128, N, 0, 1);
+    const uint32_t id = idesc_bf16(128, N, mode == 2 ? 1 : 0, 1);
     for (int ks = 0; ks < K / 16; ++ks) {
-      const uint64_t ad = sdesc_sw128(base + (uint32_t)(ks / 4) * 16384u + (uint32_t)(ks % 4) * 32u, 16u, 1024u);
+      const uint64_t ad = mode == 2 ? sdesc_sw128(base + (uint32_t)ks * 2048u, (uint32_t)K * 128u, 1024u)
+                                    : sdesc_sw128(base + (uint32_t)(ks / 4) * 16384u + (uint32_t)(ks % 4) * 32u, 16u, 1024u);
       const uint64_t bd = sdesc_sw128(bbase + (uint32_t)ks * 2048u, (uint32_t)K * 128u, 1024u);
       mma_bf16(tmem, ad, bd, id, ks > 0 ? 1u : 0u);
     }

@@ -140,6 +140,20 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
          (1ull << 46);
 }
 
+// Shared-memory matrix descriptor with the 128-byte swizzle (layout type 2),
+// sm_100 version bit; the tile base must be 1024-byte aligned. Rows are 128
+// bytes (64 bf16), the 16-byte chunk c of row r stored at chunk c ^ (r % 8).
+//   K-major operand (rows = M or N, columns = K): SBO = 1024 between 8-row
+//     groups; the K step of 16 elements adds 32 bytes inside the row, and every
+//     64 columns of K start a new box of rows.
+//   MN-major operand (rows = K, columns = M or N): SBO = 1024 between 8-row
+//     groups along K, LBO = the distance between 64-column boxes along M/N; the
+//     K step of 16 rows adds 2048 bytes.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+
 // ---- MMA issue (single thread) ---------------------------------------------
 
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
@@ -190,6 +204,33 @@ __device__ __forceinline__ void mma_tiles(uint32_t d_tmem, const Tile& A, const 
   }
 }
 
+// A staged operand in 128-byte-swizzled rows: bf16 hi and lo planes (each
+// 1024-byte aligned), row r of the matrix in 64-column boxes `box` bytes apart.
+// Written row by row (put_sw), it is read here as the MN-major operand (rows =
+// K): a sweep whose 8 threads per shared-memory phase store 8 consecutive
+// 16-byte pieces of one row lands them in 8 distinct bank groups.
+struct SwTile {
+  uint32_t hi, lo;
+  uint32_t box;
+};
+
+// D[tmem] (+)= A * B over `ksteps` steps of K = 16, A an MN-major SwTile (M =
+// its columns, K = its rows), B a no-swizzle Tile; nsplit as in mma_tiles.
+__device__ __forceinline__ void mma_tiles_swa(uint32_t d_tmem, const SwTile& A, const Tile& B, int ksteps,
+                                              uint32_t idesc, int nsplit, bool accumulate) {
+  for (int j = 0; j < ksteps; ++j) {
+    const uint32_t oa = j * 2048u, ob = j * 2u * B.lbo;
+    const uint64_t ah = sdesc_sw128(A.hi + oa, A.box, 1024u), bh = sdesc(B.hi + ob, B.lbo, B.sbo);
+    mma_bf16(d_tmem, ah, bh, idesc, (accumulate || j > 0) ? 1u : 0u);
+    if (nsplit == 3) {
+      mma_bf16(d_tmem, ah, sdesc(B.lo + ob, B.lbo, B.sbo), idesc, 1u);
+      mma_bf16(d_tmem, sdesc_sw128(A.lo + oa, A.box, 1024u), bh, idesc, 1u);
+    } else if (nsplit == 2) {
+      mma_bf16(d_tmem, sdesc_sw128(A.lo + oa, A.box, 1024u), bh, idesc, 1u);
+    }
+  }
+}
+
 // ---- operand staging (any thread) ------------------------------------------
 
 __device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
@@ -212,6 +253,15 @@ __device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo
 __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
   MUIR_SMEM_GUARD(addr, 16u);
   *reinterpret_cast<uint4*>(__cvta_shared_to_generic(addr)) = v;
+}
+
+// Row r, columns c8..c8+7 of a SwTile.
+__device__ __forceinline__ void put_sw(const SwTile& t, int r, int c8, const float (&x)[8]) {
+  uint4 hi, lo;
+  split8(x, hi, lo);
+  const uint32_t off = (uint32_t)(c8 >> 6) * t.box + (uint32_t)r * 128u + ((uint32_t)(((c8 >> 3) & 7) ^ (r & 7)) << 4);
+  sts128(t.hi + off, hi);
+  sts128(t.lo + off, lo);
 }
 
 // K-major (natural view, lbo = 128): 8 consecutive contraction indices k8..k8+7 of MN row m.

@@ -23,13 +23,6 @@
 
 namespace muir {
 
-// Shared-memory matrix descriptor with the 128-byte swizzle (layout type 2),
-// sm_100 version bit; the tile base must be 1024-byte aligned.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
-         (1ull << 46) | (2ull << 61);
-}
-
 // One 2-D box of `tmap` at element coordinates (x = column, y = row) into shared
 // memory at dst, completing as transaction bytes on bar. x * 2 bytes must be a
 // multiple of 16 (x a multiple of 8 for bf16).

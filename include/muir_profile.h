@@ -26,10 +26,11 @@
  * receives 1 if the wait saw the phase complete, else 0.
  *
  * muir_selftest_sw128(): D[128,N] = A[128,K] * B[K,N] with bf16 A and B
- * (row-major device buffers) and fp32 D, through the 128-byte-swizzled operand
- * tiles of the TMA-fed kernels: A as the K-major operand, B as the MN-major
- * one, loaded by TMA boxes (use_tma != 0) or written by the threads in the same
- * layout. K in {64, 128}, N in {64, 128, 256}.
+ * (row-major device buffers) and fp32 D, through 128-byte-swizzled operand
+ * tiles: A as the K-major operand and B as the MN-major one, loaded by TMA boxes
+ * (mode 1) or written by the threads in the same layout (mode 0); mode 2 has the
+ * threads store A transposed, as the MN-major operand (rows = K). K in {64, 128},
+ * N in {64, 128, 256}; another mode is MUIR_ERR_INVALID_ARG.
  */
 #ifndef MUIR_PROFILE_H
 #define MUIR_PROFILE_H
@@ -50,7 +51,7 @@ int64_t muir_launch_count(void);
 int muir_selftest_gemm(const float* A, const float* B, float* D, int32_t N, int32_t K, int32_t a_mode,
                        int32_t b_mode, int32_t nsplit, void* stream);
 int muir_selftest_wait(uint64_t limit_ns, int32_t arrive, int32_t* out, void* stream);
-int muir_selftest_sw128(const void* A, const void* B, float* D, int32_t N, int32_t K, int32_t use_tma, void* stream);
+int muir_selftest_sw128(const void* A, const void* B, float* D, int32_t N, int32_t K, int32_t mode, void* stream);
 
 #ifdef __cplusplus
 }

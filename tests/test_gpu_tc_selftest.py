@@ -31,12 +31,15 @@ def test_selftest_gemm(cuda_ok, a_mn, b_mn, N_, K, nsplit):
     assert err < (1e-2 if nsplit == 1 else 5e-5), err
 
 
-@pytest.mark.parametrize("use_tma", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1, 2])
 @pytest.mark.parametrize("N_,K", [(64, 64), (128, 64), (256, 128), (64, 128)])
-def test_selftest_sw128(cuda_ok, use_tma, N_, K):
-    """128-byte-swizzled operands: A K-major, B MN-major, written by the threads or
-    loaded by TMA boxes. bf16 products are exact, so only the fp32 accumulation
-    order separates the result from the fp64 matmul of the same bf16 values."""
+def test_selftest_sw128(cuda_ok, mode, N_, K):
+    """128-byte-swizzled operands: A K-major, B MN-major, written by the threads
+    (mode 0) or loaded by TMA boxes (mode 1); mode 2 stores A transposed and reads
+    it as the MN-major operand. bf16 products are exact, so only the fp32
+    accumulation order separates the result from the fp64 matmul of the same bf16
+    values."""
+    use_tma = mode
     lib = N.load()
     g = torch.Generator().manual_seed(7 * N_ + K + 1000 * use_tma)
     A = torch.randn(128, K, generator=g).bfloat16()
