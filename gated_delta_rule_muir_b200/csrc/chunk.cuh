@@ -684,8 +684,15 @@ __global__ void __launch_bounds__(256, 1) solve_kernel(ChunkParams p) {
 //   phase 2: Phi -> 384, Psi -> 128 (Z consumed)
 //   phase 3: Oloc -> 256 (Ut consumed), Q' -> 0 (W consumed)
 // Shared memory: one A tile and two MN-major B tiles (128 x 128 bf16 hi+lo
-// each). Negated operands are staged negated.
+// each). Negated operands are staged negated. The MN-major tiles the threads
+// stage (B1, B2, and A when it holds (X*Gsuf)^T) leave 16 bytes between the
+// 8-column blocks (SBO = Cs*16 + 16): the staging sweep reads token rows whole,
+// and the 8 threads of a shared-memory phase, which store 8 consecutive column
+// blocks of one row, then land in 8 distinct bank groups.
 // ---------------------------------------------------------------------------
+constexpr uint32_t kMapsPlane = 128u * 128u * 2u + 16u * 16u;  // one padded bf16 plane, at most 16 column blocks
+constexpr size_t maps_smem_bytes() { return 6u * kMapsPlane; }
+
 template <int DK, int DV, typename T, int NS>
 __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   extern __shared__ __align__(128) uint8_t sm[];
@@ -695,15 +702,18 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
-  constexpr uint32_t TBY = 128u * 128u * 2u;
+  constexpr uint32_t TBP = kMapsPlane;
+  static_assert(DK <= 128 && DV <= 128, "maps tiles hold at most 16 column blocks");
   const uint32_t base = smem_u32(sm);
   const uint32_t kstride = (uint32_t)Cs * 16u;  // every tile here contracts over the Cs tokens
+  const uint32_t kpad = kstride + 16u;          // column-block stride of the thread-staged tiles
   const uint32_t H = sq_half(Cs);
-  const Tile A{base, base + H, 128u, kstride};  // bulk-copied Gram / T image, or a staged operand
-  const Tile B1{base + 2 * TBY, base + 3 * TBY, 128u, kstride};
-  const Tile B2{base + 4 * TBY, base + 5 * TBY, 128u, kstride};
+  const Tile A{base, base + H, 128u, kstride};  // bulk-copied Gram / T image
+  const Tile As{base, base + TBP, 128u, kpad};  // the same memory holding a staged (X*Gsuf)^T
+  const Tile B1{base + 2 * TBP, base + 3 * TBP, 128u, kpad};
+  const Tile B2{base + 4 * TBP, base + 5 * TBP, 128u, kpad};
   if (tid == 0) mbar_init(&bar_cp, 1);
-  zero_smem(base + 2 * TBY, 4 * TBY);
+  zero_smem(base + 2 * TBP, 4 * TBP);
   TcCta cta;
   cta.init(&tslot, &bar, 512);
   const float* dec = p.dec + (int64_t)blockIdx.x * 4 * Cs * DK;
@@ -751,7 +761,7 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   };
   // (X * Gsuf)^T as an MN-major A operand (M = channel, K = token), X = k or e k, scaled by sign.
   auto stage_suffixed = [&](bool erase, float sign) {
-    stage_prod<T, true, DK>(A, p, s, Cs, static_cast<const T*>(p.k), erase ? static_cast<const T*>(p.e) : nullptr,
+    stage_prod<T, true, DK>(As, p, s, Cs, static_cast<const T*>(p.k), erase ? static_cast<const T*>(p.e) : nullptr,
                             gsuf, sign);
   };
   const uint32_t idK = idesc_bf16(128, DK, 0, 1), idV = idesc_bf16(128, DV, 0, 1);
@@ -788,11 +798,11 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   //   D_Phi = (A*Gsuf)^T W (Phi = Diag(Gam_C) - D_Phi in the epilogue), Psi = (A*Gsuf)^T (-Ut) + (K*Gsuf)^T U
   tmem_to_b(B1, cW, DK, 1.f);
   stage_suffixed(true, 1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cPhi, A, B1, Cs / 16, idKt, NS, false); });
+  drv.run([&] { mma_tiles(cta.tmem + cPhi, As, B1, Cs / 16, idKt, NS, false); });
   tmem_to_b(B1, cUt, DV, -1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B1, Cs / 16, idVt, NS, false); });
+  drv.run([&] { mma_tiles(cta.tmem + cPsi, As, B1, Cs / 16, idVt, NS, false); });
   stage_suffixed(false, 1.f);
-  drv.run([&] { mma_tiles(cta.tmem + cPsi, A, B2, Cs / 16, idVt, NS, true); });
+  drv.run([&] { mma_tiles(cta.tmem + cPsi, As, B2, Cs / 16, idVt, NS, true); });
   // ---- phase 3: Oloc = N^qa (-Ut) + N^qk U, and N^qa W (Q' = Qt*Gam - N^qa W in the epilogue)
   load_img(G + 3 * sq_bytes(Cs));  // N^qa
   drv.run([&] { mma_tiles(cta.tmem + cOl, A, B1, Cs / 16, idV, NS, false); });  // B1 holds -Ut
@@ -803,7 +813,7 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   // back by the epilogue's TMEM rows. The 16-byte chunk j of row t is stored at
   // chunk j ^ (t & 7), so that 8 consecutive rows reading the same chunk hit 8
   // distinct bank groups.
-  float* qgam = reinterpret_cast<float*>(sm + 2 * TBY);
+  float* qgam = reinterpret_cast<float*>(sm + 2 * TBP);
   {
     constexpr int BT = 4;
     const T* gp = static_cast<const T*>(p.g);
