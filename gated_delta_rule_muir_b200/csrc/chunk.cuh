@@ -219,12 +219,13 @@ __device__ __forceinline__ void bulk_g2s_big(uint32_t dst, const uint8_t* src, u
 // back converted. In two steps: raw_issue (thread 0 starts the copy on `bar`,
 // whose transaction count the caller has set) and, once the copy has landed,
 // raw_convert (every thread; ends without a barrier). stage_raw does both.
-__device__ __forceinline__ void raw_issue(const Tile& t, const float* src, int rows, int cols, uint64_t* bar) {
+template <typename OpTile>
+__device__ __forceinline__ void raw_issue(const OpTile& t, const float* src, int rows, int cols, uint64_t* bar) {
   if (threadIdx.x == 0)
     bulk_g2s_big(t.hi, reinterpret_cast<const uint8_t*>(src), (uint32_t)rows * (uint32_t)cols * 4u, bar);
 }
-template <bool MN>
-__device__ __forceinline__ void raw_convert(const Tile& t, int rows, int cols, float sign) {
+template <bool MN, typename OpTile>
+__device__ __forceinline__ void raw_convert(const OpTile& t, int rows, int cols, float sign) {
   constexpr int NT = 256, MAXP = 128 * 128 / 8 / NT;
   const float4* raw = reinterpret_cast<const float4*>(__cvta_shared_to_generic(t.hi));
   const int np = rows * cols / 8;
@@ -235,7 +236,8 @@ __device__ __forceinline__ void raw_convert(const Tile& t, int rows, int cols, f
     const int x = threadIdx.x + k * NT;
     if (x < np) {
       int r, c8;
-      piece_of_rot(x, g, r, c8);
+      if constexpr (std::is_same_v<OpTile, SwTile>) piece_of_swz(x, g, r, c8);
+      else piece_of_rot(x, g, r, c8);
       const int e = r * g + (c8 >> 3);
       const float4 a = raw[2 * e], b = raw[2 * e + 1];
       v[k][0] = sign * a.x; v[k][1] = sign * a.y; v[k][2] = sign * a.z; v[k][3] = sign * a.w;
@@ -248,9 +250,10 @@ __device__ __forceinline__ void raw_convert(const Tile& t, int rows, int cols, f
     const int x = threadIdx.x + k * NT;
     if (x < np) {
       int r, c8;
-      piece_of_rot(x, g, r, c8);
-      if (MN) put_mn(t, r, c8, v[k]);
-      else put_k(t, r, c8, v[k]);
+      if constexpr (std::is_same_v<OpTile, SwTile>) piece_of_swz(x, g, r, c8);
+      else piece_of_rot(x, g, r, c8);
+      if constexpr (MN) put_mn(t, r, c8, v[k]);
+      else put_op(t, r, c8, v[k]);
     }
   }
 }
@@ -275,9 +278,9 @@ __device__ __forceinline__ bool stage_raw(const Tile& t, const float* src, int r
 // inputs (b may be null), f a contiguous fp32 [rows][COLS] matrix (may be
 // null). 256 threads; BT tokens per thread per batch with every load of a batch
 // issued before any is used.
-template <typename T, bool MN, int COLS>
-__device__ __forceinline__ void stage_prod(const Tile& t, const ChunkParams& p, const SubIdx& s, int rows, const T* a,
-                                           const T* b, const float* f, float sign) {
+template <typename T, bool MN, int COLS, typename OpTile>
+__device__ __forceinline__ void stage_prod(const OpTile& t, const ChunkParams& p, const SubIdx& s, int rows,
+                                           const T* a, const T* b, const float* f, float sign) {
   constexpr int NT = 256, BT = sizeof(T) == 2 ? 4 : 2, G = COLS / 8;
   for (int x0 = threadIdx.x; x0 < rows * G; x0 += BT * NT) {
     Pack8<T> pa[BT], pb[BT];
@@ -314,8 +317,8 @@ __device__ __forceinline__ void stage_prod(const Tile& t, const ChunkParams& p, 
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) va[j] *= sign;
-        if (MN) put_mn(t, r, c8, va);
-        else put_k(t, r, c8, va);
+        if constexpr (MN) put_mn(t, r, c8, va);
+        else put_op(t, r, c8, va);
       }
     }
   }
@@ -503,8 +506,6 @@ __device__ __forceinline__ void tree_tables(const float* pre, float* ftab, int C
 // with all loads of a batch issued before any is used. Pieces go by row_piece,
 // which keeps a thread on the same 8 channels throughout: rv holds r there.
 // The operand tiles are no-swizzle Tiles (put_k) or SwTiles (put_sw).
-__device__ __forceinline__ void put_op(const Tile& t, int r, int c8, const float (&x)[8]) { put_k(t, r, c8, x); }
-__device__ __forceinline__ void put_op(const SwTile& t, int r, int c8, const float (&x)[8]) { put_sw(t, r, c8, x); }
 
 template <int DK, typename T, typename OpTile>
 __device__ __forceinline__ void stage_level(const ChunkParams& p, const SubIdx& s, const float* pre,

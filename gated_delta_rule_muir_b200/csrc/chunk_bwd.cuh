@@ -189,7 +189,10 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
   const Tile QtT{base, base + g.half, DK * 16u, 128u};       // Q'^T: M = key channel, K = token
   const Tile A{base + 2 * TB, base + 3 * TB, 128u, DK * 16u};  // W: rows = tokens, K = key channel
   const Tile B{base + 4 * TB, base + 5 * TB, 128u, DK * 16u};  // S0: K = key channel, N = value column
-  const Tile Bo{base + 4 * TB, base + 5 * TB, 128u, (uint32_t)Cs * 16u};  // dO: K = token, N = value column
+  // dO: K = token, N = value column, staged by a row-major sweep; a 16-byte pad
+  // between the 8-column blocks keeps the stores of a shared-memory phase in 8
+  // distinct bank groups
+  const Tile Bo{base + 4 * TB, base + 5 * TB + 256u, 128u, (uint32_t)Cs * 16u + 16u};
   if (tid == 0) {
     mbar_init(&bar_cp, 1);
     mbar_init(&bar_s, 1);
@@ -296,17 +299,21 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
   constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
-  const uint32_t base = smem_u32(sm);
-  constexpr uint32_t TB = 128u * 128u * 2u;
+  const uint32_t base = (smem_u32(sm) + 1023u) & ~1023u;  // swizzled tiles start on 1024-byte boundaries
+  constexpr uint32_t TB = 128u * 128u * 2u, TBP = TB + 256u;
   const uint32_t ks = (uint32_t)Cs * 16u;
   const uint32_t H = sq_half(Cs);
-  const Tile AT{base, base + H, ks, 128u};         // transposed view of a Gram / T image: M = column, K = row
-  const Tile Ak{base, base + TB, 128u, DK * 16u};  // staged operand over channels (K = DK)
-  const Tile B1{base + 2 * TB, base + 3 * TB, 128u, ks};
-  const Tile B2{base + 4 * TB, base + 5 * TB, 128u, DK * 16u};
-  const Tile B3{base + 4 * TB, base + 5 * TB, 128u, ks};
+  const Tile AT{base, base + H, ks, 128u};      // transposed view of a Gram / T image: M = column, K = row
+  const auto Ak = kmajor_tile<DK>(base, TB);  // staged operand over channels (K = DK), row-major sweep
+  // dO, staged by a row-major sweep as an MN-major tile: a 16-byte pad between
+  // the 8-column blocks puts the 8 stores of a shared-memory phase (8
+  // consecutive column blocks of one token row) in 8 distinct bank groups
+  const Tile B1{base + 2 * TB, base + 2 * TB + TBP, 128u, ks + 16u};
+  const uint32_t b2 = base + 2 * TB + 2 * TBP;
+  const Tile B2{b2, b2 + TB, 128u, DK * 16u};
+  const Tile B3{b2, b2 + TB, 128u, ks};
   if (tid == 0) mbar_init(&bar_cp, 1);
-  zero_smem(base + 2 * TB, 4 * TB);
+  zero_smem(base + 2 * TB, 2 * TBP + 2 * TB);
   TcCta cta;
   cta.init(&tslot, &bar, 512);
   MmaSync drv{&bar, 0u, true};
@@ -348,9 +355,9 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
                              gsuf, 1.f);
   };
   stage_suf(true);
-  drv.run([&] { mma_tiles(cta.tmem + cP, Ak, B2, DK / 16, idK, NS, true); });  // -dP = N^qa^T dO + (A*Gsuf) dS_C
+  drv.run([&] { mma_ops(cta.tmem + cP, kview(Ak), NoSw{B2}, DK / 16, idK, NS, true); });  // -dP = N^qa^T dO + (A*Gsuf) dS_C
   stage_suf(false);
-  drv.run([&] { mma_tiles(cta.tmem + cU, Ak, B2, DK / 16, idK, NS, true); });  // + (K*Gsuf) dS_C
+  drv.run([&] { mma_ops(cta.tmem + cU, kview(Ak), NoSw{B2}, DK / 16, idK, NS, true); });  // + (K*Gsuf) dS_C
   // dP (TMEM, negated) -> B3 (K = token), then dZ = T^T dP
   issue_img(p.tt + u * sq_bytes(Cs));  // T^T
   for (int c = wg * 16; c < DV; c += 32) {
@@ -441,11 +448,15 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   constexpr int NT = 256;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t u = blockIdx.x;
-  const uint32_t base = smem_u32(sm);
+  const uint32_t base = (smem_u32(sm) + 1023u) & ~1023u;  // swizzled tiles start on 1024-byte boundaries
+  uint8_t* const sma = sm + (base - smem_u32(sm));
   constexpr uint32_t TB = 128u * 128u * 2u;
-  const Tile R0{base, base + TB, 128u, DV * 16u};
-  const Tile R1{base + 2 * TB, base + 3 * TB, 128u, DV * 16u};
-  const Tile R2{base + 4 * TB, base + 5 * TB, 128u, DV * 16u};
+  // Every operand is K-major over the DV value columns (rows = tokens or key
+  // channels). With DV a multiple of 64 the rows are 128-byte swizzled, so that
+  // the row-major staging sweeps store without bank conflicts.
+  const auto R0 = kmajor_tile<DV>(base, TB);
+  const auto R1 = kmajor_tile<DV>(base + 2 * TB, TB);
+  const auto R2 = kmajor_tile<DV>(base + 4 * TB, TB);
   zero_smem(base, 6 * TB);
   if (tid == 0) mbar_init(&bar_cp, 1);
   uint32_t cph = 0;
@@ -454,14 +465,15 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   MmaSync drv{&bar, 0u, true};
   const uint32_t lane = tmem_lane_base(warp);
   const int t = tid & 127, wg = tid >> 7;  // TMEM row; warpgroups split the columns
-  auto stage_dO = [&](const Tile& dst) {  // z * dy (dy alone without z)
+  using RT = std::remove_const_t<decltype(R0)>;
+  auto stage_dO = [&](const RT& dst) {  // z * dy (dy alone without z)
     stage_prod<T, false, DV>(dst, p, s, Cs, static_cast<const T*>(p.dy), static_cast<const T*>(p.z), nullptr, 1.f);
   };
-  auto stage_U = [&](const Tile& dst) {  // w * v
+  auto stage_U = [&](const RT& dst) {  // w * v
     stage_prod<T, false, DV>(dst, p, s, Cs, static_cast<const T*>(p.v), static_cast<const T*>(p.w), nullptr, 1.f);
   };
   // Rows of a [Cs][N] TMEM result -> dst (fp32, row-major, row stride ld), optional mask.
-  float* scratch = reinterpret_cast<float*>(sm + 6 * TB);
+  float* scratch = reinterpret_cast<float*>(sma + 6 * TB);
   auto drain = [&](uint32_t col, int n, float* dst, int64_t ld, int mask) {
     drain_rows(cta.tmem + lane + 0u, col, n, dst, ld, Cs, scratch, drv.ok, [&](int row, int c, float(&v)[32]) {
 #pragma unroll
@@ -511,16 +523,16 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   raw_convert<false>(R0, DK, DV, 1.f);
   raw_convert<false>(R2, Cs, DV, -1.f);
   drv.run([&] {
-    mma_tiles(cta.tmem + 0, R1, R0, DV / 16, idK, NS, false);
-    mma_tiles(cta.tmem + 128, R2, R0, DV / 16, idK, NS, false);
+    mma_ops(cta.tmem + 0, kview(R1), kview(R0), DV / 16, idK, NS, false);
+    mma_ops(cta.tmem + 128, kview(R2), kview(R0), DV / 16, idK, NS, false);
   });
   drain(0, DK, g4 + 2 * Cs * DK, DK, 0);    // dKs
   drain(128, DK, g4 + 3 * Cs * DK, DK, 0);  // dAs
   // pass 2: R1 = U, R2 = -P stay; R0 = dO, then dZ
   stage_dO(R0);
   drv.run([&] {
-    mma_tiles(cta.tmem + 0, R0, R1, DV / 16, idC, NS, false);    // dN^qk
-    mma_tiles(cta.tmem + 128, R0, R2, DV / 16, idC, NS, false);  // dN^qa
+    mma_ops(cta.tmem + 0, kview(R0), kview(R1), DV / 16, idC, NS, false);    // dN^qk
+    mma_ops(cta.tmem + 128, kview(R0), kview(R2), DV / 16, idC, NS, false);  // dN^qa
   });
   if (tid == 0) mbar_expect_tx(&bar_cp, mat_csdv);
   raw_issue(R0, q.dZ + u * Cs * DV, Cs, DV, &bar_cp);
@@ -529,8 +541,8 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   raw_wait();
   raw_convert<false>(R0, Cs, DV, 1.f);
   drv.run([&] {
-    mma_tiles(cta.tmem + 256, R0, R1, DV / 16, idC, NS, false);  // dM^kk
-    mma_tiles(cta.tmem + 384, R0, R2, DV / 16, idC, NS, false);  // dM^ka
+    mma_ops(cta.tmem + 256, kview(R0), kview(R1), DV / 16, idC, NS, false);  // dM^kk
+    mma_ops(cta.tmem + 384, kview(R0), kview(R2), DV / 16, idC, NS, false);  // dM^ka
   });
   // pass 3: R0 = dZ stays, R1 = S0, R2 = dO
   if (tid == 0) mbar_expect_tx(&bar_cp, mat_dkdv);
@@ -541,8 +553,8 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   raw_wait();
   raw_convert<false>(R1, DK, DV, 1.f);
   drv.run([&] {
-    mma_tiles(cta.tmem + 0, R2, R1, DV / 16, idK, NS, false);    // dQp
-    mma_tiles(cta.tmem + 128, R0, R1, DV / 16, idK, NS, false);  // dKp
+    mma_ops(cta.tmem + 0, kview(R2), kview(R1), DV / 16, idK, NS, false);    // dQp
+    mma_ops(cta.tmem + 128, kview(R0), kview(R1), DV / 16, idK, NS, false);  // dKp
   });
   drain(0, DK, g4 + 0 * Cs * DK, DK, 0);
   drain(128, DK, g4 + 1 * Cs * DK, DK, 0);
@@ -688,7 +700,7 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
       stage_level<DK, T>(p, s, pre, suf, ftab + lev * nb * DK, rv, Cs, lb, side == 1, side == 0, OP, OP);
       drv.run([&] {
         if constexpr (DK % 64 == 0)
-          mma_tiles_swa(cta.tmem + 128 * lev, OP, side == 0 ? GT : transposed(GT), Cs / 16, id, NS, false);
+          mma_ops(cta.tmem + 128 * lev, SwMN{OP}, NoSw{side == 0 ? GT : transposed(GT)}, Cs / 16, id, NS, false);
         else
           mma_tiles(cta.tmem + 128 * lev, transposed(OP), side == 0 ? GT : transposed(GT), Cs / 16, id, NS, false);
       });

@@ -185,50 +185,75 @@ struct Tile {
 
 __device__ __forceinline__ Tile transposed(const Tile& t) { return Tile{t.hi, t.lo, t.sbo, t.lbo}; }
 
-// D[tmem] (+)= A * B for one tile pair covering `ksteps` MMA steps of K = 16.
-// M = 128 rows of A (lanes of D), N columns of B. nsplit = 1 (hi*hi), 3
-// (hi*hi + hi*lo + lo*hi), or 2 (hi*hi + A.lo*B.hi, for a B exact in bf16).
-__device__ __forceinline__ void mma_tiles(uint32_t d_tmem, const Tile& A, const Tile& B, int ksteps, uint32_t idesc,
-                                          int nsplit, bool accumulate) {
-  for (int j = 0; j < ksteps; ++j) {
-    const uint32_t oa = j * 2u * A.lbo, ob = j * 2u * B.lbo;
-    const uint64_t ah = sdesc(A.hi + oa, A.lbo, A.sbo), bh = sdesc(B.hi + ob, B.lbo, B.sbo);
-    mma_bf16(d_tmem, ah, bh, idesc, (accumulate || j > 0) ? 1u : 0u);
-    if (nsplit == 3) {
-      const uint64_t al = sdesc(A.lo + oa, A.lbo, A.sbo), bl = sdesc(B.lo + ob, B.lbo, B.sbo);
-      mma_bf16(d_tmem, ah, bl, idesc, 1u);
-      mma_bf16(d_tmem, al, bh, idesc, 1u);
-    } else if (nsplit == 2) {
-      mma_bf16(d_tmem, sdesc(A.lo + oa, A.lbo, A.sbo), bh, idesc, 1u);
-    }
-  }
-}
-
 // A staged operand in 128-byte-swizzled rows: bf16 hi and lo planes (each
 // 1024-byte aligned), row r of the matrix in 64-column boxes `box` bytes apart.
-// Written row by row (put_sw), it is read here as the MN-major operand (rows =
-// K): a sweep whose 8 threads per shared-memory phase store 8 consecutive
-// 16-byte pieces of one row lands them in 8 distinct bank groups.
+// Written row by row (put_sw), it is read as the K-major operand (rows = M or
+// N) or the MN-major one (rows = K): a sweep whose 8 threads per shared-memory
+// phase store 8 consecutive 16-byte pieces of one row lands them in 8 distinct
+// bank groups.
 struct SwTile {
   uint32_t hi, lo;
   uint32_t box;
 };
 
-// D[tmem] (+)= A * B over `ksteps` steps of K = 16, A an MN-major SwTile (M =
-// its columns, K = its rows), B a no-swizzle Tile; nsplit as in mma_tiles.
-__device__ __forceinline__ void mma_tiles_swa(uint32_t d_tmem, const SwTile& A, const Tile& B, int ksteps,
-                                              uint32_t idesc, int nsplit, bool accumulate) {
+// Operand views for the MMA loop below: each gives the shared-memory descriptor
+// of its hi or lo plane at MMA step j (K = 16 per step).
+//   NoSw: a no-swizzle Tile as stored (its lbo is the K-direction stride).
+//   SwK:  a SwTile read K-major (rows = M or N, columns = K).
+//   SwMN: a SwTile read MN-major (rows = K, columns = M or N).
+struct NoSw {
+  Tile t;
+  __device__ __forceinline__ uint64_t desc(int j, bool lo) const {
+    return sdesc((lo ? t.lo : t.hi) + (uint32_t)j * 2u * t.lbo, t.lbo, t.sbo);
+  }
+};
+struct SwK {
+  SwTile t;
+  __device__ __forceinline__ uint64_t desc(int j, bool lo) const {
+    return sdesc_sw128((lo ? t.lo : t.hi) + (uint32_t)(j >> 2) * t.box + (uint32_t)(j & 3) * 32u, 16u, 1024u);
+  }
+};
+struct SwMN {
+  SwTile t;
+  __device__ __forceinline__ uint64_t desc(int j, bool lo) const {
+    return sdesc_sw128((lo ? t.lo : t.hi) + (uint32_t)j * 2048u, t.box, 1024u);
+  }
+};
+
+// D[tmem] (+)= A * B over `ksteps` MMA steps of K = 16. M = 128 rows of A
+// (lanes of D), N columns of B. nsplit = 1 (hi*hi), 3 (hi*hi + hi*lo + lo*hi),
+// or 2 (hi*hi + A.lo*B.hi, for a B exact in bf16).
+template <typename OA, typename OB>
+__device__ __forceinline__ void mma_ops(uint32_t d_tmem, const OA& A, const OB& B, int ksteps, uint32_t idesc,
+                                        int nsplit, bool accumulate) {
   for (int j = 0; j < ksteps; ++j) {
-    const uint32_t oa = j * 2048u, ob = j * 2u * B.lbo;
-    const uint64_t ah = sdesc_sw128(A.hi + oa, A.box, 1024u), bh = sdesc(B.hi + ob, B.lbo, B.sbo);
+    const uint64_t ah = A.desc(j, false), bh = B.desc(j, false);
     mma_bf16(d_tmem, ah, bh, idesc, (accumulate || j > 0) ? 1u : 0u);
     if (nsplit == 3) {
-      mma_bf16(d_tmem, ah, sdesc(B.lo + ob, B.lbo, B.sbo), idesc, 1u);
-      mma_bf16(d_tmem, sdesc_sw128(A.lo + oa, A.box, 1024u), bh, idesc, 1u);
+      mma_bf16(d_tmem, ah, B.desc(j, true), idesc, 1u);
+      mma_bf16(d_tmem, A.desc(j, true), bh, idesc, 1u);
     } else if (nsplit == 2) {
-      mma_bf16(d_tmem, sdesc_sw128(A.lo + oa, A.box, 1024u), bh, idesc, 1u);
+      mma_bf16(d_tmem, A.desc(j, true), bh, idesc, 1u);
     }
   }
+}
+
+// A K-major operand tile over COLS columns (rows = M or N, at most 128; hi and
+// lo planes `plane` bytes apart, base 1024-byte aligned): 128-byte-swizzled rows
+// when COLS is a multiple of 64, the no-swizzle layout otherwise (rows of 64
+// bytes cannot take the 128-byte swizzle). kview gives its K-major MMA view.
+template <int COLS>
+__device__ __forceinline__ auto kmajor_tile(uint32_t a, uint32_t plane) {
+  if constexpr (COLS % 64 == 0) return SwTile{a, a + plane, 128u * 128u};
+  else return Tile{a, a + plane, 128u, (uint32_t)COLS * 16u};
+}
+__device__ __forceinline__ SwK kview(const SwTile& t) { return SwK{t}; }
+__device__ __forceinline__ NoSw kview(const Tile& t) { return NoSw{t}; }
+
+// The no-swizzle pair, the common case.
+__device__ __forceinline__ void mma_tiles(uint32_t d_tmem, const Tile& A, const Tile& B, int ksteps, uint32_t idesc,
+                                          int nsplit, bool accumulate) {
+  mma_ops(d_tmem, NoSw{A}, NoSw{B}, ksteps, idesc, nsplit, accumulate);
 }
 
 // ---- operand staging (any thread) ------------------------------------------
@@ -273,6 +298,10 @@ __device__ __forceinline__ void put_k(const Tile& t, int m, int k8, const float 
   sts128(t.lo + off, lo);
 }
 
+// Row r (the K-major view's M or N index), columns c8..c8+7 of either kind of tile.
+__device__ __forceinline__ void put_op(const Tile& t, int r, int c8, const float (&x)[8]) { put_k(t, r, c8, x); }
+__device__ __forceinline__ void put_op(const SwTile& t, int r, int c8, const float (&x)[8]) { put_sw(t, r, c8, x); }
+
 // Staging sweeps over a rows x (8 G) matrix in 8-element pieces (G a power of
 // two, rows a multiple of 8). put_k and put_mn store a piece to the bank group
 // given by its row & 7, and a 128-bit shared-memory access serves a warp in four
@@ -316,6 +345,16 @@ __device__ __forceinline__ void piece_of_rot(int x, int G, int& r, int& c8) {
   const int lg = 31 - __clz(G);
   r = ((x >> (3 + lg)) << 3) | (x & 7);
   c8 = (((x >> 3) + (x & 7)) & (G - 1)) << 3;
+}
+// The same for a SwTile destination (G >= 8): row i of the phase takes column
+// block c ^ (i / 2). The reads then fall on the four 32-byte positions of a
+// 128-byte line twice each, as with the rotation, and the swizzled stores (chunk
+// (c ^ (i / 2)) ^ i for rows i = 0..7) hit 8 distinct bank groups; the rotation
+// would put all 8 of them in one.
+__device__ __forceinline__ void piece_of_swz(int x, int G, int& r, int& c8) {
+  const int lg = 31 - __clz(G);
+  r = ((x >> (3 + lg)) << 3) | (x & 7);
+  c8 = (((x >> 3) & (G - 1)) ^ ((x & 7) >> 1)) << 3;
 }
 
 // 8 values that are exact in bf16, already packed (uint4 of 8 bf16): the hi
