@@ -425,13 +425,13 @@ def bench_decode(dev, steps, warmup, pk, graph=True):
         with torch.cuda.stream(side):
             layer_calls()  # warm-up outside the capture
         torch.cuda.current_stream().wait_stream(side)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg):
             layer_calls()
         for _ in range(max(warmup, 3)):
-            graph.replay()
-        ms_g = time_steps(graph.replay, reps, False) / reps
-        del graph
+            cg.replay()
+        ms_g = time_steps(cg.replay, reps, False) / reps
+        del cg
         gbs_g = (state_bytes + io_bytes) / (ms_g * 1e-3) / 1e9
         out[f"batch{nb}"] = {"ms_per_token": round(ms, 4), "GB_s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 3),
                              "graph24_ms_per_token": round(ms_g, 4), "graph24_GB_s": round(gbs_g, 1),
