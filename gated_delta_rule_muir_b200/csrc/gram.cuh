@@ -24,9 +24,12 @@
 //
 // Staging: thread (g, J) owns channels 8g..8g+7 of 8-block J and walks its 8
 // tokens in order (forward for an upper block, backward for a lower one), so the
-// running sum stays in registers. Inside every 8-row group of XL and YL the rows
-// are permuted by XOR with J & 7: the 8 threads of a shared-memory phase then
-// store to 8 distinct bank groups. The epilogue undoes the permutation.
+// running sum stays in registers. The channel group varies fastest across the
+// threads, so that a warp's load reads whole token rows (two rows of 256 bytes
+// for dk = 128, not sixteen 32-byte pieces of sixteen rows), and XL and YL have
+// 128-byte-swizzled rows (dk a multiple of 64), in which the 8 threads of a
+// shared-memory phase, 8 consecutive channel groups of one row, store to 8
+// distinct bank groups.
 //
 // TMEM: two 128-column slots, used by alternate levels; a level's results are
 // drained while the next level's product runs. With bf16 inputs and one MMA pass
@@ -38,37 +41,26 @@
 namespace muir {
 
 // 8 floats as one bf16 row piece of a K-major tile: the hi plane, and with NS > 1 the lo plane too.
-template <int NS>
-__device__ __forceinline__ void put_row(const Tile& t, int m, int k8, const float (&x)[8]) {
+__device__ __forceinline__ uint32_t row_piece_off(const Tile& t, int m, int k8) {
+  return (uint32_t)(m >> 3) * t.sbo + (uint32_t)(k8 >> 3) * 128u + (uint32_t)(m & 7) * 16u;
+}
+__device__ __forceinline__ uint32_t row_piece_off(const SwTile& t, int m, int k8) {
+  return (uint32_t)(k8 >> 6) * t.box + (uint32_t)m * 128u + ((uint32_t)(((k8 >> 3) & 7) ^ (m & 7)) << 4);
+}
+template <int NS, typename OpTile>
+__device__ __forceinline__ void put_row(const OpTile& t, int m, int k8, const float (&x)[8]) {
   if constexpr (NS == 1) {
     uint4 hi;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
 #pragma unroll
     for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-    sts128(t.hi + (uint32_t)(m >> 3) * t.sbo + (uint32_t)(k8 >> 3) * 128u + (uint32_t)(m & 7) * 16u, hi);
+    sts128(t.hi + row_piece_off(t, m, k8), hi);
   } else {
-    put_k(t, m, k8, x);
+    put_op(t, m, k8, x);
   }
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
-
-// v[j] <- v[j ^ pm] for a run-time pm in [0, 8), by three stages of conditional
-// swaps with fixed indices (an index computed at run time would put v in local
-// memory).
-__device__ __forceinline__ void xor_permute8(float (&v)[8], int pm) {
-#pragma unroll
-  for (int bit = 1; bit < 8; bit <<= 1) {
-    const bool sw = (pm & bit) != 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j & bit) continue;
-      const float a = v[j], c = v[j | bit];
-      v[j] = sw ? c : a;
-      v[j | bit] = sw ? a : c;
-    }
-  }
-}
 
 // 2^x for x <= 0 with the hardware's approximate base-2 exponential (relative
 // error near 2^-22); results below the normal range flush to 0, the correct
@@ -81,7 +73,8 @@ __device__ __forceinline__ float exp2_neg(float x) {
 
 template <int DK>
 constexpr uint32_t gram_smem_bytes(int NS) {
-  return 2u * (NS > 1 ? 2u : 1u) * 128u * DK * 2u  // XL, YL: hi planes, and lo planes for NS > 1
+  return 1024u                                      // alignment of the swizzled tiles
+         + 2u * (NS > 1 ? 2u : 1u) * 128u * DK * 2u  // XL, YL: hi planes, and lo planes for NS > 1
          + 16u * DK * 4u                     // totals of the 8-blocks (log2)
          + 4u * 8u * DK * 4u                 // rows of one diagonal block: k, qt, a, alpha
          + kZeroBuf;
@@ -100,10 +93,12 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
   const int lnb = Cs == 128 ? 4 : 3;   // log2(nb)
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const uint32_t base = smem_u32(sm);
-  const Tile XL{base, base + (PL - 1) * LB, 128u, DK * 16u};
-  const Tile YL{base + PL * LB, base + (2 * PL - 1) * LB, 128u, DK * 16u};
-  float* tot = reinterpret_cast<float*>(sm + 2 * PL * LB);  // [16][DK]
+  const uint32_t base = (smem_u32(sm) + 1023u) & ~1023u;  // swizzled tiles start on 1024-byte boundaries
+  uint8_t* const sma = sm + (base - smem_u32(sm));
+  const auto XL = kmajor_tile<DK>(base, (PL - 1) * LB);
+  const auto YL = kmajor_tile<DK>(base + PL * LB, (PL - 1) * LB);
+  constexpr bool kSw = DK % 64 == 0;
+  float* tot = reinterpret_cast<float*>(sma + 2 * PL * LB);  // [16][DK]
   float* drow = tot + 16 * DK;                               // [4][8][DK]
   const uint32_t zbuf = base + 2 * PL * LB + (16u * DK + 4u * 8u * DK) * 4u;
   uint8_t* out = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
@@ -111,7 +106,14 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
   const int64_t row0 = toff(p, s.b, s.tok0, s.h, DK);  // token 0 of the unit, channel 0
 
   if (Cs < 128) {  // rows >= Cs of the operands stay zero
-    for (uint32_t pl = 0; pl < 2u * PL; ++pl) zero_smem(base + pl * LB + (uint32_t)Cs * DK * 2u, (128u - Cs) * DK * 2u);
+    for (uint32_t pl = 0; pl < 2u * PL; ++pl) {
+      if constexpr (kSw) {  // in every 64-column box of 128 rows
+        for (uint32_t bx = 0; bx < DK / 64; ++bx)
+          zero_smem(base + pl * LB + bx * 16384u + (uint32_t)Cs * 128u, (128u - Cs) * 128u);
+      } else {
+        zero_smem(base + pl * LB + (uint32_t)Cs * DK * 2u, (128u - Cs) * DK * 2u);
+      }
+    }
   }
   TcCta cta;
   cta.init(&tslot, &bar, 256);
@@ -131,8 +133,8 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
   }
 
   // ---- staging thread (g, J): channels 8g.., 8-block J --------------------
-  const int sg = tid / nb, sJ = tid % nb;
-  const bool stager = sg < G;
+  const int sg = tid % G, sJ = tid / G;
+  const bool stager = sJ < nb;
   const int c8 = sg * 8;
   if (stager) {
     // totals of the 8-block in log2 units
@@ -177,13 +179,10 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
     }
     const int lo = upper ? P : P - b;  // first token of the half
     const int rbase = pv * 2 * b;
-    // upper blocks walk forward and lower ones backward: with (J & 7) ^ 7 for the
-    // lower ones, the 8 threads of a phase hit 8 distinct row offsets at every step
-    const int perm = upper ? (sJ & 7) : (sJ & 7) ^ 7;
     const T* x1p = upper ? qp : ep;                  // q (then r g q) or e (then e k)
     const T* x2p = upper && gp ? gp : kp;            // g, or a stand-in that is not used
     const bool use_g = upper && gp != nullptr;
-    const Tile dst = upper ? XL : YL;
+    const auto dst = upper ? XL : YL;
     float rl[8];  // r of these channels (loaded here: an array captured by the lambda would live in local memory)
     ld8f(p.r + (int64_t)s.h * DK + c8, rl);
     float run[8];
@@ -222,7 +221,7 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
           kk[j] *= f;
         }
         const int uu = 8 * sJ + w8 - lo, q8 = uu >> 3;
-        const int m = rbase + 8 * q8 + (w8 ^ perm);
+        const int m = rbase + 8 * q8 + w8;
         put_row<NS>(dst, m, c8, kk);
         put_row<NS>(dst, m + b, c8, x1);
       }
@@ -238,9 +237,7 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
     const int pv = rho / (2 * b);
     const int X = (rho / b) & 1, within = rho % b;
     const int P = (2 * pv + 1) * b;
-    const int q8 = within >> 3;
-    const int J = (P >> 3) + q8;
-    const int t = P + 8 * q8 + ((within & 7) ^ (J & 7));  // an upper block: XOR with J & 7
+    const int t = P + within;
     const bool on = rho < Cs;
     // this warpgroup's columns of the row's pivot: Y = wg, [pv*2b + wg*b, + b)
     for (int cq = 0; cq < b; cq += 8) {
@@ -255,12 +252,7 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] = pv == pw ? v0[j] : v1[j];
       }
-      if (on) {
-        const int Jl = ((P - b) >> 3) + (cq >> 3);  // the lower 8-block of these columns
-        const int pm = (Jl & 7) ^ 7;                 // a lower block
-        xor_permute8(v, pm);  // v[j] <- v[j ^ pm]
-        sq_put(out + (2 * X + wg) * sq_bytes(Cs), Cs, t, P - b + cq, v);
-      }
+      if (on) sq_put(out + (2 * X + wg) * sq_bytes(Cs), Cs, t, P - b + cq, v);
     }
   };
 
@@ -373,7 +365,7 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      mma_tiles(cta.tmem + (uint32_t)(lev & 1) * 128u, XL, YL, DK / 16, id, NS, false);
+      mma_ops(cta.tmem + (uint32_t)(lev & 1) * 128u, kview(XL), kview(YL), DK / 16, id, NS, false);
       mma_commit(&bar);
     }
     // the diagonal-block rows are fetched level by level, so that no prefetched
