@@ -157,14 +157,22 @@ template <> struct Pack8<__nv_bfloat16> {
   }
 };
 
-// 8 floats to global memory in one 32-byte store (p 32-byte aligned).
+// 8 floats to global memory: one 32-byte store where p is 32-byte aligned, two
+// 16-byte stores where it is only 16-byte aligned (the C ABI requires 16 bytes
+// of its callers' pointers, and a 32-byte vector store to an address that is
+// not 32-byte aligned is a fault).
 __device__ __forceinline__ void stg256(float* p, const float (&v)[8]) {
-  asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
-               "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
-               : "memory");
+  if ((reinterpret_cast<uintptr_t>(p) & 31u) == 0) {
+    asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+                 "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+                 : "memory");
+  } else {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
 }
 
-// 16 floats (p 32-byte aligned) in two 32-byte stores.
+// 16 floats (p 16-byte aligned) in two 32-byte stores (see stg256).
 __device__ __forceinline__ void stg_row16(float* p, const float (&v)[16]) {
   float a[8], b[8];
 #pragma unroll
