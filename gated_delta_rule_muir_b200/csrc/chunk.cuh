@@ -360,6 +360,84 @@ __device__ __forceinline__ void drain_rows(uint32_t tmem_lane_addr, uint32_t col
   }
 }
 
+// ---- 32 x 32 row blocks through a per-warp scratch ---------------------------
+// An epilogue thread owns one row (its TMEM lane), so a thread-per-row load or
+// store of a row-major matrix touches 32 lines per instruction. These helpers
+// move the 32 rows [row0, row0 + 32) x columns [c, c + 32) that a warp owns in
+// whole lines instead: 16-byte asynchronous copies (cp.async) into a scratch
+// block, and stores of 4 rows x 128 bytes (fp32) or 8 rows x 64 bytes (bf16)
+// per instruction out of it. In an fp32 block (4 KB) the 16-byte piece j of row
+// r sits at piece j ^ (r & 7); in a bf16 block (2 KB) piece q of row r at
+// q ^ (r & 3): conflict-free for the row-wise and the line-wise accesses alike.
+// Rows >= nrows are neither loaded nor stored.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <typename T>
+constexpr uint32_t row_block_bytes() { return sizeof(T) == 4 ? 4096u : 2048u; }
+
+template <typename T>
+__device__ __forceinline__ void rows_fill(uint32_t blk, const T* src, int64_t ld, int row0, int nrows, int c) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = (lane >> 3) + 4 * i, j = lane & 7;
+      if (row0 + r < nrows)
+        cp_async16(blk + (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)), src + (int64_t)(row0 + r) * ld + c + 4 * j);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = (lane >> 2) + 8 * i, q = lane & 3;
+      if (row0 + r < nrows)
+        cp_async16(blk + (uint32_t)(r * 64 + ((q ^ (r & 3)) << 4)), src + (int64_t)(row0 + r) * ld + c + 8 * q);
+    }
+  }
+}
+
+// Columns 8q .. 8q+7 of row r of a block, as floats.
+template <typename T>
+__device__ __forceinline__ void row8_get(const uint8_t* blk, int r, int q, float (&o)[8]) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(blk + r * 128 + (((2 * q) ^ (r & 7)) << 4));
+    const float4 b = *reinterpret_cast<const float4*>(blk + r * 128 + (((2 * q + 1) ^ (r & 7)) << 4));
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  } else {
+    Pack8<__nv_bfloat16> pk;
+    pk.u = *reinterpret_cast<const uint4*>(blk + r * 64 + ((q ^ (r & 3)) << 4));
+    pk.get(o);
+  }
+}
+__device__ __forceinline__ void row8_put(uint8_t* blk, int r, int q, const float (&v)[8]) {
+  *reinterpret_cast<float4*>(blk + r * 128 + (((2 * q) ^ (r & 7)) << 4)) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(blk + r * 128 + (((2 * q + 1) ^ (r & 7)) << 4)) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// An fp32 block out to the row-major matrix dst (element type T) in whole lines.
+template <typename T>
+__device__ __forceinline__ void rows_store(const uint8_t* blk, T* dst, int64_t ld, int row0, int nrows, int c) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (sizeof(T) == 4) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = (lane >> 3) + 4 * i, j = lane & 7;
+      const float4 a = *reinterpret_cast<const float4*>(blk + r * 128 + ((j ^ (r & 7)) << 4));
+      if (row0 + r < nrows) *reinterpret_cast<float4*>(dst + (int64_t)(row0 + r) * ld + c + 4 * j) = a;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = (lane >> 2) + 8 * i, q = lane & 3;
+      float v[8];
+      row8_get<float>(blk, r, q, v);
+      if (row0 + r < nrows) Elt<T>::st8(dst + (int64_t)(row0 + r) * ld + c + 8 * q, v);
+    }
+  }
+}
+
 // CTA prologue shared by the tensor-core kernels: TMEM allocation + mbarrier.
 struct TcCta {
   uint32_t tmem;

@@ -224,51 +224,64 @@ __global__ void __launch_bounds__(256, 1) bwd_pe_kernel(ChunkParams p, BwdBufs q
   const float* olu = p.ol + u * Cs * DV;
   float* P = q.P + u * Cs * DV;
   {
-    // every load of the row is issued before the accumulators are read
-    constexpr int NC = DV / 32;  // 16-column chunks per thread
-    const bool on = t < Cs && drv.ok, wdz = p.dz && p.z;
-    const int64_t o = toff(p, s.b, s.tok0 + (t < Cs ? t : 0), s.h, DV);
-    Pack8<float> pu[NC][2], po[NC][2];
-    Pack8<T> pd[NC][2];
-    if (on) {
+    // P = W S0 + Ut and dz = dy * (Q' S0 + Oloc) by 32 x 32 row blocks (rows_fill,
+    // rows_store): Ut, Oloc and dy come in and P, dz go out in whole lines. All
+    // shared memory is free here, the MMAs having completed.
+    const int ln = tid & 31, row0 = 32 * (warp & 3);
+    const bool wdz = p.dz && p.z;
+    const int64_t ts = (int64_t)p.H * DV;
+    const int64_t o0 = toff(p, s.b, s.tok0, s.h, DV);
+    constexpr uint32_t FB = row_block_bytes<float>(), CB = 2 * FB + row_block_bytes<T>();  // Ut, Oloc, dy blocks
+    constexpr int NCK = (DV + 63) / 64;  // 32-column chunks per warp
+    static_assert(8u * NCK * CB <= 6u * 128u * 128u * 2u, "row blocks exceed the tiles' shared memory");
+    const uint32_t wb = base + (uint32_t)warp * NCK * CB;
+    uint8_t* const wsm = sm + (wb - base);
+    if (drv.ok) {
+      int k = 0;
+      for (int c = wg * 32; c < DV; c += 64, ++k) {
+        rows_fill<float>(wb + k * CB, Ut, DV, row0, Cs, c);
+        if (wdz) {
+          rows_fill<float>(wb + k * CB + FB, olu, DV, row0, Cs, c);
+          rows_fill<T>(wb + k * CB + 2 * FB, static_cast<const T*>(p.dy) + o0, ts, row0, Cs, c);
+        }
+      }
+    }
+    cp_async_wait_all();
+    __syncwarp();
+    {
+      int k = 0;
+      for (int c = wg * 32; c < DV; c += 64, ++k) {
+        uint8_t* bu = wsm + k * CB;
+        float v[32];
+        tmem_ld32(cta.tmem + lane + c, v);
 #pragma unroll
-      for (int k = 0; k < NC; ++k)
+        for (int q8 = 0; q8 < 4; ++q8) {
+          float a8[8];
+          row8_get<float>(bu, ln, q8, a8);
 #pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          const int c = wg * 16 + 32 * k + 8 * h8;
-          pu[k][h8].ld(Ut + t * DV + c);
-          if (wdz) {
-            pd[k][h8].ld(static_cast<const T*>(p.dy) + o + c);
-            po[k][h8].ld(olu + (int64_t)t * DV + c);
+          for (int j = 0; j < 8; ++j) a8[j] += v[8 * q8 + j];
+          row8_put(bu, ln, q8, a8);
+        }
+        if (wdz) {
+          tmem_ld32(cta.tmem + lane + 128 + c, v);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            float ol8[8], dd[8];
+            row8_get<float>(bu + FB, ln, q8, ol8);
+            row8_get<T>(bu + 2 * FB, ln, q8, dd);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) ol8[j] = dd[j] * (v[8 * q8 + j] + ol8[j]);
+            row8_put(bu + FB, ln, q8, ol8);
           }
         }
-    }
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      const int c = wg * 16 + 32 * k;
-      float v[16], w[16];
-      tmem_ld16(cta.tmem + lane + c, v);
-      tmem_ld16(cta.tmem + lane + 128 + c, w);
-      if (!on) continue;
-      float pv[16];
-#pragma unroll
-      for (int h8 = 0; h8 < 2; ++h8) {
-        float a8[8];
-        pu[k][h8].get(a8);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) pv[8 * h8 + j] = v[8 * h8 + j] + a8[j];
       }
-      stg_row16(P + t * DV + c, pv);
-      if (wdz) {
-#pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          float dd[8], ol8[8], out[8];
-          pd[k][h8].get(dd);
-          po[k][h8].get(ol8);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) out[j] = dd[j] * (w[8 * h8 + j] + ol8[j]);
-          Elt<T>::st8(static_cast<T*>(p.dz) + o + c + 8 * h8, out);
-        }
+    }
+    __syncwarp();
+    if (drv.ok) {
+      int k = 0;
+      for (int c = wg * 32; c < DV; c += 64, ++k) {
+        rows_store<float>(wsm + k * CB, P, DV, row0, Cs, c);
+        if (wdz) rows_store<T>(wsm + k * CB + FB, static_cast<T*>(p.dz) + o0, ts, row0, Cs, c);
       }
     }
   }
