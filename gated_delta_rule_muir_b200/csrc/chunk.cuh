@@ -1331,8 +1331,7 @@ __global__ void apply_map_kernel(const float* __restrict__ Phi, const float* __r
 // A = Q' tiles of the map image (bulk copy, K-major over key channels),
 // B = S0 (MN-major: K = key channel, N = value column), bulk-copied raw and
 // converted in place (stage_raw). 256 threads: TMEM row t = tid % 128, the two
-// warpgroups take alternate 16-column chunks; every load of a row's Oloc and z
-// is issued before the accumulator is read.
+// warpgroups take alternate 32-column chunks.
 // ---------------------------------------------------------------------------
 template <int DK, int DV, typename T, int NS>
 __global__ void __launch_bounds__(256, 1) out_kernel(ChunkParams p, const uint8_t* ma, const float* ol, int units,
@@ -1372,43 +1371,58 @@ __global__ void __launch_bounds__(256, 1) out_kernel(ChunkParams p, const uint8_
         mma_tiles(cta.tmem + j * DV, Q, Sb, DK / 16, id, NS, false);
       }
     });
+  // y = z * (Q' S0 + Oloc) by 32 x 32 row blocks (rows_fill, rows_store): Oloc and
+  // z come in and y goes out in whole lines, through shared memory that is free
+  // once the products have completed.
   const uint32_t lane = tmem_lane_base(warp);
-  const int t = tid & 127, wg = tid >> 7;
-  constexpr int NC = DV / 32;  // 16-column chunks per thread
+  const int ln = tid & 31, row0 = 32 * (warp & 3), wg = tid >> 7;
+  constexpr uint32_t FB = row_block_bytes<float>(), CB = FB + row_block_bytes<T>();  // Oloc (then y), z
+  constexpr int NCK = (DV + 63) / 64;  // 32-column chunks per warp
+  const uint32_t wb = base + (uint32_t)warp * NCK * CB;
+  auto gen = [&](uint32_t x) { return sm + (x - base); };  // shared address -> generic pointer
   const float* olu = ol + uid * ulen * DV;
   const T* zp = static_cast<const T*>(p.z);
+  const int64_t ts = (int64_t)p.H * DV;
+  const int64_t y0 = toff(p, b, (int64_t)n * ulen, h, DV);  // token 0 of the unit
   for (int j = 0; j < nq; ++j) {
-    const int tt = j * 128 + t;
-    const bool on = tt < ulen && drv.ok;
-    const int64_t yo = toff(p, b, (int64_t)n * ulen + (on ? tt : 0), h, DV);  // rows past the unit: unused
-    Pack8<float> pa[NC][2];
-    Pack8<T> pz[NC][2];
-    if (on) {
-#pragma unroll
-      for (int k = 0; k < NC; ++k)
-#pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          const int c = wg * 16 + 32 * k + 8 * h8;
-          pa[k][h8].ld(olu + (int64_t)tt * DV + c);
-          pz[k][h8].ld_or_one(zp ? zp + yo + c : nullptr);  // y = o when z is absent
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      const int c = wg * 16 + 32 * k;
-      float v[16];
-      tmem_ld16(cta.tmem + lane + j * DV + c, v);
-      if (!on) continue;
-#pragma unroll
-      for (int h8 = 0; h8 < 2; ++h8) {
-        float a8[8], z8[8], o8[8];
-        pa[k][h8].get(a8);
-        pz[k][h8].get(z8);
-#pragma unroll
-        for (int e2 = 0; e2 < 8; ++e2) o8[e2] = (v[8 * h8 + e2] + a8[e2]) * z8[e2];
-        Elt<T>::st8(static_cast<T*>(p.y) + yo + c + 8 * h8, o8);
+    const int nrj = ulen - j * 128 < 128 ? ulen - j * 128 : 128;  // rows of this 128-row tile
+    const int64_t yj = y0 + (int64_t)j * 128 * ts;
+    if (drv.ok) {
+      int k = 0;
+      for (int c = wg * 32; c < DV; c += 64, ++k) {
+        rows_fill<float>(wb + k * CB, olu + (int64_t)j * 128 * DV, DV, row0, nrj, c);
+        if (zp) rows_fill<T>(wb + k * CB + FB, zp + yj, ts, row0, nrj, c);
       }
     }
+    cp_async_wait_all();
+    __syncwarp();
+    {
+      int k = 0;
+      for (int c = wg * 32; c < DV; c += 64, ++k) {
+        float v[32];
+        tmem_ld32(cta.tmem + lane + j * DV + c, v);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          float a8[8], z8[8];
+          row8_get<float>(gen(wb + k * CB), ln, q8, a8);
+          if (zp) {
+            row8_get<T>(gen(wb + k * CB + FB), ln, q8, z8);
+          } else {  // y = o when z is absent
+#pragma unroll
+            for (int e2 = 0; e2 < 8; ++e2) z8[e2] = 1.f;
+          }
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) a8[e2] = (v[8 * q8 + e2] + a8[e2]) * z8[e2];
+          row8_put(gen(wb + k * CB), ln, q8, a8);
+        }
+      }
+    }
+    __syncwarp();
+    if (drv.ok) {
+      int k = 0;
+      for (int c = wg * 32; c < DV; c += 64, ++k) rows_store<T>(gen(wb + k * CB), static_cast<T*>(p.y) + yj, ts, row0, nrj, c);
+    }
+    __syncwarp();
   }
   cta.finish();
 }

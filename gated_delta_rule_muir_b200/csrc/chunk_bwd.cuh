@@ -402,43 +402,60 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
     }
   }
   wait_img();
-  // dU -> dv = w dU and dw = v dU, straight into the gradients; this thread's w
-  // and v pieces are loaded while the last product runs
-  constexpr int NCH = DV / 32;  // 16-column chunks per thread
-  const int64_t vo = toff(p, s.b, s.tok0 + (t < Cs ? t : 0), s.h, DV);  // rows past the unit: unused
-  Pack8<T> pw[NCH][2], pv[NCH][2];
+  // dU -> dv = w dU and dw = v dU by 32 x 32 row blocks (rows_fill, rows_store):
+  // w and v come in whole lines, into dO's tile (free since its two products)
+  // while the last product runs where they fit there, and dv, dw go out through
+  // the A tile's memory once that product has completed.
+  constexpr uint32_t IB = row_block_bytes<T>(), OB = row_block_bytes<float>();
+  constexpr int NCK = (DV + 63) / 64;  // 32-column chunks per warp
+  constexpr bool kFillUnder = 8u * NCK * 2u * IB <= 2u * TBP;
+  static_assert(8u * 2u * OB <= 2u * TB, "output row blocks exceed the A tile");
+  static_assert(8u * NCK * 2u * IB <= 2u * TB + 2u * TBP, "input row blocks exceed the free tiles");
+  const int ln = tid & 31, row0 = 32 * (warp & 3);
+  const int64_t ts = (int64_t)p.H * DV, o0 = toff(p, s.b, s.tok0, s.h, DV);
+  const uint32_t inb = base + 2 * TB + (uint32_t)warp * NCK * 2u * IB;  // after the A tile
+  const uint32_t outb = base + (uint32_t)warp * 2u * OB;
+  auto gen = [&](uint32_t x) { return sm + (x - smem_u32(sm)); };  // shared address -> generic pointer
+  auto fill = [&] {
+    if (drv.ok) {
+      int k = 0;
+      for (int c = wg * 32; c < DV; c += 64, ++k) {
+        rows_fill<T>(inb + 2u * k * IB, static_cast<const T*>(p.w) + o0, ts, row0, Cs, c);
+        rows_fill<T>(inb + (2u * k + 1u) * IB, static_cast<const T*>(p.v) + o0, ts, row0, Cs, c);
+      }
+    }
+    cp_async_wait_all();
+  };
   drv.run_overlap([&] { mma_tiles(cta.tmem + cU, AT, B3, Cs / 16, idT, NS, true); },
                   [&] {
-                    if (t < Cs) {
-#pragma unroll
-                      for (int k = 0; k < NCH; ++k)
-#pragma unroll
-                        for (int h8 = 0; h8 < 2; ++h8) {
-                          const int c = wg * 16 + 32 * k + 8 * h8;
-                          pw[k][h8].ld(static_cast<const T*>(p.w) + vo + c);
-                          pv[k][h8].ld(static_cast<const T*>(p.v) + vo + c);
-                        }
-                    }
+                    if constexpr (kFillUnder) fill();
                   });
+  if constexpr (!kFillUnder) fill();
+  __syncwarp();
+  {
+    int k = 0;
+    for (int c = wg * 32; c < DV; c += 64, ++k) {
+      float v[32];
+      tmem_ld32(cta.tmem + lane + cU + c, v);
 #pragma unroll
-  for (int k = 0; k < NCH; ++k) {
-    const int c = wg * 16 + 32 * k;
-    float v[16];
-    tmem_ld16(cta.tmem + lane + cU + c, v);
-    if (t < Cs && drv.ok) {
-#pragma unroll
-      for (int h8 = 0; h8 < 2; ++h8) {
-        float ww[8], vv[8], a8[8], b8[8];
-        pw[k][h8].get(ww);
-        pv[k][h8].get(vv);
+      for (int q8 = 0; q8 < 4; ++q8) {
+        float ww[8], vv[8];
+        row8_get<T>(gen(inb + 2u * k * IB), ln, q8, ww);
+        row8_get<T>(gen(inb + (2u * k + 1u) * IB), ln, q8, vv);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          a8[j] = ww[j] * v[8 * h8 + j];
-          b8[j] = vv[j] * v[8 * h8 + j];
+          ww[j] *= v[8 * q8 + j];
+          vv[j] *= v[8 * q8 + j];
         }
-        Elt<T>::st8(static_cast<T*>(q.dv) + vo + c + 8 * h8, a8);
-        Elt<T>::st8(static_cast<T*>(q.dw) + vo + c + 8 * h8, b8);
+        row8_put(gen(outb), ln, q8, ww);
+        row8_put(gen(outb + OB), ln, q8, vv);
       }
+      __syncwarp();
+      if (drv.ok) {
+        rows_store<T>(gen(outb), static_cast<T*>(q.dv) + o0, ts, row0, Cs, c);
+        rows_store<T>(gen(outb + OB), static_cast<T*>(q.dw) + o0, ts, row0, Cs, c);
+      }
+      __syncwarp();
     }
   }
   cta.finish();
