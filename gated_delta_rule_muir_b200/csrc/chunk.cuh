@@ -857,21 +857,15 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
   tmem_to_b(B1, cZ, DV, 1.f);
   wait_img();
   drv.run([&] { mma_tiles(cta.tmem + cUt, A, B1, Cs / 16, idV, NS, false); });
-  if (p.wsave) {  // the backward pass reuses W and Ut
+  auto no_mask = [](int, int, float(&)[32]) {};
+  if (p.wsave) {  // the backward pass reuses W and Ut: out in whole lines through
+                  // the A tile's memory (its last product has completed)
     float* wo = p.wsave + (int64_t)blockIdx.x * Cs * DK;
     float* uo = p.usave + (int64_t)blockIdx.x * Cs * DV;
-    for (int c = wg * 16; c < DK; c += 32) {
-      float v[16];
-      tmem_ld16(cta.tmem + lane + cW + c, v);
-      if (t < Cs)
-        stg_row16(wo + t * DK + c, v);
-    }
-    for (int c = wg * 16; c < DV; c += 32) {
-      float v[16];
-      tmem_ld16(cta.tmem + lane + cUt + c, v);
-      if (t < Cs)
-        stg_row16(uo + t * DV + c, v);
-    }
+    float* scr = reinterpret_cast<float*>(sm);
+    drain_rows(cta.tmem + lane, cW, DK, wo, DK, Cs, scr, drv.ok, no_mask);
+    drain_rows(cta.tmem + lane, cUt, DV, uo, DV, Cs, scr, drv.ok, no_mask);
+    __syncthreads();  // the scratch is read before (X*Gsuf)^T is staged over it
   }
   // ---- phase 2, A = (A*Gsuf)^T staged once for both of its products:
   //   D_Phi = (A*Gsuf)^T W (Phi = Diag(Gam_C) - D_Phi in the epilogue), Psi = (A*Gsuf)^T (-Ut) + (K*Gsuf)^T U
@@ -982,13 +976,8 @@ __global__ void __launch_bounds__(256, 1) maps_kernel(ChunkParams p) {
       map_put_q(ma, mg, DK, t, c + 8, b8);
     }
   }
-  for (int c = wg * 16; c < DV; c += 32) {
-    float v[16];
-    tmem_ld16(cta.tmem + lane + cOl + c, v);
-    if (t < Cs && drv.ok) {
-      stg_row16(ol + (int64_t)t * DV + c, v);
-    }
-  }
+  // Oloc out in whole lines through B2's memory (its last product has completed)
+  drain_rows(cta.tmem + lane, cOl, DV, ol, DV, Cs, reinterpret_cast<float*>(sm + 4 * TBP), drv.ok, no_mask);
   cta.finish();
 }
 

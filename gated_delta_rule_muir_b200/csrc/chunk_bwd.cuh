@@ -397,10 +397,11 @@ __global__ void __launch_bounds__(256, 1) bwd_dz_kernel(ChunkParams p, BwdBufs q
       for (int j = 0; j < 8; ++j) { a8[j] = v[j]; b8[j] = v[8 + j]; }
       put_mn(B3, t, c, a8);
       put_mn(B3, t, c + 8, b8);
-      if (drv.ok)
-        stg_row16(dZo + t * DV + c, v);
     }
   }
+  // dZ out in whole lines through dO's memory (free since its two products)
+  drain_rows(cta.tmem + lane, cZ, DV, dZo, DV, Cs, reinterpret_cast<float*>(sm + (base + 2 * TB - smem_u32(sm))),
+             drv.ok, [](int, int, float(&)[32]) {});
   wait_img();
   // dU -> dv = w dU and dw = v dU by 32 x 32 row blocks (rows_fill, rows_store):
   // w and v come in whole lines, into dO's tile (free since its two products)
