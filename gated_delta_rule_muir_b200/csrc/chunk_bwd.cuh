@@ -810,12 +810,26 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
           al[tt] = expf(__ldg(p.la + o));
         }
       }
-      const float* sc = side == 0 ? pre : suf;
+      // the block-relative decay products of these 16 tokens, formed from their
+      // alphas in the decay kernel's order (so equal to its pre and suf tables):
+      // pre_t from the block start through t (left phase), suf_s over the tokens
+      // after s to the block end (right phase)
+      if (side == 0) {
+        float run = 1.f;
 #pragma unroll
-      for (int tt = 0; tt < SB; ++tt) {
-        const float f = sc[(SB * J + tt) * DK + i];
-        acc[0][tt] *= f;
-        acc[1][tt] *= f;
+        for (int tt = 0; tt < SB; ++tt) {
+          run *= al[tt];
+          acc[0][tt] *= run;
+          acc[1][tt] *= run;
+        }
+      } else {
+        float run = 1.f;
+#pragma unroll
+        for (int tt = SB - 1; tt >= 0; --tt) {
+          acc[0][tt] *= run;
+          acc[1][tt] *= run;
+          run *= al[tt];
+        }
       }
       // Diagonal block, exact: pairs ss < tt inside the block go by sub-pivots
       // (halves of 8, 4, 2, 1 tokens), where Gam_{tt<-ss} = fac_tt * fac_ss with
