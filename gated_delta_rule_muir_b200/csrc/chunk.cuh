@@ -496,46 +496,53 @@ struct Rows {
 };
 
 // ---------------------------------------------------------------------------
-// decay_kernel: one CTA per unit, thread = key channel.
+// decay_kernel: one CTA per unit, thread = (16-token block, key channel).
 //   pre[t]  = prod_{u=start(block)..t} alpha_u     suf[t]  = prod_{u=t+1..end(block)} alpha_u
 //   gam[t]  = prod_{u=0..t} alpha_u               gsuf[t] = prod_{u=t+1..Cs-1} alpha_u
 // built as running products of alphas inside blocks and products of whole-block
-// totals across blocks (no division, every factor in [0, 1]).
+// totals across blocks (no division, every factor in [0, 1]). Each thread walks
+// its block's 16 tokens; the block totals meet in shared memory, and the
+// products across blocks are taken in token order (before a block) and in
+// reverse token order (after it).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) decay_kernel(ChunkParams p) {
-  const int dk = p.dk, Cs = p.Cs;
+__global__ void __launch_bounds__(1024) decay_kernel(ChunkParams p) {
+  __shared__ float tot[8][128];  // block totals: Cs / 16 <= 8 blocks, dk <= 128 channels
+  const int dk = p.dk, Cs = p.Cs, nb = Cs / SB;
   const SubIdx s = sub_of(p, blockIdx.x, p.nsub, Cs);
-  const int i = threadIdx.x;
-  if (i >= dk) return;
+  const int i = threadIdx.x % dk, jb = threadIdx.x / dk;
+  const bool on = jb < nb;
   float* pre = p.dec + (int64_t)blockIdx.x * 4 * Cs * dk;
   float* suf = pre + Cs * dk;
   float* gam = suf + Cs * dk;
   float* gsuf = gam + Cs * dk;
-  const float* la = p.la + toff(p, s.b, s.tok0, s.h, dk) + i;
   const int64_t stride = (int64_t)p.H * dk;
-  float run = 1.f, before = 1.f;
-#pragma unroll 16
-  for (int t = 0; t < Cs; ++t) {
-    const float a = expf(__ldg(la + t * stride));
-    if ((t & (SB - 1)) == 0) {
-      before *= run;
-      run = a;
-    } else {
-      run *= a;
+  const float* la = p.la + toff(p, s.b, s.tok0 + (on ? jb * SB : 0), s.h, dk) + i;
+  float a[SB], pr[SB];
+  float run = 1.f;
+  if (on) {
+#pragma unroll
+    for (int u = 0; u < SB; ++u) a[u] = expf(__ldg(la + u * stride));
+#pragma unroll
+    for (int u = 0; u < SB; ++u) {
+      run *= a[u];
+      pr[u] = run;
+      pre[(jb * SB + u) * dk + i] = run;
     }
-    pre[t * dk + i] = run;
-    gam[t * dk + i] = before * run;
+    tot[jb][i] = run;
   }
-  float after = 1.f, srun = 1.f;
-#pragma unroll 16
-  for (int t = Cs - 1; t >= 0; --t) {
-    if ((t & (SB - 1)) == SB - 1) {
-      srun = 1.f;
-      if (t + SB < Cs) after *= pre[(t + SB) * dk + i];
-    }
-    suf[t * dk + i] = srun;
-    gsuf[t * dk + i] = srun * after;
-    srun *= expf(__ldg(la + t * stride));
+  __syncthreads();
+  if (!on) return;
+  float before = 1.f, after = 1.f;
+  for (int J = 0; J < jb; ++J) before *= tot[J][i];
+  for (int J = nb - 1; J > jb; --J) after *= tot[J][i];
+  float srun = 1.f;
+#pragma unroll
+  for (int u = SB - 1; u >= 0; --u) {
+    const int o = (jb * SB + u) * dk + i;
+    gam[o] = before * pr[u];
+    suf[o] = srun;
+    gsuf[o] = srun * after;
+    srun *= a[u];
   }
 }
 
