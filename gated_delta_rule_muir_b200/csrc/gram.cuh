@@ -76,7 +76,7 @@ constexpr uint32_t gram_smem_bytes(int NS) {
   return 1024u                                      // alignment of the swizzled tiles
          + 2u * (NS > 1 ? 2u : 1u) * 128u * DK * 2u  // XL, YL: hi planes, and lo planes for NS > 1
          + 16u * DK * 4u                     // totals of the 8-blocks (log2)
-         + 4u * 8u * DK * 4u                 // rows of one diagonal block: k, qt, a, alpha
+         + 4u * 16u * DK * 4u                // rows of two diagonal blocks: k, qt, a, alpha
          + kZeroBuf;
 }
 
@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
   const auto YL = kmajor_tile<DK>(base + PL * LB, (PL - 1) * LB);
   constexpr bool kSw = DK % 64 == 0;
   float* tot = reinterpret_cast<float*>(sma + 2 * PL * LB);  // [16][DK]
-  float* drow = tot + 16 * DK;                               // [4][8][DK]
-  const uint32_t zbuf = base + 2 * PL * LB + (16u * DK + 4u * 8u * DK) * 4u;
+  float* drow = tot + 16 * DK;                               // [4][16][DK]
+  const uint32_t zbuf = base + 2 * PL * LB + (16u * DK + 4u * 16u * DK) * 4u;
   uint8_t* out = p.gr + (int64_t)blockIdx.x * 4 * sq_bytes(Cs);
   const int64_t tok_stride = (int64_t)p.H * DK;
   const int64_t row0 = toff(p, s.b, s.tok0, s.h, DK);  // token 0 of the unit, channel 0
@@ -256,16 +256,17 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
     }
   };
 
-  // ---- the 8x8 diagonal blocks, one per step, on the CUDA cores ------------
-  // thread (row t, lane ln of 32) holds CH = DK/32 channels; for s = t, t-1, ...
-  // the running product Gam_{t<-s} = Gam_{t<-s+1} alpha_{s+1} scales both right
-  // operands; the 32 partial sums (4 Grams x 8 columns) are reduced over the 32
-  // lanes of the row, after which lane ln holds Gram ln/8, column ln%8.
-  const int npieces = 8 * G;
+  // ---- the 8x8 diagonal blocks, two per step, on the CUDA cores -----------
+  // warp w takes row w of block J (w + 1 pairs) and row 7 - w of block J + 1
+  // (8 - w pairs): 9 pairs for every warp. Thread (row t, lane ln of 32) holds
+  // CD = DK/32 channels; for s = t, t-1, ... the running product
+  // Gam_{t<-s} = Gam_{t<-s+1} alpha_{s+1} scales both right operands; the 32
+  // partial sums (4 Grams x 8 columns) are reduced over the 32 lanes of the row,
+  // after which lane ln holds Gram ln/8, column ln%8.
   Pack8<T> fk, fe, fq, fg;
   Pack8<float> fl;
-  auto fetch = [&](int J) {
-    if (tid < npieces) {
+  auto fetch = [&](int J, int nblk) {  // rows of blocks J .. J + nblk - 1, one piece per thread
+    if (tid < nblk * 8 * G) {
       const int tok = tid / G, cg = tid % G;
       const int64_t o = row0 + (int64_t)(8 * J + tok) * tok_stride + 8 * cg;
       fk.ld(kp + o);
@@ -275,8 +276,8 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
       fl.ld(p.la + o);
     }
   };
-  auto put_rows = [&] {
-    if (tid < npieces) {
+  auto put_rows = [&](int nblk) {
+    if (tid < nblk * 8 * G) {
       const int tok = tid / G, cg = tid % G;
       float kk[8], ee[8], qq[8], gg[8], la[8], rr[8];
       fk.get(kk);
@@ -292,24 +293,20 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
         qq[j] = rr[j] * gg[j] * qq[j];
       }
       float* d0 = drow + tok * DK + 8 * cg;
-      Elt<float>::st8(d0 + 0 * 8 * DK, kk);
-      Elt<float>::st8(d0 + 1 * 8 * DK, qq);
-      Elt<float>::st8(d0 + 2 * 8 * DK, ee);
-      Elt<float>::st8(d0 + 3 * 8 * DK, la);
+      Elt<float>::st8(d0 + 0 * 16 * DK, kk);
+      Elt<float>::st8(d0 + 1 * 16 * DK, qq);
+      Elt<float>::st8(d0 + 2 * 16 * DK, ee);
+      Elt<float>::st8(d0 + 3 * 16 * DK, la);
     }
   };
   constexpr int CD = DK / 32;  // channels per lane in the diagonal blocks
-  // block J; its rows were fetched before, those of block `next` (if any) are
-  // fetched here, under this block's arithmetic
-  auto diag_step = [&](int J, int next) {
-    __syncthreads();  // drow is free
-    put_rows();
-    __syncthreads();
-    if (next >= 0) fetch(next);
-    const int t = tid >> 5, ln = tid & 31, c0 = ln * CD;
+  // row t of block J, whose rows sit at drow tokens 8 blk ..
+  auto diag_row = [&](int J, int blk, int t) {
+    const int ln = tid & 31, c0 = ln * CD;
+    const float* dr = drow + blk * 8 * DK;
     float xk[CD], xq[CD], gm[CD];
-    lds_vec(drow + 0 * 8 * DK + t * DK + c0, xk);
-    lds_vec(drow + 1 * 8 * DK + t * DK + c0, xq);
+    lds_vec(dr + 0 * 16 * DK + t * DK + c0, xk);
+    lds_vec(dr + 1 * 16 * DK + t * DK + c0, xq);
 #pragma unroll
     for (int j = 0; j < CD; ++j) gm[j] = 1.f;
     float v[32];
@@ -318,9 +315,9 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       if (ss <= t) {
         float yk[CD], ya[CD], al[CD];
-        lds_vec(drow + 0 * 8 * DK + ss * DK + c0, yk);
-        lds_vec(drow + 2 * 8 * DK + ss * DK + c0, ya);
-        lds_vec(drow + 3 * 8 * DK + ss * DK + c0, al);
+        lds_vec(dr + 0 * 16 * DK + ss * DK + c0, yk);
+        lds_vec(dr + 2 * 16 * DK + ss * DK + c0, ya);
+        lds_vec(dr + 3 * 16 * DK + ss * DK + c0, al);
 #pragma unroll
         for (int j = 0; j < CD; ++j) {
           yk[j] *= gm[j];
@@ -353,6 +350,18 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
     *reinterpret_cast<__nv_bfloat16*>(img + o) = hb;
     *reinterpret_cast<__nv_bfloat16*>(img + sq_half(Cs) + o) = lb;
   };
+  // blocks J (.. J + 1 when nblk = 2); their rows were fetched before, those of
+  // the next step (nnext blocks from `next`, if any) are fetched here, under this
+  // step's arithmetic
+  auto diag_step = [&](int J, int nblk, int next, int nnext) {
+    __syncthreads();  // drow is free
+    put_rows(nblk);
+    __syncthreads();
+    if (next >= 0) fetch(next, nnext);
+    const int w = tid >> 5;
+    diag_row(J, 0, w);
+    if (nblk == 2) diag_row(J + 1, 1, 7 - w);
+  };
 
   const uint32_t id = idesc_bf16(128, Cs, 0, 0);
   uint32_t phase = 0;
@@ -371,9 +380,13 @@ __global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) gram_kernel(ChunkParams 
     // the diagonal-block rows are fetched level by level, so that no prefetched
     // registers stay live across the staging
     const int it1 = (lev + 1) * nb / nlev;
-    if (it < it1) fetch(it);
+    if (it < it1) fetch(it, it1 - it < 2 ? it1 - it : 2);
     if (lev > 0) drain(lev - 1);  // the other slot, complete since the last wait
-    for (; it < it1; ++it) diag_step(it, it + 1 < it1 ? it + 1 : -1);
+    while (it < it1) {
+      const int nblk = it1 - it < 2 ? it1 - it : 2, nx = it + nblk;
+      diag_step(it, nblk, nx < it1 ? nx : -1, it1 - nx < 2 ? it1 - nx : 2);
+      it = nx;
+    }
     ok = __syncthreads_and(tid == 0 ? (mbar_wait(&bar, phase) ? 1 : 0) : 1) != 0;  // one poller
     phase ^= 1u;
     tc_fence_after();
