@@ -44,10 +44,12 @@ def _start(lib: str, extra: list[str], verbose: bool):
     return subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
 
 
-def _finish(proc, lib: str) -> None:
+def _finish(proc, lib: str, verbose: bool) -> None:
     out, err = proc.communicate()
     if proc.returncode != 0:
         raise RuntimeError(f"nvcc failed ({proc.returncode}):\n{out}\n{err}")
+    if verbose and (out or err):
+        print(out + err, file=sys.stderr)  # e.g. the -Xptxas -v report
     os.replace(lib + ".tmp", lib)
 
 
@@ -59,7 +61,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     if check and (force or needs_build(CHECK_LIB)):
         jobs.append((CHECK_LIB, _start(CHECK_LIB, [*(extra or []), "-DMUIR_CHECK"], verbose)))
     for lib, proc in jobs:
-        _finish(proc, lib)
+        _finish(proc, lib, verbose)
     return LIB
 
 

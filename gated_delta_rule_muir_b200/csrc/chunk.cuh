@@ -1330,8 +1330,8 @@ __global__ void apply_map_kernel(const float* __restrict__ Phi, const float* __r
 // warpgroups take alternate 32-column chunks.
 // ---------------------------------------------------------------------------
 template <int DK, int DV, typename T, int NS>
-__global__ void __launch_bounds__(256, 1) out_kernel(ChunkParams p, const uint8_t* ma, const float* ol, int units,
-                                                     int ulen) {
+__global__ void __launch_bounds__(256, NS == 1 ? 2 : 1) out_kernel(ChunkParams p, const uint8_t* ma, const float* ol,
+                                                                   int units, int ulen) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ uint64_t bar, bar_cp, bar_s0;
   __shared__ uint32_t tslot;
@@ -1343,7 +1343,10 @@ __global__ void __launch_bounds__(256, 1) out_kernel(ChunkParams p, const uint8_
   const MapGeom g = map_geom(DK, ulen);
   const int nq = g.ntile - 1;
   const uint32_t base = smem_u32(sm);
-  const uint32_t s_off = (uint32_t)nq * g.tile;
+  // one pass reads only the hi planes of Q', so only they are copied: with
+  // chunk 128 the CTA then needs 96 KB and two share an SM
+  const uint32_t qt = NS == 1 ? g.half : g.tile;  // shared bytes per Q' tile
+  const uint32_t s_off = (uint32_t)nq * qt;
   const Tile Sb{base + s_off, base + s_off + DK * DV * 2u, 128u, DK * 16u};
   if (tid == 0) {
     mbar_init(&bar_cp, 1);
@@ -1352,8 +1355,12 @@ __global__ void __launch_bounds__(256, 1) out_kernel(ChunkParams p, const uint8_
   TcCta cta;
   cta.init(&tslot, &bar, tmem_cols_for(nq * DV));
   if (tid == 0) {
-    mbar_expect_tx(&bar_cp, nq * g.tile);
-    bulk_g2s_big(base, ma + uid * g.unit + g.tile, nq * g.tile, &bar_cp);
+    mbar_expect_tx(&bar_cp, nq * qt);
+    if (NS == 1) {
+      for (int j = 0; j < nq; ++j) bulk_g2s_big(base + j * qt, ma + uid * g.unit + (1 + j) * g.tile, qt, &bar_cp);
+    } else {
+      bulk_g2s_big(base, ma + uid * g.unit + g.tile, nq * g.tile, &bar_cp);
+    }
   }
   uint32_t ph_s0 = 0;
   const bool s0_ok = stage_raw<true>(Sb, p.S_chunks + uid * DK * DV, DK, DV, 1.f, &bar_s0, ph_s0);
@@ -1363,7 +1370,7 @@ __global__ void __launch_bounds__(256, 1) out_kernel(ChunkParams p, const uint8_
   if (drv.ok)
     drv.run([&] {
       for (int j = 0; j < nq; ++j) {
-        const Tile Q{base + j * g.tile, base + j * g.tile + g.half, 128u, DK * 16u};
+        const Tile Q{base + j * qt, base + j * qt + (NS == 1 ? 0u : g.half), 128u, DK * 16u};
         mma_tiles(cta.tmem + j * DV, Q, Sb, DK / 16, id, NS, false);
       }
     });
