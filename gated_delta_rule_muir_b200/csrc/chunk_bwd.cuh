@@ -531,64 +531,96 @@ __global__ void __launch_bounds__(256, 1) bwd_grads_kernel(ChunkParams p, BwdBuf
   if (tid == 0) mbar_expect_tx(&bar_cp, mat_dkdv + mat_csdv);
   raw_issue(R0, q.dSC + u * DK * DV, DK, DV, &bar_cp);
   raw_issue(R2, q.P + u * Cs * DV, Cs, DV, &bar_cp);
-  if (tid < DK) {
+  if (warp < 4) {
     // Everything that reaches the unit's last cumulative log-decay L_{C-1}: the
     // decay of S0 (Gam_C dGam_C, dGam_C = rowsum(dS_C * S0)) plus the suffix
     // factors of K_s and A_s (sum_s K_s dK_s + A_s dA_s, with dK_s = U dS_C^T and
     // dA_s = -P dS_C^T). Since S_C = Diag(Gam_C) S0 + K_s^T U - A_s^T P, the sum
     // is rowsum(dS_C * S_C), with S_C the next unit's start state (or the state
-    // after the sequence's last unit).
-    const float* d = q.dSC + u * DK * DV + tid * DV;
-    const float* sc = (s.n + 1 < p.nsub ? q.S_chunks + (u + 1) * DK * DV
-                                        : p.S_end + ((int64_t)s.b * p.H + s.h) * DK * DV) + tid * DV;
-    float acc = 0.f;
-#pragma unroll 4
-    for (int j = 0; j < DV; j += 4) {
-      const float4 a = *reinterpret_cast<const float4*>(d + j), c = *reinterpret_cast<const float4*>(sc + j);
-      acc += a.x * c.x + a.y * c.y + a.z * c.z + a.w * c.w;
+    // after the sequence's last unit). The first four warps take a row at a time,
+    // each load reading whole lines, while the other four start staging U.
+    const float* d0 = q.dSC + u * DK * DV;
+    const float* s0 = s.n + 1 < p.nsub ? q.S_chunks + (u + 1) * DK * DV
+                                       : p.S_end + ((int64_t)s.b * p.H + s.h) * DK * DV;
+    const int ln = tid & 31;
+    constexpr int RB = 8;  // rows per batch of loads
+    for (int r0 = warp; r0 < DK; r0 += 4 * RB) {
+      float acc[RB];
+#pragma unroll
+      for (int k = 0; k < RB; ++k) {
+        const int row = r0 + 4 * k;
+        acc[k] = 0.f;
+        if (row < DK && 4 * ln < DV) {
+          const float4 a = *reinterpret_cast<const float4*>(d0 + row * DV + 4 * ln);
+          const float4 c = *reinterpret_cast<const float4*>(s0 + row * DV + 4 * ln);
+          acc[k] = a.x * c.x + a.y * c.y + a.z * c.z + a.w * c.w;
+        }
+      }
+      for (int j = 128; j < DV; j += 128) {  // wider rows than one line per lane
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+          const int row = r0 + 4 * k;
+          if (row < DK) {
+            const float4 a = *reinterpret_cast<const float4*>(d0 + row * DV + j + 4 * ln);
+            const float4 c = *reinterpret_cast<const float4*>(s0 + row * DV + j + 4 * ln);
+            acc[k] += a.x * c.x + a.y * c.y + a.z * c.z + a.w * c.w;
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < RB; ++k) {
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], m);
+        const int row = r0 + 4 * k;
+        if (ln == 0 && row < DK) q.eC[u * DK + row] = acc[k];
+      }
     }
-    q.eC[u * DK + tid] = acc;
   }
   stage_U(R1);
   raw_wait();
   raw_convert<false>(R0, DK, DV, 1.f);
   raw_convert<false>(R2, Cs, DV, -1.f);
+  // TMEM: two pairs of 128-column accumulators, [0, 256) and [256, 512), taken in
+  // turn, so that the drain of one pass runs while the tensor core does the next.
   drv.run([&] {
     mma_ops(cta.tmem + 0, kview(R1), kview(R0), DV / 16, idK, NS, false);
     mma_ops(cta.tmem + 128, kview(R2), kview(R0), DV / 16, idK, NS, false);
   });
-  drain(0, DK, g4 + 2 * Cs * DK, DK, 0);    // dKs
-  drain(128, DK, g4 + 3 * Cs * DK, DK, 0);  // dAs
-  // pass 2: R1 = U, R2 = -P stay; R0 = dO, then dZ
+  // pass 2a: R1 = U, R2 = -P stay; R0 = dO
   stage_dO(R0);
-  drv.run([&] {
-    mma_ops(cta.tmem + 0, kview(R0), kview(R1), DV / 16, idC, NS, false);    // dN^qk
-    mma_ops(cta.tmem + 128, kview(R0), kview(R2), DV / 16, idC, NS, false);  // dN^qa
-  });
+  drv.run_overlap([&] {
+                    mma_ops(cta.tmem + 256, kview(R0), kview(R1), DV / 16, idC, NS, false);  // dN^qk
+                    mma_ops(cta.tmem + 384, kview(R0), kview(R2), DV / 16, idC, NS, false);  // dN^qa
+                  },
+                  [&] {
+                    drain(0, DK, g4 + 2 * Cs * DK, DK, 0);    // dKs
+                    drain(128, DK, g4 + 3 * Cs * DK, DK, 0);  // dAs
+                  });
+  // pass 2b: R0 = dZ
   if (tid == 0) mbar_expect_tx(&bar_cp, mat_csdv);
   raw_issue(R0, q.dZ + u * Cs * DV, Cs, DV, &bar_cp);
-  drain(0, Cs, dG + 2 * Cs * Cs, Cs, 2);
-  drain(128, Cs, dG + 3 * Cs * Cs, Cs, 2);
+  drain(256, Cs, dG + 2 * Cs * Cs, Cs, 2);
   raw_wait();
   raw_convert<false>(R0, Cs, DV, 1.f);
-  drv.run([&] {
-    mma_ops(cta.tmem + 256, kview(R0), kview(R1), DV / 16, idC, NS, false);  // dM^kk
-    mma_ops(cta.tmem + 384, kview(R0), kview(R2), DV / 16, idC, NS, false);  // dM^ka
-  });
+  drv.run_overlap([&] {
+                    mma_ops(cta.tmem + 0, kview(R0), kview(R1), DV / 16, idC, NS, false);    // dM^kk
+                    mma_ops(cta.tmem + 128, kview(R0), kview(R2), DV / 16, idC, NS, false);  // dM^ka
+                  },
+                  [&] { drain(384, Cs, dG + 3 * Cs * Cs, Cs, 2); });
   // pass 3: R0 = dZ stays, R1 = S0, R2 = dO
   if (tid == 0) mbar_expect_tx(&bar_cp, mat_dkdv);
   raw_issue(R1, q.S_chunks + u * DK * DV, DK, DV, &bar_cp);
   stage_dO(R2);
-  drain(256, Cs, dG + 0 * Cs * Cs, Cs, 1);
-  drain(384, Cs, dG + 1 * Cs * Cs, Cs, 1);
+  drain(0, Cs, dG + 0 * Cs * Cs, Cs, 1);
   raw_wait();
   raw_convert<false>(R1, DK, DV, 1.f);
-  drv.run([&] {
-    mma_ops(cta.tmem + 0, kview(R2), kview(R1), DV / 16, idK, NS, false);    // dQp
-    mma_ops(cta.tmem + 128, kview(R0), kview(R1), DV / 16, idK, NS, false);  // dKp
-  });
-  drain(0, DK, g4 + 0 * Cs * DK, DK, 0);
-  drain(128, DK, g4 + 1 * Cs * DK, DK, 0);
+  drv.run_overlap([&] {
+                    mma_ops(cta.tmem + 256, kview(R2), kview(R1), DV / 16, idK, NS, false);  // dQp
+                    mma_ops(cta.tmem + 384, kview(R0), kview(R1), DV / 16, idK, NS, false);  // dKp
+                  },
+                  [&] { drain(128, Cs, dG + 1 * Cs * Cs, Cs, 1); });
+  drain(256, DK, g4 + 0 * Cs * DK, DK, 0);
+  drain(384, DK, g4 + 1 * Cs * DK, DK, 0);
   cta.finish();
 }
 
