@@ -24,11 +24,13 @@
 // with suf_s = prod_{u=s+1..end(I)}, pre_t = prod_{u=start(J)..t} and mid the
 // product of whole blocks in between: every factor is a product of alphas, so
 // it lies in [0, 1] and nothing is divided. Off-diagonal Gram blocks then are
-// tensor-core GEMMs of pivot-scaled operands; the 16x16 diagonal blocks are
-// computed exactly on the CUDA cores with running products.
+// tensor-core GEMMs of pivot-scaled operands; the diagonal blocks (8x8 in the
+// forward Grams, 16x16 in their backward) are computed exactly on the CUDA
+// cores with running products.
 //
 // Kernels (one CTA per (batch, head, unit of Cs = min(chunk, 128) tokens) unless noted):
 //   decay_kernel      pre, suf, Gam_t, Gsuf_t            -> workspace
+//                     (a thread per 16-token block and key channel)
 //   gram_kernel       the 4 Grams (gram.cuh): blocks across the binary tree of
 //                     8-token blocks on tcgen05 (one product per level), the
 //                     exact 8x8 diagonal blocks on the CUDA cores meanwhile
@@ -36,7 +38,7 @@
 //                     T21 = -T22 M21 T11 on tcgen05 (block-Neumann recursion)
 //   maps_kernel       W, Ut, Phi, Psi, Q', Oloc (tcgen05)  -> workspace
 //   compose_kernel    (chunk 256) composes two 128-token half-chunk maps
-//   scan_kernel       sequential over chunks per (batch, head, 32-column slab):
+//   scan_kernel       sequential over chunks per (batch, head, kSlab-column slab):
 //                     S_C = Phi S0 + Psi (tcgen05), states -> workspace
 //   out_kernel        chunk-parallel y = z * (Q' S0 + Oloc) (tcgen05)
 #pragma once

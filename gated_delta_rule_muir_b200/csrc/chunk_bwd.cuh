@@ -947,7 +947,7 @@ __global__ void __launch_bounds__(256, 1) bwd_gram_kernel(ChunkParams p, BwdBufs
 }
 
 // ---------------------------------------------------------------------------
-// bwd_final_kernel: per unit, thread = key channel i (then value channel j):
+// bwd_final_kernel: per unit, thread = key channel i:
 //   dL_t = k dKl + qt dQl - k dKr - a dAr + Kp dKp + Qp dQp - Ks dKs - As dAs
 //   dL_{C-1} += sum_s (Ks dKs + As dAs) + Gam_C dGam_C = rowsum(dS_C * S_C)
 //   dlog_alpha_t = sum_{u >= t} dL_u
